@@ -1,0 +1,367 @@
+"""Benchmark of the SGA hot path on B200: decode at 128K context (batch 32).
+
+One step = one pass of the whole path over one batch of queries: the indexer
+over every cached position, top-2048 selection, sparse latent attention and the
+head gate.  The three C-ABI calls issued per step (sga_index_scores,
+sga_topk_select, sga_sparse_mla_attend) are exactly the launches sga_forward
+makes; they are issued separately so CUDA events on the same stream can time
+each kernel inside the timed region.
+
+Prints one JSON line (rank 0).  `--impl reference` times the fp64 CPU oracle
+on the host cores instead (a bounded sample of the same workload).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "SGA decode queries/s at 128K ctx; achieved HBM GB/s vs 8 TB/s roofline"
+UNIT = "queries/s"
+NOMINAL_HBM_GBS = 8000.0
+FALLBACK_HBM_GBS = 6650.0
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default=None, help="workload name (default: decode_b32_ctx128k)")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-sample-queries", type=int, default=0, help="oracle sample size (0 = auto)")
+    return ap.parse_args()
+
+
+def algorithmic_bytes_per_query(ctx: int, top_k: int = 2048) -> dict:
+    """Bytes the method must move per decode query (intermediate scores excluded).
+
+    k_idx: every causal key once (ctx * 128 * 2), q_idx 64*128*2, w 64*2,
+    gathered latent rows top_k * 576 * 2, q 64*576*2, gate 64*2, out 64*512*4,
+    idx top_k * 4.
+    """
+    parts = dict(k_idx=ctx * 256, q_idx=16384, w=128, kv_rows=top_k * 1152, q=73728, gate=128, out=131072,
+                 idx=top_k * 4)
+    parts["total"] = sum(parts.values())
+    parts["indexer"] = parts["k_idx"] + parts["q_idx"] + parts["w"]
+    return parts
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def kernel_counters(kernel_file: str):
+    """ncu DRAM traffic per launch for the dominant kernel, if taken on the current source."""
+    path = os.path.join(ROOT, "profiles", "counters.json")
+    src = os.path.join(ROOT, "sparse_gated_attention_b200", "csrc", kernel_file)
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        entry = d[kernel_file]
+        sha = hashlib.sha256(open(src, "rb").read()).hexdigest()
+        if entry.get("source_sha256") != sha:
+            return None
+        return entry
+    except Exception:
+        return None
+
+
+class ClockSampler:
+    """Samples nvidia-smi clocks and throttle reasons while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu_index = gpu_index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu_index), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        self.lines = []
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except Exception:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [ln for ln in out.splitlines() if ln.strip()]
+        return False
+
+    def summary(self):
+        if not getattr(self, "lines", None):
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                smax = float(f[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def cpu_baseline(wl, n_queries: int = 0, min_seconds: float = 10.0, max_queries: int = 400):
+    """The oracle, as it stands, on a bounded sample of the workload (host cores).
+
+    n_queries > 0 runs exactly that many queries; otherwise queries are run
+    until min_seconds of CPU time have passed (at most max_queries)."""
+    import oracle
+    from sparse_gated_attention_b200 import synth
+
+    sample = synth.custom(batch=1, n_q=1, ctx=wl.ctx, first_pos=wl.first_pos if wl.n_q == 1 else wl.ctx - 1,
+                          k_range=wl.k_range, name=wl.name + "_sample")
+    x = synth.make_inputs(sample, device="cpu", seed=0)
+    oracle.build()
+    threads = oracle.hardware_threads()
+    t0 = time.perf_counter()
+    done = 0
+    while True:
+        oracle.forward(x["q_idx"], x["w"], x["k_idx"], x["q"], x["kv"], x["gate"], x["q_pos"], n_threads=threads)
+        done += 1
+        dt = time.perf_counter() - t0
+        if (n_queries > 0 and done >= n_queries) or (n_queries <= 0 and (dt >= min_seconds or done >= max_queries)):
+            break
+    n_queries = done
+    return {"value": n_queries / dt, "unit": UNIT, "cores": threads, "kind": "oracle",
+            "sample": f"{n_queries} decode queries of {wl.name} (1 sequence, ctx {wl.ctx}, full path, fp64)",
+            "seconds": dt}
+
+
+def run_reference(args, wl, rank):
+    if rank != 0:
+        return
+    steps, warm = args.steps, args.warmup
+    nq = args.cpu_sample_queries or 1
+    for _ in range(warm):
+        cpu_baseline(wl, nq)
+    times = []
+    vals = []
+    for _ in range(steps):
+        r = cpu_baseline(wl, nq)
+        times.append(r["seconds"])
+        vals.append(r)
+    total = sum(times)
+    value = steps * nq / total
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus, "steps": steps,
+        "warmup": warm, "ms_per_step": 1000.0 * total / steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": config_of(wl),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": vals[0]["cores"], "kind": "oracle",
+                         "sample": vals[0]["sample"] + " per step"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def config_of(wl):
+    return {"workload": wl.name, "batch": wl.batch, "queries_per_seq": wl.n_q, "ctx": wl.ctx, "top_k": wl.top_k,
+            "heads": 64, "latent": 576, "index_heads": 64, "index_dim": 128,
+            "l2": "inputs larger than L2 (k_idx+kv rows ~1.16 GB/step vs 126 MB L2), no flush",
+            "parallelism": "replicas"}
+
+
+def main():
+    args = parse_args()
+    from sparse_gated_attention_b200 import synth
+
+    wl = synth.WORKLOADS[args.workload or synth.HEADLINE]
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        run_reference(args, wl, rank)
+        return
+
+    import sparse_gated_attention_b200 as sga
+
+    torch.cuda.set_device(local_rank)
+    dist = None
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    dev = torch.device("cuda", local_rank)
+    sga.load_library()
+
+    x = synth.make_inputs(wl, device=dev, seed=rank)
+    B, T, L, K = wl.batch, wl.n_q, wl.ctx, wl.top_k
+    rows = B * T
+    dims = sga.make_dims(B, T, L, K)
+    ws_all = sga.alloc_workspace(dims, sga.OP_FORWARD, dev)
+    ws_idx = sga.alloc_workspace(dims, sga.OP_INDEX_SCORES, dev)
+    ws_topk = sga.alloc_workspace(dims, sga.OP_TOPK_SELECT, dev)
+    ws_att = sga.alloc_workspace(dims, sga.OP_SPARSE_MLA_ATTEND, dev)
+    scores = torch.empty((B, T, L), dtype=torch.float32, device=dev)
+    idx = torch.empty((B, T, K), dtype=torch.int32, device=dev)
+    out = torch.empty((B, T, 64, 512), dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    splits = 1
+    from sparse_gated_attention_b200 import _binding  # noqa: F401
+
+    att_ws_bytes = sga.workspace_size(dims, sga.OP_SPARSE_MLA_ATTEND)
+    launches_per_step = 3 + (1 if att_ws_bytes > 256 else 0)
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        sga.index_scores(x["q_idx"], x["w"], x["k_idx"], x["q_pos"], scores=scores, ws=ws_idx, stream=stream)
+        if ev is not None:
+            ev[1].record(stream)
+        sga.topk_select(scores, x["q_pos"], top_k=K, idx=idx, ws=ws_topk, stream=stream)
+        if ev is not None:
+            ev[2].record(stream)
+        sga.sparse_mla_attend(x["q"], x["kv"], idx, x["gate"], out=out, ws=ws_att, stream=stream)
+        if ev is not None:
+            ev[3].record(stream)
+
+    for _ in range(max(args.warmup, 3)):
+        step()
+    torch.cuda.synchronize(dev)
+    for w in (ws_idx, ws_topk, ws_att):
+        st = sga.device_status(w)
+        if st != 0:
+            raise RuntimeError(f"device status {st} after warm-up")
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    with ClockSampler(local_rank) as clk:
+        time.sleep(0.3)
+        start.record(stream)
+        for i in range(args.steps):
+            step(evs[i])
+        stop.record(stream)
+        torch.cuda.synchronize(dev)
+    elapsed_ms = start.elapsed_time(stop)
+    if dist is not None:
+        t = torch.tensor([elapsed_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        elapsed_ms = float(t.item())
+    k1 = [e[0].elapsed_time(e[1]) for e in evs]
+    k2 = [e[1].elapsed_time(e[2]) for e in evs]
+    k3 = [e[2].elapsed_time(e[3]) for e in evs]
+
+    # ---- end to end through sga_forward with host buffers (cache resident on the device)
+    host = {k: x[k].cpu().pin_memory() for k in ("q_idx", "w", "q", "gate", "q_pos")}
+    dev_in = {k: torch.empty_like(x[k]) for k in host}
+    out_h = torch.empty((B, T, 64, 512), dtype=torch.float32).pin_memory()
+    idx_h = torch.empty((B, T, K), dtype=torch.int32).pin_memory()
+    h2d = sum(v.numel() * v.element_size() for v in host.values())
+    d2h = out_h.numel() * 4 + idx_h.numel() * 4
+
+    def e2e_step():
+        for k in host:
+            dev_in[k].copy_(host[k], non_blocking=True)
+        sga.forward(dev_in["q_idx"], dev_in["w"], x["k_idx"], dev_in["q"], x["kv"], dev_in["gate"], dev_in["q_pos"],
+                    top_k=K, idx_out=idx, out=out, ws=ws_all, stream=stream)
+        out_h.copy_(out, non_blocking=True)
+        idx_h.copy_(idx, non_blocking=True)
+
+    for _ in range(3):
+        e2e_step()
+    torch.cuda.synchronize(dev)
+    if dist is not None:
+        dist.barrier()
+    s2, e2 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s2.record(stream)
+    for _ in range(args.steps):
+        e2e_step()
+    e2.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = s2.elapsed_time(e2)
+    if dist is not None:
+        t = torch.tensor([e2e_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    if sga.device_status(ws_all) != 0:
+        raise RuntimeError("device status set during the end-to-end run")
+
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+
+    ms_per_step = elapsed_ms / args.steps
+    total_queries = rows * args.steps * world
+    value = total_queries / (elapsed_ms / 1e3)
+    ab = algorithmic_bytes_per_query(L, K)
+    peak, peak_kind = measured_peaks()
+    k1_ms = statistics.mean(k1)
+    k1_bytes = ab["indexer"] * rows
+    k1_gbs = k1_bytes / (k1_ms * 1e-3) / 1e9
+    counters = kernel_counters("sga_index.cu")
+    traffic = None
+    if counters and counters.get("workload") == wl.name:
+        traffic = counters.get("dram_bytes_per_launch")
+    path_gbs = ab["total"] * rows / (ms_per_step * 1e-3) / 1e9
+
+    cpu = None
+    if not args.no_cpu_baseline and world == 1:
+        cpu = cpu_baseline(wl, args.cpu_sample_queries)
+        cpu.pop("seconds", None)
+
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic", "config": config_of(wl),
+        "roofline": {"bound": "hbm", "kernel": "sga_index_kernel", "achieved": k1_gbs, "peak": peak, "unit": "GB/s",
+                     "frac": k1_gbs / peak, "peak_kind": peak_kind, "traffic": traffic,
+                     "algorithmic_bytes_per_launch": k1_bytes},
+        "path_roofline": {"achieved_gbs": path_gbs, "frac_of_8tbs": path_gbs / NOMINAL_HBM_GBS,
+                          "frac_of_measured": path_gbs / peak, "bytes_per_query": ab["total"]},
+        "stages_ms": {"index": k1_ms, "topk": statistics.mean(k2), "attend": statistics.mean(k3)},
+        "cpu_baseline": cpu,
+        "e2e": {"value": total_queries / (e2e_ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h},
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clk.summary(),
+    }
+    print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

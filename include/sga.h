@@ -1,0 +1,168 @@
+/*
+ * sga.h - C ABI of libsga, the B200 (sm_100a) hot path of Sparse Gated
+ * Attention (SGA), the attention of the A.X K2 model.
+ *
+ * For each query the path scores every causal past position with a DSA-style
+ * indexer, keeps the top K (= 2048) positions, runs MLA-style attention in the
+ * latent form (64 heads sharing one 576-wide latent row per token; the first
+ * 512 dims are the value) over only those positions, and multiplies each
+ * head's output by a sigmoid gate.  Sources:
+ *   - archdb "A.X K2", token-selection field: DSA-style indexer, top-2048
+ *     tokens per query, 64 indexer heads of dim 128, ReLU-scored;
+ *     indexer-key-width field: 128 per token.
+ *   - archdb "A.X K2", attention fields: 64 query heads, qk head dim 192
+ *     (128 nope + 64 rope), v head dim 128, KV latent 512, shared rope key 64.
+ *   - archdb "A.X K2", gate field: head-specific sigmoid gate on the attention
+ *     output before o_proj.
+ *   - arXiv abstract "A.X K2 Technical Report": each query reads only 2,048
+ *     positions.
+ * The indexer score is the DSA-style reading
+ *     score(t,s) = sum_j w[t,j] * max(0, q_idx[t,j,:] . k_idx[s,:]),
+ * since the pages name the parts but print no formula.
+ *
+ * Conventions shared by every call
+ *   - All tensors are dense, row-major, innermost dimension contiguous, and live
+ *     in device memory owned by the caller.  bf16 tensors are passed as their
+ *     16-bit patterns (sga_bf16_t).  Pointers to bf16 inputs must be 16-byte
+ *     aligned (they are read by the Tensor Memory Accelerator).
+ *   - B = dims.batch sequences, T = dims.n_q queries per sequence,
+ *     L = dims.kv_stride cache rows per sequence, K = dims.top_k.
+ *     q_pos[b*T + i] is the absolute position t of query i of sequence b;
+ *     positions 0..t are its candidates, so 0 <= t < L is required.
+ *   - Every call is asynchronous on `stream` (a cudaStream_t; NULL = legacy
+ *     default stream), allocates nothing, and does not synchronise.
+ *   - The return value reports host-side validation and launch errors only.
+ *     Errors found on the device (a position or index out of range, a
+ *     bounded wait that ran out) are written to a status word at the start of
+ *     the workspace; read it with sga_get_device_status.  The first device
+ *     error is kept until sga_clear_device_status.
+ *   - Workspace: caller-allocated device memory of at least
+ *     sga_workspace_size(dims, op) bytes, 256-byte aligned.  A zero-filled
+ *     workspace starts with a clear status.  Calls that share a workspace must
+ *     be ordered on one stream.
+ *   - No C++ exception crosses this interface.
+ */
+#ifndef SGA_H_
+#define SGA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define SGA_API __attribute__((visibility("default")))
+#else
+#define SGA_API
+#endif
+
+typedef uint16_t sga_bf16_t; /* bfloat16 bit pattern */
+typedef void* sga_stream_t;  /* cudaStream_t */
+
+typedef enum {
+  SGA_OK = 0,
+  SGA_ERR_INVALID_ARG = 1, /* null/misaligned pointer, bad size, unsupported shape */
+  SGA_ERR_UNSUPPORTED = 2, /* no sm_100 device, or a size beyond the compiled limits */
+  SGA_ERR_WORKSPACE = 3,   /* workspace null, misaligned or too small */
+  SGA_ERR_CUDA = 4,        /* a CUDA runtime call or kernel launch failed */
+  SGA_ERR_TIMEOUT = 5,     /* device: a bounded wait inside a kernel ran out */
+  SGA_ERR_DEVICE_ARG = 6   /* device: a position or index outside its range */
+} sga_status_t;
+
+typedef enum {
+  SGA_OP_INDEX_SCORES = 0,
+  SGA_OP_TOPK_SELECT = 1,
+  SGA_OP_SPARSE_MLA_ATTEND = 2,
+  SGA_OP_FORWARD = 3
+} sga_op_t;
+
+typedef struct {
+  int32_t batch;     /* B >= 1 */
+  int32_t n_q;       /* T >= 1 queries per sequence */
+  int32_t kv_stride; /* L >= 1 cache rows per sequence (capacity) */
+  int32_t top_k;     /* K: a multiple of 64 in [64, 2048]; the method uses 2048 */
+} sga_dims_t;
+
+/* Compiled model constants (archdb "A.X K2" attention, indexer and gate fields). */
+#define SGA_INDEX_HEADS 64 /* Hi */
+#define SGA_INDEX_DIM 128  /* Di */
+#define SGA_HEADS 64       /* H */
+#define SGA_QK_DIM 576     /* Dq = 512 latent + 64 rope */
+#define SGA_V_DIM 512      /* Dv: the latent part is the value */
+#define SGA_TOP_K 2048
+#define SGA_MAX_TOP_K 2048
+/* Softmax scale 192^-0.5 (qk head dim 192 = 128 nope + 64 rope). */
+#define SGA_SOFTMAX_SCALE 0.07216878364870322
+#define SGA_MAX_KV_STRIDE (1 << 30) /* positions are int32; rows * L must fit in int32 */
+
+/* ABI version of this header (bumped on any incompatible change). */
+SGA_API int32_t sga_abi_version(void);
+
+/* Human-readable name of a status code (static string). */
+SGA_API const char* sga_status_string(sga_status_t status);
+
+/* Bytes of workspace `op` needs for `dims`.  SGA_OP_FORWARD covers every op.
+ * Returns SGA_ERR_INVALID_ARG for bad dims or a null `bytes`. */
+SGA_API sga_status_t sga_workspace_size(const sga_dims_t* dims, sga_op_t op, size_t* bytes);
+
+/* Step 1, the indexer (archdb "A.X K2", token-selection field):
+ *   scores[b,i,s] = sum_j w[b,i,j] * max(0, sum_d q_idx[b,i,j,d] * k_idx[b,s,d])
+ * for 0 <= s <= t = q_pos[b,i].  Entries with s > t are left unwritten.
+ *   q_idx  [B][T][64][128] bf16     w      [B][T][64] bf16
+ *   k_idx  [B][L][128] bf16         q_pos  [B][T] int32
+ *   scores [B][T][L] fp32 (output; 16-byte aligned)
+ * Accumulation is fp32; integer-valued inputs whose scores stay below 2^24
+ * give exact scores.  Device error: t outside [0, L) (the row is skipped). */
+SGA_API sga_status_t sga_index_scores(const sga_dims_t* dims, const sga_bf16_t* q_idx, const sga_bf16_t* w,
+                              const sga_bf16_t* k_idx, const int32_t* q_pos, float* scores, void* ws,
+                              size_t ws_bytes, sga_stream_t stream);
+
+/* Step 2, top-K selection (archdb "A.X K2", token-selection field; arXiv
+ * abstract "A.X K2 Technical Report": each query reads 2,048 positions):
+ * for each query, the K positions s <= t with the largest scores[b,i,s],
+ * equal scores going to the lower position (-0.0 counts as +0.0); if t+1 <= K
+ * every position 0..t is kept.  idx[b,i,:] lists them in ascending order,
+ * followed by -1 in unused slots.
+ *   scores [B][T][L] fp32 (entries s > t are not read)   q_pos [B][T] int32
+ *   idx    [B][T][K] int32 (output)
+ * NaN scores give an unspecified selection.  Device error: t outside [0, L). */
+SGA_API sga_status_t sga_topk_select(const sga_dims_t* dims, const float* scores, const int32_t* q_pos, int32_t* idx,
+                             void* ws, size_t ws_bytes, sga_stream_t stream);
+
+/* Steps 3 and 4, sparse MLA attention in latent form plus the head gate
+ * (archdb "A.X K2", attention and gate fields): for each query and head h,
+ *   z_s   = (q[b,i,h,:] . kv[b,s,:]) * 192^-0.5     for s in idx[b,i,:], s >= 0
+ *   o     = sum_s softmax(z)_s * kv[b,s,0:512]
+ *   out[b,i,h,:] = o / (1 + exp(-gate[b,i,h]))      (gate == NULL: no gate)
+ *   q    [B][T][64][576] bf16        kv  [B][L][576] bf16
+ *   idx  [B][T][K] int32, any order, -1 = empty slot (positions are not
+ *        compared with q_pos here; duplicates count twice)
+ *   gate [B][T][64] bf16 or NULL     out [B][T][64][512] fp32 (output)
+ * A query with no valid slot gets zeros.  Device error: an index outside
+ * [-1, L) (the slot is treated as empty). */
+SGA_API sga_status_t sga_sparse_mla_attend(const sga_dims_t* dims, const sga_bf16_t* q, const sga_bf16_t* kv,
+                                   const int32_t* idx, const sga_bf16_t* gate, float* out, void* ws,
+                                   size_t ws_bytes, sga_stream_t stream);
+
+/* The whole path: sga_index_scores -> sga_topk_select -> sga_sparse_mla_attend,
+ * with the scores and (when idx_out is NULL) the indices kept in the workspace.
+ * idx_out [B][T][K] int32 may be NULL; other arguments as above. */
+SGA_API sga_status_t sga_forward(const sga_dims_t* dims, const sga_bf16_t* q_idx, const sga_bf16_t* w,
+                         const sga_bf16_t* k_idx, const sga_bf16_t* q, const sga_bf16_t* kv,
+                         const sga_bf16_t* gate, const int32_t* q_pos, int32_t* idx_out, float* out, void* ws,
+                         size_t ws_bytes, sga_stream_t stream);
+
+/* Synchronises `stream` and returns in *device_status the first device-side
+ * error recorded in the workspace (an sga_status_t value, SGA_OK if none). */
+SGA_API sga_status_t sga_get_device_status(const void* ws, sga_stream_t stream, int32_t* device_status);
+
+/* Clears the workspace status word (asynchronously on `stream`). */
+SGA_API sga_status_t sga_clear_device_status(void* ws, sga_stream_t stream);
+
+#ifdef __cplusplus
+} /* extern "C" */
+#endif
+
+#endif /* SGA_H_ */

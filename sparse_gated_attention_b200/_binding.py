@@ -1,0 +1,216 @@
+"""ctypes binding of libsga (include/sga.h): argument marshalling only.
+
+Every step of the path runs in the CUDA library; this module checks tensor
+shapes, dtypes and devices, allocates outputs and workspaces with PyTorch when
+the caller does not pass them, and forwards raw pointers and the current CUDA
+stream.  There is no fallback: if libsga.so is missing or the device is not an
+sm_100 GPU the calls raise.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libsga.so")
+
+INDEX_HEADS = 64
+INDEX_DIM = 128
+HEADS = 64
+QK_DIM = 576
+V_DIM = 512
+TOP_K = 2048
+
+OP_INDEX_SCORES, OP_TOPK_SELECT, OP_SPARSE_MLA_ATTEND, OP_FORWARD = 0, 1, 2, 3
+STATUS_NAMES = {0: "SGA_OK", 1: "SGA_ERR_INVALID_ARG", 2: "SGA_ERR_UNSUPPORTED", 3: "SGA_ERR_WORKSPACE",
+                4: "SGA_ERR_CUDA", 5: "SGA_ERR_TIMEOUT", 6: "SGA_ERR_DEVICE_ARG"}
+
+EXPORTED = ["sga_abi_version", "sga_status_string", "sga_workspace_size", "sga_index_scores", "sga_topk_select",
+            "sga_sparse_mla_attend", "sga_forward", "sga_get_device_status", "sga_clear_device_status"]
+
+
+class SGAError(RuntimeError):
+    def __init__(self, call: str, status: int):
+        super().__init__(f"{call} failed: {STATUS_NAMES.get(status, status)}")
+        self.status = status
+
+
+class Dims(ctypes.Structure):
+    _fields_ = [("batch", ctypes.c_int32), ("n_q", ctypes.c_int32), ("kv_stride", ctypes.c_int32),
+                ("top_k", ctypes.c_int32)]
+
+
+_lib = None
+
+
+def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
+    """Loads libsga.so (built in-tree by ``sparse_gated_attention_b200.build``)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise RuntimeError(f"libsga.so not found at {path}: build it with `python -m sparse_gated_attention_b200.build`")
+    lib = ctypes.CDLL(path)
+    P, i32, sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_size_t
+    D = ctypes.POINTER(Dims)
+    sig = {
+        "sga_abi_version": (i32, []),
+        "sga_status_string": (ctypes.c_char_p, [ctypes.c_int]),
+        "sga_workspace_size": (ctypes.c_int, [D, ctypes.c_int, ctypes.POINTER(sz)]),
+        "sga_index_scores": (ctypes.c_int, [D, P, P, P, P, P, P, sz, P]),
+        "sga_topk_select": (ctypes.c_int, [D, P, P, P, P, sz, P]),
+        "sga_sparse_mla_attend": (ctypes.c_int, [D, P, P, P, P, P, P, sz, P]),
+        "sga_forward": (ctypes.c_int, [D, P, P, P, P, P, P, P, P, P, P, sz, P]),
+        "sga_get_device_status": (ctypes.c_int, [P, P, ctypes.POINTER(i32)]),
+        "sga_clear_device_status": (ctypes.c_int, [P, P]),
+    }
+    for name, (res, args) in sig.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    _lib = lib
+    return lib
+
+
+def _check(call: str, status: int) -> None:
+    if status != 0:
+        raise SGAError(call, status)
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _ptr(t):
+    return ctypes.c_void_p(0 if t is None else t.data_ptr())
+
+
+def _need(t, name, dtype, shape=None):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name}: expected a torch.Tensor")
+    if t.device.type != "cuda":
+        raise ValueError(f"{name}: must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name}: expected {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name}: must be contiguous")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name}: expected shape {tuple(shape)}, got {tuple(t.shape)}")
+    return t
+
+
+def make_dims(batch: int, n_q: int, kv_stride: int, top_k: int = TOP_K) -> Dims:
+    return Dims(int(batch), int(n_q), int(kv_stride), int(top_k))
+
+
+def workspace_size(dims: Dims, op: int = OP_FORWARD) -> int:
+    out = ctypes.c_size_t(0)
+    _check("sga_workspace_size", load_library().sga_workspace_size(ctypes.byref(dims), int(op), ctypes.byref(out)))
+    return int(out.value)
+
+
+def alloc_workspace(dims: Dims, op: int = OP_FORWARD, device=None) -> torch.Tensor:
+    """A zero-filled workspace (zero = clear device status)."""
+    n = workspace_size(dims, op)
+    return torch.zeros(n, dtype=torch.uint8, device=device or "cuda")
+
+
+def device_status(ws: torch.Tensor, stream=None) -> int:
+    v = ctypes.c_int32(0)
+    _check("sga_get_device_status", load_library().sga_get_device_status(_ptr(ws), _stream(stream), ctypes.byref(v)))
+    return int(v.value)
+
+
+def clear_device_status(ws: torch.Tensor, stream=None) -> None:
+    _check("sga_clear_device_status", load_library().sga_clear_device_status(_ptr(ws), _stream(stream)))
+
+
+def index_scores(q_idx, w, k_idx, q_pos, scores=None, ws=None, stream=None):
+    """Indexer scores [B,T,L] fp32 (entries after each query's position are not written)."""
+    B, T = q_idx.shape[0], q_idx.shape[1]
+    L = k_idx.shape[1]
+    _need(q_idx, "q_idx", torch.bfloat16, (B, T, INDEX_HEADS, INDEX_DIM))
+    _need(w, "w", torch.bfloat16, (B, T, INDEX_HEADS))
+    _need(k_idx, "k_idx", torch.bfloat16, (B, L, INDEX_DIM))
+    _need(q_pos, "q_pos", torch.int32, (B, T))
+    dims = make_dims(B, T, L)
+    if scores is None:
+        scores = torch.empty((B, T, L), dtype=torch.float32, device=q_idx.device)
+    _need(scores, "scores", torch.float32, (B, T, L))
+    if ws is None:
+        ws = alloc_workspace(dims, OP_INDEX_SCORES, q_idx.device)
+    _check("sga_index_scores", load_library().sga_index_scores(
+        ctypes.byref(dims), _ptr(q_idx), _ptr(w), _ptr(k_idx), _ptr(q_pos), _ptr(scores), _ptr(ws), ws.numel(),
+        _stream(stream)))
+    return scores
+
+
+def topk_select(scores, q_pos, top_k: int = TOP_K, idx=None, ws=None, stream=None):
+    """Top-k positions [B,T,K] int32, ascending, -1 padded (ties -> lower position)."""
+    B, T, L = scores.shape
+    _need(scores, "scores", torch.float32, (B, T, L))
+    _need(q_pos, "q_pos", torch.int32, (B, T))
+    dims = make_dims(B, T, L, top_k)
+    if idx is None:
+        idx = torch.empty((B, T, top_k), dtype=torch.int32, device=scores.device)
+    _need(idx, "idx", torch.int32, (B, T, top_k))
+    if ws is None:
+        ws = alloc_workspace(dims, OP_TOPK_SELECT, scores.device)
+    _check("sga_topk_select", load_library().sga_topk_select(
+        ctypes.byref(dims), _ptr(scores), _ptr(q_pos), _ptr(idx), _ptr(ws), ws.numel(), _stream(stream)))
+    return idx
+
+
+def sparse_mla_attend(q, kv, idx, gate=None, out=None, ws=None, stream=None):
+    """Sparse latent attention + sigmoid head gate -> out [B,T,64,512] fp32."""
+    B, T = q.shape[0], q.shape[1]
+    L = kv.shape[1]
+    K = idx.shape[-1]
+    _need(q, "q", torch.bfloat16, (B, T, HEADS, QK_DIM))
+    _need(kv, "kv", torch.bfloat16, (B, L, QK_DIM))
+    _need(idx, "idx", torch.int32, (B, T, K))
+    if gate is not None:
+        _need(gate, "gate", torch.bfloat16, (B, T, HEADS))
+    dims = make_dims(B, T, L, K)
+    if out is None:
+        out = torch.empty((B, T, HEADS, V_DIM), dtype=torch.float32, device=q.device)
+    _need(out, "out", torch.float32, (B, T, HEADS, V_DIM))
+    if ws is None:
+        ws = alloc_workspace(dims, OP_SPARSE_MLA_ATTEND, q.device)
+    _check("sga_sparse_mla_attend", load_library().sga_sparse_mla_attend(
+        ctypes.byref(dims), _ptr(q), _ptr(kv), _ptr(idx), _ptr(gate), _ptr(out), _ptr(ws), ws.numel(),
+        _stream(stream)))
+    return out
+
+
+def forward(q_idx, w, k_idx, q, kv, gate, q_pos, top_k: int = TOP_K, idx_out=None, out=None, ws=None,
+            stream=None, return_idx: bool = True):
+    """The whole path.  Returns (idx [B,T,K] or None, out [B,T,64,512])."""
+    B, T = q_idx.shape[0], q_idx.shape[1]
+    L = k_idx.shape[1]
+    _need(q_idx, "q_idx", torch.bfloat16, (B, T, INDEX_HEADS, INDEX_DIM))
+    _need(w, "w", torch.bfloat16, (B, T, INDEX_HEADS))
+    _need(k_idx, "k_idx", torch.bfloat16, (B, L, INDEX_DIM))
+    _need(q, "q", torch.bfloat16, (B, T, HEADS, QK_DIM))
+    _need(kv, "kv", torch.bfloat16, (B, L, QK_DIM))
+    if gate is not None:
+        _need(gate, "gate", torch.bfloat16, (B, T, HEADS))
+    _need(q_pos, "q_pos", torch.int32, (B, T))
+    dims = make_dims(B, T, L, top_k)
+    if idx_out is None and return_idx:
+        idx_out = torch.empty((B, T, top_k), dtype=torch.int32, device=q.device)
+    if idx_out is not None:
+        _need(idx_out, "idx_out", torch.int32, (B, T, top_k))
+    if out is None:
+        out = torch.empty((B, T, HEADS, V_DIM), dtype=torch.float32, device=q.device)
+    _need(out, "out", torch.float32, (B, T, HEADS, V_DIM))
+    if ws is None:
+        ws = alloc_workspace(dims, OP_FORWARD, q.device)
+    _check("sga_forward", load_library().sga_forward(
+        ctypes.byref(dims), _ptr(q_idx), _ptr(w), _ptr(k_idx), _ptr(q), _ptr(kv), _ptr(gate), _ptr(q_pos),
+        _ptr(idx_out), _ptr(out), _ptr(ws), ws.numel(), _stream(stream)))
+    return idx_out, out

@@ -1,0 +1,245 @@
+// C ABI of libsga: argument validation, workspace layout, tensor-map encoding
+// and kernel launches.  See include/sga.h for the contract of each call.
+#include <cudaTypedefs.h>
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <mutex>
+
+#include "../../include/sga.h"
+#include "sga_internal.cuh"
+
+namespace sga {
+namespace {
+
+constexpr size_t kAlign = 256;
+constexpr size_t kStatusBytes = 256;
+
+size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+
+struct Layout {
+  size_t bitmap = 0, part_o = 0, part_ml = 0, scores = 0, idx = 0, total = 0;
+  int splits = 1;
+};
+
+bool dims_ok(const sga_dims_t* d) {
+  if (!d) return false;
+  if (d->batch < 1 || d->n_q < 1 || d->kv_stride < 1 || d->kv_stride > SGA_MAX_KV_STRIDE) return false;
+  if (d->top_k < 64 || d->top_k > SGA_MAX_TOP_K || d->top_k % 64 != 0) return false;
+  const long long rows = static_cast<long long>(d->batch) * d->n_q;
+  // row indices of the flattened [rows*64] query matrices and [B*L] caches are int32
+  if (rows * 64 > INT32_MAX || static_cast<long long>(d->batch) * d->kv_stride > INT32_MAX) return false;
+  return true;
+}
+
+Layout make_layout(const sga_dims_t& d, sga_op_t op) {
+  Layout l;
+  const size_t rows = static_cast<size_t>(d.batch) * d.n_q;
+  size_t off = kStatusBytes;
+  if (op == SGA_OP_TOPK_SELECT || op == SGA_OP_FORWARD) {
+    l.bitmap = off;
+    off += align_up(rows * topk_bitmap_words(d.kv_stride) * 4);
+  }
+  if (op == SGA_OP_SPARSE_MLA_ATTEND || op == SGA_OP_FORWARD) {
+    l.splits = attend_splits(static_cast<int>(rows), d.top_k);
+    if (l.splits > 1) {
+      l.part_o = off;
+      off += align_up(rows * l.splits * SGA_HEADS * SGA_V_DIM * 4);
+      l.part_ml = off;
+      off += align_up(rows * l.splits * SGA_HEADS * 2 * 4);
+    }
+  }
+  if (op == SGA_OP_FORWARD) {
+    l.scores = off;
+    off += align_up(rows * static_cast<size_t>(d.kv_stride) * 4);
+    l.idx = off;
+    off += align_up(rows * static_cast<size_t>(d.top_k) * 4);
+  }
+  l.total = off;
+  return l;
+}
+
+bool aligned(const void* p, size_t a) { return p && (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+std::once_flag g_encode_once;
+
+// Checks that the current device is an sm_100 part and returns its SM count.
+sga_status_t device_info(int* num_sms) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    cudaGetLastError();
+    return SGA_ERR_UNSUPPORTED;
+  }
+  int major = 0, sms = 0;
+  if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+    cudaGetLastError();
+    return SGA_ERR_UNSUPPORTED;
+  }
+  if (major != 10) return SGA_ERR_UNSUPPORTED;
+  *num_sms = sms;
+  return SGA_OK;
+}
+
+sga_status_t check_ws(void* ws, size_t ws_bytes, const sga_dims_t& d, sga_op_t op, Layout* l) {
+  *l = make_layout(d, op);
+  if (!ws || !aligned(ws, kAlign)) return SGA_ERR_WORKSPACE;
+  if (ws_bytes < l->total) return SGA_ERR_WORKSPACE;
+  return SGA_OK;
+}
+
+sga_status_t from_cuda(cudaError_t e) { return e == cudaSuccess ? SGA_OK : SGA_ERR_CUDA; }
+
+template <class T>
+T* at(void* ws, size_t off) {
+  return reinterpret_cast<T*>(static_cast<uint8_t*>(ws) + off);
+}
+
+}  // namespace
+
+cudaError_t make_tmap_bf16_2d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer,
+                              uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer) {
+  std::call_once(g_encode_once, []() {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+    cudaGetLastError();
+  });
+  if (!g_encode) return cudaErrorNotSupported;
+  const cuuint64_t dims[2] = {inner, outer};
+  const cuuint64_t strides[1] = {row_bytes};
+  const cuuint32_t box[2] = {box_inner, box_outer};
+  const cuuint32_t estr[2] = {1, 1};
+  const CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
+                              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+}  // namespace sga
+
+using namespace sga;
+
+extern "C" {
+
+int32_t sga_abi_version(void) { return 1; }
+
+const char* sga_status_string(sga_status_t s) {
+  switch (s) {
+    case SGA_OK: return "SGA_OK";
+    case SGA_ERR_INVALID_ARG: return "SGA_ERR_INVALID_ARG";
+    case SGA_ERR_UNSUPPORTED: return "SGA_ERR_UNSUPPORTED";
+    case SGA_ERR_WORKSPACE: return "SGA_ERR_WORKSPACE";
+    case SGA_ERR_CUDA: return "SGA_ERR_CUDA";
+    case SGA_ERR_TIMEOUT: return "SGA_ERR_TIMEOUT";
+    case SGA_ERR_DEVICE_ARG: return "SGA_ERR_DEVICE_ARG";
+  }
+  return "SGA_ERR_UNKNOWN";
+}
+
+sga_status_t sga_workspace_size(const sga_dims_t* dims, sga_op_t op, size_t* bytes) {
+  if (!dims_ok(dims) || !bytes || op < SGA_OP_INDEX_SCORES || op > SGA_OP_FORWARD) return SGA_ERR_INVALID_ARG;
+  *bytes = make_layout(*dims, op).total;
+  return SGA_OK;
+}
+
+sga_status_t sga_index_scores(const sga_dims_t* dims, const sga_bf16_t* q_idx, const sga_bf16_t* w,
+                              const sga_bf16_t* k_idx, const int32_t* q_pos, float* scores, void* ws,
+                              size_t ws_bytes, sga_stream_t stream) {
+  if (!dims_ok(dims)) return SGA_ERR_INVALID_ARG;
+  if (!aligned(q_idx, 16) || !aligned(w, 16) || !aligned(k_idx, 16) || !aligned(q_pos, 4) || !aligned(scores, 16))
+    return SGA_ERR_INVALID_ARG;
+  Layout l;
+  sga_status_t st = check_ws(ws, ws_bytes, *dims, SGA_OP_INDEX_SCORES, &l);
+  if (st != SGA_OK) return st;
+  int sms = 0;
+  if ((st = device_info(&sms)) != SGA_OK) return st;
+  IndexArgs a{q_idx, w, k_idx, q_pos, scores, at<int>(ws, 0), dims->batch, dims->n_q, dims->kv_stride};
+  return from_cuda(launch_index_scores(a, sms, static_cast<cudaStream_t>(stream)));
+}
+
+sga_status_t sga_topk_select(const sga_dims_t* dims, const float* scores, const int32_t* q_pos, int32_t* idx,
+                             void* ws, size_t ws_bytes, sga_stream_t stream) {
+  if (!dims_ok(dims)) return SGA_ERR_INVALID_ARG;
+  if (!aligned(scores, 4) || !aligned(q_pos, 4) || !aligned(idx, 16)) return SGA_ERR_INVALID_ARG;
+  Layout l;
+  sga_status_t st = check_ws(ws, ws_bytes, *dims, SGA_OP_TOPK_SELECT, &l);
+  if (st != SGA_OK) return st;
+  int sms = 0;
+  if ((st = device_info(&sms)) != SGA_OK) return st;
+  TopkArgs a{scores, q_pos, idx, at<uint32_t>(ws, l.bitmap), at<int>(ws, 0), dims->batch * dims->n_q,
+             dims->kv_stride, dims->top_k};
+  return from_cuda(launch_topk(a, static_cast<cudaStream_t>(stream)));
+}
+
+sga_status_t sga_sparse_mla_attend(const sga_dims_t* dims, const sga_bf16_t* q, const sga_bf16_t* kv,
+                                   const int32_t* idx, const sga_bf16_t* gate, float* out, void* ws,
+                                   size_t ws_bytes, sga_stream_t stream) {
+  if (!dims_ok(dims)) return SGA_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(kv, 16) || !aligned(idx, 16) || !aligned(out, 16) ||
+      (gate && !aligned(gate, 2)))
+    return SGA_ERR_INVALID_ARG;
+  Layout l;
+  sga_status_t st = check_ws(ws, ws_bytes, *dims, SGA_OP_SPARSE_MLA_ATTEND, &l);
+  if (st != SGA_OK) return st;
+  int sms = 0;
+  if ((st = device_info(&sms)) != SGA_OK) return st;
+  AttendArgs a{q, kv, idx, gate, out, l.splits > 1 ? at<float>(ws, l.part_o) : nullptr,
+               l.splits > 1 ? at<float>(ws, l.part_ml) : nullptr, at<int>(ws, 0), dims->batch, dims->n_q,
+               dims->kv_stride, dims->top_k};
+  return from_cuda(launch_attend(a, static_cast<cudaStream_t>(stream)));
+}
+
+sga_status_t sga_forward(const sga_dims_t* dims, const sga_bf16_t* q_idx, const sga_bf16_t* w,
+                         const sga_bf16_t* k_idx, const sga_bf16_t* q, const sga_bf16_t* kv,
+                         const sga_bf16_t* gate, const int32_t* q_pos, int32_t* idx_out, float* out, void* ws,
+                         size_t ws_bytes, sga_stream_t stream) {
+  if (!dims_ok(dims)) return SGA_ERR_INVALID_ARG;
+  if (!aligned(q_idx, 16) || !aligned(w, 16) || !aligned(k_idx, 16) || !aligned(q, 16) || !aligned(kv, 16) ||
+      !aligned(q_pos, 4) || !aligned(out, 16) || (gate && !aligned(gate, 2)) || (idx_out && !aligned(idx_out, 16)))
+    return SGA_ERR_INVALID_ARG;
+  Layout l;
+  sga_status_t st = check_ws(ws, ws_bytes, *dims, SGA_OP_FORWARD, &l);
+  if (st != SGA_OK) return st;
+  int sms = 0;
+  if ((st = device_info(&sms)) != SGA_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int* status = at<int>(ws, 0);
+  float* scores = at<float>(ws, l.scores);
+  int32_t* idx = idx_out ? idx_out : at<int32_t>(ws, l.idx);
+  const int rows = dims->batch * dims->n_q;
+  IndexArgs ia{q_idx, w, k_idx, q_pos, scores, status, dims->batch, dims->n_q, dims->kv_stride};
+  cudaError_t e = launch_index_scores(ia, sms, s);
+  if (e != cudaSuccess) return SGA_ERR_CUDA;
+  TopkArgs ta{scores, q_pos, idx, at<uint32_t>(ws, l.bitmap), status, rows, dims->kv_stride, dims->top_k};
+  e = launch_topk(ta, s);
+  if (e != cudaSuccess) return SGA_ERR_CUDA;
+  AttendArgs aa{q, kv, idx, gate, out, l.splits > 1 ? at<float>(ws, l.part_o) : nullptr,
+                l.splits > 1 ? at<float>(ws, l.part_ml) : nullptr, status, dims->batch, dims->n_q,
+                dims->kv_stride, dims->top_k};
+  return from_cuda(launch_attend(aa, s));
+}
+
+sga_status_t sga_get_device_status(const void* ws, sga_stream_t stream, int32_t* device_status) {
+  if (!ws || !device_status) return SGA_ERR_INVALID_ARG;
+  int32_t v = 0;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (cudaMemcpyAsync(&v, ws, sizeof v, cudaMemcpyDeviceToHost, s) != cudaSuccess ||
+      cudaStreamSynchronize(s) != cudaSuccess) {
+    cudaGetLastError();
+    return SGA_ERR_CUDA;
+  }
+  *device_status = v;
+  return SGA_OK;
+}
+
+sga_status_t sga_clear_device_status(void* ws, sga_stream_t stream) {
+  if (!ws) return SGA_ERR_INVALID_ARG;
+  return from_cuda(cudaMemsetAsync(ws, 0, kStatusBytes, static_cast<cudaStream_t>(stream)));
+}
+
+}  // extern "C"

@@ -1,0 +1,302 @@
+// Step 1: the DSA-style indexer (archdb "A.X K2", token-selection field: 64
+// indexer heads of dim 128, ReLU-scored; indexer-key-width field: 128 per token).
+//
+//   scores[row, s] = sum_j w[row, j] * max(0, q_idx[row, j, :] . k_idx[b, s, :]),  s <= t
+//
+// Design (decode is HBM-bound: the 256 B index key of every past token is read
+// once and is ~93% of the bytes of the whole path at 128K context):
+//   * A persistent grid, one CTA per SM, walks a contiguous range of
+//     (query, 128-key tile) work items.
+//   * Warp 0 streams 128-key x 128-dim bf16 tiles of k_idx with TMA (128-byte
+//     swizzle, L2 evict-first) through a 5-stage shared-memory ring, and the
+//     query's 64 x 128 indexer matrix into a double buffer when the query
+//     changes.
+//   * Warp 1 issues tcgen05.mma (M = 128 keys, N = 64 heads, K = 128 dims in 8
+//     steps of 16) into one of four 64-column TMEM accumulators.
+//   * Warps 2-5 (one per TMEM lane quarter) read a key's 64 head dots with
+//     tcgen05.ld, apply ReLU, the per-head weight and the head sum in fp32,
+//     mask s > t and store the score (32 consecutive keys per warp: one
+//     128-byte store).
+#include "sga_internal.cuh"
+#include "sga_ptx.cuh"
+
+namespace sga {
+namespace {
+
+constexpr int kKeys = 128;    // keys per tile: MMA M
+constexpr int kDim = 128;     // indexer dim: MMA K
+constexpr int kHeads = 64;    // indexer heads: MMA N
+constexpr int kStages = 5;
+constexpr int kABox = kKeys * 64 * 2;  // one 128-byte-wide column strip of a tile
+constexpr int kAStage = 2 * kABox;     // 32 KB
+constexpr int kQBox = kHeads * 64 * 2;
+constexpr int kQBuf = 2 * kQBox;       // 16 KB
+constexpr int kAcc = 4;
+constexpr int kTmemCols = kAcc * kHeads;  // 256
+constexpr int kThreads = 192;
+constexpr int kNumBars = 2 * kStages + 4 + 2 * kAcc + 1;
+constexpr size_t kSmemBytes = 1024 + kStages * kAStage + 2 * kQBuf + kNumBars * 8 + 16;
+
+static_assert(kDim == 2 * 64, "two 128-byte strips per key row");
+
+struct IndexParams {
+  const uint16_t* w;
+  const int32_t* q_pos;
+  float* scores;
+  int* status;
+  int n_q, kv_stride, tiles_per_row;
+  long long total_tiles;
+};
+
+// Work item j -> (query row, first key).  Returns false for tiles that lie past
+// the query position (or rows whose position is invalid).
+__device__ __forceinline__ bool tile_info(const IndexParams& p, long long j, int& row, int& key0, int& t) {
+  row = static_cast<int>(j / p.tiles_per_row);
+  key0 = static_cast<int>(j % p.tiles_per_row) * kKeys;
+  t = __ldg(p.q_pos + row);
+  if (t < 0 || t >= p.kv_stride) return false;
+  return key0 <= t;
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+    sga_index_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap qmap,
+                     IndexParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t a_base = smem_u32(smem);
+  const uint32_t q_base = a_base + kStages * kAStage;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kStages * kAStage + 2 * kQBuf);
+  const uint32_t bar0 = smem_u32(bars);
+  auto full = [&](int s) { return bar0 + 8u * s; };
+  auto empty = [&](int s) { return bar0 + 8u * (kStages + s); };
+  auto qfull = [&](int s) { return bar0 + 8u * (2 * kStages + s); };
+  auto qempty = [&](int s) { return bar0 + 8u * (2 * kStages + 2 + s); };
+  auto accfull = [&](int s) { return bar0 + 8u * (2 * kStages + 4 + s); };
+  auto accempty = [&](int s) { return bar0 + 8u * (2 * kStages + 4 + kAcc + s); };
+  const uint32_t done_bar = bar0 + 8u * (2 * kStages + 4 + 2 * kAcc);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + kNumBars);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(full(s), 1);
+      mbar_init(empty(s), 1);
+    }
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(qfull(s), 1);
+      mbar_init(qempty(s), 1);
+    }
+    for (int s = 0; s < kAcc; ++s) {
+      mbar_init(accfull(s), 1);
+      mbar_init(accempty(s), 4 * 32);
+    }
+    mbar_init(done_bar, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tmap(&kmap);
+    prefetch_tmap(&qmap);
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_slot), kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  const long long j0 = p.total_tiles * blockIdx.x / gridDim.x;
+  const long long j1 = p.total_tiles * (blockIdx.x + 1) / gridDim.x;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      const uint64_t pol_stream = policy_evict_first();
+      const uint64_t pol_keep = policy_evict_last();
+      long long n = 0, qc = 0;
+      int cur_row = -1;
+      bool ok = true;
+      for (long long j = j0; j < j1; ++j) {
+        int row, key0, t;
+        if (!tile_info(p, j, row, key0, t)) {
+          if (t < 0 || t >= p.kv_stride) record_status(p.status, kStatusDeviceArg);
+          continue;
+        }
+        if (row != cur_row) {
+          const int slot = static_cast<int>(qc & 1);
+          if (!mbar_wait(qempty(slot), static_cast<uint32_t>((qc >> 1) & 1) ^ 1u, abort_flag)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(qfull(slot), kQBuf);
+          tma_load_2d(q_base + slot * kQBuf, &qmap, qfull(slot), 0, row * kHeads, pol_keep);
+          tma_load_2d(q_base + slot * kQBuf + kQBox, &qmap, qfull(slot), 64, row * kHeads, pol_keep);
+          ++qc;
+          cur_row = row;
+        }
+        const int st = static_cast<int>(n % kStages);
+        if (!mbar_wait(empty(st), static_cast<uint32_t>((n / kStages) & 1) ^ 1u, abort_flag)) {
+          ok = false;
+          break;
+        }
+        mbar_arrive_expect_tx(full(st), kAStage);
+        const int y = (row / p.n_q) * p.kv_stride + key0;
+        tma_load_2d(a_base + st * kAStage, &kmap, full(st), 0, y, pol_stream);
+        tma_load_2d(a_base + st * kAStage + kABox, &kmap, full(st), 64, y, pol_stream);
+        ++n;
+      }
+      if (!ok) {
+        record_status(p.status, kStatusTimeout);
+        *abort_flag = 1;
+        // Let the copies already issued land before the CTA retires.
+        volatile int never = 0;
+        for (long long m = (n > kStages ? n - kStages : 0); m < n; ++m)
+          mbar_wait(full(static_cast<int>(m % kStages)), static_cast<uint32_t>((m / kStages) & 1), &never);
+        for (long long m = (qc > 2 ? qc - 2 : 0); m < qc; ++m)
+          mbar_wait(qfull(static_cast<int>(m & 1)), static_cast<uint32_t>((m >> 1) & 1), &never);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_bf16_f32(kKeys, kHeads, false, false);
+      long long n = 0, qc = 0, an = 0;
+      int cur_row = -1, cur_q = 0;
+      bool ok = true;
+      for (long long j = j0; j < j1 && ok; ++j) {
+        int row, key0, t;
+        if (!tile_info(p, j, row, key0, t)) continue;
+        if (row != cur_row) {
+          if (cur_row >= 0) mma_commit(qempty(cur_q));  // frees the previous query's buffer
+          const int slot = static_cast<int>(qc & 1);
+          if (!mbar_wait(qfull(slot), static_cast<uint32_t>((qc >> 1) & 1), abort_flag)) {
+            ok = false;
+            break;
+          }
+          cur_q = slot;
+          ++qc;
+          cur_row = row;
+        }
+        const int acc = static_cast<int>(an % kAcc);
+        if (!mbar_wait(accempty(acc), static_cast<uint32_t>((an / kAcc) & 1) ^ 1u, abort_flag)) {
+          ok = false;
+          break;
+        }
+        const int st = static_cast<int>(n % kStages);
+        if (!mbar_wait(full(st), static_cast<uint32_t>((n / kStages) & 1), abort_flag)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d = tmem_base + static_cast<uint32_t>(acc * kHeads);
+#pragma unroll
+        for (int k = 0; k < kDim / 16; ++k) {
+          const uint32_t a_addr = a_base + st * kAStage + (k >> 2) * kABox + (k & 3) * 32;
+          const uint32_t b_addr = q_base + cur_q * kQBuf + (k >> 2) * kQBox + (k & 3) * 32;
+          mma_bf16(d, sdesc_sw128(a_addr, 16, 1024), sdesc_sw128(b_addr, 16, 1024), idesc, k > 0 ? 1u : 0u);
+        }
+        mma_commit(empty(st));
+        mma_commit(accfull(acc));
+        ++n;
+        ++an;
+      }
+      if (!ok) {
+        record_status(p.status, kStatusTimeout);
+        *abort_flag = 1;
+      }
+      // Every MMA this thread issued has finished once done_bar flips.
+      mma_commit(done_bar);
+      volatile int never = 0;
+      mbar_wait(done_bar, 0, &never);
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int quarter = warp & 3;  // TMEM lanes 32*quarter .. +31 (warp % 4 rule)
+    long long an = 0;
+    int cur_row = -1;
+    float wv[kHeads];
+    for (long long j = j0; j < j1; ++j) {
+      int row, key0, t;
+      if (!tile_info(p, j, row, key0, t)) continue;
+      if (row != cur_row) {
+        const uint4* wp = reinterpret_cast<const uint4*>(p.w + static_cast<size_t>(row) * kHeads);
+#pragma unroll
+        for (int c = 0; c < kHeads / 8; ++c) {
+          const uint4 u = __ldg(wp + c);
+          const uint32_t x[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            wv[8 * c + 2 * e] = __uint_as_float(x[e] << 16);
+            wv[8 * c + 2 * e + 1] = __uint_as_float(x[e] & 0xFFFF0000u);
+          }
+        }
+        cur_row = row;
+      }
+      const int acc = static_cast<int>(an % kAcc);
+      if (!mbar_wait(accfull(acc), static_cast<uint32_t>((an / kAcc) & 1), abort_flag)) {
+        record_status(p.status, kStatusTimeout);
+        *abort_flag = 1;
+        break;
+      }
+      tc_fence_after();
+      float v0[32], v1[32];
+      const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + static_cast<uint32_t>(acc * kHeads);
+      tmem_ld32(taddr, v0);
+      tmem_ld32(taddr + 32, v1);
+      tc_fence_before();
+      mbar_arrive(accempty(acc));
+      float s = 0.f;
+#pragma unroll
+      for (int h = 0; h < 32; ++h) s = fmaf(wv[h], fmaxf(v0[h], 0.f), s);
+#pragma unroll
+      for (int h = 0; h < 32; ++h) s = fmaf(wv[32 + h], fmaxf(v1[h], 0.f), s);
+      const int key = key0 + quarter * 32 + lane;
+      if (key <= t) p.scores[static_cast<size_t>(row) * p.kv_stride + key] = s;
+      ++an;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, kTmemCols);
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_index_scores(const IndexArgs& a, int num_sms, cudaStream_t stream) {
+  const int rows = a.batch * a.n_q;
+  const int tiles_per_row = (a.kv_stride + kKeys - 1) / kKeys;
+  const long long total = static_cast<long long>(rows) * tiles_per_row;
+  if (total == 0) return cudaSuccess;
+  CUtensorMap kmap, qmap;
+  cudaError_t e = make_tmap_bf16_2d(&kmap, a.k_idx, kDim, static_cast<uint64_t>(a.batch) * a.kv_stride, kDim * 2,
+                                    64, kKeys);
+  if (e != cudaSuccess) return e;
+  e = make_tmap_bf16_2d(&qmap, a.q_idx, kDim, static_cast<uint64_t>(rows) * kHeads, kDim * 2, 64, kHeads);
+  if (e != cudaSuccess) return e;
+  e = cudaFuncSetAttribute(sga_index_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(kSmemBytes));
+  if (e != cudaSuccess) return e;
+  IndexParams p;
+  p.w = a.w;
+  p.q_pos = a.q_pos;
+  p.scores = a.scores;
+  p.status = a.status;
+  p.n_q = a.n_q;
+  p.kv_stride = a.kv_stride;
+  p.tiles_per_row = tiles_per_row;
+  p.total_tiles = total;
+  const int grid = static_cast<int>(total < num_sms ? total : num_sms);
+  sga_index_kernel<<<grid, kThreads, kSmemBytes, stream>>>(kmap, qmap, p);
+  return cudaGetLastError();
+}
+
+}  // namespace sga

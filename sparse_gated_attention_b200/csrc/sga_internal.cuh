@@ -1,0 +1,55 @@
+// Launch interfaces between the C-ABI layer (sga_api.cu) and the kernels.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace sga {
+
+// ---- indexer (step 1) --------------------------------------------------------
+struct IndexArgs {
+  const uint16_t* q_idx;  // [rows][64][128]
+  const uint16_t* w;      // [rows][64]
+  const uint16_t* k_idx;  // [B][L][128]
+  const int32_t* q_pos;   // [rows]
+  float* scores;          // [rows][L]
+  int* status;
+  int batch, n_q, kv_stride;
+};
+cudaError_t launch_index_scores(const IndexArgs& a, int num_sms, cudaStream_t stream);
+
+// ---- top-k (step 2) ------------------------------------------------------------
+struct TopkArgs {
+  const float* scores;  // [rows][L]
+  const int32_t* q_pos; // [rows]
+  int32_t* idx;         // [rows][K]
+  uint32_t* bitmap;     // [rows][words_per_row] scratch
+  int* status;
+  int rows, kv_stride, top_k;
+};
+size_t topk_bitmap_words(int kv_stride);
+cudaError_t launch_topk(const TopkArgs& a, cudaStream_t stream);
+
+// ---- sparse attention + gate (steps 3-4) -----------------------------------------
+struct AttendArgs {
+  const uint16_t* q;     // [rows][64][576]
+  const uint16_t* kv;    // [B][L][576]
+  const int32_t* idx;    // [rows][K]
+  const uint16_t* gate;  // [rows][64] or null
+  float* out;            // [rows][64][512]
+  float* part_o;         // [rows][splits][64][512] scratch (splits > 1)
+  float* part_ml;        // [rows][splits][64][2] scratch (splits > 1)
+  int* status;
+  int batch, n_q, kv_stride, top_k;
+};
+int attend_splits(int rows, int top_k);
+cudaError_t launch_attend(const AttendArgs& a, cudaStream_t stream);
+
+// ---- tensor maps -------------------------------------------------------------------
+// 2-D bf16 tensor map: `inner` elements per row, `outer` rows, rows `row_bytes`
+// apart, box {box_inner, box_outer}, 128-byte swizzle.
+cudaError_t make_tmap_bf16_2d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer,
+                              uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer);
+
+}  // namespace sga

@@ -1,0 +1,111 @@
+"""Host-side checks of the C ABI: the library loads, exports every entry point
+that include/sga.h declares, sizes workspaces and rejects bad arguments before
+touching the GPU.  No kernel is launched here."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import sparse_gated_attention_b200 as sga
+from sparse_gated_attention_b200 import build as sga_build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    sga_build.build()
+    return sga.load_library()
+
+
+def declared_symbols():
+    text = open(os.path.join(ROOT, "include", "sga.h")).read()
+    return sorted(set(re.findall(r"SGA_API\s+[\w\s\*]+?\b(sga_\w+)\s*\(", text)))
+
+
+def test_header_declares_the_four_steps():
+    names = declared_symbols()
+    for n in ["sga_index_scores", "sga_topk_select", "sga_sparse_mla_attend", "sga_forward"]:
+        assert n in names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = declared_symbols()
+    assert names and set(names) == set(sga.EXPORTED)
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+def test_abi_version_and_status_strings(lib):
+    assert lib.sga_abi_version() == 1
+    assert lib.sga_status_string(0) == b"SGA_OK"
+    assert lib.sga_status_string(5) == b"SGA_ERR_TIMEOUT"
+    assert lib.sga_status_string(99) == b"SGA_ERR_UNKNOWN"
+
+
+def test_workspace_sizes(lib):
+    d = sga.make_dims(32, 1, 131072)
+    idx_ws = sga.workspace_size(d, sga.OP_INDEX_SCORES)
+    topk_ws = sga.workspace_size(d, sga.OP_TOPK_SELECT)
+    att_ws = sga.workspace_size(d, sga.OP_SPARSE_MLA_ATTEND)
+    fwd_ws = sga.workspace_size(d, sga.OP_FORWARD)
+    assert idx_ws == 256
+    assert topk_ws == 256 + 32 * (131072 // 32) * 4
+    # 32 queries -> 4 splits of the 2048 slots; partial O + (m, l)
+    assert att_ws == 256 + 32 * 4 * 64 * 512 * 4 + 32 * 4 * 64 * 2 * 4
+    assert fwd_ws >= topk_ws + att_ws - 256 + 32 * 131072 * 4 + 32 * 2048 * 4
+    # prefill: 4096 queries fill the GPU without splitting
+    p = sga.make_dims(1, 4096, 131072)
+    assert sga.workspace_size(p, sga.OP_SPARSE_MLA_ATTEND) == 256
+
+
+@pytest.mark.parametrize("dims", [(0, 1, 100, 2048), (1, 0, 100, 2048), (1, 1, 0, 2048), (1, 1, 100, 100),
+                                  (1, 1, 100, 4096), (1, 1, 100, 0), (70000, 1, 1 << 20, 2048)])
+def test_bad_dims_rejected(lib, dims):
+    d = sga.make_dims(*dims)
+    out = ctypes.c_size_t(0)
+    assert lib.sga_workspace_size(ctypes.byref(d), 3, ctypes.byref(out)) == 1
+
+
+def test_null_and_misaligned_pointers_rejected_on_host(lib):
+    d = sga.make_dims(1, 1, 4096)
+    P = ctypes.c_void_p
+    good = P(0x100000)
+    odd = P(0x100002)
+    ws = P(0x200000)
+    # null inputs
+    assert lib.sga_index_scores(ctypes.byref(d), None, good, good, good, good, ws, 1 << 20, None) == 1
+    assert lib.sga_topk_select(ctypes.byref(d), good, good, None, ws, 1 << 20, None) == 1
+    assert lib.sga_sparse_mla_attend(ctypes.byref(d), good, None, good, None, good, ws, 1 << 20, None) == 1
+    # misaligned bf16 input (TMA needs 16-byte alignment)
+    assert lib.sga_index_scores(ctypes.byref(d), good, good, odd, good, good, ws, 1 << 20, None) == 1
+    assert lib.sga_sparse_mla_attend(ctypes.byref(d), odd, good, good, None, good, ws, 1 << 20, None) == 1
+    # workspace: null, misaligned, too small
+    assert lib.sga_topk_select(ctypes.byref(d), good, good, good, None, 1 << 20, None) == 3
+    assert lib.sga_topk_select(ctypes.byref(d), good, good, good, P(0x200010), 1 << 20, None) == 3
+    assert lib.sga_topk_select(ctypes.byref(d), good, good, good, ws, 64, None) == 3
+    assert lib.sga_get_device_status(None, None, None) == 1
+    assert lib.sga_clear_device_status(None, None) == 1
+
+
+def test_binding_refuses_cpu_tensors():
+    import torch
+
+    q = torch.zeros((1, 1, 64, 576), dtype=torch.bfloat16)
+    kv = torch.zeros((1, 8, 576), dtype=torch.bfloat16)
+    idx = torch.zeros((1, 1, 64), dtype=torch.int32)
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        sga.sparse_mla_attend(q, kv, idx)
+
+
+def test_binding_fails_loudly_without_library(tmp_path):
+    from sparse_gated_attention_b200 import _binding
+
+    saved = _binding._lib
+    _binding._lib = None
+    try:
+        with pytest.raises(RuntimeError, match="libsga.so not found"):
+            _binding.load_library(str(tmp_path / "missing.so"))
+    finally:
+        _binding._lib = saved
