@@ -19,7 +19,7 @@ constexpr size_t kStatusBytes = 256;
 size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 
 struct Layout {
-  size_t bitmap = 0, part_o = 0, part_ml = 0, scores = 0, idx = 0, total = 0;
+  size_t bitmap = 0, part_o = 0, part_ml = 0, scores = 0, idx = 0, hist = 0, total = 0;
   int splits = 1;
 };
 
@@ -55,6 +55,8 @@ Layout make_layout(const sga_dims_t& d, sga_op_t op) {
     off += align_up(rows * static_cast<size_t>(d.kv_stride) * 4);
     l.idx = off;
     off += align_up(rows * static_cast<size_t>(d.top_k) * 4);
+    l.hist = off;
+    off += align_up(rows * 4096 * 4);
   }
   l.total = off;
   return l;
@@ -158,7 +160,7 @@ sga_status_t sga_index_scores(const sga_dims_t* dims, const sga_bf16_t* q_idx, c
   if (st != SGA_OK) return st;
   int sms = 0;
   if ((st = device_info(&sms)) != SGA_OK) return st;
-  IndexArgs a{q_idx, w, k_idx, q_pos, scores, at<int>(ws, 0), dims->batch, dims->n_q, dims->kv_stride};
+  IndexArgs a{q_idx, w, k_idx, q_pos, scores, nullptr, at<int>(ws, 0), dims->batch, dims->n_q, dims->kv_stride};
   return from_cuda(launch_index_scores(a, sms, static_cast<cudaStream_t>(stream)));
 }
 
@@ -171,8 +173,8 @@ sga_status_t sga_topk_select(const sga_dims_t* dims, const float* scores, const 
   if (st != SGA_OK) return st;
   int sms = 0;
   if ((st = device_info(&sms)) != SGA_OK) return st;
-  TopkArgs a{scores, q_pos, idx, at<uint32_t>(ws, l.bitmap), at<int>(ws, 0), dims->batch * dims->n_q,
-             dims->kv_stride, dims->top_k};
+  TopkArgs a{scores,          q_pos, idx, at<uint32_t>(ws, l.bitmap), nullptr, at<int>(ws, 0),
+             dims->batch * dims->n_q, dims->kv_stride, dims->top_k};
   return from_cuda(launch_topk(a, static_cast<cudaStream_t>(stream)));
 }
 
@@ -212,10 +214,14 @@ sga_status_t sga_forward(const sga_dims_t* dims, const sga_bf16_t* q_idx, const 
   float* scores = at<float>(ws, l.scores);
   int32_t* idx = idx_out ? idx_out : at<int32_t>(ws, l.idx);
   const int rows = dims->batch * dims->n_q;
-  IndexArgs ia{q_idx, w, k_idx, q_pos, scores, status, dims->batch, dims->n_q, dims->kv_stride};
-  cudaError_t e = launch_index_scores(ia, sms, s);
+  // The indexer counts the first radix level of the selection as it writes the scores.
+  uint32_t* hist = at<uint32_t>(ws, l.hist);
+  cudaError_t e = cudaMemsetAsync(hist, 0, static_cast<size_t>(rows) * 4096 * 4, s);
   if (e != cudaSuccess) return SGA_ERR_CUDA;
-  TopkArgs ta{scores, q_pos, idx, at<uint32_t>(ws, l.bitmap), status, rows, dims->kv_stride, dims->top_k};
+  IndexArgs ia{q_idx, w, k_idx, q_pos, scores, hist, status, dims->batch, dims->n_q, dims->kv_stride};
+  e = launch_index_scores(ia, sms, s);
+  if (e != cudaSuccess) return SGA_ERR_CUDA;
+  TopkArgs ta{scores, q_pos, idx, at<uint32_t>(ws, l.bitmap), hist, status, rows, dims->kv_stride, dims->top_k};
   e = launch_topk(ta, s);
   if (e != cudaSuccess) return SGA_ERR_CUDA;
   AttendArgs aa{q, kv, idx, gate, out, l.splits > 1 ? at<float>(ws, l.part_o) : nullptr,

@@ -10,15 +10,18 @@
 //   * Shared memory: Q (9 swizzled 64x64 boxes, 72 KB, loaded once by TMA), a
 //     17-slot ring of 8 KB boxes holding gathered rows, and P (hi and lo bf16
 //     parts, 8 KB each).
-//   * Warp 0 gathers a 64-row tile as 9 boxes [rope dims 512..575, then value
-//     dims 0..63, ..., 448..511] with TMA tile::gather4 (4 rows per
-//     instruction, 16 lanes issuing), plus a 64-bit mask of non-empty slots.
-//   * Warp 1 issues tcgen05.mma: S_j = Q C_j^T (M = 64 heads, N = 64 rows,
+//   * Warps 0-3 gather a 64-row tile as 9 boxes [rope dims 512..575, then
+//     value dims 0..63, ..., 448..511] with 16-byte cp.async copies written
+//     straight into the 128-byte-swizzled layout (each warp instruction moves
+//     four full 128-byte row strips; empty slots are zero-filled without a
+//     read), completing on the box's mbarrier.  Warp 0 also publishes a 64-bit
+//     mask of non-empty slots per tile and loads Q with TMA.
+//   * Warp 4 issues tcgen05.mma: S_j = Q C_j^T (M = 64 heads, N = 64 rows,
 //     K = 576) into one of two TMEM S buffers, and O += P_j V_j as 8 MMAs of
 //     M = 64, N = 64 dims, K = 64 rows each, for P_hi and P_lo (P split into
 //     two bf16 parts keeps ~16 mantissa bits of P).  S_{j+1} is issued before
 //     PV_j so the softmax of tile j overlaps the next QK^T.
-//   * Warps 2-5 (one per TMEM lane quarter, 16 heads each) run the softmax in
+//   * Warps 5-8 (one per TMEM lane quarter, 16 heads each) run the softmax in
 //     the log2 domain with a lazy running max (O in TMEM is rescaled only when
 //     the max grows by more than 2^8), write P to shared memory in the
 //     swizzled K-major layout, and finally scale O by sigmoid(g)/l.
@@ -45,7 +48,9 @@ constexpr int kRing = 17;       // >= 8 value boxes of tile j + 9 boxes of tile 
 constexpr int kQBytes = 9 * kBox;
 constexpr int kPBytes = kHeads * kTile * 2;
 constexpr int kMaskRing = 4;
-constexpr int kThreads = 192;
+constexpr int kProducers = 128;  // warps 0-3
+constexpr int kMmaWarp = 4;
+constexpr int kThreads = 288;
 constexpr int kTmemCols = 512;
 constexpr int kSCol = 256;
 // barriers: full[17] empty[17] q_full s_full[2] s_free[2] p_full p_free o_full mask_full[4] mask_empty[4]
@@ -57,6 +62,7 @@ static_assert(kSmemBytes <= 232448, "shared memory budget");
 static_assert(kRing >= 2 * kBoxesPerTile - 1, "ring must hold a tile's values plus the next tile");
 
 struct AttendParams {
+  const uint16_t* kv;
   const int32_t* idx;
   const uint16_t* gate;
   float* out;
@@ -75,8 +81,7 @@ __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
-    sga_attend_kernel(const __grid_constant__ CUtensorMap kvmap, const __grid_constant__ CUtensorMap qmap,
-                      AttendParams p) {
+    sga_attend_kernel(const __grid_constant__ CUtensorMap qmap, AttendParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t ring = smem_u32(smem);
@@ -108,7 +113,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kRing; ++s) {
-      mbar_init(full(s), 1);
+      mbar_init(full(s), kProducers);  // one cp.async arrival per producer thread
       mbar_init(empty(s), 1);
     }
     mbar_init(q_full, 1);
@@ -126,11 +131,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     *abort_flag = 0;
     fence_barrier_init();
   }
-  if (warp == 0 && lane == 0) {
-    prefetch_tmap(&kvmap);
-    prefetch_tmap(&qmap);
-  }
-  if (warp == 1) {
+  if (warp == 0 && lane == 0) prefetch_tmap(&qmap);
+  if (warp == kMmaWarp) {
     tmem_alloc(smem_u32(tmem_slot), kTmemCols);
     tmem_relinquish();
   }
@@ -139,69 +141,78 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == 0) {
-    // ------------------------------------------------------------ gather producer
+  if (warp < kProducers / 32) {
+    // ------------------------------------------------------------ gather producers
     const int b = row / p.n_q;
     const int32_t* idx_row = p.idx + static_cast<size_t>(row) * p.top_k + static_cast<size_t>(split) * ntiles * kTile;
-    long long issued = 0;
+    const uint16_t* kv_b = p.kv + static_cast<size_t>(b) * p.kv_stride * kDq;
+    const int ptid = threadIdx.x;
+    const int part = ptid & 7;   // 16-byte chunk of a 128-byte row strip
+    const int rsub = ptid >> 3;  // rows rsub + 16 i, i = 0..3
     bool ok = true;
-    if (lane == 0) {
+    if (ptid == 0) {
       mbar_arrive_expect_tx(q_full, kQBytes);
       const uint64_t pol = policy_evict_first();
       for (int c = 0; c < 9; ++c) tma_load_2d(q_s + c * kBox, &qmap, q_full, c * 64, row * kHeads, pol);
     }
     for (int j = 0; j < ntiles && ok; ++j) {
-      const int2 v = __ldg(reinterpret_cast<const int2*>(idx_row + j * kTile) + lane);
-      const bool ok0 = v.x >= 0 && v.x < p.kv_stride;
-      const bool ok1 = v.y >= 0 && v.y < p.kv_stride;
-      if ((v.x < -1 || v.x >= p.kv_stride) || (v.y < -1 || v.y >= p.kv_stride))
-        record_status(p.status, kStatusDeviceArg);
-      const int y0 = b * p.kv_stride + (ok0 ? v.x : 0);
-      const int y1 = b * p.kv_stride + (ok1 ? v.y : 0);
-      // 64-bit mask of filled slots: bit r <-> tile row r (lane l holds rows 2l, 2l+1)
-      uint64_t m = (static_cast<uint64_t>(ok0) << (2 * lane)) | (static_cast<uint64_t>(ok1) << (2 * lane + 1));
+      if (warp == 0) {
+        const int2 v = __ldg(reinterpret_cast<const int2*>(idx_row + j * kTile) + lane);
+        const bool ok0 = v.x >= 0 && v.x < p.kv_stride;
+        const bool ok1 = v.y >= 0 && v.y < p.kv_stride;
+        if ((v.x < -1 || v.x >= p.kv_stride) || (v.y < -1 || v.y >= p.kv_stride))
+          record_status(p.status, kStatusDeviceArg);
+        // 64-bit mask of filled slots: bit r <-> tile row r (lane l holds rows 2l, 2l+1)
+        uint64_t m = (static_cast<uint64_t>(ok0) << (2 * lane)) | (static_cast<uint64_t>(ok1) << (2 * lane + 1));
 #pragma unroll
-      for (int o = 16; o > 0; o >>= 1) m |= __shfl_xor_sync(0xFFFFFFFFu, m, o);
-      // rows 4g .. 4g+3 for lane g < 16
-      const int g = lane & 15;
-      const int r0 = __shfl_sync(0xFFFFFFFFu, y0, 2 * g);
-      const int r1 = __shfl_sync(0xFFFFFFFFu, y1, 2 * g);
-      const int r2 = __shfl_sync(0xFFFFFFFFu, y0, 2 * g + 1);
-      const int r3 = __shfl_sync(0xFFFFFFFFu, y1, 2 * g + 1);
-      if (lane == 0) {
-        const int mb = j % kMaskRing;
-        if (mbar_wait(mask_empty(mb), static_cast<uint32_t>((j / kMaskRing) & 1) ^ 1u, abort_flag)) {
-          masks[mb] = m;
-          mbar_arrive(mask_full(mb));
-        } else {
-          ok = false;
+        for (int o = 16; o > 0; o >>= 1) m |= __shfl_xor_sync(0xFFFFFFFFu, m, o);
+        if (lane == 0) {
+          const int mb = j % kMaskRing;
+          if (mbar_wait(mask_empty(mb), static_cast<uint32_t>((j / kMaskRing) & 1) ^ 1u, abort_flag)) {
+            masks[mb] = m;
+            mbar_arrive(mask_full(mb));
+          } else {
+            ok = false;
+          }
         }
+        ok = __shfl_sync(0xFFFFFFFFu, ok ? 1 : 0, 0) != 0;
+        if (!ok) break;
       }
-      ok = __shfl_sync(0xFFFFFFFFu, ok ? 1 : 0, 0) != 0;
-      for (int c = 0; c < kBoxesPerTile && ok; ++c) {
+      const uint16_t* src[4];
+      uint32_t nbytes[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int s = __ldg(idx_row + j * kTile + rsub + 16 * i);
+        const bool valid = s >= 0 && s < p.kv_stride;
+        src[i] = kv_b + static_cast<size_t>(valid ? s : 0) * kDq + part * 8;
+        nbytes[i] = valid ? 16u : 0u;
+      }
+      for (int c = 0; c < kBoxesPerTile; ++c) {
         const long long n = static_cast<long long>(j) * kBoxesPerTile + c;
         const int slot = static_cast<int>(n % kRing);
-        int waited = 1;
-        if (lane == 0) {
-          waited = mbar_wait(empty(slot), static_cast<uint32_t>((n / kRing) & 1) ^ 1u, abort_flag) ? 1 : 0;
-          if (waited) mbar_arrive_expect_tx(full(slot), kBox);
+        if (!mbar_wait(empty(slot), static_cast<uint32_t>((n / kRing) & 1) ^ 1u, abort_flag)) {
+          ok = false;
+          break;
         }
-        ok = __shfl_sync(0xFFFFFFFFu, waited, 0) != 0;
-        if (!ok) break;
-        const int x = c == 0 ? kDv : (c - 1) * 64;
-        if (lane < 16) tma_gather4(ring + slot * kBox + lane * 512, &kvmap, full(slot), x, r0, r1, r2, r3);
-        issued = n + 1;
+        const int dim0 = c == 0 ? kDv : (c - 1) * 64;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int r = rsub + 16 * i;
+          cp_async_16(ring + slot * kBox + r * 128 + ((part ^ (r & 7)) << 4), src[i] + dim0, nbytes[i]);
+        }
+        cp_async_arrive_noinc(full(slot));
       }
     }
-    if (!ok && lane == 0) {
+    asm volatile("cp.async.wait_all;" ::: "memory");
+    if (!ok) {
       record_status(p.status, kStatusTimeout);
       *abort_flag = 1;
-      volatile int never = 0;
-      for (long long m = (issued > kRing ? issued - kRing : 0); m < issued; ++m)
-        mbar_wait(full(static_cast<int>(m % kRing)), static_cast<uint32_t>((m / kRing) & 1), &never);
-      mbar_wait(q_full, 0, &never);
+      if (ptid == 0) {
+        volatile int never = 0;
+        mbar_wait(q_full, 0, &never);
+      }
     }
-  } else if (warp == 1) {
+  } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       constexpr uint32_t idesc_qk = idesc_bf16_f32(kHeads, kTile, false, false);
@@ -216,6 +227,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const long long n = static_cast<long long>(j) * kBoxesPerTile + c;
           const int slot = static_cast<int>(n % kRing);
           if (!mbar_wait(full(slot), static_cast<uint32_t>((n / kRing) & 1), abort_flag)) return false;
+          fence_proxy_async_smem();  // the box was written by cp.async (generic proxy)
           tc_fence_after();
           if (c == 0) rope_slot = slot;
           const int qbox = c == 0 ? 8 : c - 1;  // Q box covering the same dims
@@ -391,7 +403,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 1) {
+  if (warp == kMmaWarp) {
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);
   }
@@ -457,15 +469,14 @@ cudaError_t launch_attend(const AttendArgs& a, cudaStream_t stream) {
   const int rows = a.batch * a.n_q;
   if (rows == 0) return cudaSuccess;
   const int splits = attend_splits(rows, a.top_k);
-  CUtensorMap kvmap, qmap;
-  cudaError_t e = make_tmap_bf16_2d(&kvmap, a.kv, kDq, static_cast<uint64_t>(a.batch) * a.kv_stride, kDq * 2, 64, 1);
-  if (e != cudaSuccess) return e;
-  e = make_tmap_bf16_2d(&qmap, a.q, kDq, static_cast<uint64_t>(rows) * kHeads, kDq * 2, 64, kHeads);
+  CUtensorMap qmap;
+  cudaError_t e = make_tmap_bf16_2d(&qmap, a.q, kDq, static_cast<uint64_t>(rows) * kHeads, kDq * 2, 64, kHeads);
   if (e != cudaSuccess) return e;
   e = cudaFuncSetAttribute(sga_attend_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            static_cast<int>(kSmemBytes));
   if (e != cudaSuccess) return e;
   AttendParams p;
+  p.kv = a.kv;
   p.idx = a.idx;
   p.gate = a.gate;
   p.out = a.out;
@@ -478,7 +489,7 @@ cudaError_t launch_attend(const AttendArgs& a, cudaStream_t stream) {
   p.splits = splits;
   p.tiles_per_split = a.top_k / kTile / splits;
   p.scale_log2 = static_cast<float>(0.07216878364870322 * 1.4426950408889634);
-  sga_attend_kernel<<<rows * splits, kThreads, kSmemBytes, stream>>>(kvmap, qmap, p);
+  sga_attend_kernel<<<rows * splits, kThreads, kSmemBytes, stream>>>(qmap, p);
   e = cudaGetLastError();
   if (e != cudaSuccess || splits == 1) return e;
   sga_combine_kernel<<<rows * kHeads, 128, 0, stream>>>(a.part_o, a.part_ml, a.gate, a.out, splits);

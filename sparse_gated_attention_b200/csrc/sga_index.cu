@@ -16,7 +16,10 @@
 //   * Warps 2-5 (one per TMEM lane quarter) read a key's 64 head dots with
 //     tcgen05.ld, apply ReLU, the per-head weight and the head sum in fp32,
 //     mask s > t and store the score (32 consecutive keys per warp: one
-//     128-byte store).
+//     128-byte store).  When the caller asks for it, they also count each
+//     score's top 12 order bits into a per-query shared-memory histogram that
+//     is added to global memory when the query changes: the first level of
+//     the top-k radix select, computed while the scores are still in registers.
 #include "sga_internal.cuh"
 #include "sga_ptx.cuh"
 
@@ -35,7 +38,9 @@ constexpr int kAcc = 4;
 constexpr int kTmemCols = kAcc * kHeads;  // 256
 constexpr int kThreads = 192;
 constexpr int kNumBars = 2 * kStages + 4 + 2 * kAcc + 1;
-constexpr size_t kSmemBytes = 1024 + kStages * kAStage + 2 * kQBuf + kNumBars * 8 + 16;
+constexpr int kHistBytes = kTopkHistBins * 4;
+constexpr int kEpiThreads = 128;
+constexpr size_t kSmemBytes = 1024 + kStages * kAStage + 2 * kQBuf + kHistBytes + kNumBars * 8 + 16;
 
 static_assert(kDim == 2 * 64, "two 128-byte strips per key row");
 
@@ -43,6 +48,7 @@ struct IndexParams {
   const uint16_t* w;
   const int32_t* q_pos;
   float* scores;
+  uint32_t* hist;  // [rows][kTopkHistBins] or null
   int* status;
   int n_q, kv_stride, tiles_per_row;
   long long total_tiles;
@@ -65,7 +71,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t a_base = smem_u32(smem);
   const uint32_t q_base = a_base + kStages * kAStage;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kStages * kAStage + 2 * kQBuf);
+  uint32_t* hist_s = reinterpret_cast<uint32_t*>(smem + kStages * kAStage + 2 * kQBuf);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kStages * kAStage + 2 * kQBuf + kHistBytes);
   const uint32_t bar0 = smem_u32(bars);
   auto full = [&](int s) { return bar0 + 8u * s; };
   auto empty = [&](int s) { return bar0 + 8u * (kStages + s); };
@@ -217,13 +224,32 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else {
     // ------------------------------------------------------------ epilogue
     const int quarter = warp & 3;  // TMEM lanes 32*quarter .. +31 (warp % 4 rule)
+    const int et = threadIdx.x - 64;
+    const bool with_hist = p.hist != nullptr;
     long long an = 0;
     int cur_row = -1;
     float wv[kHeads];
+    // Adds the shared histogram of `r` to global memory and clears it.
+    auto flush_hist = [&](int r) {
+      named_barrier(1, kEpiThreads);
+      for (int b = et; b < kTopkHistBins; b += kEpiThreads) {
+        const uint32_t v = hist_s[b];
+        if (v) {
+          atomicAdd(p.hist + static_cast<size_t>(r) * kTopkHistBins + b, v);
+          hist_s[b] = 0;
+        }
+      }
+      named_barrier(1, kEpiThreads);
+    };
+    if (with_hist) {
+      for (int b = et; b < kTopkHistBins; b += kEpiThreads) hist_s[b] = 0;
+      named_barrier(1, kEpiThreads);
+    }
     for (long long j = j0; j < j1; ++j) {
       int row, key0, t;
       if (!tile_info(p, j, row, key0, t)) continue;
       if (row != cur_row) {
+        if (with_hist && cur_row >= 0) flush_hist(cur_row);
         const uint4* wp = reinterpret_cast<const uint4*>(p.w + static_cast<size_t>(row) * kHeads);
 #pragma unroll
         for (int c = 0; c < kHeads / 8; ++c) {
@@ -256,9 +282,13 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
       for (int h = 0; h < 32; ++h) s = fmaf(wv[32 + h], fmaxf(v1[h], 0.f), s);
       const int key = key0 + quarter * 32 + lane;
-      if (key <= t) p.scores[static_cast<size_t>(row) * p.kv_stride + key] = s;
+      if (key <= t) {
+        p.scores[static_cast<size_t>(row) * p.kv_stride + key] = s;
+        if (with_hist) atomicAdd(hist_s + (order_bits(s) >> (32 - kTopkHistBits)), 1u);
+      }
       ++an;
     }
+    if (with_hist && cur_row >= 0) flush_hist(cur_row);
   }
 
   tc_fence_before();
@@ -289,6 +319,7 @@ cudaError_t launch_index_scores(const IndexArgs& a, int num_sms, cudaStream_t st
   p.w = a.w;
   p.q_pos = a.q_pos;
   p.scores = a.scores;
+  p.hist = a.hist;
   p.status = a.status;
   p.n_q = a.n_q;
   p.kv_stride = a.kv_stride;

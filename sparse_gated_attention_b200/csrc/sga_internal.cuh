@@ -14,6 +14,7 @@ struct IndexArgs {
   const uint16_t* k_idx;  // [B][L][128]
   const int32_t* q_pos;   // [rows]
   float* scores;          // [rows][L]
+  uint32_t* hist;         // [rows][4096] first-level top-k histogram (zeroed by the caller) or null
   int* status;
   int batch, n_q, kv_stride;
 };
@@ -21,14 +22,16 @@ cudaError_t launch_index_scores(const IndexArgs& a, int num_sms, cudaStream_t st
 
 // ---- top-k (step 2) ------------------------------------------------------------
 struct TopkArgs {
-  const float* scores;  // [rows][L]
-  const int32_t* q_pos; // [rows]
-  int32_t* idx;         // [rows][K]
-  uint32_t* bitmap;     // [rows][words_per_row] scratch
+  const float* scores;   // [rows][L]
+  const int32_t* q_pos;  // [rows]
+  int32_t* idx;          // [rows][K]
+  uint32_t* bitmap;      // [rows][words_per_row] scratch
+  const uint32_t* hist;  // [rows][4096] histogram of the top 12 order bits, or null
   int* status;
   int rows, kv_stride, top_k;
 };
 size_t topk_bitmap_words(int kv_stride);
+int topk_cluster_size(int rows);
 cudaError_t launch_topk(const TopkArgs& a, cudaStream_t stream);
 
 // ---- sparse attention + gate (steps 3-4) -----------------------------------------
