@@ -6,28 +6,34 @@
 // For one query: Q [64 heads x 576], rows C_s [576] for s in idx,
 //   S = Q C^T * 192^-0.5,  P = softmax_s(S),  O = P C[:, 0:512],  out = O * sigmoid(g)
 //
-// Kernel design (one CTA per (query, split of the K selected slots)):
-//   * Shared memory: Q (9 swizzled 64x64 boxes, 72 KB, loaded once by TMA), a
-//     17-slot ring of 8 KB boxes holding gathered rows, and P (hi and lo bf16
-//     parts, 8 KB each).
-//   * Warps 0-3 gather a 64-row tile as 9 boxes [rope dims 512..575, then
-//     value dims 0..63, ..., 448..511] with 16-byte cp.async copies written
-//     straight into the 128-byte-swizzled layout (each warp instruction moves
-//     four full 128-byte row strips; empty slots are zero-filled without a
-//     read), completing on the box's mbarrier.  Warp 0 also publishes a 64-bit
-//     mask of non-empty slots per tile and loads Q with TMA.
-//   * Warp 4 issues tcgen05.mma: S_j = Q C_j^T (M = 64 heads, N = 64 rows,
-//     K = 576) into one of two TMEM S buffers, and O += P_j V_j as 8 MMAs of
-//     M = 64, N = 64 dims, K = 64 rows each, for P_hi and P_lo (P split into
-//     two bf16 parts keeps ~16 mantissa bits of P).  S_{j+1} is issued before
-//     PV_j so the softmax of tile j overlaps the next QK^T.
-//   * Warps 5-8 (one per TMEM lane quarter, 16 heads each) run the softmax in
-//     the log2 domain with a lazy running max (O in TMEM is rescaled only when
-//     the max grows by more than 2^8), write P to shared memory in the
-//     swizzled K-major layout, and finally scale O by sigmoid(g)/l.
-//   * TMEM (512 columns): O for dims 0..255 in lanes 0-15 of each quarter and
-//     dims 256..511 in lanes 16-31 (the two half-lane interleaves of the M = 64
-//     accumulator layout), columns 0..255; S buffers at columns 256 and 320.
+// Kernel design (one CTA per (query, split of the K selected slots); the
+// selected rows are processed in chunks of 128):
+//   * tcgen05.mma costs a fixed ~70 cycles per instruction below M x N =
+//     128 x 128 and ~220 when consecutive MMAs change accumulator, so every
+//     MMA here is 64 x 128 (QK^T) or 128 x 64 (PV) and runs in long chains on
+//     one accumulator.
+//   * QK^T: S_j [64 heads x 128 rows] = Q C_j^T, M = 64, N = 128, K = 576, Q
+//     (72 KB, 9 swizzled boxes, TMA) in shared memory, S in TMEM (two buffers).
+//   * PV in transposed form: O^T [512 dims x 64 heads] += V_j^T P_j^T as four
+//     M = 128 dim blocks, N = 64 heads, K = 128 rows; A = V^T read straight
+//     from the gathered rows (MN-major), B = P^T from the softmax (K-major).
+//     P is split into two bf16 parts (hi + lo, ~16 mantissa bits) so the
+//     result keeps the accuracy of an fp32 P.
+//   * Gathered rows stream through a 3-slot ring of 32 KB slots (128 rows x
+//     128 dims) in MMA consumption order: QK(j) takes 5 slots (dims 0..511
+//     and the rope dims 512..575), PV(j-1) takes 4 slots of value dims.  The
+//     value rows are gathered a second time for PV (they are still in L2), so
+//     shared memory only holds data in flight.  Issue order QK(j), PV(j-1) lets
+//     the softmax of chunk j-1 overlap QK^T of chunk j.
+//   * Warps 0-3 gather with 16-byte cp.async written straight into the
+//     128-byte-swizzled layout (empty slots zero-filled without a read);
+//     warp 0 also publishes the validity mask of each chunk and loads Q.
+//     Warp 4 issues the MMAs.  Warps 5-8 (one per TMEM lane quarter) run the
+//     softmax in the log2 domain with a lazy running max (O is rescaled only
+//     when the max grows by more than 2^8) and the epilogue.
+//   * TMEM (512 columns): O^T in columns 0..255 (dim block b at 64 b, all
+//     lanes), S buffers at columns 256 and 384 (M = 64 layout: lanes 0-15 of
+//     each quarter).
 //   * With several splits per query the CTA writes (O, m, l) partials and a
 //     small combine kernel merges them and applies the gate.
 #include <math.h>
@@ -41,25 +47,30 @@ namespace {
 constexpr int kHeads = 64;
 constexpr int kDq = 576;
 constexpr int kDv = 512;
-constexpr int kTile = 64;
-constexpr int kBox = 64 * 128;  // 64 rows x 64 bf16 (128 B per row)
-constexpr int kBoxesPerTile = 9;
-constexpr int kRing = 17;       // >= 8 value boxes of tile j + 9 boxes of tile j+1
-constexpr int kQBytes = 9 * kBox;
-constexpr int kPBytes = kHeads * kTile * 2;
+constexpr int kChunk = 128;                   // selected rows per chunk
+constexpr int kBoxBytes = kChunk * 128;       // 128 rows x 64 dims bf16
+constexpr int kSlotBytes = 2 * kBoxBytes;     // 128 rows x 128 dims
+constexpr int kRing = 3;
+constexpr int kQBox = kHeads * 128;           // 64 heads x 64 dims
+constexpr int kQBytes = 9 * kQBox;
+constexpr int kPAtom = kHeads * 128;          // 64 heads x 64 rows
+constexpr int kPBytes = 2 * kPAtom;           // 64 heads x 128 rows
+constexpr int kQkSlots = 5;
+constexpr int kPvSlots = 4;
 constexpr int kMaskRing = 4;
-constexpr int kProducers = 128;  // warps 0-3
+constexpr int kProducers = 128;               // warps 0-3
 constexpr int kMmaWarp = 4;
+constexpr int kSoftmaxThreads = 128;          // warps 5-8
 constexpr int kThreads = 288;
 constexpr int kTmemCols = 512;
 constexpr int kSCol = 256;
-// barriers: full[17] empty[17] q_full s_full[2] s_free[2] p_full p_free o_full mask_full[4] mask_empty[4]
+// barriers: full[3] empty[3] q_full s_full[2] s_free[2] p_full p_free o_full mask_full[4] mask_empty[4]
 constexpr int kNumBars = 2 * kRing + 1 + 2 + 2 + 3 + 2 * kMaskRing;
-constexpr size_t kSmemBytes = 1024 + kRing * kBox + kQBytes + 2 * kPBytes + kNumBars * 8 + kMaskRing * 8 + 16;
+constexpr size_t kSmemBytes = 1024 + kRing * kSlotBytes + kQBytes + 2 * kPBytes + kNumBars * 8 +
+                              kMaskRing * 16 + kHeads * 4 + 16;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 
 static_assert(kSmemBytes <= 232448, "shared memory budget");
-static_assert(kRing >= 2 * kBoxesPerTile - 1, "ring must hold a tile's values plus the next tile");
 
 struct AttendParams {
   const uint16_t* kv;
@@ -69,7 +80,7 @@ struct AttendParams {
   float* part_o;
   float* part_ml;
   int* status;
-  int n_q, kv_stride, top_k, splits, tiles_per_split;
+  int n_q, kv_stride, top_k, splits, chunks_per_split;
   float scale_log2;
 };
 
@@ -80,16 +91,32 @@ __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
   return *reinterpret_cast<const uint32_t*>(&v);
 }
 
+// Slot sequence shared by the gather producers and the MMA issuer:
+// QK(0), QK(1), PV(0), QK(2), PV(1), ..., QK(n-1), PV(n-2), PV(n-1).
+struct SlotStep {
+  int chunk, pv, pair;
+};
+__device__ __forceinline__ SlotStep slot_step(int k, int n) {
+  if (k < kQkSlots) return {0, 0, k};
+  const int r = k - kQkSlots;
+  const int blk = r / (kQkSlots + kPvSlots), off = r % (kQkSlots + kPvSlots);
+  if (blk < n - 1) {
+    if (off < kQkSlots) return {blk + 1, 0, off};
+    return {blk, 1, off - kQkSlots};
+  }
+  return {n - 1, 1, off};  // trailing PV(n-1)
+}
+
 __global__ void __launch_bounds__(kThreads, 1)
     sga_attend_kernel(const __grid_constant__ CUtensorMap qmap, AttendParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t ring = smem_u32(smem);
-  const uint32_t q_s = ring + kRing * kBox;
+  const uint32_t q_s = ring + kRing * kSlotBytes;
   const uint32_t p_hi = q_s + kQBytes;
   const uint32_t p_lo = p_hi + kPBytes;
-  uint8_t* p_hi_ptr = smem + kRing * kBox + kQBytes;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kRing * kBox + kQBytes + 2 * kPBytes);
+  uint8_t* p_hi_ptr = smem + kRing * kSlotBytes + kQBytes;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kRing * kSlotBytes + kQBytes + 2 * kPBytes);
   const uint32_t bar0 = smem_u32(bars);
   auto full = [&](int s) { return bar0 + 8u * s; };
   auto empty = [&](int s) { return bar0 + 8u * (kRing + s); };
@@ -101,15 +128,18 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t o_full = bar0 + 8u * (2 * kRing + 7);
   auto mask_full = [&](int b) { return bar0 + 8u * (2 * kRing + 8 + b); };
   auto mask_empty = [&](int b) { return bar0 + 8u * (2 * kRing + 8 + kMaskRing + b); };
-  uint64_t* masks = bars + kNumBars;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(masks + kMaskRing);
+  uint64_t* masks = bars + kNumBars;                                // [kMaskRing][2]
+  float* head_f = reinterpret_cast<float*>(masks + 2 * kMaskRing);  // [64] per-head factors
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(head_f + kHeads);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int row = blockIdx.x / p.splits;
   const int split = blockIdx.x % p.splits;
-  const int ntiles = p.tiles_per_split;
+  const int nchunks = p.chunks_per_split;
+  const int slot_base = split * nchunks * kChunk;  // first selected slot of this split
+  const int nsteps = nchunks * (kQkSlots + kPvSlots);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kRing; ++s) {
@@ -119,14 +149,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(q_full, 1);
     for (int b = 0; b < 2; ++b) {
       mbar_init(s_full(b), 1);
-      mbar_init(s_free(b), 128);
+      mbar_init(s_free(b), kSoftmaxThreads);
     }
-    mbar_init(p_full, 128);
+    mbar_init(p_full, kSoftmaxThreads);
     mbar_init(p_free, 1);
     mbar_init(o_full, 1);
     for (int b = 0; b < kMaskRing; ++b) {
       mbar_init(mask_full(b), 1);
-      mbar_init(mask_empty(b), 128);
+      mbar_init(mask_empty(b), kSoftmaxThreads);
     }
     *abort_flag = 0;
     fence_barrier_init();
@@ -144,32 +174,44 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp < kProducers / 32) {
     // ------------------------------------------------------------ gather producers
     const int b = row / p.n_q;
-    const int32_t* idx_row = p.idx + static_cast<size_t>(row) * p.top_k + static_cast<size_t>(split) * ntiles * kTile;
+    const int32_t* idx_row = p.idx + static_cast<size_t>(row) * p.top_k;
     const uint16_t* kv_b = p.kv + static_cast<size_t>(b) * p.kv_stride * kDq;
     const int ptid = threadIdx.x;
     const int part = ptid & 7;   // 16-byte chunk of a 128-byte row strip
-    const int rsub = ptid >> 3;  // rows rsub + 16 i, i = 0..3
+    const int rsub = ptid >> 3;  // rows rsub + 16 i, i = 0..7
     bool ok = true;
     if (ptid == 0) {
       mbar_arrive_expect_tx(q_full, kQBytes);
       const uint64_t pol = policy_evict_first();
-      for (int c = 0; c < 9; ++c) tma_load_2d(q_s + c * kBox, &qmap, q_full, c * 64, row * kHeads, pol);
+      for (int c = 0; c < 9; ++c) tma_load_2d(q_s + c * kQBox, &qmap, q_full, c * 64, row * kHeads, pol);
     }
-    for (int j = 0; j < ntiles && ok; ++j) {
-      if (warp == 0) {
-        const int2 v = __ldg(reinterpret_cast<const int2*>(idx_row + j * kTile) + lane);
-        const bool ok0 = v.x >= 0 && v.x < p.kv_stride;
-        const bool ok1 = v.y >= 0 && v.y < p.kv_stride;
-        if ((v.x < -1 || v.x >= p.kv_stride) || (v.y < -1 || v.y >= p.kv_stride))
-          record_status(p.status, kStatusDeviceArg);
-        // 64-bit mask of filled slots: bit r <-> tile row r (lane l holds rows 2l, 2l+1)
-        uint64_t m = (static_cast<uint64_t>(ok0) << (2 * lane)) | (static_cast<uint64_t>(ok1) << (2 * lane + 1));
+    for (int k = 0; k < nsteps && ok; ++k) {
+      const SlotStep st = slot_step(k, nchunks);
+      const int first = slot_base + st.chunk * kChunk;
+      if (!st.pv && st.pair == 0 && warp == 0) {
+        // validity mask of this chunk's 128 slots (bit r <-> chunk row r)
+        uint64_t m[2];
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) m |= __shfl_xor_sync(0xFFFFFFFFu, m, o);
+        for (int h = 0; h < 2; ++h) {
+          bool v0 = false, v1 = false;
+          const int r0 = first + 64 * h + 2 * lane;
+          if (r0 < p.top_k) {
+            const int2 v = __ldg(reinterpret_cast<const int2*>(idx_row + r0));
+            v0 = v.x >= 0 && v.x < p.kv_stride;
+            v1 = v.y >= 0 && v.y < p.kv_stride;
+            if (v.x < -1 || v.x >= p.kv_stride || v.y < -1 || v.y >= p.kv_stride)
+              record_status(p.status, kStatusDeviceArg);
+          }
+          uint64_t x = (static_cast<uint64_t>(v0) << (2 * lane)) | (static_cast<uint64_t>(v1) << (2 * lane + 1));
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1) x |= __shfl_xor_sync(0xFFFFFFFFu, x, o);
+          m[h] = x;
+        }
         if (lane == 0) {
-          const int mb = j % kMaskRing;
-          if (mbar_wait(mask_empty(mb), static_cast<uint32_t>((j / kMaskRing) & 1) ^ 1u, abort_flag)) {
-            masks[mb] = m;
+          const int mb = st.chunk % kMaskRing;
+          if (mbar_wait(mask_empty(mb), static_cast<uint32_t>((st.chunk / kMaskRing) & 1) ^ 1u, abort_flag)) {
+            masks[2 * mb] = m[0];
+            masks[2 * mb + 1] = m[1];
             mbar_arrive(mask_full(mb));
           } else {
             ok = false;
@@ -178,30 +220,26 @@ __global__ void __launch_bounds__(kThreads, 1)
         ok = __shfl_sync(0xFFFFFFFFu, ok ? 1 : 0, 0) != 0;
         if (!ok) break;
       }
-      const uint16_t* src[4];
-      uint32_t nbytes[4];
+      const int slot = k % kRing;
+      if (!mbar_wait(empty(slot), static_cast<uint32_t>((k / kRing) & 1) ^ 1u, abort_flag)) {
+        ok = false;
+        break;
+      }
+      const bool two = st.pv || st.pair < 4;  // the rope slot holds one 64-dim box
+      const int dim0 = st.pair * 128;
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const int s = __ldg(idx_row + j * kTile + rsub + 16 * i);
+      for (int i = 0; i < 8; ++i) {
+        const int r = rsub + 16 * i;
+        const int sidx = first + r;
+        int s = -1;
+        if (sidx < p.top_k) s = __ldg(idx_row + sidx);
         const bool valid = s >= 0 && s < p.kv_stride;
-        src[i] = kv_b + static_cast<size_t>(valid ? s : 0) * kDq + part * 8;
-        nbytes[i] = valid ? 16u : 0u;
+        const uint16_t* src = kv_b + static_cast<size_t>(valid ? s : 0) * kDq + dim0 + part * 8;
+        const uint32_t dst = ring + slot * kSlotBytes + r * 128 + ((part ^ (r & 7)) << 4);
+        cp_async_16(dst, src, valid ? 16u : 0u);
+        if (two) cp_async_16(dst + kBoxBytes, src + 64, valid ? 16u : 0u);
       }
-      for (int c = 0; c < kBoxesPerTile; ++c) {
-        const long long n = static_cast<long long>(j) * kBoxesPerTile + c;
-        const int slot = static_cast<int>(n % kRing);
-        if (!mbar_wait(empty(slot), static_cast<uint32_t>((n / kRing) & 1) ^ 1u, abort_flag)) {
-          ok = false;
-          break;
-        }
-        const int dim0 = c == 0 ? kDv : (c - 1) * 64;
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const int r = rsub + 16 * i;
-          cp_async_16(ring + slot * kBox + r * 128 + ((part ^ (r & 7)) << 4), src[i] + dim0, nbytes[i]);
-        }
-        cp_async_arrive_noinc(full(slot));
-      }
+      cp_async_arrive_noinc(full(slot));
     }
     asm volatile("cp.async.wait_all;" ::: "memory");
     if (!ok) {
@@ -215,52 +253,70 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      constexpr uint32_t idesc_qk = idesc_bf16_f32(kHeads, kTile, false, false);
-      constexpr uint32_t idesc_pv = idesc_bf16_f32(kHeads, 64, false, true);
+      constexpr uint32_t idesc_qk = idesc_bf16_f32(kHeads, kChunk, false, false);
+      constexpr uint32_t idesc_pv = idesc_bf16_f32(128, kHeads, true, false);
       bool ok = mbar_wait(q_full, 0, abort_flag);
+      int k = 0;  // slot counter
+      auto take_slot = [&](uint32_t& addr) -> bool {
+        const int slot = k % kRing;
+        if (!mbar_wait(full(slot), static_cast<uint32_t>((k / kRing) & 1), abort_flag)) return false;
+        fence_proxy_async_smem();  // written by cp.async (generic proxy)
+        tc_fence_after();
+        addr = ring + slot * kSlotBytes;
+        return true;
+      };
       auto issue_qk = [&](int j) -> bool {
         const int sb = j & 1;
         if (!mbar_wait(s_free(sb), static_cast<uint32_t>((j >> 1) & 1) ^ 1u, abort_flag)) return false;
-        const uint32_t d = tmem + kSCol + sb * kTile;
-        int rope_slot = 0;
-        for (int c = 0; c < kBoxesPerTile; ++c) {
-          const long long n = static_cast<long long>(j) * kBoxesPerTile + c;
-          const int slot = static_cast<int>(n % kRing);
-          if (!mbar_wait(full(slot), static_cast<uint32_t>((n / kRing) & 1), abort_flag)) return false;
-          fence_proxy_async_smem();  // the box was written by cp.async (generic proxy)
-          tc_fence_after();
-          if (c == 0) rope_slot = slot;
-          const int qbox = c == 0 ? 8 : c - 1;  // Q box covering the same dims
+        tc_fence_after();
+        const uint32_t d = tmem + kSCol + sb * kChunk;
+        for (int pr = 0; pr < kQkSlots; ++pr) {
+          uint32_t sa;
+          if (!take_slot(sa)) return false;
+          const int nbox = pr == 4 ? 1 : 2;
+          for (int bx = 0; bx < nbox; ++bx) {
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk) {
-            mma_bf16(d, sdesc_sw128(q_s + qbox * kBox + kk * 32, 16, 1024),
-                     sdesc_sw128(ring + slot * kBox + kk * 32, 16, 1024), idesc_qk, (c | kk) != 0 ? 1u : 0u);
+            for (int kk = 0; kk < 4; ++kk) {
+              mma_bf16(d, sdesc_sw128(q_s + (2 * pr + bx) * kQBox + kk * 32, 16, 1024),
+                       sdesc_sw128(sa + bx * kBoxBytes + kk * 32, 16, 1024), idesc_qk,
+                       (pr | bx | kk) != 0 ? 1u : 0u);
+            }
           }
+          mma_commit(empty(k % kRing));
+          ++k;
         }
         mma_commit(s_full(sb));
-        mma_commit(empty(rope_slot));  // rope dims are not needed for P V
         return true;
       };
-      if (ok && ntiles > 0) ok = issue_qk(0);
-      for (int j = 0; j < ntiles && ok; ++j) {
-        if (j + 1 < ntiles && !(ok = issue_qk(j + 1))) break;
-        if (!(ok = mbar_wait(p_full, static_cast<uint32_t>(j & 1), abort_flag))) break;
+      auto issue_pv = [&](int j) -> bool {
+        if (!mbar_wait(p_full, static_cast<uint32_t>(j & 1), abort_flag)) return false;
         tc_fence_after();
-        for (int c = 1; c < kBoxesPerTile; ++c) {
-          const long long n = static_cast<long long>(j) * kBoxesPerTile + c;
-          const int slot = static_cast<int>(n % kRing);
-          const int vbox = c - 1;
-          const uint32_t d = vbox < 4 ? tmem + vbox * 64 : tmem + (16u << 16) + (vbox - 4) * 64;
+        for (int pr = 0; pr < kPvSlots; ++pr) {
+          uint32_t sa;
+          if (!take_slot(sa)) return false;
+          const uint32_t d = tmem + pr * kHeads;  // O^T block: dims 128 pr .. +127
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk) {
-            const uint64_t bdesc = sdesc_sw128(ring + slot * kBox + kk * 2048, kBox, 1024);
-            mma_bf16(d, sdesc_sw128(p_hi + kk * 32, 16, 1024), bdesc, idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
-            mma_bf16(d, sdesc_sw128(p_lo + kk * 32, 16, 1024), bdesc, idesc_pv, 1u);
+          for (int kk = 0; kk < 8; ++kk) {
+            // A = V^T: M = 128 dims spread over the slot's two boxes, K = rows 16 kk ..
+            const uint64_t adesc = sdesc_sw128(sa + kk * 2048, kBoxBytes, 1024);
+#pragma unroll
+            for (int part = 0; part < 2; ++part) {
+              const uint64_t bdesc =
+                  sdesc_sw128((part ? p_lo : p_hi) + (kk >> 2) * kPAtom + (kk & 3) * 32, 16, 1024);
+              mma_bf16(d, adesc, bdesc, idesc_pv, (j > 0 || kk > 0 || part > 0) ? 1u : 0u);
+            }
           }
-          mma_commit(empty(slot));
+          mma_commit(empty(k % kRing));
+          ++k;
         }
         mma_commit(p_free);
+        return true;
+      };
+      for (int j = 0; j < nchunks && ok; ++j) {
+        ok = issue_qk(j);
+        if (ok && j > 0) ok = issue_pv(j - 1);
       }
+      if (ok && nchunks > 0) ok = issue_pv(nchunks - 1);
       if (!ok) {
         record_status(p.status, kStatusTimeout);
         *abort_flag = 1;
@@ -274,38 +330,29 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else {
     // ------------------------------------------------------------ softmax + epilogue
     const int quarter = warp & 3;
-    const int hl = lane & 15;
-    const int head = quarter * 16 + hl;
+    const int head = quarter * 16 + (lane & 15);  // lanes 0-15 own this head's S row
+    const bool owner = lane < 16;
     const uint32_t lane_addr = static_cast<uint32_t>(quarter * 32) << 16;
     float m_ref = -INFINITY, l_run = 0.f;
     bool ok = true;
-    for (int j = 0; j < ntiles; ++j) {
+    for (int j = 0; j < nchunks; ++j) {
       const int sb = j & 1;
       if (!(ok = mbar_wait(s_full(sb), static_cast<uint32_t>((j >> 1) & 1), abort_flag))) break;
       tc_fence_after();
-      float s[64];
-      {
-        float a0[32], a1[32];
-        tmem_ld32(tmem + lane_addr + kSCol + sb * kTile, a0);
-        tmem_ld32(tmem + lane_addr + kSCol + sb * kTile + 32, a1);
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          s[i] = a0[i];
-          s[32 + i] = a1[i];
-        }
-      }
-      tc_fence_before();
-      mbar_arrive(s_free(sb));
       const int mb = j % kMaskRing;
       if (!(ok = mbar_wait(mask_full(mb), static_cast<uint32_t>((j / kMaskRing) & 1), abort_flag))) break;
-      const uint64_t mask = masks[mb];
+      const uint64_t mk0 = masks[2 * mb], mk1 = masks[2 * mb + 1];
       mbar_arrive(mask_empty(mb));
-
+      const uint32_t s_addr = tmem + lane_addr + kSCol + sb * kChunk;
+      // pass 1: row max of the masked, scaled logits
       float mt = -INFINITY;
+      for (int c = 0; c < 4; ++c) {
+        float v[32];
+        tmem_ld32(s_addr + c * 32, v);
+        const uint32_t bits = static_cast<uint32_t>((c < 2 ? mk0 : mk1) >> (32 * (c & 1)));
 #pragma unroll
-      for (int i = 0; i < 64; ++i) {
-        s[i] = ((mask >> i) & 1ull) ? s[i] * p.scale_log2 : -INFINITY;
-        mt = fmaxf(mt, s[i]);
+        for (int i = 0; i < 32; ++i)
+          if ((bits >> i) & 1u) mt = fmaxf(mt, v[i] * p.scale_log2);
       }
       float alpha = 1.f;
       bool resc = false;
@@ -316,53 +363,58 @@ __global__ void __launch_bounds__(kThreads, 1)
         m_ref = mt;
         resc = true;
       }
-      float psum = 0.f;
-      if (m_ref == -INFINITY) {
-#pragma unroll
-        for (int i = 0; i < 64; ++i) s[i] = 0.f;
-      } else {
-#pragma unroll
-        for (int i = 0; i < 64; ++i) {
-          s[i] = exp2f(s[i] - m_ref);
-          psum += s[i];
-        }
-      }
-      l_run = l_run * alpha + psum;
-
       // PV_{j-1} must be done before P and O are touched.
       if (!(ok = mbar_wait(p_free, static_cast<uint32_t>(j & 1) ^ 1u, abort_flag))) break;
       tc_fence_after();
-      const bool any_resc = __any_sync(0xFFFFFFFFu, lane < 16 && resc);
-      if (any_resc) {
-        const float a = __shfl_sync(0xFFFFFFFFu, (lane < 16 && resc) ? alpha : 1.f, hl);
-        for (int c = 0; c < 8; ++c) {
-          float o[32];
-          tmem_ld32(tmem + lane_addr + c * 32, o);
+      if (owner) head_f[head] = alpha;
+      if (named_barrier_or(1, kSoftmaxThreads, owner && resc)) {
+        // O^T[dim][head] *= alpha[head]: every lane holds one dim of each block
+        for (int blk = 0; blk < 4; ++blk) {
+          for (int c = 0; c < 2; ++c) {
+            float o[32];
+            tmem_ld32(tmem + lane_addr + blk * kHeads + c * 32, o);
 #pragma unroll
-          for (int i = 0; i < 32; ++i) o[i] *= a;
-          tmem_st32(tmem + lane_addr + c * 32, o);
-        }
-      }
-      if (lane < 16) {
-        // P[head][row] in the 128-byte-swizzled K-major layout (8 rows per 1 KB atom)
-        const uint32_t rbase = (head >> 3) * 1024 + (head & 7) * 128;
-#pragma unroll
-        for (int c8 = 0; c8 < 8; ++c8) {
-          uint32_t hi[4], lo[4];
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const float x0 = s[8 * c8 + 2 * e], x1 = s[8 * c8 + 2 * e + 1];
-            hi[e] = pack_bf16(x0, x1);
-            const float h0 = __uint_as_float(hi[e] << 16), h1 = __uint_as_float(hi[e] & 0xFFFF0000u);
-            lo[e] = pack_bf16(x0 - h0, x1 - h1);
+            for (int i = 0; i < 32; ++i) o[i] *= head_f[c * 32 + i];
+            tmem_st32(tmem + lane_addr + blk * kHeads + c * 32, o);
           }
-          const uint32_t off = rbase + ((c8 ^ (head & 7)) << 4);
-          *reinterpret_cast<uint4*>(p_hi_ptr + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
-          *reinterpret_cast<uint4*>(p_hi_ptr + kPBytes + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+        }
+        named_barrier(1, kSoftmaxThreads);
+      }
+      // pass 2: P = 2^(s - m) as bf16 hi + lo into P[head][row] (K-major, 128-byte swizzle)
+      float psum = 0.f;
+      const uint32_t rbase = (head >> 3) * 1024 + (head & 7) * 128;
+      for (int c = 0; c < 4; ++c) {
+        float v[32];
+        tmem_ld32(s_addr + c * 32, v);
+        const uint32_t bits = static_cast<uint32_t>((c < 2 ? mk0 : mk1) >> (32 * (c & 1)));
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          const float x = (((bits >> i) & 1u) && m_ref != -INFINITY) ? exp2f(v[i] * p.scale_log2 - m_ref) : 0.f;
+          v[i] = x;
+          psum += x;
+        }
+        if (owner) {
+#pragma unroll
+          for (int g = 0; g < 4; ++g) {  // 8 rows = one 16-byte chunk
+            uint32_t hi[4], lo[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const float x0 = v[8 * g + 2 * e], x1 = v[8 * g + 2 * e + 1];
+              hi[e] = pack_bf16(x0, x1);
+              const float h0 = __uint_as_float(hi[e] << 16), h1 = __uint_as_float(hi[e] & 0xFFFF0000u);
+              lo[e] = pack_bf16(x0 - h0, x1 - h1);
+            }
+            const int r0 = c * 32 + g * 8;  // chunk row of the first value
+            const uint32_t off = (r0 >> 6) * kPAtom + rbase + ((((r0 & 63) >> 3) ^ (head & 7)) << 4);
+            *reinterpret_cast<uint4*>(p_hi_ptr + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+            *reinterpret_cast<uint4*>(p_hi_ptr + kPBytes + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+          }
         }
       }
-      fence_proxy_async_smem();
+      l_run = l_run * alpha + psum;
       tc_fence_before();
+      mbar_arrive(s_free(sb));
+      fence_proxy_async_smem();
       mbar_arrive(p_full);
     }
     if (!ok) {
@@ -370,30 +422,34 @@ __global__ void __launch_bounds__(kThreads, 1)
       *abort_flag = 1;
     } else if (mbar_wait(o_full, 0, abort_flag)) {
       tc_fence_after();
-      const float m_h = __shfl_sync(0xFFFFFFFFu, m_ref, hl);
-      const float l_h = __shfl_sync(0xFFFFFFFFu, l_run, hl);
-      const int part = lane >> 4;  // 0: dims 0..255, 1: dims 256..511
-      float factor = 1.f;
-      float* dst;
-      if (p.splits == 1) {
-        const float g = p.gate ? sigmoidf_(bf16_bits_to_float(p.gate[static_cast<size_t>(row) * kHeads + head])) : 1.f;
-        factor = l_h > 0.f ? g / l_h : 0.f;
-        dst = p.out + (static_cast<size_t>(row) * kHeads + head) * kDv + part * 256;
-      } else {
-        const size_t slot = (static_cast<size_t>(row) * p.splits + split) * kHeads + head;
-        dst = p.part_o + slot * kDv + part * 256;
-        if (lane < 16) {
-          p.part_ml[slot * 2 + 0] = m_h;
-          p.part_ml[slot * 2 + 1] = l_h;
+      // per-head factor: gate / l (one split) or 1 (partials)
+      const size_t pslot = (static_cast<size_t>(row) * p.splits + split) * kHeads;
+      if (owner) {
+        float f = 1.f;
+        if (p.splits == 1) {
+          const float g =
+              p.gate ? sigmoidf_(bf16_bits_to_float(p.gate[static_cast<size_t>(row) * kHeads + head])) : 1.f;
+          f = l_run > 0.f ? g / l_run : 0.f;
+        } else {
+          p.part_ml[(pslot + head) * 2 + 0] = m_ref;
+          p.part_ml[(pslot + head) * 2 + 1] = l_run;
         }
+        head_f[head] = f;
       }
-      for (int c = 0; c < 8; ++c) {
-        float o[32];
-        tmem_ld32(tmem + lane_addr + c * 32, o);
-        float4* d4 = reinterpret_cast<float4*>(dst + c * 32);
+      named_barrier(1, kSoftmaxThreads);
+      // O^T block b: this lane holds dim 128 b + 32 quarter + lane for all 64 heads
+      float* base = p.splits == 1 ? p.out + static_cast<size_t>(row) * kHeads * kDv : p.part_o + pslot * kDv;
+      for (int blk = 0; blk < 4; ++blk) {
+        const int dim = 128 * blk + 32 * quarter + lane;
+        for (int c = 0; c < 2; ++c) {
+          float o[32];
+          tmem_ld32(tmem + lane_addr + blk * kHeads + c * 32, o);
 #pragma unroll
-        for (int i = 0; i < 8; ++i)
-          d4[i] = make_float4(o[4 * i] * factor, o[4 * i + 1] * factor, o[4 * i + 2] * factor, o[4 * i + 3] * factor);
+          for (int i = 0; i < 32; ++i) {
+            const int h = c * 32 + i;
+            base[static_cast<size_t>(h) * kDv + dim] = o[i] * head_f[h];
+          }
+        }
       }
     } else {
       record_status(p.status, kStatusTimeout);
@@ -457,10 +513,10 @@ __global__ void __launch_bounds__(128) sga_combine_kernel(const float* __restric
 
 // Splits of the K slots per query so that rows * splits fills ~148 SMs once.
 int attend_splits(int rows, int top_k) {
-  const int tiles = top_k / kTile;
+  const int chunks = (top_k + kChunk - 1) / kChunk;
   int best = 1;
-  for (int s = 1; s <= tiles && s <= 64; ++s) {
-    if (tiles % s == 0 && static_cast<long long>(rows) * s <= 148) best = s;
+  for (int s = 1; s <= chunks && s <= 64; ++s) {
+    if (chunks % s == 0 && static_cast<long long>(rows) * s <= 148) best = s;
   }
   return best;
 }
@@ -487,7 +543,7 @@ cudaError_t launch_attend(const AttendArgs& a, cudaStream_t stream) {
   p.kv_stride = a.kv_stride;
   p.top_k = a.top_k;
   p.splits = splits;
-  p.tiles_per_split = a.top_k / kTile / splits;
+  p.chunks_per_split = (a.top_k + kChunk - 1) / kChunk / splits;
   p.scale_log2 = static_cast<float>(0.07216878364870322 * 1.4426950408889634);
   sga_attend_kernel<<<rows * splits, kThreads, kSmemBytes, stream>>>(qmap, p);
   e = cudaGetLastError();
