@@ -39,7 +39,7 @@ Layout make_layout(const sga_dims_t& d, sga_op_t op) {
   size_t off = kStatusBytes;
   if (op == SGA_OP_TOPK_SELECT || op == SGA_OP_FORWARD) {
     l.bitmap = off;
-    off += align_up(rows * topk_bitmap_words(d.kv_stride) * 4);
+    off += align_up(rows * 2 * topk_bitmap_words(d.kv_stride) * 4);  // selection + tie bitmaps
   }
   if (op == SGA_OP_SPARSE_MLA_ATTEND || op == SGA_OP_FORWARD) {
     l.splits = attend_splits(static_cast<int>(rows), d.top_k);

@@ -3,23 +3,33 @@
 // only 2,048 positions).  Larger score first; equal scores go to the lower
 // position; output ascending, -1 padded.
 //
-// Each candidate s gets a unique 64-bit key
-//     order_bits(score[s]) << 32  |  (0xFFFFFFFF - s)
-// so "larger key" is exactly the selection order and the K-th largest key is a
-// single threshold.  One thread-block cluster of C CTAs (1024 threads each)
-// handles one query; CTA r owns a contiguous segment of the positions.
-//   1. MSD radix select over the keys, 12 bits per level.  Each CTA counts its
-//      segment into a shared-memory histogram; every CTA then sums the C
-//      histograms through distributed shared memory, so all agree on the bin
-//      that holds the threshold.  Levels stop once that bin fits the leader's
-//      candidate list (8192 keys).  When the indexer has already counted the
-//      first level (sga_forward) that pass is skipped.
-//   2. One pass over the segments: a selection bitmap word per 32 positions
-//      (warp ballot) marks keys above the bin; keys inside the bin are appended
-//      to the leader CTA's candidate list through distributed shared memory.
-//   3. The leader finishes the select among the candidates in shared memory,
-//      sets their bitmap bits, and emits the set bits in position order
-//      (per-thread popcounts + block scan).
+// Scores are ranked through order_bits (an order-preserving 32-bit image of
+// the float).  The K-th largest score key K* splits the positions into
+// "above" (all selected) and "ties" (key == K*, of which the lowest positions
+// fill the remaining slots); nothing else needs ordering.  One thread-block
+// cluster of C CTAs (1024 threads each) handles one query; CTA r owns a
+// contiguous segment of positions (a multiple of 128), which streams through a
+// 3-slot shared-memory ring of 32 KB bulk copies (TMA) so that every pass over
+// it reads shared memory while the next chunks are in flight.
+//   1. MSD radix select over the score key, 12/12/8 bits per level.  Each CTA
+//      counts its segment into a shared-memory histogram and all CTAs sum the
+//      C histograms through distributed shared memory, so every CTA finds the
+//      same bin.  Levels stop when that bin fits a candidate list (4096 keys)
+//      or holds a single key.  Under sga_forward the indexer has already
+//      counted the first level, so that pass is skipped.
+//   2. One pass over the segment, four positions per thread: per 32
+//      positions a selection word (keys above the bin) and a tie word (keys
+//      in the bin, once the bin is a single key) are assembled from per-lane
+//      nibbles with three shuffles; keys in a wider bin go to the CTA's
+//      candidate list.
+//   3. Every CTA copies all candidate lists over distributed shared memory,
+//      narrows them to K* itself (no leader), marks its own candidates in its
+//      own words and publishes two counts (selected, ties).
+//   4. Every CTA emits its own segment: popcounts, two block scans and the
+//      other CTAs' counts give each set bit its output slot; ties are taken in
+//      position order until the K slots are full.
+// The selection and tie words of a segment stay in shared memory (segments up
+// to 65536 positions) or in the workspace (longer segments).
 #include <cooperative_groups.h>
 
 #include "sga_internal.cuh"
@@ -35,10 +45,16 @@ constexpr int kWarps = kThreads / 32;
 constexpr int kBits = kTopkHistBits;  // 12
 constexpr int kBins = kTopkHistBins;  // 4096
 constexpr int kBinsPerThread = kBins / kThreads;
-constexpr int kCandCap = 8192;
+constexpr int kCandCap = 4096;
 constexpr int kMaxCluster = 8;
-constexpr int kUnroll = 4;
-constexpr size_t kSmemBytes = 2 * kBins * 4 + kCandCap * 8;
+constexpr int kChunk = 8192;           // scores per ring slot (32 KB)
+constexpr int kRingSlots = 3;
+constexpr int kSegWordsSmem = 2048;    // bitmap words per segment kept in shared memory
+constexpr int kMaxWordsPerThread = 8;  // bitmap words kept in registers per emission batch
+constexpr size_t kRingBytes = kRingSlots * kChunk * 4;
+constexpr int kWarpStage = 64;         // per-warp staging of candidates before one shared atomic
+constexpr size_t kSmemBytes =
+    kRingBytes + 2 * kBins * 4 + kCandCap * 8 + 2 * kSegWordsSmem * 4 + kWarps * kWarpStage * 8 + 4 * 8;
 
 struct TopkParams {
   const float* scores;
@@ -50,10 +66,6 @@ struct TopkParams {
   int kv_stride, top_k;
   long long words_per_row;
 };
-
-__device__ __forceinline__ uint64_t sel_key(float f, int s) {
-  return (static_cast<uint64_t>(order_bits(f)) << 32) | static_cast<uint64_t>(0xFFFFFFFFu - static_cast<uint32_t>(s));
-}
 
 // Inclusive block scan of one value per thread; also returns the block total.
 __device__ __forceinline__ uint32_t block_inclusive_scan(uint32_t v, uint32_t* warp_buf, uint32_t& total) {
@@ -86,8 +98,7 @@ struct Narrow {
 };
 
 // Finds the bin holding the `need`-th largest key: fewer than `need` keys lie
-// in higher bins, at least `need` in this bin or higher.  Bins only up to
-// `nbins` are used (the last level can be narrower than 12 bits).
+// in higher bins, at least `need` in this bin or higher.
 __device__ __forceinline__ Narrow find_bin(const uint32_t* hist, uint32_t need, uint32_t* warp_buf, Narrow* out) {
   const int i = threadIdx.x;
   uint32_t h[kBinsPerThread];
@@ -115,20 +126,64 @@ __device__ __forceinline__ Narrow find_bin(const uint32_t* hist, uint32_t need, 
   return *out;
 }
 
+// Four consecutive scores starting at s; positions >= end are read as 0 (the
+// caller masks them).  The vector form needs rows that start 16-byte aligned.
+template <bool kVec>
+__device__ __forceinline__ float4 load4(const float* sc, int s, int end) {
+  if (kVec) return __ldg(reinterpret_cast<const float4*>(sc + s));
+  float4 v;
+  v.x = s < end ? __ldg(sc + s) : 0.f;
+  v.y = s + 1 < end ? __ldg(sc + s + 1) : 0.f;
+  v.z = s + 2 < end ? __ldg(sc + s + 2) : 0.f;
+  v.w = s + 3 < end ? __ldg(sc + s + 3) : 0.f;
+  return v;
+}
+
+// Smallest / largest float whose order_bits lies in [lo_key, hi_key] (NaN bit
+// patterns at the ends of the key range map to -inf / +inf).
+__device__ __forceinline__ float key_to_float_lo(uint32_t k) {
+  if (k <= 0x007FFFFFu) return -INFINITY;
+  return __uint_as_float((k & 0x80000000u) ? (k ^ 0x80000000u) : ~k);
+}
+__device__ __forceinline__ float key_to_float_hi(uint32_t k) {
+  if (k >= 0xFF800000u) return INFINITY;
+  if (k == 0x7FFFFFFFu) k = 0x7FFFFFFEu;  // the key of -0.0: zeros fold onto +0.0, which lies above
+  return __uint_as_float((k & 0x80000000u) ? (k ^ 0x80000000u) : ~k);
+}
+
+// Merges a 4-bit nibble per lane into one 32-bit word per 8 lanes (lane 8w then
+// holds the word for positions 32w .. 32w+31 of the warp's 128).
+__device__ __forceinline__ uint32_t nibbles_to_word(uint32_t nib, int lane) {
+  uint32_t w = nib << (4 * (lane & 7));
+  w |= __shfl_xor_sync(0xFFFFFFFFu, w, 1);
+  w |= __shfl_xor_sync(0xFFFFFFFFu, w, 2);
+  w |= __shfl_xor_sync(0xFFFFFFFFu, w, 4);
+  return w;
+}
+
+template <bool kVec>
 __global__ void __launch_bounds__(kThreads, 1) sga_topk_kernel(TopkParams p) {
-  extern __shared__ __align__(16) uint8_t smem_raw[];
-  uint32_t* lhist = reinterpret_cast<uint32_t*>(smem_raw);
+  extern __shared__ __align__(128) uint8_t smem_raw[];
+  float* ring = reinterpret_cast<float*>(smem_raw);
+  uint32_t* lhist = reinterpret_cast<uint32_t*>(smem_raw + kRingBytes);
   uint32_t* ghist = lhist + kBins;
-  uint64_t* cand = reinterpret_cast<uint64_t*>(smem_raw + 2 * kBins * 4);
+  uint64_t* cand = reinterpret_cast<uint64_t*>(ghist + kBins);
+  uint32_t* selw_s = reinterpret_cast<uint32_t*>(cand + kCandCap);
+  uint32_t* tiew_s = selw_s + kSegWordsSmem;
+  uint64_t* wstage = reinterpret_cast<uint64_t*>(tiew_s + kSegWordsSmem) + (threadIdx.x >> 5) * kWarpStage;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(tiew_s + kSegWordsSmem) + kWarps * kWarpStage;  // full[3], hist
   __shared__ uint32_t warp_buf[kWarps];
+  __shared__ uint32_t warp_buf2[kWarps];
   __shared__ Narrow narrow;
-  __shared__ uint32_t cand_n;
+  __shared__ uint32_t cand_n;     // candidates of this CTA's segment
+  __shared__ uint32_t counts[2];  // this segment's (selected, ties), read by the whole cluster
+  __shared__ int abort_flag;
 
   cg::cluster_group cluster = cg::this_cluster();
   const int C = static_cast<int>(cluster.num_blocks());
   const int rank = static_cast<int>(cluster.block_rank());
   const int row = blockIdx.x / C;
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int tid = threadIdx.x, lane = tid & 31;
   const int K = p.top_k;
   int32_t* out = p.idx + static_cast<size_t>(row) * K;
   const int t = __ldg(p.q_pos + row);
@@ -146,15 +201,72 @@ __global__ void __launch_bounds__(kThreads, 1) sga_topk_kernel(TopkParams p) {
     return;
   }
   const float* sc = p.scores + static_cast<size_t>(row) * p.kv_stride;
-  uint32_t* bits = p.bitmap + static_cast<size_t>(row) * p.words_per_row;
-  const int per = (((n + C - 1) / C) + 31) & ~31;
+  const int per = (((n + C - 1) / C) + 127) & ~127;
   const int s0 = min(rank * per, n), s1 = min(s0 + per, n);
-  if (tid == 0) cand_n = 0;
+  const int nch = (s1 - s0 + kChunk - 1) / kChunk;
+  // selection / tie words of this segment: shared memory when they fit, else the workspace
+  const int wbeg = s0 >> 5, wend = (s1 + 31) >> 5;
+  const bool words_in_smem = wend - wbeg <= kSegWordsSmem;
+  uint32_t* gsel = p.bitmap + static_cast<size_t>(row) * 2 * p.words_per_row;
+  uint32_t* selw = words_in_smem ? selw_s : gsel;
+  uint32_t* tiew = words_in_smem ? tiew_s : gsel + p.words_per_row;
+  const int woff = words_in_smem ? wbeg : 0;
+  const uint32_t bar0 = smem_u32(bars);
+  auto full = [&](int slot) { return bar0 + 8u * slot; };
+  const uint32_t hist_bar = bar0 + 8u * kRingSlots;
+  if (tid == 0) {
+    cand_n = 0;
+    abort_flag = 0;
+    for (int i = 0; i <= kRingSlots; ++i) mbar_init(bar0 + 8u * i, 1);
+    fence_barrier_init();
+  }
+  __syncthreads();
 
-  // ---- 1. radix levels until the threshold bin fits the candidate list
-  uint64_t prefix = 0, mask = 0;
+  // Chunk j of the segment into ring slot (g % 3); g counts chunks over all passes.
+  auto issue = [&](int g, int j) {
+    const int slot = g % kRingSlots;
+    const int pos = s0 + j * kChunk;
+    const int cnt = min(kChunk, s1 - pos);
+    const uint32_t bytes = static_cast<uint32_t>((cnt + 3) & ~3) * 4u;
+    mbar_arrive_expect_tx(full(slot), bytes);
+    bulk_load(smem_u32(ring + slot * kChunk), sc + pos, bytes, full(slot));
+  };
+  if (kVec && tid == 0) {
+    if (p.hist) {
+      mbar_arrive_expect_tx(hist_bar, kBins * 4);
+      bulk_load(smem_u32(ghist), p.hist + static_cast<size_t>(row) * kBins, kBins * 4, hist_bar);
+    }
+    for (int j = 0; j < min(kRingSlots, nch); ++j) issue(j, j);
+  }
+  int consumed = 0;  // chunks consumed by earlier passes
+  // One pass over the segment: body(pos, chunk data in shared memory (or null), count).
+  auto stream = [&](auto&& body) {
+    if (kVec) {
+      if (consumed > 0 && tid == 0)
+        for (int j = 0; j < min(kRingSlots, nch); ++j) issue(consumed + j, j);
+      for (int j = 0; j < nch; ++j) {
+        const int g = consumed + j, slot = g % kRingSlots;
+        if (!mbar_wait(full(slot), static_cast<uint32_t>((g / kRingSlots) & 1), &abort_flag))
+          record_status(p.status, kStatusTimeout);
+        const int pos = s0 + j * kChunk;
+        body(pos, ring + slot * kChunk, min(kChunk, s1 - pos));
+        __syncthreads();  // slot fully read
+        if (tid == 0 && j + kRingSlots < nch) issue(g + kRingSlots, j + kRingSlots);
+      }
+      consumed += nch;
+    } else {
+      for (int pos = s0; pos < s1; pos += kChunk) body(pos, nullptr, min(kChunk, s1 - pos));
+    }
+  };
+  auto load4s = [&](const float* d, int f, int s) -> float4 {
+    if (kVec) return reinterpret_cast<const float4*>(d)[f];
+    return load4<false>(sc, s, s1);
+  };
+
+  // ---- 1. radix levels on the score key until the bin fits the candidate list or is one key
+  uint32_t prefix = 0, mask = 0;
   uint32_t need = static_cast<uint32_t>(K);
-  int shift = 64;
+  int shift = 32;
   uint32_t bucket = 0;
   bool first = true;
   while (true) {
@@ -162,28 +274,28 @@ __global__ void __launch_bounds__(kThreads, 1) sga_topk_kernel(TopkParams p) {
     shift -= width;
     const uint32_t dmask = (1u << width) - 1u;
     if (first && p.hist) {
-      const uint32_t* hrow = p.hist + static_cast<size_t>(row) * kBins;
-      for (int b = tid; b < kBins; b += kThreads) ghist[b] = __ldg(hrow + b);
+      if (kVec) {
+        if (!mbar_wait(hist_bar, 0, &abort_flag)) record_status(p.status, kStatusTimeout);
+      } else {
+        const uint32_t* hrow = p.hist + static_cast<size_t>(row) * kBins;
+        for (int b = tid; b < kBins; b += kThreads) ghist[b] = __ldg(hrow + b);
+      }
       __syncthreads();
     } else {
       for (int b = tid; b < kBins; b += kThreads) lhist[b] = 0;
       __syncthreads();
-      for (int base = s0; base < s1; base += kUnroll * kThreads) {
-        float v[kUnroll];
+      stream([&](int pos, const float* d, int cnt) {
+        for (int f = tid; 4 * f < cnt; f += kThreads) {
+          const int s = pos + 4 * f;
+          const float4 v = load4s(d, f, s);
+          const float e[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-        for (int u = 0; u < kUnroll; ++u) {
-          const int s = base + u * kThreads + tid;
-          v[u] = s < s1 ? __ldg(sc + s) : 0.f;
-        }
-#pragma unroll
-        for (int u = 0; u < kUnroll; ++u) {
-          const int s = base + u * kThreads + tid;
-          if (s < s1) {
-            const uint64_t c = sel_key(v[u], s);
-            if ((c & mask) == prefix) atomicAdd(lhist + (static_cast<uint32_t>(c >> shift) & dmask), 1u);
+          for (int j = 0; j < 4; ++j) {
+            const uint32_t k = order_bits(e[j]);
+            if (s + j < s1 && (k & mask) == prefix) atomicAdd(lhist + ((k >> shift) & dmask), 1u);
           }
         }
-      }
+      });
       cluster.sync();
       for (int b = tid; b < kBins; b += kThreads) {
         uint32_t acc = 0;
@@ -194,103 +306,222 @@ __global__ void __launch_bounds__(kThreads, 1) sga_topk_kernel(TopkParams p) {
     }
     first = false;
     const Narrow nr = find_bin(ghist, need, warp_buf, &narrow);
-    prefix |= static_cast<uint64_t>(nr.digit) << shift;
-    mask |= static_cast<uint64_t>(dmask) << shift;
+    prefix |= nr.digit << shift;
+    mask |= dmask << shift;
     need -= nr.above;
     bucket = nr.count;
     if (bucket <= kCandCap || shift == 0) break;
   }
+  // A bin that is a single key holds exact ties: they go straight to the tie words.
+  const bool resolved = shift == 0;
 
-  // ---- 2. bitmap of keys above the bin; keys in the bin -> leader's candidate list
-  cluster.sync();  // the leader's cand_n is initialised
-  uint64_t* lead_cand = cluster.map_shared_rank(cand, 0);
-  uint32_t* lead_n = cluster.map_shared_rank(&cand_n, 0);
-  for (int base = s0; base < s1; base += kUnroll * kThreads) {
-    float v[kUnroll];
+  // ---- 2. one pass over the segment: selection / tie words and local candidates.
+  // The bin is the key range [prefix, prefix | ~mask]; as floats, "above" is
+  // f > f_hi and "in the bin" is f_lo <= f <= f_hi, so most positions cost two
+  // compares and warps with nothing to record skip the word assembly.
+  const float f_lo = key_to_float_lo(prefix), f_hi = key_to_float_hi(prefix | ~mask);
+  for (int w = wbeg + tid; w < wend; w += kThreads) {
+    selw[w - woff] = 0u;
+    tiew[w - woff] = 0u;
+  }
+  __syncthreads();
+  uint32_t my_sel = 0, my_tie = 0;
+  uint32_t wcount = 0;  // staged candidates of this warp (same value in every lane)
+  auto flush_stage = [&]() {
+    if (wcount == 0) return;
+    __syncwarp();  // staged entries written by other lanes are visible
+    uint32_t base = 0;
+    if (lane == 0) base = atomicAdd(&cand_n, wcount);
+    base = __shfl_sync(0xFFFFFFFFu, base, 0);
+    for (uint32_t i = lane; i < wcount; i += 32)
+      if (base + i < kCandCap) cand[base + i] = wstage[i];
+    __syncwarp();
+    wcount = 0;
+  };
+  stream([&](int pos, const float* d, int cnt) {
+    for (int f = tid; f < kChunk / 4; f += kThreads) {  // same trip count in every lane
+      const int s = pos + 4 * f;
+      const float4 v = 4 * f < cnt ? load4s(d, f, s) : make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
+      const float e[4] = {v.x, v.y, v.z, v.w};
+      uint32_t nib_above = 0, nib_bin = 0;
 #pragma unroll
-    for (int u = 0; u < kUnroll; ++u) {
-      const int s = base + u * kThreads + tid;
-      v[u] = s < s1 ? __ldg(sc + s) : 0.f;
-    }
-#pragma unroll
-    for (int u = 0; u < kUnroll; ++u) {
-      const int s = base + u * kThreads + tid;
-      bool above = false, in_bin = false;
-      uint64_t c = 0;
-      if (s < s1) {
-        c = sel_key(v[u], s);
-        above = (c & mask) > prefix;
-        in_bin = (c & mask) == prefix;
+      for (int j = 0; j < 4; ++j) {
+        const bool valid = s + j < s1;
+        nib_above |= static_cast<uint32_t>(valid && e[j] > f_hi) << j;
+        nib_bin |= static_cast<uint32_t>(valid && e[j] >= f_lo && e[j] <= f_hi) << j;
       }
-      const uint32_t word = __ballot_sync(0xFFFFFFFFu, above);
-      const int first_pos = base + u * kThreads + warp * 32;
-      if (lane == 0 && first_pos < s1) bits[first_pos >> 5] = word;
-      const uint32_t cm = __ballot_sync(0xFFFFFFFFu, in_bin);
-      if (cm) {
-        uint32_t off = 0;
-        if (lane == 0) off = atomicAdd(lead_n, static_cast<uint32_t>(__popc(cm)));
-        off = __shfl_sync(0xFFFFFFFFu, off, 0);
-        if (in_bin) {
-          const uint32_t r = off + __popc(cm & ((1u << lane) - 1u));
-          if (r < kCandCap) lead_cand[r] = c;
+      if (!__any_sync(0xFFFFFFFFu, (nib_above | nib_bin) != 0)) continue;
+      my_sel += __popc(nib_above);
+      const uint32_t wa = nibbles_to_word(nib_above, lane);
+      const uint32_t wb = nibbles_to_word(nib_bin, lane);
+      if ((lane & 7) == 0 && s < s1) {
+        if (wa) selw[(s >> 5) - woff] = wa;
+        if (resolved && wb) tiew[(s >> 5) - woff] = wb;
+      }
+      if (resolved) {
+        my_tie += __popc(nib_bin);
+      } else if (__any_sync(0xFFFFFFFFu, nib_bin != 0)) {
+        // stage this lane's in-bin keys in the warp's buffer: warp prefix of the per-lane counts
+        const uint32_t c4 = __popc(nib_bin);
+        uint32_t incl = c4;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const uint32_t y = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+          if (lane >= o) incl += y;
+        }
+        const uint32_t total = __shfl_sync(0xFFFFFFFFu, incl, 31);
+        if (wcount + total > kWarpStage) flush_stage();
+        uint64_t* dst = wstage + wcount;
+        uint32_t off = incl - c4;
+        if (total > kWarpStage) {  // more than a buffer in one step: straight to the list
+          uint32_t base = 0;
+          if (lane == 31) base = atomicAdd(&cand_n, total);
+          base = __shfl_sync(0xFFFFFFFFu, base, 31);
+          dst = cand;
+          off += base;
+        }
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          if ((nib_bin >> j) & 1u) {
+            if (dst != cand || off < kCandCap)
+              dst[off] = (static_cast<uint64_t>(order_bits(e[j])) << 32) | (0xFFFFFFFFu - static_cast<uint32_t>(s + j));
+            ++off;
+          }
+        }
+        if (total <= kWarpStage) wcount += total;
+      }
+    }
+  });
+  if (!resolved) flush_stage();
+  cluster.sync();  // segments scanned, candidate lists complete
+
+  // ---- 3. every CTA: all candidates -> K*; mark own candidates; publish counts
+  if (!resolved) {
+    const uint32_t own = min(cand_n, static_cast<uint32_t>(kCandCap));
+    uint32_t offs[kMaxCluster + 1];
+    int src_rank[kMaxCluster];
+    offs[0] = own;
+    int m = 0;
+    for (int r = 0; r < C; ++r) {
+      if (r == rank) continue;
+      src_rank[m] = r;
+      offs[m + 1] = offs[m] + *cluster.map_shared_rank(&cand_n, r);
+      ++m;
+    }
+    const uint32_t nc = min(offs[m], static_cast<uint32_t>(kCandCap));
+    for (uint32_t g = own + tid; g < nc; g += kThreads) {
+      int q = 0;
+      while (q < m - 1 && g >= offs[q + 1]) ++q;
+      cand[g] = cluster.map_shared_rank(cand, src_rank[q])[g - offs[q]];
+    }
+    cluster.sync();  // remote lists read; each CTA extended its own list behind its own entries
+    uint64_t kmask = static_cast<uint64_t>(mask) << 32, kpref = static_cast<uint64_t>(prefix) << 32;
+    while (shift > 0) {
+      const int width = shift >= kBits ? kBits : shift;
+      shift -= width;
+      const uint32_t dmask = (1u << width) - 1u;
+      for (int b = tid; b < kBins; b += kThreads) ghist[b] = 0;
+      __syncthreads();
+      for (uint32_t i = tid; i < nc; i += kThreads) {
+        const uint64_t c = cand[i];
+        if ((c & kmask) == kpref) atomicAdd(ghist + (static_cast<uint32_t>(c >> (32 + shift)) & dmask), 1u);
+      }
+      __syncthreads();
+      const Narrow nr = find_bin(ghist, need, warp_buf, &narrow);
+      kpref |= static_cast<uint64_t>(nr.digit) << (32 + shift);
+      kmask |= static_cast<uint64_t>(dmask) << (32 + shift);
+      need -= nr.above;
+    }
+    // own candidates (the first `own` entries) -> selection or tie bits in own words
+    for (uint32_t i = tid; i < own; i += kThreads) {
+      const uint64_t c = cand[i];
+      const uint64_t hi = c & kmask;
+      if (hi >= kpref) {
+        const uint32_t s = 0xFFFFFFFFu - static_cast<uint32_t>(c);
+        const bool tie = hi == kpref;
+        atomicOr((tie ? tiew : selw) + ((s >> 5) - woff), 1u << (s & 31));
+        if (tie) {
+          ++my_tie;
+        } else {
+          ++my_sel;
         }
       }
     }
   }
-  cluster.sync();  // all candidates appended, all bitmap words written
-  if (rank != 0) return;
+  uint32_t seg_sel, seg_tie;
+  block_inclusive_scan(my_sel, warp_buf, seg_sel);
+  block_inclusive_scan(my_tie, warp_buf2, seg_tie);
+  if (tid == 0) {
+    counts[0] = seg_sel;
+    counts[1] = seg_tie;
+  }
+  cluster.sync();  // counts published, own words marked
+  uint32_t sel_before = 0, tie_before = 0, sel_all = 0, tie_all = 0;
+  for (int r = 0; r < C; ++r) {
+    const uint32_t* rc = cluster.map_shared_rank(counts, r);
+    const uint32_t a = rc[0], b = rc[1];
+    if (r < rank) {
+      sel_before += a;
+      tie_before += b;
+    }
+    sel_all += a;
+    tie_all += b;
+  }
+  cluster.sync();  // every CTA has read every count
+  const uint32_t take_all = static_cast<uint32_t>(K) > sel_all ? static_cast<uint32_t>(K) - sel_all : 0u;
+  if (rank == 0 && tid == 0 &&
+      (sel_all > static_cast<uint32_t>(K) || sel_all + tie_all < static_cast<uint32_t>(K)))
+    record_status(p.status, kStatusDeviceArg);
 
-  // ---- 3. leader: finish the select inside the candidate list
-  const uint32_t nc = cand_n < kCandCap ? cand_n : kCandCap;
-  while (need < bucket && shift > 0) {
-    const int width = shift >= kBits ? kBits : shift;
-    shift -= width;
-    const uint32_t dmask = (1u << width) - 1u;
-    for (int b = tid; b < kBins; b += kThreads) ghist[b] = 0;
-    __syncthreads();
-    for (uint32_t i = tid; i < nc; i += kThreads) {
-      const uint64_t c = cand[i];
-      if ((c & mask) == prefix) atomicAdd(ghist + (static_cast<uint32_t>(c >> shift) & dmask), 1u);
+  // ---- 4. emit this segment in position order
+  uint32_t sel_run = sel_before, tie_run = tie_before;
+  for (int wb = wbeg; wb < wend; wb += kThreads * kMaxWordsPerThread) {
+    const int w0 = wb + tid * kMaxWordsPerThread;
+    uint32_t sw[kMaxWordsPerThread], tw[kMaxWordsPerThread];
+    uint32_t cs = 0, ct = 0;
+#pragma unroll
+    for (int i = 0; i < kMaxWordsPerThread; ++i) {
+      const bool in = w0 + i < wend;
+      sw[i] = in ? selw[w0 + i - woff] : 0u;
+      tw[i] = in ? tiew[w0 + i - woff] : 0u;
+      cs += __popc(sw[i]);
+      ct += __popc(tw[i]);
     }
-    __syncthreads();
-    const Narrow nr = find_bin(ghist, need, warp_buf, &narrow);
-    prefix |= static_cast<uint64_t>(nr.digit) << shift;
-    mask |= static_cast<uint64_t>(dmask) << shift;
-    need -= nr.above;
-    bucket = nr.count;
-  }
-  for (uint32_t i = tid; i < nc; i += kThreads) {
-    const uint64_t c = cand[i];
-    if ((c & mask) >= prefix) {
-      const uint32_t s = 0xFFFFFFFFu - static_cast<uint32_t>(c);
-      atomicOr(bits + (s >> 5), 1u << (s & 31));
+    uint32_t bs, bt;
+    const uint32_t s_incl = block_inclusive_scan(cs, warp_buf, bs);
+    const uint32_t t_incl = block_inclusive_scan(ct, warp_buf2, bt);
+    const uint32_t tb = tie_run + t_incl - ct;
+    uint32_t pos = sel_run + (s_incl - cs) + min(tb, take_all);
+    uint32_t ties_left = tb < take_all ? take_all - tb : 0u;
+#pragma unroll
+    for (int i = 0; i < kMaxWordsPerThread; ++i) {
+      uint32_t t2 = tw[i], keep = 0;
+      while (t2 && ties_left) {
+        const uint32_t low = t2 & (0u - t2);
+        keep |= low;
+        t2 ^= low;
+        --ties_left;
+      }
+      uint32_t mm = sw[i] | keep;
+      while (mm) {
+        const int b = __ffs(mm) - 1;
+        mm &= mm - 1;
+        if (pos < static_cast<uint32_t>(K)) out[pos] = (w0 + i) * 32 + b;
+        ++pos;
+      }
     }
+    sel_run += bs;
+    tie_run += bt;
   }
-  __syncthreads();
-
-  // ---- emit set bits in position order
-  const int words = (n + 31) >> 5;
-  const int per_t = (words + kThreads - 1) / kThreads;
-  const int w0 = min(tid * per_t, words), w1 = min(w0 + per_t, words);
-  uint32_t cnt = 0;
-  for (int wi = w0; wi < w1; ++wi) cnt += __popc(__ldcg(bits + wi));
-  uint32_t total;
-  uint32_t pos = block_inclusive_scan(cnt, warp_buf, total) - cnt;
-  for (int wi = w0; wi < w1; ++wi) {
-    uint32_t m = __ldcg(bits + wi);
-    while (m) {
-      const int b = __ffs(m) - 1;
-      m &= m - 1;
-      if (pos < static_cast<uint32_t>(K)) out[pos] = wi * 32 + b;
-      ++pos;
-    }
+  if (rank == 0) {
+    const uint32_t emitted = sel_all + min(tie_all, take_all);
+    for (int j = static_cast<int>(emitted) + tid; j < K; j += kThreads) out[j] = -1;
   }
-  if (tid == 0 && (total != static_cast<uint32_t>(K) || cand_n > kCandCap)) record_status(p.status, kStatusDeviceArg);
-  for (int j = static_cast<int>(total) + tid; j < K; j += kThreads) out[j] = -1;
 }
 
 }  // namespace
 
+// Words of one bitmap per row; the workspace holds two per row (selected, ties).
 size_t topk_bitmap_words(int kv_stride) { return (static_cast<size_t>(kv_stride) + 31) / 32; }
 
 // CTAs per query: enough to fill the GPU once, at most kMaxCluster.
@@ -302,7 +533,9 @@ int topk_cluster_size(int rows) {
 
 cudaError_t launch_topk(const TopkArgs& a, cudaStream_t stream) {
   if (a.rows == 0) return cudaSuccess;
-  cudaError_t e = cudaFuncSetAttribute(sga_topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  const bool vec = (a.kv_stride % 4 == 0) && (reinterpret_cast<uintptr_t>(a.scores) % 16 == 0);
+  auto kernel = vec ? sga_topk_kernel<true> : sga_topk_kernel<false>;
+  cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(kSmemBytes));
   if (e != cudaSuccess) return e;
   TopkParams p;
@@ -328,7 +561,7 @@ cudaError_t launch_topk(const TopkArgs& a, cudaStream_t stream) {
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, sga_topk_kernel, p);
+  return cudaLaunchKernelEx(&cfg, kernel, p);
 }
 
 }  // namespace sga
