@@ -7,32 +7,31 @@
 //   S = Q C^T * 192^-0.5,  P = softmax_s(S),  O = P C[:, 0:512],  out = O * sigmoid(g)
 //
 // Kernel design (one CTA per (query, split of the K selected slots); the
-// selected rows are processed in chunks of 128):
-//   * tcgen05.mma costs a fixed ~70 cycles per instruction below M x N =
-//     128 x 128 and ~220 when consecutive MMAs change accumulator, so every
-//     MMA here is 64 x 128 (QK^T) or 128 x 64 (PV) and runs in long chains on
-//     one accumulator.
-//   * QK^T: S_j [64 heads x 128 rows] = Q C_j^T, M = 64, N = 128, K = 576, Q
-//     (72 KB, 9 swizzled boxes, TMA) in shared memory, S in TMEM (two buffers).
+// selected rows are processed in chunks of 64, each gathered exactly once):
+//   * QK^T: S_j [64 heads x 64 rows] = Q C_j^T, M = 64, N = 64, K = 576, with
+//     Q (72 KB, 9 swizzled boxes, TMA) in shared memory and S in TMEM (two
+//     buffers).
 //   * PV in transposed form: O^T [512 dims x 64 heads] += V_j^T P_j^T as four
-//     M = 128 dim blocks, N = 64 heads, K = 128 rows; A = V^T read straight
+//     M = 128 dim blocks, N = 64 heads, K = 64 rows; A = V^T read straight
 //     from the gathered rows (MN-major), B = P^T from the softmax (K-major).
 //     P is split into two bf16 parts (hi + lo, ~16 mantissa bits) so the
-//     result keeps the accuracy of an fp32 P.
-//   * Gathered rows stream through a 3-slot ring of 32 KB slots (128 rows x
-//     128 dims) in MMA consumption order: QK(j) takes 5 slots (dims 0..511
-//     and the rope dims 512..575), PV(j-1) takes 4 slots of value dims.  The
-//     value rows are gathered a second time for PV (they are still in L2), so
-//     shared memory only holds data in flight.  Issue order QK(j), PV(j-1) lets
-//     the softmax of chunk j-1 overlap QK^T of chunk j.
+//     result keeps the accuracy of an fp32 P.  tcgen05.mma costs ~70 cycles
+//     per instruction at these sizes and ~220 when consecutive MMAs change
+//     accumulator, so each accumulator gets its MMAs back to back.
+//   * The value dims of a chunk arrive as four 16 KB "pair" slots (two
+//     swizzled 64-dim boxes each, so one M = 128 block of V^T has a fixed box
+//     stride) in an 8-slot ring, i.e. two chunks; the rope dims use one 8 KB
+//     slot that is freed right after QK^T.  QK^T(j+1) is issued before PV(j),
+//     so the softmax of chunk j overlaps the next QK^T and chunk j+2 streams in
+//     while chunk j's values wait for P.
 //   * Warps 0-3 gather with 16-byte cp.async written straight into the
 //     128-byte-swizzled layout (empty slots zero-filled without a read);
 //     warp 0 also publishes the validity mask of each chunk and loads Q.
-//     Warp 4 issues the MMAs.  Warps 5-8 (one per TMEM lane quarter) run the
-//     softmax in the log2 domain with a lazy running max (O is rescaled only
-//     when the max grows by more than 2^8) and the epilogue.
+//     Warp 4 issues the MMAs.  Warps 5-8 (one per TMEM lane quarter, 16 heads
+//     each) run the softmax in the log2 domain with a lazy running max (O is
+//     rescaled only when the max grows by more than 2^8) and the epilogue.
 //   * TMEM (512 columns): O^T in columns 0..255 (dim block b at 64 b, all
-//     lanes), S buffers at columns 256 and 384 (M = 64 layout: lanes 0-15 of
+//     lanes), S buffers at columns 256 and 320 (M = 64 layout: lanes 0-15 of
 //     each quarter).
 //   * With several splits per query the CTA writes (O, m, l) partials and a
 //     small combine kernel merges them and applies the gate.
@@ -47,27 +46,26 @@ namespace {
 constexpr int kHeads = 64;
 constexpr int kDq = 576;
 constexpr int kDv = 512;
-constexpr int kChunk = 128;                   // selected rows per chunk
-constexpr int kBoxBytes = kChunk * 128;       // 128 rows x 64 dims bf16
-constexpr int kSlotBytes = 2 * kBoxBytes;     // 128 rows x 128 dims
-constexpr int kRing = 3;
-constexpr int kQBox = kHeads * 128;           // 64 heads x 64 dims
+constexpr int kChunk = 64;                  // selected rows per chunk
+constexpr int kBoxBytes = kChunk * 128;     // 64 rows x 64 dims bf16
+constexpr int kPairBytes = 2 * kBoxBytes;   // 64 rows x 128 dims
+constexpr int kPairsPerChunk = 4;           // value dims 0..511
+constexpr int kPairRing = 8;                // two chunks of value pairs
+constexpr int kQBox = kHeads * 128;         // 64 heads x 64 dims
 constexpr int kQBytes = 9 * kQBox;
-constexpr int kPAtom = kHeads * 128;          // 64 heads x 64 rows
-constexpr int kPBytes = 2 * kPAtom;           // 64 heads x 128 rows
-constexpr int kQkSlots = 5;
-constexpr int kPvSlots = 4;
+constexpr int kPBytes = kHeads * kChunk * 2;  // 64 heads x 64 rows bf16
 constexpr int kMaskRing = 4;
-constexpr int kProducers = 128;               // warps 0-3
+constexpr int kProducers = 128;             // warps 0-3
 constexpr int kMmaWarp = 4;
-constexpr int kSoftmaxThreads = 128;          // warps 5-8
+constexpr int kSoftmaxThreads = 128;        // warps 5-8
 constexpr int kThreads = 288;
 constexpr int kTmemCols = 512;
 constexpr int kSCol = 256;
-// barriers: full[3] empty[3] q_full s_full[2] s_free[2] p_full p_free o_full mask_full[4] mask_empty[4]
-constexpr int kNumBars = 2 * kRing + 1 + 2 + 2 + 3 + 2 * kMaskRing;
-constexpr size_t kSmemBytes = 1024 + kRing * kSlotBytes + kQBytes + 2 * kPBytes + kNumBars * 8 +
-                              kMaskRing * 16 + kHeads * 4 + 16;
+// barriers: pair_full[8] pair_empty[8] rope_full rope_empty q_full s_full[2] s_free[2]
+//           p_full p_free o_full mask_full[4] mask_empty[4]
+constexpr int kNumBars = 2 * kPairRing + 2 + 1 + 2 + 2 + 3 + 2 * kMaskRing;
+constexpr size_t kSmemBytes = 1024 + kPairRing * kPairBytes + kBoxBytes + kQBytes + 2 * kPBytes + kNumBars * 8 +
+                              kMaskRing * 8 + kHeads * 4 + 16;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 
 static_assert(kSmemBytes <= 232448, "shared memory budget");
@@ -91,45 +89,32 @@ __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
   return *reinterpret_cast<const uint32_t*>(&v);
 }
 
-// Slot sequence shared by the gather producers and the MMA issuer:
-// QK(0), QK(1), PV(0), QK(2), PV(1), ..., QK(n-1), PV(n-2), PV(n-1).
-struct SlotStep {
-  int chunk, pv, pair;
-};
-__device__ __forceinline__ SlotStep slot_step(int k, int n) {
-  if (k < kQkSlots) return {0, 0, k};
-  const int r = k - kQkSlots;
-  const int blk = r / (kQkSlots + kPvSlots), off = r % (kQkSlots + kPvSlots);
-  if (blk < n - 1) {
-    if (off < kQkSlots) return {blk + 1, 0, off};
-    return {blk, 1, off - kQkSlots};
-  }
-  return {n - 1, 1, off};  // trailing PV(n-1)
-}
-
 __global__ void __launch_bounds__(kThreads, 1)
     sga_attend_kernel(const __grid_constant__ CUtensorMap qmap, AttendParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  const uint32_t ring = smem_u32(smem);
-  const uint32_t q_s = ring + kRing * kSlotBytes;
+  const uint32_t pairs = smem_u32(smem);
+  const uint32_t rope = pairs + kPairRing * kPairBytes;
+  const uint32_t q_s = rope + kBoxBytes;
   const uint32_t p_hi = q_s + kQBytes;
   const uint32_t p_lo = p_hi + kPBytes;
-  uint8_t* p_hi_ptr = smem + kRing * kSlotBytes + kQBytes;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kRing * kSlotBytes + kQBytes + 2 * kPBytes);
+  uint8_t* p_hi_ptr = smem + kPairRing * kPairBytes + kBoxBytes + kQBytes;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(p_hi_ptr + 2 * kPBytes);
   const uint32_t bar0 = smem_u32(bars);
-  auto full = [&](int s) { return bar0 + 8u * s; };
-  auto empty = [&](int s) { return bar0 + 8u * (kRing + s); };
-  const uint32_t q_full = bar0 + 8u * (2 * kRing);
-  auto s_full = [&](int b) { return bar0 + 8u * (2 * kRing + 1 + b); };
-  auto s_free = [&](int b) { return bar0 + 8u * (2 * kRing + 3 + b); };
-  const uint32_t p_full = bar0 + 8u * (2 * kRing + 5);
-  const uint32_t p_free = bar0 + 8u * (2 * kRing + 6);
-  const uint32_t o_full = bar0 + 8u * (2 * kRing + 7);
-  auto mask_full = [&](int b) { return bar0 + 8u * (2 * kRing + 8 + b); };
-  auto mask_empty = [&](int b) { return bar0 + 8u * (2 * kRing + 8 + kMaskRing + b); };
-  uint64_t* masks = bars + kNumBars;                                // [kMaskRing][2]
-  float* head_f = reinterpret_cast<float*>(masks + 2 * kMaskRing);  // [64] per-head factors
+  auto pair_full = [&](int s) { return bar0 + 8u * s; };
+  auto pair_empty = [&](int s) { return bar0 + 8u * (kPairRing + s); };
+  const uint32_t rope_full = bar0 + 8u * (2 * kPairRing);
+  const uint32_t rope_empty = rope_full + 8u;
+  const uint32_t q_full = rope_full + 16u;
+  auto s_full = [&](int b) { return q_full + 8u * (1 + b); };
+  auto s_free = [&](int b) { return q_full + 8u * (3 + b); };
+  const uint32_t p_full = q_full + 8u * 5;
+  const uint32_t p_free = q_full + 8u * 6;
+  const uint32_t o_full = q_full + 8u * 7;
+  auto mask_full = [&](int b) { return q_full + 8u * (8 + b); };
+  auto mask_empty = [&](int b) { return q_full + 8u * (8 + kMaskRing + b); };
+  uint64_t* masks = bars + kNumBars;
+  float* head_f = reinterpret_cast<float*>(masks + kMaskRing);  // [64] per-head factors
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(head_f + kHeads);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -139,13 +124,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int split = blockIdx.x % p.splits;
   const int nchunks = p.chunks_per_split;
   const int slot_base = split * nchunks * kChunk;  // first selected slot of this split
-  const int nsteps = nchunks * (kQkSlots + kPvSlots);
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kRing; ++s) {
-      mbar_init(full(s), kProducers);  // one cp.async arrival per producer thread
-      mbar_init(empty(s), 1);
+    for (int s = 0; s < kPairRing; ++s) {
+      mbar_init(pair_full(s), kProducers);  // one cp.async arrival per producer thread
+      mbar_init(pair_empty(s), 1);
     }
+    mbar_init(rope_full, kProducers);
+    mbar_init(rope_empty, 1);
     mbar_init(q_full, 1);
     for (int b = 0; b < 2; ++b) {
       mbar_init(s_full(b), 1);
@@ -178,40 +164,33 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint16_t* kv_b = p.kv + static_cast<size_t>(b) * p.kv_stride * kDq;
     const int ptid = threadIdx.x;
     const int part = ptid & 7;   // 16-byte chunk of a 128-byte row strip
-    const int rsub = ptid >> 3;  // rows rsub + 16 i, i = 0..7
+    const int rsub = ptid >> 3;  // rows rsub + 16 i, i = 0..3
     bool ok = true;
     if (ptid == 0) {
       mbar_arrive_expect_tx(q_full, kQBytes);
       const uint64_t pol = policy_evict_first();
       for (int c = 0; c < 9; ++c) tma_load_2d(q_s + c * kQBox, &qmap, q_full, c * 64, row * kHeads, pol);
     }
-    for (int k = 0; k < nsteps && ok; ++k) {
-      const SlotStep st = slot_step(k, nchunks);
-      const int first = slot_base + st.chunk * kChunk;
-      if (!st.pv && st.pair == 0 && warp == 0) {
-        // validity mask of this chunk's 128 slots (bit r <-> chunk row r)
-        uint64_t m[2];
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          bool v0 = false, v1 = false;
-          const int r0 = first + 64 * h + 2 * lane;
-          if (r0 < p.top_k) {
-            const int2 v = __ldg(reinterpret_cast<const int2*>(idx_row + r0));
-            v0 = v.x >= 0 && v.x < p.kv_stride;
-            v1 = v.y >= 0 && v.y < p.kv_stride;
-            if (v.x < -1 || v.x >= p.kv_stride || v.y < -1 || v.y >= p.kv_stride)
-              record_status(p.status, kStatusDeviceArg);
-          }
-          uint64_t x = (static_cast<uint64_t>(v0) << (2 * lane)) | (static_cast<uint64_t>(v1) << (2 * lane + 1));
-#pragma unroll
-          for (int o = 16; o > 0; o >>= 1) x |= __shfl_xor_sync(0xFFFFFFFFu, x, o);
-          m[h] = x;
+    for (int j = 0; j < nchunks && ok; ++j) {
+      const int first = slot_base + j * kChunk;
+      if (warp == 0) {
+        // validity mask of this chunk's 64 slots (bit r <-> chunk row r)
+        bool v0 = false, v1 = false;
+        const int r0 = first + 2 * lane;
+        if (r0 < p.top_k) {
+          const int2 v = __ldg(reinterpret_cast<const int2*>(idx_row + r0));
+          v0 = v.x >= 0 && v.x < p.kv_stride;
+          v1 = v.y >= 0 && v.y < p.kv_stride;
+          if (v.x < -1 || v.x >= p.kv_stride || v.y < -1 || v.y >= p.kv_stride)
+            record_status(p.status, kStatusDeviceArg);
         }
+        uint64_t m = (static_cast<uint64_t>(v0) << (2 * lane)) | (static_cast<uint64_t>(v1) << (2 * lane + 1));
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) m |= __shfl_xor_sync(0xFFFFFFFFu, m, o);
         if (lane == 0) {
-          const int mb = st.chunk % kMaskRing;
-          if (mbar_wait(mask_empty(mb), static_cast<uint32_t>((st.chunk / kMaskRing) & 1) ^ 1u, abort_flag)) {
-            masks[2 * mb] = m[0];
-            masks[2 * mb + 1] = m[1];
+          const int mb = j % kMaskRing;
+          if (mbar_wait(mask_empty(mb), static_cast<uint32_t>((j / kMaskRing) & 1) ^ 1u, abort_flag)) {
+            masks[mb] = m;
             mbar_arrive(mask_full(mb));
           } else {
             ok = false;
@@ -220,26 +199,47 @@ __global__ void __launch_bounds__(kThreads, 1)
         ok = __shfl_sync(0xFFFFFFFFu, ok ? 1 : 0, 0) != 0;
         if (!ok) break;
       }
-      const int slot = k % kRing;
-      if (!mbar_wait(empty(slot), static_cast<uint32_t>((k / kRing) & 1) ^ 1u, abort_flag)) {
-        ok = false;
-        break;
-      }
-      const bool two = st.pv || st.pair < 4;  // the rope slot holds one 64-dim box
-      const int dim0 = st.pair * 128;
+      // this thread's four rows of the chunk
+      const uint16_t* src[4];
+      uint32_t nbytes[4];
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const int r = rsub + 16 * i;
-        const int sidx = first + r;
+      for (int i = 0; i < 4; ++i) {
+        const int sidx = first + rsub + 16 * i;
         int s = -1;
         if (sidx < p.top_k) s = __ldg(idx_row + sidx);
         const bool valid = s >= 0 && s < p.kv_stride;
-        const uint16_t* src = kv_b + static_cast<size_t>(valid ? s : 0) * kDq + dim0 + part * 8;
-        const uint32_t dst = ring + slot * kSlotBytes + r * 128 + ((part ^ (r & 7)) << 4);
-        cp_async_16(dst, src, valid ? 16u : 0u);
-        if (two) cp_async_16(dst + kBoxBytes, src + 64, valid ? 16u : 0u);
+        src[i] = kv_b + static_cast<size_t>(valid ? s : 0) * kDq + part * 8;
+        nbytes[i] = valid ? 16u : 0u;
       }
-      cp_async_arrive_noinc(full(slot));
+      // rope dims 512..575 -> the rope slot
+      if (!mbar_wait(rope_empty, static_cast<uint32_t>(j & 1) ^ 1u, abort_flag)) {
+        ok = false;
+        break;
+      }
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int r = rsub + 16 * i;
+        cp_async_16(rope + r * 128 + ((part ^ (r & 7)) << 4), src[i] + kDv, nbytes[i]);
+      }
+      cp_async_arrive_noinc(rope_full);
+      // value dims 128 q .. 128 q + 127 -> pair slot (4 j + q) mod 8
+      for (int q = 0; q < kPairsPerChunk; ++q) {
+        const int n = j * kPairsPerChunk + q;
+        const int slot = n % kPairRing;
+        if (!mbar_wait(pair_empty(slot), static_cast<uint32_t>((n / kPairRing) & 1) ^ 1u, abort_flag)) {
+          ok = false;
+          break;
+        }
+        const uint32_t base = pairs + slot * kPairBytes;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int r = rsub + 16 * i;
+          const uint32_t dst = base + r * 128 + ((part ^ (r & 7)) << 4);
+          cp_async_16(dst, src[i] + 128 * q, nbytes[i]);
+          cp_async_16(dst + kBoxBytes, src[i] + 128 * q + 64, nbytes[i]);
+        }
+        cp_async_arrive_noinc(pair_full(slot));
+      }
     }
     asm volatile("cp.async.wait_all;" ::: "memory");
     if (!ok) {
@@ -256,13 +256,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       constexpr uint32_t idesc_qk = idesc_bf16_f32(kHeads, kChunk, false, false);
       constexpr uint32_t idesc_pv = idesc_bf16_f32(128, kHeads, true, false);
       bool ok = mbar_wait(q_full, 0, abort_flag);
-      int k = 0;  // slot counter
-      auto take_slot = [&](uint32_t& addr) -> bool {
-        const int slot = k % kRing;
-        if (!mbar_wait(full(slot), static_cast<uint32_t>((k / kRing) & 1), abort_flag)) return false;
+      auto wait_full = [&](uint32_t bar, uint32_t parity) -> bool {
+        if (!mbar_wait(bar, parity, abort_flag)) return false;
         fence_proxy_async_smem();  // written by cp.async (generic proxy)
         tc_fence_after();
-        addr = ring + slot * kSlotBytes;
         return true;
       };
       auto issue_qk = [&](int j) -> bool {
@@ -270,20 +267,24 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!mbar_wait(s_free(sb), static_cast<uint32_t>((j >> 1) & 1) ^ 1u, abort_flag)) return false;
         tc_fence_after();
         const uint32_t d = tmem + kSCol + sb * kChunk;
-        for (int pr = 0; pr < kQkSlots; ++pr) {
-          uint32_t sa;
-          if (!take_slot(sa)) return false;
-          const int nbox = pr == 4 ? 1 : 2;
-          for (int bx = 0; bx < nbox; ++bx) {
+        if (!wait_full(rope_full, static_cast<uint32_t>(j & 1))) return false;
 #pragma unroll
-            for (int kk = 0; kk < 4; ++kk) {
-              mma_bf16(d, sdesc_sw128(q_s + (2 * pr + bx) * kQBox + kk * 32, 16, 1024),
-                       sdesc_sw128(sa + bx * kBoxBytes + kk * 32, 16, 1024), idesc_qk,
-                       (pr | bx | kk) != 0 ? 1u : 0u);
-            }
+        for (int kk = 0; kk < 4; ++kk)
+          mma_bf16(d, sdesc_sw128(q_s + 8 * kQBox + kk * 32, 16, 1024), sdesc_sw128(rope + kk * 32, 16, 1024),
+                   idesc_qk, kk > 0 ? 1u : 0u);
+        mma_commit(rope_empty);  // rope dims are not needed for P V
+        for (int q = 0; q < kPairsPerChunk; ++q) {
+          const int n = j * kPairsPerChunk + q;
+          const int slot = n % kPairRing;
+          if (!wait_full(pair_full(slot), static_cast<uint32_t>((n / kPairRing) & 1))) return false;
+          const uint32_t base = pairs + slot * kPairBytes;
+#pragma unroll
+          for (int bx = 0; bx < 2; ++bx) {
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+              mma_bf16(d, sdesc_sw128(q_s + (2 * q + bx) * kQBox + kk * 32, 16, 1024),
+                       sdesc_sw128(base + bx * kBoxBytes + kk * 32, 16, 1024), idesc_qk, 1u);
           }
-          mma_commit(empty(k % kRing));
-          ++k;
         }
         mma_commit(s_full(sb));
         return true;
@@ -291,32 +292,30 @@ __global__ void __launch_bounds__(kThreads, 1)
       auto issue_pv = [&](int j) -> bool {
         if (!mbar_wait(p_full, static_cast<uint32_t>(j & 1), abort_flag)) return false;
         tc_fence_after();
-        for (int pr = 0; pr < kPvSlots; ++pr) {
-          uint32_t sa;
-          if (!take_slot(sa)) return false;
-          const uint32_t d = tmem + pr * kHeads;  // O^T block: dims 128 pr .. +127
+        for (int q = 0; q < kPairsPerChunk; ++q) {
+          const int slot = (j * kPairsPerChunk + q) % kPairRing;
+          const uint32_t base = pairs + slot * kPairBytes;
+          const uint32_t d = tmem + q * kHeads;  // O^T block: dims 128 q .. +127
 #pragma unroll
-          for (int kk = 0; kk < 8; ++kk) {
-            // A = V^T: M = 128 dims spread over the slot's two boxes, K = rows 16 kk ..
-            const uint64_t adesc = sdesc_sw128(sa + kk * 2048, kBoxBytes, 1024);
+          for (int kk = 0; kk < 4; ++kk) {
+            // A = V^T: M = 128 dims over the pair's two boxes, K = rows 16 kk ..
+            const uint64_t adesc = sdesc_sw128(base + kk * 2048, kBoxBytes, 1024);
 #pragma unroll
             for (int part = 0; part < 2; ++part) {
-              const uint64_t bdesc =
-                  sdesc_sw128((part ? p_lo : p_hi) + (kk >> 2) * kPAtom + (kk & 3) * 32, 16, 1024);
+              const uint64_t bdesc = sdesc_sw128((part ? p_lo : p_hi) + kk * 32, 16, 1024);
               mma_bf16(d, adesc, bdesc, idesc_pv, (j > 0 || kk > 0 || part > 0) ? 1u : 0u);
             }
           }
-          mma_commit(empty(k % kRing));
-          ++k;
+          mma_commit(pair_empty(slot));
         }
         mma_commit(p_free);
         return true;
       };
+      if (ok && nchunks > 0) ok = issue_qk(0);
       for (int j = 0; j < nchunks && ok; ++j) {
-        ok = issue_qk(j);
-        if (ok && j > 0) ok = issue_pv(j - 1);
+        if (j + 1 < nchunks && !(ok = issue_qk(j + 1))) break;
+        ok = issue_pv(j);
       }
-      if (ok && nchunks > 0) ok = issue_pv(nchunks - 1);
       if (!ok) {
         record_status(p.status, kStatusTimeout);
         *abort_flag = 1;
@@ -339,20 +338,28 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int sb = j & 1;
       if (!(ok = mbar_wait(s_full(sb), static_cast<uint32_t>((j >> 1) & 1), abort_flag))) break;
       tc_fence_after();
+      float s[64];
+      {
+        float a0[32], a1[32];
+        tmem_ld32(tmem + lane_addr + kSCol + sb * kChunk, a0);
+        tmem_ld32(tmem + lane_addr + kSCol + sb * kChunk + 32, a1);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          s[i] = a0[i];
+          s[32 + i] = a1[i];
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(s_free(sb));
       const int mb = j % kMaskRing;
       if (!(ok = mbar_wait(mask_full(mb), static_cast<uint32_t>((j / kMaskRing) & 1), abort_flag))) break;
-      const uint64_t mk0 = masks[2 * mb], mk1 = masks[2 * mb + 1];
+      const uint64_t mk = masks[mb];
       mbar_arrive(mask_empty(mb));
-      const uint32_t s_addr = tmem + lane_addr + kSCol + sb * kChunk;
-      // pass 1: row max of the masked, scaled logits
       float mt = -INFINITY;
-      for (int c = 0; c < 4; ++c) {
-        float v[32];
-        tmem_ld32(s_addr + c * 32, v);
-        const uint32_t bits = static_cast<uint32_t>((c < 2 ? mk0 : mk1) >> (32 * (c & 1)));
 #pragma unroll
-        for (int i = 0; i < 32; ++i)
-          if ((bits >> i) & 1u) mt = fmaxf(mt, v[i] * p.scale_log2);
+      for (int i = 0; i < 64; ++i) {
+        s[i] = ((mk >> i) & 1ull) ? s[i] * p.scale_log2 : -INFINITY;
+        mt = fmaxf(mt, s[i]);
       }
       float alpha = 1.f;
       bool resc = false;
@@ -363,6 +370,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         m_ref = mt;
         resc = true;
       }
+      float psum = 0.f;
+#pragma unroll
+      for (int i = 0; i < 64; ++i) {
+        s[i] = m_ref == -INFINITY ? 0.f : exp2f(s[i] - m_ref);
+        psum += s[i];
+      }
+      l_run = l_run * alpha + psum;
       // PV_{j-1} must be done before P and O are touched.
       if (!(ok = mbar_wait(p_free, static_cast<uint32_t>(j & 1) ^ 1u, abort_flag))) break;
       tc_fence_after();
@@ -380,41 +394,26 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         named_barrier(1, kSoftmaxThreads);
       }
-      // pass 2: P = 2^(s - m) as bf16 hi + lo into P[head][row] (K-major, 128-byte swizzle)
-      float psum = 0.f;
-      const uint32_t rbase = (head >> 3) * 1024 + (head & 7) * 128;
-      for (int c = 0; c < 4; ++c) {
-        float v[32];
-        tmem_ld32(s_addr + c * 32, v);
-        const uint32_t bits = static_cast<uint32_t>((c < 2 ? mk0 : mk1) >> (32 * (c & 1)));
+      if (owner) {
+        // P[head][row] in the 128-byte-swizzled K-major layout (8 heads per 1 KB atom)
+        const uint32_t rbase = (head >> 3) * 1024 + (head & 7) * 128;
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const float x = (((bits >> i) & 1u) && m_ref != -INFINITY) ? exp2f(v[i] * p.scale_log2 - m_ref) : 0.f;
-          v[i] = x;
-          psum += x;
-        }
-        if (owner) {
+        for (int c8 = 0; c8 < 8; ++c8) {
+          uint32_t hi[4], lo[4];
 #pragma unroll
-          for (int g = 0; g < 4; ++g) {  // 8 rows = one 16-byte chunk
-            uint32_t hi[4], lo[4];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const float x0 = v[8 * g + 2 * e], x1 = v[8 * g + 2 * e + 1];
-              hi[e] = pack_bf16(x0, x1);
-              const float h0 = __uint_as_float(hi[e] << 16), h1 = __uint_as_float(hi[e] & 0xFFFF0000u);
-              lo[e] = pack_bf16(x0 - h0, x1 - h1);
-            }
-            const int r0 = c * 32 + g * 8;  // chunk row of the first value
-            const uint32_t off = (r0 >> 6) * kPAtom + rbase + ((((r0 & 63) >> 3) ^ (head & 7)) << 4);
-            *reinterpret_cast<uint4*>(p_hi_ptr + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
-            *reinterpret_cast<uint4*>(p_hi_ptr + kPBytes + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+          for (int e = 0; e < 4; ++e) {
+            const float x0 = s[8 * c8 + 2 * e], x1 = s[8 * c8 + 2 * e + 1];
+            hi[e] = pack_bf16(x0, x1);
+            const float h0 = __uint_as_float(hi[e] << 16), h1 = __uint_as_float(hi[e] & 0xFFFF0000u);
+            lo[e] = pack_bf16(x0 - h0, x1 - h1);
           }
+          const uint32_t off = rbase + ((c8 ^ (head & 7)) << 4);
+          *reinterpret_cast<uint4*>(p_hi_ptr + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+          *reinterpret_cast<uint4*>(p_hi_ptr + kPBytes + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
         }
       }
-      l_run = l_run * alpha + psum;
-      tc_fence_before();
-      mbar_arrive(s_free(sb));
       fence_proxy_async_smem();
+      tc_fence_before();
       mbar_arrive(p_full);
     }
     if (!ok) {

@@ -161,6 +161,31 @@ __device__ __forceinline__ uint32_t nibbles_to_word(uint32_t nib, int lane) {
   return w;
 }
 
+// Chunk j of the segment [s0, s1) into ring slot g % kRingSlots (bulk copy,
+// completing on that slot's mbarrier); g counts chunks over all passes.
+__device__ __forceinline__ void ring_issue(float* ring, uint32_t bar0, const float* sc, int s0, int s1, int g, int j) {
+  const int slot = g % kRingSlots;
+  const int pos = s0 + j * kChunk;
+  const int cnt = min(kChunk, s1 - pos);
+  const uint32_t bytes = static_cast<uint32_t>((cnt + 3) & ~3) * 4u;
+  mbar_arrive_expect_tx(bar0 + 8u * slot, bytes);
+  bulk_load(smem_u32(ring + slot * kChunk), sc + pos, bytes, bar0 + 8u * slot);
+}
+
+// Moves a warp's staged candidates to the CTA list with one shared atomic; returns 0.
+__device__ __forceinline__ uint32_t flush_stage(uint32_t wcount, const uint64_t* wstage, uint64_t* cand,
+                                                uint32_t* cand_n, int lane) {
+  if (wcount == 0) return 0;
+  __syncwarp();  // staged entries written by other lanes are visible
+  uint32_t base = 0;
+  if (lane == 0) base = atomicAdd(cand_n, wcount);
+  base = __shfl_sync(0xFFFFFFFFu, base, 0);
+  for (uint32_t i = lane; i < wcount; i += 32)
+    if (base + i < kCandCap) cand[base + i] = wstage[i];
+  __syncwarp();
+  return 0;
+}
+
 template <bool kVec>
 __global__ void __launch_bounds__(kThreads, 1) sga_topk_kernel(TopkParams p) {
   extern __shared__ __align__(128) uint8_t smem_raw[];
@@ -212,7 +237,6 @@ __global__ void __launch_bounds__(kThreads, 1) sga_topk_kernel(TopkParams p) {
   uint32_t* tiew = words_in_smem ? tiew_s : gsel + p.words_per_row;
   const int woff = words_in_smem ? wbeg : 0;
   const uint32_t bar0 = smem_u32(bars);
-  auto full = [&](int slot) { return bar0 + 8u * slot; };
   const uint32_t hist_bar = bar0 + 8u * kRingSlots;
   if (tid == 0) {
     cand_n = 0;
@@ -221,47 +245,14 @@ __global__ void __launch_bounds__(kThreads, 1) sga_topk_kernel(TopkParams p) {
     fence_barrier_init();
   }
   __syncthreads();
-
-  // Chunk j of the segment into ring slot (g % 3); g counts chunks over all passes.
-  auto issue = [&](int g, int j) {
-    const int slot = g % kRingSlots;
-    const int pos = s0 + j * kChunk;
-    const int cnt = min(kChunk, s1 - pos);
-    const uint32_t bytes = static_cast<uint32_t>((cnt + 3) & ~3) * 4u;
-    mbar_arrive_expect_tx(full(slot), bytes);
-    bulk_load(smem_u32(ring + slot * kChunk), sc + pos, bytes, full(slot));
-  };
   if (kVec && tid == 0) {
     if (p.hist) {
       mbar_arrive_expect_tx(hist_bar, kBins * 4);
       bulk_load(smem_u32(ghist), p.hist + static_cast<size_t>(row) * kBins, kBins * 4, hist_bar);
     }
-    for (int j = 0; j < min(kRingSlots, nch); ++j) issue(j, j);
+    for (int j = 0; j < min(kRingSlots, nch); ++j) ring_issue(ring, bar0, sc, s0, s1, j, j);
   }
-  int consumed = 0;  // chunks consumed by earlier passes
-  // One pass over the segment: body(pos, chunk data in shared memory (or null), count).
-  auto stream = [&](auto&& body) {
-    if (kVec) {
-      if (consumed > 0 && tid == 0)
-        for (int j = 0; j < min(kRingSlots, nch); ++j) issue(consumed + j, j);
-      for (int j = 0; j < nch; ++j) {
-        const int g = consumed + j, slot = g % kRingSlots;
-        if (!mbar_wait(full(slot), static_cast<uint32_t>((g / kRingSlots) & 1), &abort_flag))
-          record_status(p.status, kStatusTimeout);
-        const int pos = s0 + j * kChunk;
-        body(pos, ring + slot * kChunk, min(kChunk, s1 - pos));
-        __syncthreads();  // slot fully read
-        if (tid == 0 && j + kRingSlots < nch) issue(g + kRingSlots, j + kRingSlots);
-      }
-      consumed += nch;
-    } else {
-      for (int pos = s0; pos < s1; pos += kChunk) body(pos, nullptr, min(kChunk, s1 - pos));
-    }
-  };
-  auto load4s = [&](const float* d, int f, int s) -> float4 {
-    if (kVec) return reinterpret_cast<const float4*>(d)[f];
-    return load4<false>(sc, s, s1);
-  };
+  int consumed = 0;  // ring chunks consumed by earlier passes (mbarrier phase bookkeeping)
 
   // ---- 1. radix levels on the score key until the bin fits the candidate list or is one key
   uint32_t prefix = 0, mask = 0;
@@ -284,18 +275,28 @@ __global__ void __launch_bounds__(kThreads, 1) sga_topk_kernel(TopkParams p) {
     } else {
       for (int b = tid; b < kBins; b += kThreads) lhist[b] = 0;
       __syncthreads();
-      stream([&](int pos, const float* d, int cnt) {
+      if (kVec && consumed > 0 && tid == 0)
+        for (int j = 0; j < min(kRingSlots, nch); ++j) ring_issue(ring, bar0, sc, s0, s1, consumed + j, j);
+      for (int j = 0; j < nch; ++j) {
+        const int g = consumed + j, slot = g % kRingSlots;
+        if (kVec && !mbar_wait(bar0 + 8u * slot, static_cast<uint32_t>((g / kRingSlots) & 1), &abort_flag))
+          record_status(p.status, kStatusTimeout);
+        const int pos = s0 + j * kChunk, cnt = min(kChunk, s1 - pos);
+        const float4* d4 = reinterpret_cast<const float4*>(ring + slot * kChunk);
         for (int f = tid; 4 * f < cnt; f += kThreads) {
           const int s = pos + 4 * f;
-          const float4 v = load4s(d, f, s);
+          const float4 v = kVec ? d4[f] : load4<false>(sc, s, s1);
           const float e[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            const uint32_t k = order_bits(e[j]);
-            if (s + j < s1 && (k & mask) == prefix) atomicAdd(lhist + ((k >> shift) & dmask), 1u);
+          for (int q = 0; q < 4; ++q) {
+            const uint32_t k = order_bits(e[q]);
+            if (s + q < s1 && (k & mask) == prefix) atomicAdd(lhist + ((k >> shift) & dmask), 1u);
           }
         }
-      });
+        __syncthreads();  // slot fully read
+        if (kVec && tid == 0 && j + kRingSlots < nch) ring_issue(ring, bar0, sc, s0, s1, g + kRingSlots, j + kRingSlots);
+      }
+      if (kVec) consumed += nch;
       cluster.sync();
       for (int b = tid; b < kBins; b += kThreads) {
         uint32_t acc = 0;
@@ -327,28 +328,25 @@ __global__ void __launch_bounds__(kThreads, 1) sga_topk_kernel(TopkParams p) {
   __syncthreads();
   uint32_t my_sel = 0, my_tie = 0;
   uint32_t wcount = 0;  // staged candidates of this warp (same value in every lane)
-  auto flush_stage = [&]() {
-    if (wcount == 0) return;
-    __syncwarp();  // staged entries written by other lanes are visible
-    uint32_t base = 0;
-    if (lane == 0) base = atomicAdd(&cand_n, wcount);
-    base = __shfl_sync(0xFFFFFFFFu, base, 0);
-    for (uint32_t i = lane; i < wcount; i += 32)
-      if (base + i < kCandCap) cand[base + i] = wstage[i];
-    __syncwarp();
-    wcount = 0;
-  };
-  stream([&](int pos, const float* d, int cnt) {
+  if (kVec && consumed > 0 && tid == 0)
+    for (int j = 0; j < min(kRingSlots, nch); ++j) ring_issue(ring, bar0, sc, s0, s1, consumed + j, j);
+  for (int j = 0; j < nch; ++j) {
+    const int g = consumed + j, slot = g % kRingSlots;
+    if (kVec && !mbar_wait(bar0 + 8u * slot, static_cast<uint32_t>((g / kRingSlots) & 1), &abort_flag))
+      record_status(p.status, kStatusTimeout);
+    const int pos = s0 + j * kChunk, cnt = min(kChunk, s1 - pos);
+    const float4* d4 = reinterpret_cast<const float4*>(ring + slot * kChunk);
     for (int f = tid; f < kChunk / 4; f += kThreads) {  // same trip count in every lane
       const int s = pos + 4 * f;
-      const float4 v = 4 * f < cnt ? load4s(d, f, s) : make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
+      float4 v = make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
+      if (4 * f < cnt) v = kVec ? d4[f] : load4<false>(sc, s, s1);
       const float e[4] = {v.x, v.y, v.z, v.w};
       uint32_t nib_above = 0, nib_bin = 0;
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const bool valid = s + j < s1;
-        nib_above |= static_cast<uint32_t>(valid && e[j] > f_hi) << j;
-        nib_bin |= static_cast<uint32_t>(valid && e[j] >= f_lo && e[j] <= f_hi) << j;
+      for (int q = 0; q < 4; ++q) {
+        const bool valid = s + q < s1;
+        nib_above |= static_cast<uint32_t>(valid && e[q] > f_hi) << q;
+        nib_bin |= static_cast<uint32_t>(valid && e[q] >= f_lo && e[q] <= f_hi) << q;
       }
       if (!__any_sync(0xFFFFFFFFu, (nib_above | nib_bin) != 0)) continue;
       my_sel += __popc(nib_above);
@@ -370,29 +368,37 @@ __global__ void __launch_bounds__(kThreads, 1) sga_topk_kernel(TopkParams p) {
           if (lane >= o) incl += y;
         }
         const uint32_t total = __shfl_sync(0xFFFFFFFFu, incl, 31);
-        if (wcount + total > kWarpStage) flush_stage();
-        uint64_t* dst = wstage + wcount;
-        uint32_t off = incl - c4;
+        if (wcount + total > kWarpStage) wcount = flush_stage(wcount, wstage, cand, &cand_n, lane);
         if (total > kWarpStage) {  // more than a buffer in one step: straight to the list
           uint32_t base = 0;
           if (lane == 31) base = atomicAdd(&cand_n, total);
-          base = __shfl_sync(0xFFFFFFFFu, base, 31);
-          dst = cand;
-          off += base;
-        }
+          base = __shfl_sync(0xFFFFFFFFu, base, 31) + incl - c4;
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          if ((nib_bin >> j) & 1u) {
-            if (dst != cand || off < kCandCap)
-              dst[off] = (static_cast<uint64_t>(order_bits(e[j])) << 32) | (0xFFFFFFFFu - static_cast<uint32_t>(s + j));
-            ++off;
+          for (int q = 0; q < 4; ++q) {
+            if ((nib_bin >> q) & 1u) {
+              if (base < kCandCap)
+                cand[base] = (static_cast<uint64_t>(order_bits(e[q])) << 32) | (0xFFFFFFFFu - static_cast<uint32_t>(s + q));
+              ++base;
+            }
           }
+        } else {
+          uint32_t off = wcount + incl - c4;
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            if ((nib_bin >> q) & 1u) {
+              wstage[off] = (static_cast<uint64_t>(order_bits(e[q])) << 32) | (0xFFFFFFFFu - static_cast<uint32_t>(s + q));
+              ++off;
+            }
+          }
+          wcount += total;
         }
-        if (total <= kWarpStage) wcount += total;
       }
     }
-  });
-  if (!resolved) flush_stage();
+    __syncthreads();  // slot fully read
+    if (kVec && tid == 0 && j + kRingSlots < nch) ring_issue(ring, bar0, sc, s0, s1, g + kRingSlots, j + kRingSlots);
+  }
+  if (kVec) consumed += nch;
+  if (!resolved) wcount = flush_stage(wcount, wstage, cand, &cand_n, lane);
   cluster.sync();  // segments scanned, candidate lists complete
 
   // ---- 3. every CTA: all candidates -> K*; mark own candidates; publish counts
