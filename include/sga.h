@@ -161,6 +161,32 @@ SGA_API sga_status_t sga_get_device_status(const void* ws, sga_stream_t stream, 
 /* Clears the workspace status word (asynchronously on `stream`). */
 SGA_API sga_status_t sga_clear_device_status(void* ws, sga_stream_t stream);
 
+/* Bytes of device memory inside the library that sga_topk_select_noalloc uses
+ * as its scratch (a status word plus the selection bitmaps). */
+#define SGA_NOALLOC_SCRATCH_BYTES (256 + 4 * 1024 * 1024)
+
+/* sga_topk_select without a caller workspace.  No counterpart on the pages:
+ * this entry point exists for callers that cannot allocate device memory,
+ * for example a custom operator inside another inference engine whose plugin
+ * interface hands over only its input and output buffers: it cannot lend a
+ * workspace and must not call cudaMalloc, which would synchronise the device
+ * and step outside the engine's memory budget.
+ *   The scratch is one static device array of SGA_NOALLOC_SCRATCH_BYTES that
+ * every GPU which loads the library keeps until the process exits.  The
+ * selection bitmaps need 2 * B * T * ceil(L / 32) * 4 bytes; larger sizes are
+ * rejected with SGA_ERR_WORKSPACE before anything is launched.  This call
+ * allocates nothing and calls no allocating routine.  The first call on each
+ * device looks up the array's device address (cudaGetSymbolAddress) with that
+ * device current; make that first call before any stream capture.  Every call
+ * shares the array, which keeps the last call's contents; each call clears
+ * what must start at zero (the status word; the kernel zeroes its bitmap
+ * words before use).  Calls that overlap on the GPU race on the array, so
+ * order them on one stream.  Device-side errors are not reported (the status
+ * word is private to the library); all other arguments, results and errors
+ * are as for sga_topk_select. */
+SGA_API sga_status_t sga_topk_select_noalloc(const sga_dims_t* dims, const float* scores, const int32_t* q_pos,
+                                             int32_t* idx, sga_stream_t stream);
+
 #ifdef __cplusplus
 } /* extern "C" */
 #endif

@@ -27,5 +27,6 @@ from ._binding import (  # noqa: F401
     make_dims,
     sparse_mla_attend,
     topk_select,
+    topk_select_noalloc,
     workspace_size,
 )

@@ -28,7 +28,9 @@ STATUS_NAMES = {0: "SGA_OK", 1: "SGA_ERR_INVALID_ARG", 2: "SGA_ERR_UNSUPPORTED",
                 4: "SGA_ERR_CUDA", 5: "SGA_ERR_TIMEOUT", 6: "SGA_ERR_DEVICE_ARG"}
 
 EXPORTED = ["sga_abi_version", "sga_status_string", "sga_workspace_size", "sga_index_scores", "sga_topk_select",
-            "sga_sparse_mla_attend", "sga_forward", "sga_get_device_status", "sga_clear_device_status"]
+            "sga_sparse_mla_attend", "sga_forward", "sga_get_device_status", "sga_clear_device_status",
+            "sga_topk_select_noalloc"]
+NOALLOC_SCRATCH_BYTES = 256 + 4 * 1024 * 1024
 
 
 class SGAError(RuntimeError):
@@ -65,6 +67,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "sga_forward": (ctypes.c_int, [D, P, P, P, P, P, P, P, P, P, P, sz, P]),
         "sga_get_device_status": (ctypes.c_int, [P, P, ctypes.POINTER(i32)]),
         "sga_clear_device_status": (ctypes.c_int, [P, P]),
+        "sga_topk_select_noalloc": (ctypes.c_int, [D, P, P, P, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -162,6 +165,20 @@ def topk_select(scores, q_pos, top_k: int = TOP_K, idx=None, ws=None, stream=Non
         ws = alloc_workspace(dims, OP_TOPK_SELECT, scores.device)
     _check("sga_topk_select", load_library().sga_topk_select(
         ctypes.byref(dims), _ptr(scores), _ptr(q_pos), _ptr(idx), _ptr(ws), ws.numel(), _stream(stream)))
+    return idx
+
+
+def topk_select_noalloc(scores, q_pos, top_k: int = TOP_K, idx=None, stream=None):
+    """Top-k without a workspace (the library's own static scratch; see sga.h)."""
+    B, T, L = scores.shape
+    _need(scores, "scores", torch.float32, (B, T, L))
+    _need(q_pos, "q_pos", torch.int32, (B, T))
+    dims = make_dims(B, T, L, top_k)
+    if idx is None:
+        idx = torch.empty((B, T, top_k), dtype=torch.int32, device=scores.device)
+    _need(idx, "idx", torch.int32, (B, T, top_k))
+    _check("sga_topk_select_noalloc", load_library().sga_topk_select_noalloc(
+        ctypes.byref(dims), _ptr(scores), _ptr(q_pos), _ptr(idx), _stream(stream)))
     return idx
 
 

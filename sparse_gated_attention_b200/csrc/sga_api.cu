@@ -249,3 +249,49 @@ sga_status_t sga_clear_device_status(void* ws, sga_stream_t stream) {
 }
 
 }  // extern "C"
+
+// ---- top-k without a caller workspace -------------------------------------------------
+// Scratch of sga_topk_select_noalloc: a status word then the selection bitmaps.  It
+// lives in the library for callers that cannot allocate device memory.  In host
+// code the symbol is only a host-side stand-in, so the device address is looked
+// up once per device (with that device current) and passed to the kernel.
+namespace {
+constexpr int kNoallocMaxDevices = 64;
+static __device__ __align__(256) unsigned char g_noalloc_scratch[SGA_NOALLOC_SCRATCH_BYTES];
+void* g_noalloc_ptr[kNoallocMaxDevices] = {};
+cudaError_t g_noalloc_err[kNoallocMaxDevices] = {};
+std::once_flag g_noalloc_once[kNoallocMaxDevices];
+}  // namespace
+
+extern "C" {
+
+sga_status_t sga_topk_select_noalloc(const sga_dims_t* dims, const float* scores, const int32_t* q_pos,
+                                     int32_t* idx, sga_stream_t stream) {
+  if (!dims_ok(dims)) return SGA_ERR_INVALID_ARG;
+  if (!aligned(scores, 4) || !aligned(q_pos, 4) || !aligned(idx, 16)) return SGA_ERR_INVALID_ARG;
+  const size_t rows = static_cast<size_t>(dims->batch) * dims->n_q;
+  const size_t bitmap_bytes = rows * 2 * topk_bitmap_words(dims->kv_stride) * 4;
+  if (kStatusBytes + bitmap_bytes > SGA_NOALLOC_SCRATCH_BYTES) return SGA_ERR_WORKSPACE;
+  int sms = 0;
+  sga_status_t st = device_info(&sms);
+  if (st != SGA_OK) return st;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kNoallocMaxDevices) {
+    cudaGetLastError();
+    return SGA_ERR_UNSUPPORTED;
+  }
+  std::call_once(g_noalloc_once[dev], [dev]() {
+    void* ptr = nullptr;
+    g_noalloc_err[dev] = cudaGetSymbolAddress(&ptr, g_noalloc_scratch);
+    if (g_noalloc_err[dev] == cudaSuccess) g_noalloc_ptr[dev] = ptr;
+  });
+  if (g_noalloc_err[dev] != cudaSuccess || !g_noalloc_ptr[dev]) return SGA_ERR_CUDA;
+  void* scratch = g_noalloc_ptr[dev];
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (cudaMemsetAsync(scratch, 0, kStatusBytes, s) != cudaSuccess) return SGA_ERR_CUDA;  // status word
+  TopkArgs a{scores,   q_pos, idx, at<uint32_t>(scratch, kStatusBytes), nullptr, at<int>(scratch, 0),
+             static_cast<int>(rows), dims->kv_stride, dims->top_k};
+  return from_cuda(launch_topk(a, s));
+}
+
+}  // extern "C"
