@@ -139,6 +139,9 @@ class ClockSampler:
                 "samples": len(sm)}
 
 
+_SAMPLE_CACHE = {}
+
+
 def cpu_baseline(wl, n_queries: int = 0, min_seconds: float = 10.0, max_queries: int = 400):
     """The oracle, as it stands, on a bounded sample of the workload (host cores).
 
@@ -147,9 +150,12 @@ def cpu_baseline(wl, n_queries: int = 0, min_seconds: float = 10.0, max_queries:
     import oracle
     from sparse_gated_attention_b200 import synth
 
-    sample = synth.custom(batch=1, n_q=1, ctx=wl.ctx, first_pos=wl.first_pos if wl.n_q == 1 else wl.ctx - 1,
-                          k_range=wl.k_range, name=wl.name + "_sample")
-    x = synth.make_inputs(sample, device="cpu", seed=0)
+    key = (wl.name, wl.ctx, wl.k_range)
+    if key not in _SAMPLE_CACHE:
+        sample = synth.custom(batch=1, n_q=1, ctx=wl.ctx, first_pos=wl.first_pos if wl.n_q == 1 else wl.ctx - 1,
+                              k_range=wl.k_range, name=wl.name + "_sample")
+        _SAMPLE_CACHE[key] = synth.make_inputs(sample, device="cpu", seed=0)
+    x = _SAMPLE_CACHE[key]
     oracle.build()
     threads = oracle.hardware_threads()
     t0 = time.perf_counter()
