@@ -8,28 +8,32 @@
 // "above" (all selected) and "ties" (key == K*, of which the lowest positions
 // fill the remaining slots); nothing else needs ordering.  One thread-block
 // cluster of C CTAs (1024 threads each) handles one query; CTA r owns a
-// contiguous segment of positions (a multiple of 128), which streams through a
-// 3-slot shared-memory ring of 32 KB bulk copies (TMA) so that every pass over
-// it reads shared memory while the next chunks are in flight.
-//   1. MSD radix select over the score key, 12/12/8 bits per level.  Each CTA
+// contiguous segment of positions (a multiple of 128).
+//
+// Resident kernel (segments of at most 32768 positions, i.e. rows up to
+// 8 x 32768): the whole segment is copied once into shared memory (four 32 KB
+// bulk copies) and every pass reads it there.  Warp w owns 1024 consecutive
+// positions of the segment and walks them 32 at a time, so a ballot over one
+// step is the 32-position word of that step in position order.
+//   1. MSD radix select over the score key, 12/12/8 bits per level: each CTA
 //      counts its segment into a shared-memory histogram and all CTAs sum the
 //      C histograms through distributed shared memory, so every CTA finds the
 //      same bin.  Levels stop when that bin fits a candidate list (4096 keys)
-//      or holds a single key.  Under sga_forward the indexer has already
-//      counted the first level, so that pass is skipped.
-//   2. One pass over the segment, four positions per thread: per 32
-//      positions a selection word (keys above the bin) and a tie word (keys
-//      in the bin, once the bin is a single key) are assembled from per-lane
-//      nibbles with three shuffles; keys in a wider bin go to the CTA's
-//      candidate list.
-//   3. Every CTA copies all candidate lists over distributed shared memory,
-//      narrows them to K* itself (no leader), marks its own candidates in its
-//      own words and publishes two counts (selected, ties).
-//   4. Every CTA emits its own segment: popcounts, two block scans and the
-//      other CTAs' counts give each set bit its output slot; ties are taken in
-//      position order until the K slots are full.
-// The selection and tie words of a segment stay in shared memory (segments up
-// to 65536 positions) or in the workspace (longer segments).
+//      or is a single key.  Under sga_forward the indexer has already counted
+//      the first level, so that pass is skipped.
+//   2. If the bin is wider than one key: one ballot pass collects the keys in
+//      the bin into the CTA's candidate list; every CTA copies all lists over
+//      distributed shared memory and narrows them to K* itself (no leader).
+//   3. One ballot pass builds, per 32 positions, a selection word (key > K*)
+//      and a tie word (key == K*); lane j keeps the words of step j.  Warp and
+//      block scans of their popcounts plus the other CTAs' two counts give
+//      each set bit its output slot; ties are taken in position order until
+//      the K slots are full.
+// Streaming kernel (longer rows): the segment streams through a 3-slot ring of
+// 32 KB bulk copies once per pass; the second step records selection / tie
+// words (shared memory up to 65536 positions, else the workspace) and stages
+// candidates per warp, own candidates are marked in the words after K* is
+// known, and the words are emitted as above.
 #include <cooperative_groups.h>
 
 #include "sga_internal.cuh"
@@ -55,6 +59,13 @@ constexpr size_t kRingBytes = kRingSlots * kChunk * 4;
 constexpr int kWarpStage = 64;         // per-warp staging of candidates before one shared atomic
 constexpr size_t kSmemBytes =
     kRingBytes + 2 * kBins * 4 + kCandCap * 8 + 2 * kSegWordsSmem * 4 + kWarps * kWarpStage * 8 + 4 * 8;
+// resident kernel
+constexpr int kResSeg = 32768;                  // positions per CTA held in shared memory (128 KB)
+constexpr int kResWarpSpan = kResSeg / kWarps;  // 1024 consecutive positions per warp
+constexpr int kResSteps = kResWarpSpan / 32;    // 32 ballot steps per warp and pass
+constexpr int kResChunks = kResSeg / kChunk;    // 4 bulk copies
+constexpr size_t kResSmemBytes = kResSeg * 4 + 2 * kBins * 4 + kCandCap * 8 + (kResChunks + 1) * 8;
+static_assert(kResSteps == 32, "lane j keeps the words of step j");
 
 struct TopkParams {
   const float* scores;
@@ -126,6 +137,70 @@ __device__ __forceinline__ Narrow find_bin(const uint32_t* hist, uint32_t need, 
   return *out;
 }
 
+// Narrows the first nc candidates (key << 32 | ~position), all in the bin
+// (prefix, mask, shift), to the exact K-th key with the radix levels of the
+// main selection.  Returns K* in the high 32 bits (kmask then covers all of
+// them); `need` becomes the number of ties at K* still to take.
+__device__ __noinline__ uint64_t refine_candidates(const uint64_t* cand, uint32_t nc, uint32_t* ghist, uint32_t prefix,
+                                                   uint32_t mask, int shift, uint32_t& need, uint32_t* warp_buf,
+                                                   Narrow* narrow, uint64_t& kmask) {
+  const int tid = threadIdx.x;
+  kmask = static_cast<uint64_t>(mask) << 32;
+  uint64_t kpref = static_cast<uint64_t>(prefix) << 32;
+  while (shift > 0) {
+    const int width = shift >= kBits ? kBits : shift;
+    shift -= width;
+    const uint32_t dmask = (1u << width) - 1u;
+    for (int b = tid; b < kBins; b += kThreads) ghist[b] = 0;
+    __syncthreads();
+    for (uint32_t i = tid; i < nc; i += kThreads) {
+      const uint64_t c = cand[i];
+      if ((c & kmask) == kpref) atomicAdd(ghist + (static_cast<uint32_t>(c >> (32 + shift)) & dmask), 1u);
+    }
+    __syncthreads();
+    const Narrow nr = find_bin(ghist, need, warp_buf, narrow);
+    kpref |= static_cast<uint64_t>(nr.digit) << (32 + shift);
+    kmask |= static_cast<uint64_t>(dmask) << (32 + shift);
+    need -= nr.above;
+  }
+  return kpref;
+}
+
+// Appends the other CTAs' candidate lists behind this CTA's `own` entries;
+// peer_n[r] is the length of CTA r's list.  Returns the total length.  The
+// caller's cluster barrier must have published every list and count, and no
+// CTA may change the first entries of its list until all have copied them.
+__device__ __forceinline__ uint32_t pull_candidates(cg::cluster_group& cluster, uint64_t* cand, uint32_t own,
+                                                    const uint32_t* peer_n) {
+  const int C = static_cast<int>(cluster.num_blocks());
+  const int rank = static_cast<int>(cluster.block_rank());
+  uint32_t nc = own;
+  for (int r = 0; r < C; ++r) {
+    if (r == rank) continue;
+    const uint32_t cnt = min(peer_n[r], static_cast<uint32_t>(kCandCap) - nc);
+    const uint64_t* src = cluster.map_shared_rank(cand, r);
+    for (uint32_t i = threadIdx.x; i < cnt; i += kThreads) cand[nc + i] = src[i];
+    nc += cnt;
+  }
+  return nc;
+}
+
+// Streaming kernel: every CTA reads the other CTAs' list lengths, copies their
+// lists behind its own `own` entries and narrows them to K* (see
+// refine_candidates).  Ends with the list complete in every CTA; the caller's
+// earlier cluster barrier must have published all lists.
+__device__ __noinline__ void narrow_candidates(cg::cluster_group& cluster, uint64_t* cand, uint32_t* cand_n, uint32_t own,
+                                               uint32_t* ghist, uint32_t prefix, uint32_t mask, int shift,
+                                               uint32_t& need, uint32_t* warp_buf, Narrow* narrow, uint64_t& kpref,
+                                               uint64_t& kmask) {
+  uint32_t peer_n[kMaxCluster];
+  const int C = static_cast<int>(cluster.num_blocks());
+  for (int r = 0; r < C; ++r) peer_n[r] = *cluster.map_shared_rank(cand_n, r);
+  const uint32_t nc = pull_candidates(cluster, cand, own, peer_n);
+  cluster.sync();  // remote lists read; each CTA extended its own list behind its own entries
+  kpref = refine_candidates(cand, nc, ghist, prefix, mask, shift, need, warp_buf, narrow, kmask);
+}
+
 // Four consecutive scores starting at s; positions >= end are read as 0 (the
 // caller masks them).  The vector form needs rows that start 16-byte aligned.
 template <bool kVec>
@@ -187,7 +262,7 @@ __device__ __forceinline__ uint32_t flush_stage(uint32_t wcount, const uint64_t*
 }
 
 template <bool kVec>
-__global__ void __launch_bounds__(kThreads, 1) sga_topk_kernel(TopkParams p) {
+__global__ void __launch_bounds__(kThreads, 1) sga_topk_stream_kernel(TopkParams p) {
   extern __shared__ __align__(128) uint8_t smem_raw[];
   float* ring = reinterpret_cast<float*>(smem_raw);
   uint32_t* lhist = reinterpret_cast<uint32_t*>(smem_raw + kRingBytes);
@@ -404,40 +479,8 @@ __global__ void __launch_bounds__(kThreads, 1) sga_topk_kernel(TopkParams p) {
   // ---- 3. every CTA: all candidates -> K*; mark own candidates; publish counts
   if (!resolved) {
     const uint32_t own = min(cand_n, static_cast<uint32_t>(kCandCap));
-    uint32_t offs[kMaxCluster + 1];
-    int src_rank[kMaxCluster];
-    offs[0] = own;
-    int m = 0;
-    for (int r = 0; r < C; ++r) {
-      if (r == rank) continue;
-      src_rank[m] = r;
-      offs[m + 1] = offs[m] + *cluster.map_shared_rank(&cand_n, r);
-      ++m;
-    }
-    const uint32_t nc = min(offs[m], static_cast<uint32_t>(kCandCap));
-    for (uint32_t g = own + tid; g < nc; g += kThreads) {
-      int q = 0;
-      while (q < m - 1 && g >= offs[q + 1]) ++q;
-      cand[g] = cluster.map_shared_rank(cand, src_rank[q])[g - offs[q]];
-    }
-    cluster.sync();  // remote lists read; each CTA extended its own list behind its own entries
-    uint64_t kmask = static_cast<uint64_t>(mask) << 32, kpref = static_cast<uint64_t>(prefix) << 32;
-    while (shift > 0) {
-      const int width = shift >= kBits ? kBits : shift;
-      shift -= width;
-      const uint32_t dmask = (1u << width) - 1u;
-      for (int b = tid; b < kBins; b += kThreads) ghist[b] = 0;
-      __syncthreads();
-      for (uint32_t i = tid; i < nc; i += kThreads) {
-        const uint64_t c = cand[i];
-        if ((c & kmask) == kpref) atomicAdd(ghist + (static_cast<uint32_t>(c >> (32 + shift)) & dmask), 1u);
-      }
-      __syncthreads();
-      const Narrow nr = find_bin(ghist, need, warp_buf, &narrow);
-      kpref |= static_cast<uint64_t>(nr.digit) << (32 + shift);
-      kmask |= static_cast<uint64_t>(dmask) << (32 + shift);
-      need -= nr.above;
-    }
+    uint64_t kpref, kmask;
+    narrow_candidates(cluster, cand, &cand_n, own, ghist, prefix, mask, shift, need, warp_buf, &narrow, kpref, kmask);
     // own candidates (the first `own` entries) -> selection or tie bits in own words
     for (uint32_t i = tid; i < own; i += kThreads) {
       const uint64_t c = cand[i];
@@ -525,6 +568,260 @@ __global__ void __launch_bounds__(kThreads, 1) sga_topk_kernel(TopkParams p) {
   }
 }
 
+// Waits (once per warp) for the bulk copy that holds this warp's positions.
+__device__ __forceinline__ void wait_own_chunk(bool& have, int wbase, int len, uint32_t bar0, volatile int* abort_flag,
+                                               int* status) {
+  if (have) return;
+  have = true;
+  if (wbase < len && !mbar_wait(bar0 + 8u * static_cast<uint32_t>(wbase / kChunk), 0, abort_flag))
+    record_status(status, kStatusTimeout);
+}
+
+template <bool kVec>
+__global__ void __launch_bounds__(kThreads, 1) sga_topk_resident_kernel(TopkParams p) {
+  extern __shared__ __align__(128) uint8_t smem_raw[];
+  float* seg = reinterpret_cast<float*>(smem_raw);
+  uint32_t* lhist = reinterpret_cast<uint32_t*>(smem_raw + kResSeg * 4);
+  uint32_t* ghist = lhist + kBins;
+  uint64_t* cand = reinterpret_cast<uint64_t*>(ghist + kBins);
+  uint64_t* bars = cand + kCandCap;  // chunk[kResChunks], hist
+  __shared__ uint32_t warp_buf[kWarps];
+  __shared__ uint32_t wsel[kWarps], wtie[kWarps];  // per-warp exclusive prefixes of the word popcounts
+  __shared__ Narrow narrow;
+  __shared__ uint32_t cand_n;
+  __shared__ uint32_t peer_n[kMaxCluster];          // candidate-list lengths, written by each CTA of the cluster
+  __shared__ uint32_t peer_counts[kMaxCluster][2];  // (selected, ties) of each CTA's segment, written by that CTA
+  __shared__ int abort_flag;
+
+  cg::cluster_group cluster = cg::this_cluster();
+  const int C = static_cast<int>(cluster.num_blocks());
+  const int rank = static_cast<int>(cluster.block_rank());
+  const int row = blockIdx.x / C;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int K = p.top_k;
+  int32_t* out = p.idx + static_cast<size_t>(row) * K;
+  const int t = __ldg(p.q_pos + row);
+  if (t < 0 || t >= p.kv_stride) {
+    if (rank == 0) {
+      if (tid == 0) record_status(p.status, kStatusDeviceArg);
+      for (int j = tid; j < K; j += kThreads) out[j] = -1;
+    }
+    return;
+  }
+  const int n = t + 1;
+  if (n <= K) {
+    if (rank == 0)
+      for (int j = tid; j < K; j += kThreads) out[j] = j < n ? j : -1;
+    return;
+  }
+  // The host picks C with C * kResSeg >= kv_stride, so every segment fits.
+  const float* sc = p.scores + static_cast<size_t>(row) * p.kv_stride;
+  const int per = (((n + C - 1) / C) + 127) & ~127;
+  const int s0 = min(rank * per, n), s1 = min(s0 + per, n);
+  const int len = s1 - s0;
+  const int nch = (len + kChunk - 1) / kChunk;
+  const uint32_t bar0 = smem_u32(bars);
+  const uint32_t hist_bar = bar0 + 8u * kResChunks;
+  if (tid == 0) {
+    cand_n = 0;
+    abort_flag = 0;
+    for (int i = 0; i <= kResChunks; ++i) mbar_init(bar0 + 8u * i, 1);
+    fence_barrier_init();
+  }
+  __syncthreads();
+  if (kVec) {
+    if (tid == 0) {
+      if (p.hist) {
+        mbar_arrive_expect_tx(hist_bar, kBins * 4);
+        bulk_load(smem_u32(ghist), p.hist + static_cast<size_t>(row) * kBins, kBins * 4, hist_bar);
+      }
+      for (int c = 0; c < nch; ++c) {
+        const int cnt = min(kChunk, len - c * kChunk);
+        // rows are 16-byte aligned and kv_stride % 4 == 0, so rounding up stays inside the row
+        const uint32_t bytes = static_cast<uint32_t>((cnt + 3) & ~3) * 4u;
+        mbar_arrive_expect_tx(bar0 + 8u * c, bytes);
+        bulk_load(smem_u32(seg + c * kChunk), sc + s0 + c * kChunk, bytes, bar0 + 8u * c);
+      }
+    }
+  } else {
+    for (int i = tid; i < len; i += kThreads) seg[i] = __ldg(sc + s0 + i);
+    if (p.hist) {
+      const uint32_t* hrow = p.hist + static_cast<size_t>(row) * kBins;
+      for (int b = tid; b < kBins; b += kThreads) ghist[b] = __ldg(hrow + b);
+    }
+    __syncthreads();
+  }
+  const int wbase = warp * kResWarpSpan;  // this warp's first position within the segment
+  bool have_seg = !kVec;
+
+  // ---- 1. radix levels on the score key until the bin fits the candidate list or is one key
+  uint32_t prefix = 0, mask = 0;
+  uint32_t need = static_cast<uint32_t>(K);
+  int shift = 32;
+  uint32_t bucket = 0;
+  bool first = true;
+  while (true) {
+    const int width = shift >= kBits ? kBits : shift;
+    shift -= width;
+    const uint32_t dmask = (1u << width) - 1u;
+    if (first && p.hist) {
+      if (kVec && !mbar_wait(hist_bar, 0, &abort_flag)) record_status(p.status, kStatusTimeout);
+      __syncthreads();
+    } else {
+      for (int b = tid; b < kBins; b += kThreads) lhist[b] = 0;
+      wait_own_chunk(have_seg, wbase, len, bar0, &abort_flag, p.status);
+      __syncthreads();
+#pragma unroll 4
+      for (int j = 0; j < kResSteps; ++j) {
+        const int i = wbase + 32 * j + lane;
+        if (i < len) {
+          const uint32_t k = order_bits(seg[i]);
+          if ((k & mask) == prefix) atomicAdd(lhist + ((k >> shift) & dmask), 1u);
+        }
+      }
+      cluster.sync();
+      for (int b = tid; b < kBins; b += kThreads) {
+        uint32_t acc = 0;
+        for (int r = 0; r < C; ++r) acc += cluster.map_shared_rank(lhist, r)[b];
+        ghist[b] = acc;
+      }
+      cluster.sync();  // every CTA has read every histogram
+    }
+    first = false;
+    const Narrow nr = find_bin(ghist, need, warp_buf, &narrow);
+    prefix |= nr.digit << shift;
+    mask |= dmask << shift;
+    need -= nr.above;
+    bucket = nr.count;
+    if (bucket <= kCandCap || shift == 0) break;
+  }
+  const bool resolved = shift == 0;  // the bin is a single key: its positions are the ties
+
+  // ---- 2. one pass: per 32 positions a word of keys above the bin and a word
+  // of keys in it (lane j keeps the words of step j).  As floats, "above" is
+  // f > f_hi and "in the bin" f_lo <= f <= f_hi.
+  wait_own_chunk(have_seg, wbase, len, bar0, &abort_flag, p.status);
+  const float f_lo = key_to_float_lo(prefix), f_hi = key_to_float_hi(prefix | ~mask);
+  uint32_t my_sel = 0, my_bin = 0;
+#pragma unroll 8
+  for (int j = 0; j < kResSteps; ++j) {
+    const int i = wbase + 32 * j + lane;
+    const float f = i < len ? seg[i] : f_lo;
+    const uint32_t sw = __ballot_sync(0xFFFFFFFFu, i < len && f > f_hi);
+    const uint32_t bw = __ballot_sync(0xFFFFFFFFu, i < len && f >= f_lo && f <= f_hi);
+    if (lane == j) {
+      my_sel = sw;
+      my_bin = bw;
+    }
+  }
+  const int lpos = wbase + 32 * lane;  // segment offset of bit 0 of this lane's words
+  uint32_t kstar = prefix;
+  uint32_t my_tie = my_bin;
+  if (!resolved) {
+    // in-bin keys -> this CTA's candidate list (one shared atomic per warp)
+    const uint32_t c = __popc(my_bin);
+    uint32_t incl = c;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t y = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    uint32_t base = 0;
+    if (lane == 31 && incl) base = atomicAdd(&cand_n, incl);
+    base = __shfl_sync(0xFFFFFFFFu, base, 31) + incl - c;
+    for (uint32_t m = my_bin; m; m &= m - 1, ++base) {
+      const int i = lpos + __ffs(m) - 1;
+      if (base < kCandCap)
+        cand[base] = (static_cast<uint64_t>(order_bits(seg[i])) << 32) | (0xFFFFFFFFu - static_cast<uint32_t>(s0 + i));
+    }
+    __syncthreads();  // this CTA's list is complete
+    if (tid < C) *cluster.map_shared_rank(&peer_n[rank], tid) = min(cand_n, static_cast<uint32_t>(kCandCap));
+    cluster.sync();  // every list and every length published
+    const uint32_t nc = pull_candidates(cluster, cand, peer_n[rank], peer_n);
+    __syncthreads();  // the whole cluster's candidates are in this CTA's list
+    uint64_t kmask;
+    kstar = static_cast<uint32_t>(refine_candidates(cand, nc, ghist, prefix, mask, shift, need, warp_buf, &narrow,
+                                                    kmask) >> 32);
+    // in-bin positions: above K* -> selected, at K* -> ties, below -> dropped
+    my_tie = 0;
+    for (uint32_t m = my_bin; m; m &= m - 1) {
+      const int b = __ffs(m) - 1;
+      const uint32_t k = order_bits(seg[lpos + b]);
+      if (k > kstar) my_sel |= 1u << b;
+      if (k == kstar) my_tie |= 1u << b;
+    }
+  }
+
+  // ---- 3. counts, their scans across warps and CTAs, emission in position order
+  const uint32_t cs = __popc(my_sel), ct = __popc(my_tie);
+  uint32_t is = cs, it = ct;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t ys = __shfl_up_sync(0xFFFFFFFFu, is, o);
+    const uint32_t yt = __shfl_up_sync(0xFFFFFFFFu, it, o);
+    if (lane >= o) {
+      is += ys;
+      it += yt;
+    }
+  }
+  if (lane == 31) {
+    wsel[warp] = is;
+    wtie[warp] = it;
+  }
+  __syncthreads();
+  if (warp == 0) {
+    const uint32_t xs = wsel[lane], xt = wtie[lane];
+    uint32_t ps = xs, pt = xt;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t ys = __shfl_up_sync(0xFFFFFFFFu, ps, o);
+      const uint32_t yt = __shfl_up_sync(0xFFFFFFFFu, pt, o);
+      if (lane >= o) {
+        ps += ys;
+        pt += yt;
+      }
+    }
+    wsel[lane] = ps - xs;
+    wtie[lane] = pt - xt;
+    const uint32_t tot_s = __shfl_sync(0xFFFFFFFFu, ps, 31), tot_t = __shfl_sync(0xFFFFFFFFu, pt, 31);
+    if (lane < C) {
+      uint32_t* dst = cluster.map_shared_rank(&peer_counts[rank][0], lane);
+      dst[0] = tot_s;
+      dst[1] = tot_t;
+    }
+  }
+  // Every count delivered.  No CTA touches another's shared memory after this
+  // barrier, so none has to wait for the others before exiting.
+  cluster.sync();
+  uint32_t sel_before = 0, tie_before = 0, sel_all = 0, tie_all = 0;
+  for (int r = 0; r < C; ++r) {
+    const uint32_t a = peer_counts[r][0], b = peer_counts[r][1];
+    if (r < rank) {
+      sel_before += a;
+      tie_before += b;
+    }
+    sel_all += a;
+    tie_all += b;
+  }
+  if (rank == 0 && tid == 0 && (sel_all + need != static_cast<uint32_t>(K) || tie_all < need))
+    record_status(p.status, kStatusDeviceArg);
+  const uint32_t sel_base = sel_before + wsel[warp] + (is - cs);
+  const uint32_t tie_base = tie_before + wtie[warp] + (it - ct);
+  const int pos0 = s0 + lpos;
+  for (uint32_t m = my_sel | my_tie; m; m &= m - 1) {
+    const int b = __ffs(m) - 1;
+    const uint32_t below = (1u << b) - 1u;
+    const uint32_t tr = tie_base + __popc(my_tie & below);
+    if (((my_tie >> b) & 1u) && tr >= need) continue;
+    const uint32_t slot = sel_base + __popc(my_sel & below) + min(tr, need);
+    if (slot < static_cast<uint32_t>(K)) out[slot] = pos0 + b;
+  }
+  if (rank == 0) {
+    const uint32_t emitted = sel_all + min(tie_all, need);
+    for (int j = static_cast<int>(emitted) + tid; j < K; j += kThreads) out[j] = -1;
+  }
+}
+
 }  // namespace
 
 // Words of one bitmap per row; the workspace holds two per row (selected, ties).
@@ -540,9 +837,13 @@ int topk_cluster_size(int rows) {
 cudaError_t launch_topk(const TopkArgs& a, cudaStream_t stream) {
   if (a.rows == 0) return cudaSuccess;
   const bool vec = (a.kv_stride % 4 == 0) && (reinterpret_cast<uintptr_t>(a.scores) % 16 == 0);
-  auto kernel = vec ? sga_topk_kernel<true> : sga_topk_kernel<false>;
-  cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(kSmemBytes));
+  // rows that fit kMaxCluster segments of kResSeg positions take the resident kernel
+  const int c_res = (a.kv_stride + kResSeg - 1) / kResSeg;
+  const bool resident = c_res <= kMaxCluster;
+  auto kernel = resident ? (vec ? sga_topk_resident_kernel<true> : sga_topk_resident_kernel<false>)
+                         : (vec ? sga_topk_stream_kernel<true> : sga_topk_stream_kernel<false>);
+  const size_t smem = resident ? kResSmemBytes : kSmemBytes;
+  cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   TopkParams p;
   p.scores = a.scores;
@@ -554,11 +855,12 @@ cudaError_t launch_topk(const TopkArgs& a, cudaStream_t stream) {
   p.kv_stride = a.kv_stride;
   p.top_k = a.top_k;
   p.words_per_row = static_cast<long long>(topk_bitmap_words(a.kv_stride));
-  const int C = topk_cluster_size(a.rows);
+  int C = topk_cluster_size(a.rows);
+  if (resident) C = max(C, c_res);
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(a.rows * C));
   cfg.blockDim = dim3(kThreads);
-  cfg.dynamicSmemBytes = kSmemBytes;
+  cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;

@@ -147,6 +147,27 @@ def test_topk_sizes(L, K, t):
     np.testing.assert_array_equal(got, want)
 
 
+# Rows of up to 8 x 32768 positions are selected with each CTA's segment held
+# in shared memory; longer rows stream.  A row stride that is not a multiple
+# of 4 takes plain loads instead of bulk copies.  Many rows with a long stride
+# give clusters of 3 and 5 CTAs.
+@pytest.mark.parametrize("rows,L,kind", [(2, 100001, "int"), (2, 100001, "ties"), (100, 70000, "int"),
+                                         (40, 131075, "ties"), (2, 300000, "int"), (2, 300000, "ties"),
+                                         (3, 300003, "int"), (1, 262145, "float")])
+def test_topk_kernel_paths(rows, L, kind):
+    rng = np.random.default_rng(rows * 7 + L)
+    if kind == "int":
+        sc = rng.integers(0, 4000, size=(rows, L)).astype(np.float64)
+    elif kind == "ties":
+        sc = rng.integers(0, 9, size=(rows, L)).astype(np.float64)
+    else:
+        sc = rng.normal(size=(rows, L)).astype(np.float32).astype(np.float64)
+    pos = rng.integers(2048, L, size=rows)
+    pos[0] = L - 1
+    got, want = run_topk(sc, pos, 2048)
+    np.testing.assert_array_equal(got, want)
+
+
 # ----------------------------------------------------------------------------- steps 3-4: attention + gate
 
 
