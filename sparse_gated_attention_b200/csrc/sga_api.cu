@@ -19,8 +19,7 @@ constexpr size_t kStatusBytes = 256;
 size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 
 struct Layout {
-  size_t bitmap = 0, part_o = 0, part_ml = 0, scores = 0, idx = 0, hist = 0, total = 0;
-  int splits = 1;
+  size_t bitmap = 0, scores = 0, idx = 0, hist = 0, total = 0;
 };
 
 bool dims_ok(const sga_dims_t* d) {
@@ -41,15 +40,8 @@ Layout make_layout(const sga_dims_t& d, sga_op_t op) {
     l.bitmap = off;
     off += align_up(rows * 2 * topk_bitmap_words(d.kv_stride) * 4);  // selection + tie bitmaps
   }
-  if (op == SGA_OP_SPARSE_MLA_ATTEND || op == SGA_OP_FORWARD) {
-    l.splits = attend_splits(static_cast<int>(rows), d.top_k);
-    if (l.splits > 1) {
-      l.part_o = off;
-      off += align_up(rows * l.splits * SGA_HEADS * SGA_V_DIM * 4);
-      l.part_ml = off;
-      off += align_up(rows * l.splits * SGA_HEADS * 2 * 4);
-    }
-  }
+  // The attention needs no workspace beyond the status word: the splits of a
+  // query merge their partial results on chip.
   if (op == SGA_OP_FORWARD) {
     l.scores = off;
     off += align_up(rows * static_cast<size_t>(d.kv_stride) * 4);
@@ -190,9 +182,7 @@ sga_status_t sga_sparse_mla_attend(const sga_dims_t* dims, const sga_bf16_t* q, 
   if (st != SGA_OK) return st;
   int sms = 0;
   if ((st = device_info(&sms)) != SGA_OK) return st;
-  AttendArgs a{q, kv, idx, gate, out, l.splits > 1 ? at<float>(ws, l.part_o) : nullptr,
-               l.splits > 1 ? at<float>(ws, l.part_ml) : nullptr, at<int>(ws, 0), dims->batch, dims->n_q,
-               dims->kv_stride, dims->top_k};
+  AttendArgs a{q, kv, idx, gate, out, at<int>(ws, 0), dims->batch, dims->n_q, dims->kv_stride, dims->top_k};
   return from_cuda(launch_attend(a, static_cast<cudaStream_t>(stream)));
 }
 
@@ -224,9 +214,7 @@ sga_status_t sga_forward(const sga_dims_t* dims, const sga_bf16_t* q_idx, const 
   TopkArgs ta{scores, q_pos, idx, at<uint32_t>(ws, l.bitmap), hist, status, rows, dims->kv_stride, dims->top_k};
   e = launch_topk(ta, s);
   if (e != cudaSuccess) return SGA_ERR_CUDA;
-  AttendArgs aa{q, kv, idx, gate, out, l.splits > 1 ? at<float>(ws, l.part_o) : nullptr,
-                l.splits > 1 ? at<float>(ws, l.part_ml) : nullptr, status, dims->batch, dims->n_q,
-                dims->kv_stride, dims->top_k};
+  AttendArgs aa{q, kv, idx, gate, out, status, dims->batch, dims->n_q, dims->kv_stride, dims->top_k};
   return from_cuda(launch_attend(aa, s));
 }
 

@@ -24,21 +24,35 @@
 //     slot that is freed right after QK^T.  QK^T(j+1) is issued before PV(j),
 //     so the softmax of chunk j overlaps the next QK^T and chunk j+2 streams in
 //     while chunk j's values wait for P.
-//   * Warps 0-3 gather with 16-byte cp.async written straight into the
-//     128-byte-swizzled layout (empty slots zero-filled without a read);
-//     warp 0 also publishes the validity mask of each chunk and loads Q.
-//     Warp 4 issues the MMAs.  Warps 5-8 (one per TMEM lane quarter, 16 heads
-//     each) run the softmax in the log2 domain with a lazy running max (O is
-//     rescaled only when the max grows by more than 2^8) and the epilogue.
+//   * Warps 0-3 gather with TMA tile::gather4 (four cache rows x one 64-dim
+//     box per instruction, written by the TMA straight into the
+//     128-byte-swizzled layout); each warp gathers 16 rows of every chunk,
+//     so four warps keep the TMA unit busy.  An empty slot gathers the
+//     sequence's row 0 and is masked out of the softmax.  Warp 0 also
+//     publishes the validity mask of each chunk and loads Q.
+//     Warp 4 issues the MMAs without blocking on any one operand: it polls
+//     the barriers and issues PV(j) as soon as P_j is written, between the
+//     value pairs of QK^T(j+1), so value slots are released (and refilled)
+//     as early as the softmax allows.  Warps 5-8 (one per TMEM lane quarter,
+//     16 heads each) run the softmax in the log2 domain with a lazy running
+//     max (O is rescaled only when the max grows by more than 2^8) and the
+//     epilogue.
 //   * TMEM (512 columns): O^T in columns 0..255 (dim block b at 64 b, all
 //     lanes), S buffers at columns 256 and 320 (M = 64 layout: lanes 0-15 of
 //     each quarter).
-//   * With several splits per query the CTA writes (O, m, l) partials and a
-//     small combine kernel merges them and applies the gate.
+//   * The splits of one query form a thread-block cluster.  Each CTA keeps its
+//     (m, l) per head in shared memory; after a cluster barrier every CTA
+//     reads all of them, scales its own O by 2^(m_r - M) g / L and stages it
+//     in its (now idle) value ring; after a second barrier CTA r sums the
+//     split outputs of dims [512 r / S, 512 (r+1) / S) over distributed shared
+//     memory and writes them.  No partials leave the chip.
+#include <cooperative_groups.h>
 #include <math.h>
 
 #include "sga_internal.cuh"
 #include "sga_ptx.cuh"
+
+namespace cg = cooperative_groups;
 
 namespace sga {
 namespace {
@@ -55,7 +69,7 @@ constexpr int kQBox = kHeads * 128;         // 64 heads x 64 dims
 constexpr int kQBytes = 9 * kQBox;
 constexpr int kPBytes = kHeads * kChunk * 2;  // 64 heads x 64 rows bf16
 constexpr int kMaskRing = 4;
-constexpr int kProducers = 128;             // warps 0-3
+constexpr int kProducerWarps = 4;          // warps 0-3
 constexpr int kMmaWarp = 4;
 constexpr int kSoftmaxThreads = 128;        // warps 5-8
 constexpr int kThreads = 288;
@@ -64,19 +78,19 @@ constexpr int kSCol = 256;
 // barriers: pair_full[8] pair_empty[8] rope_full rope_empty q_full s_full[2] s_free[2]
 //           p_full p_free o_full mask_full[4] mask_empty[4]
 constexpr int kNumBars = 2 * kPairRing + 2 + 1 + 2 + 2 + 3 + 2 * kMaskRing;
+constexpr int kMaxSplits = 8;               // splits of a query = CTAs of its cluster
 constexpr size_t kSmemBytes = 1024 + kPairRing * kPairBytes + kBoxBytes + kQBytes + 2 * kPBytes + kNumBars * 8 +
-                              kMaskRing * 8 + kHeads * 4 + 16;
+                              kMaskRing * 8 + kHeads * 4 + kHeads * 8 + 16;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 
 static_assert(kSmemBytes <= 232448, "shared memory budget");
+static_assert(kPairRing * kPairBytes == kHeads * kDv * 4, "the value ring stages one CTA's O for the split merge");
 
 struct AttendParams {
   const uint16_t* kv;
   const int32_t* idx;
   const uint16_t* gate;
   float* out;
-  float* part_o;
-  float* part_ml;
   int* status;
   int n_q, kv_stride, top_k, splits, chunks_per_split;
   float scale_log2;
@@ -84,13 +98,22 @@ struct AttendParams {
 
 __device__ __forceinline__ float sigmoidf_(float g) { return 1.0f / (1.0f + expf(-g)); }
 
+// 2^x with the hardware approximation (relative error ~2^-22; results below
+// 2^-126 flush to zero, which only drops weights far below the fp32 sum).
+__device__ __forceinline__ float fast_exp2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
   const __nv_bfloat162 v = __floats2bfloat162_rn(a, b);
   return *reinterpret_cast<const uint32_t*>(&v);
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
-    sga_attend_kernel(const __grid_constant__ CUtensorMap qmap, AttendParams p) {
+    sga_attend_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap kvmap,
+                      AttendParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t pairs = smem_u32(smem);
@@ -115,22 +138,24 @@ __global__ void __launch_bounds__(kThreads, 1)
   auto mask_empty = [&](int b) { return q_full + 8u * (8 + kMaskRing + b); };
   uint64_t* masks = bars + kNumBars;
   float* head_f = reinterpret_cast<float*>(masks + kMaskRing);  // [64] per-head factors
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(head_f + kHeads);
+  float2* own_ml = reinterpret_cast<float2*>(head_f + kHeads);   // [64] (m, l) of this split, read by the cluster
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(own_ml + kHeads);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  cg::cluster_group cluster = cg::this_cluster();
   const int row = blockIdx.x / p.splits;
-  const int split = blockIdx.x % p.splits;
+  const int split = static_cast<int>(cluster.block_rank());  // the cluster is the query's p.splits CTAs
   const int nchunks = p.chunks_per_split;
   const int slot_base = split * nchunks * kChunk;  // first selected slot of this split
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kPairRing; ++s) {
-      mbar_init(pair_full(s), kProducers);  // one cp.async arrival per producer thread
+      mbar_init(pair_full(s), kProducerWarps);  // one expect_tx arrival per producer warp
       mbar_init(pair_empty(s), 1);
     }
-    mbar_init(rope_full, kProducers);
+    mbar_init(rope_full, kProducerWarps);
     mbar_init(rope_empty, 1);
     mbar_init(q_full, 1);
     for (int b = 0; b < 2; ++b) {
@@ -147,7 +172,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     *abort_flag = 0;
     fence_barrier_init();
   }
-  if (warp == 0 && lane == 0) prefetch_tmap(&qmap);
+  if (warp == 0 && lane == 0) {
+    prefetch_tmap(&qmap);
+    prefetch_tmap(&kvmap);
+  }
   if (warp == kMmaWarp) {
     tmem_alloc(smem_u32(tmem_slot), kTmemCols);
     tmem_relinquish();
@@ -157,14 +185,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp < kProducers / 32) {
+  if (warp < kProducerWarps) {
     // ------------------------------------------------------------ gather producers
     const int b = row / p.n_q;
     const int32_t* idx_row = p.idx + static_cast<size_t>(row) * p.top_k;
-    const uint16_t* kv_b = p.kv + static_cast<size_t>(b) * p.kv_stride * kDq;
+    const int row0 = b * p.kv_stride;  // this sequence's first row in the [B * L] cache map
     const int ptid = threadIdx.x;
-    const int part = ptid & 7;   // 16-byte chunk of a 128-byte row strip
-    const int rsub = ptid >> 3;  // rows rsub + 16 i, i = 0..3
+    const int g = lane & 3;             // this lane's group of 4 rows within the warp's 16
+    const int grow = 16 * warp + 4 * g;  // first chunk row of that group
     bool ok = true;
     if (ptid == 0) {
       mbar_arrive_expect_tx(q_full, kQBytes);
@@ -199,30 +227,25 @@ __global__ void __launch_bounds__(kThreads, 1)
         ok = __shfl_sync(0xFFFFFFFFu, ok ? 1 : 0, 0) != 0;
         if (!ok) break;
       }
-      // this thread's four rows of the chunk
-      const uint16_t* src[4];
-      uint32_t nbytes[4];
+      // cache rows of this lane's group (empty or invalid slots -> row 0, masked above)
+      int y[4];
+      {
+        const int sidx = first + grow;  // a multiple of 4: one 16-byte load
+        int4 v = make_int4(-1, -1, -1, -1);
+        if (sidx < p.top_k) v = __ldg(reinterpret_cast<const int4*>(idx_row + sidx));
+        const int e[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const int sidx = first + rsub + 16 * i;
-        int s = -1;
-        if (sidx < p.top_k) s = __ldg(idx_row + sidx);
-        const bool valid = s >= 0 && s < p.kv_stride;
-        src[i] = kv_b + static_cast<size_t>(valid ? s : 0) * kDq + part * 8;
-        nbytes[i] = valid ? 16u : 0u;
+        for (int i = 0; i < 4; ++i) y[i] = row0 + ((e[i] >= 0 && e[i] < p.kv_stride) ? e[i] : 0);
       }
-      // rope dims 512..575 -> the rope slot
+      // rope dims 512..575 -> the rope slot (lanes 0-3: one group each)
       if (!mbar_wait(rope_empty, static_cast<uint32_t>(j & 1) ^ 1u, abort_flag)) {
         ok = false;
         break;
       }
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const int r = rsub + 16 * i;
-        cp_async_16(rope + r * 128 + ((part ^ (r & 7)) << 4), src[i] + kDv, nbytes[i]);
-      }
-      cp_async_arrive_noinc(rope_full);
-      // value dims 128 q .. 128 q + 127 -> pair slot (4 j + q) mod 8
+      if (lane == 0) mbar_arrive_expect_tx(rope_full, 16 * 128);
+      __syncwarp();
+      if (lane < 4) tma_gather4(rope + grow * 128, &kvmap, rope_full, kDv, y[0], y[1], y[2], y[3]);
+      // value dims 128 q .. 128 q + 127 -> pair slot (4 j + q) mod 8 (lanes 0-7: group x box)
       for (int q = 0; q < kPairsPerChunk; ++q) {
         const int n = j * kPairsPerChunk + q;
         const int slot = n % kPairRing;
@@ -231,17 +254,17 @@ __global__ void __launch_bounds__(kThreads, 1)
           break;
         }
         const uint32_t base = pairs + slot * kPairBytes;
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const int r = rsub + 16 * i;
-          const uint32_t dst = base + r * 128 + ((part ^ (r & 7)) << 4);
-          cp_async_16(dst, src[i] + 128 * q, nbytes[i]);
-          cp_async_16(dst + kBoxBytes, src[i] + 128 * q + 64, nbytes[i]);
+        if (lane == 0) mbar_arrive_expect_tx(pair_full(slot), 16 * 2 * 128);
+        __syncwarp();
+        if (lane < 8) {
+          const int bx = lane >> 2;
+          tma_gather4(base + bx * kBoxBytes + grow * 128, &kvmap, pair_full(slot), 128 * q + 64 * bx, y[0], y[1], y[2],
+                      y[3]);
         }
-        cp_async_arrive_noinc(pair_full(slot));
       }
     }
-    asm volatile("cp.async.wait_all;" ::: "memory");
+    // On a timeout the waits above have run for about a second, long after any
+    // gather issued before them has landed.
     if (!ok) {
       record_status(p.status, kStatusTimeout);
       *abort_flag = 1;
@@ -256,46 +279,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       constexpr uint32_t idesc_qk = idesc_bf16_f32(kHeads, kChunk, false, false);
       constexpr uint32_t idesc_pv = idesc_bf16_f32(128, kHeads, true, false);
       bool ok = mbar_wait(q_full, 0, abort_flag);
-      auto wait_full = [&](uint32_t bar, uint32_t parity) -> bool {
-        if (!mbar_wait(bar, parity, abort_flag)) return false;
-        fence_proxy_async_smem();  // written by cp.async (generic proxy)
-        tc_fence_after();
-        return true;
-      };
-      auto issue_qk = [&](int j) -> bool {
-        const int sb = j & 1;
-        if (!mbar_wait(s_free(sb), static_cast<uint32_t>((j >> 1) & 1) ^ 1u, abort_flag)) return false;
-        tc_fence_after();
-        const uint32_t d = tmem + kSCol + sb * kChunk;
-        if (!wait_full(rope_full, static_cast<uint32_t>(j & 1))) return false;
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk)
-          mma_bf16(d, sdesc_sw128(q_s + 8 * kQBox + kk * 32, 16, 1024), sdesc_sw128(rope + kk * 32, 16, 1024),
-                   idesc_qk, kk > 0 ? 1u : 0u);
-        mma_commit(rope_empty);  // rope dims are not needed for P V
-        for (int q = 0; q < kPairsPerChunk; ++q) {
-          const int n = j * kPairsPerChunk + q;
-          const int slot = n % kPairRing;
-          if (!wait_full(pair_full(slot), static_cast<uint32_t>((n / kPairRing) & 1))) return false;
-          const uint32_t base = pairs + slot * kPairBytes;
-#pragma unroll
-          for (int bx = 0; bx < 2; ++bx) {
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk)
-              mma_bf16(d, sdesc_sw128(q_s + (2 * q + bx) * kQBox + kk * 32, 16, 1024),
-                       sdesc_sw128(base + bx * kBoxBytes + kk * 32, 16, 1024), idesc_qk, 1u);
-          }
-        }
-        mma_commit(s_full(sb));
-        return true;
-      };
-      auto issue_pv = [&](int j) -> bool {
-        if (!mbar_wait(p_full, static_cast<uint32_t>(j & 1), abort_flag)) return false;
-        tc_fence_after();
+      // PV(j): O^T[dims 128 q ..][heads] += V_j^T (P_hi + P_lo)^T, one accumulator block per value pair
+      auto issue_pv = [&](int j) {
         for (int q = 0; q < kPairsPerChunk; ++q) {
           const int slot = (j * kPairsPerChunk + q) % kPairRing;
           const uint32_t base = pairs + slot * kPairBytes;
-          const uint32_t d = tmem + q * kHeads;  // O^T block: dims 128 q .. +127
+          const uint32_t d = tmem + q * kHeads;
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk) {
             // A = V^T: M = 128 dims over the pair's two boxes, K = rows 16 kk ..
@@ -309,12 +298,66 @@ __global__ void __launch_bounds__(kThreads, 1)
           mma_commit(pair_empty(slot));
         }
         mma_commit(p_free);
-        return true;
       };
-      if (ok && nchunks > 0) ok = issue_qk(0);
-      for (int j = 0; j < nchunks && ok; ++j) {
-        if (j + 1 < nchunks && !(ok = issue_qk(j + 1))) break;
-        ok = issue_pv(j);
+      // Non-blocking issue: PV(pv_j) as soon as P is written, else the next
+      // piece of QK^T(qk_j) (part 0: rope box once S buffer and rope slot are
+      // ready; parts 1-4: one value pair each).
+      int qk_j = 0, qk_part = 0, pv_j = 0;
+      long long idle_since = clock64();
+      while (ok && pv_j < nchunks) {
+        bool did = false;
+        if (pv_j < qk_j && mbar_test_wait(p_full, static_cast<uint32_t>(pv_j & 1))) {
+          tc_fence_after();
+          issue_pv(pv_j);
+          ++pv_j;
+          did = true;
+        } else if (qk_j < nchunks) {
+          const int sb = qk_j & 1;
+          const uint32_t d = tmem + kSCol + sb * kChunk;
+          if (qk_part == 0) {
+            if (mbar_test_wait(s_free(sb), static_cast<uint32_t>((qk_j >> 1) & 1) ^ 1u) &&
+                mbar_test_wait(rope_full, static_cast<uint32_t>(qk_j & 1))) {
+              fence_proxy_async_smem();  // written by cp.async (generic proxy)
+              tc_fence_after();
+#pragma unroll
+              for (int kk = 0; kk < 4; ++kk)
+                mma_bf16(d, sdesc_sw128(q_s + 8 * kQBox + kk * 32, 16, 1024), sdesc_sw128(rope + kk * 32, 16, 1024),
+                         idesc_qk, kk > 0 ? 1u : 0u);
+              mma_commit(rope_empty);  // rope dims are not needed for P V
+              qk_part = 1;
+              did = true;
+            }
+          } else {
+            const int q = qk_part - 1;
+            const int n = qk_j * kPairsPerChunk + q;
+            const int slot = n % kPairRing;
+            if (mbar_test_wait(pair_full(slot), static_cast<uint32_t>((n / kPairRing) & 1))) {
+              fence_proxy_async_smem();
+              tc_fence_after();
+              const uint32_t base = pairs + slot * kPairBytes;
+#pragma unroll
+              for (int bx = 0; bx < 2; ++bx) {
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk)
+                  mma_bf16(d, sdesc_sw128(q_s + (2 * q + bx) * kQBox + kk * 32, 16, 1024),
+                           sdesc_sw128(base + bx * kBoxBytes + kk * 32, 16, 1024), idesc_qk, 1u);
+              }
+              if (qk_part == kPairsPerChunk) {
+                mma_commit(s_full(sb));
+                ++qk_j;
+                qk_part = 0;
+              } else {
+                ++qk_part;
+              }
+              did = true;
+            }
+          }
+        }
+        if (did) {
+          idle_since = clock64();
+        } else if (*abort_flag || clock64() - idle_since > kWaitBudgetCycles) {
+          ok = false;
+        }
       }
       if (!ok) {
         record_status(p.status, kStatusTimeout);
@@ -355,12 +398,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!(ok = mbar_wait(mask_full(mb), static_cast<uint32_t>((j / kMaskRing) & 1), abort_flag))) break;
       const uint64_t mk = masks[mb];
       mbar_arrive(mask_empty(mb));
-      float mt = -INFINITY;
+      // row max as eight independent chains (one warp per scheduler: latency, not issue, bounds this)
+      float mp[8];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) mp[k] = -INFINITY;
 #pragma unroll
       for (int i = 0; i < 64; ++i) {
         s[i] = ((mk >> i) & 1ull) ? s[i] * p.scale_log2 : -INFINITY;
-        mt = fmaxf(mt, s[i]);
+        mp[i & 7] = fmaxf(mp[i & 7], s[i]);
       }
+      const float mt = fmaxf(fmaxf(fmaxf(mp[0], mp[1]), fmaxf(mp[2], mp[3])),
+                             fmaxf(fmaxf(mp[4], mp[5]), fmaxf(mp[6], mp[7])));
       float alpha = 1.f;
       bool resc = false;
       if (m_ref == -INFINITY) {
@@ -370,12 +418,20 @@ __global__ void __launch_bounds__(kThreads, 1)
         m_ref = mt;
         resc = true;
       }
-      float psum = 0.f;
+      float ps[8];
 #pragma unroll
-      for (int i = 0; i < 64; ++i) {
-        s[i] = m_ref == -INFINITY ? 0.f : exp2f(s[i] - m_ref);
-        psum += s[i];
+      for (int k = 0; k < 8; ++k) ps[k] = 0.f;
+      if (m_ref == -INFINITY) {  // every slot so far is empty: all weights are zero
+#pragma unroll
+        for (int i = 0; i < 64; ++i) s[i] = 0.f;
+      } else {
+#pragma unroll
+        for (int i = 0; i < 64; ++i) {
+          s[i] = fast_exp2(s[i] - m_ref);
+          ps[i & 7] += s[i];
+        }
       }
+      const float psum = ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7]));
       l_run = l_run * alpha + psum;
       // PV_{j-1} must be done before P and O are touched.
       if (!(ok = mbar_wait(p_free, static_cast<uint32_t>(j & 1) ^ 1u, abort_flag))) break;
@@ -416,44 +472,110 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_before();
       mbar_arrive(p_full);
     }
-    if (!ok) {
-      record_status(p.status, kStatusTimeout);
-      *abort_flag = 1;
-    } else if (mbar_wait(o_full, 0, abort_flag)) {
-      tc_fence_after();
-      // per-head factor: gate / l (one split) or 1 (partials)
-      const size_t pslot = (static_cast<size_t>(row) * p.splits + split) * kHeads;
-      if (owner) {
-        float f = 1.f;
-        if (p.splits == 1) {
-          const float g =
-              p.gate ? sigmoidf_(bf16_bits_to_float(p.gate[static_cast<size_t>(row) * kHeads + head])) : 1.f;
-          f = l_run > 0.f ? g / l_run : 0.f;
-        } else {
-          p.part_ml[(pslot + head) * 2 + 0] = m_ref;
-          p.part_ml[(pslot + head) * 2 + 1] = l_run;
-        }
-        head_f[head] = f;
-      }
-      named_barrier(1, kSoftmaxThreads);
-      // O^T block b: this lane holds dim 128 b + 32 quarter + lane for all 64 heads
-      float* base = p.splits == 1 ? p.out + static_cast<size_t>(row) * kHeads * kDv : p.part_o + pslot * kDv;
-      for (int blk = 0; blk < 4; ++blk) {
-        const int dim = 128 * blk + 32 * quarter + lane;
-        for (int c = 0; c < 2; ++c) {
-          float o[32];
-          tmem_ld32(tmem + lane_addr + blk * kHeads + c * 32, o);
-#pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            const int h = c * 32 + i;
-            base[static_cast<size_t>(h) * kDv + dim] = o[i] * head_f[h];
-          }
-        }
-      }
-    } else {
+    const bool have_o = ok && mbar_wait(o_full, 0, abort_flag);
+    if (!have_o) {
       record_status(p.status, kStatusTimeout);
       *abort_flag = 1;
     }
+    if (owner) own_ml[head] = make_float2(m_ref, l_run);
+  }
+
+  // ---- split merge: out = g / L * sum_r 2^(m_r - M) O_r with M = max_r m_r and
+  // L = sum_r 2^(m_r - M) l_r (per head).  Every thread of the cluster takes
+  // part in its barriers, on every path.
+  const int S = p.splits;
+  float* o_stage = reinterpret_cast<float*>(smem);  // [64][512] fp32 in the value ring
+  if (S > 1) {
+    cluster.sync();  // every split's (m, l) published; all MMAs of every CTA done
+  } else {
+    __syncthreads();
+  }
+  if (warp > kMmaWarp && lane < 16) {
+    const int head = (warp & 3) * 16 + lane;
+    const float g = p.gate ? sigmoidf_(bf16_bits_to_float(p.gate[static_cast<size_t>(row) * kHeads + head])) : 1.f;
+    float f;
+    if (S == 1) {
+      const float l = own_ml[head].y;
+      f = l > 0.f ? g / l : 0.f;
+    } else {
+      // every split's (m, l) for this head, all loads in flight at once
+      float2 ml[kMaxSplits];
+#pragma unroll
+      for (int r = 0; r < kMaxSplits; ++r)
+        ml[r] = r < S ? *cluster.map_shared_rank(&own_ml[head], r) : make_float2(-INFINITY, 0.f);
+      float mx = -INFINITY;
+#pragma unroll
+      for (int r = 0; r < kMaxSplits; ++r) mx = fmaxf(mx, ml[r].x);
+      float L = 0.f;
+#pragma unroll
+      for (int r = 0; r < kMaxSplits; ++r)
+        if (ml[r].x != -INFINITY) L += exp2f(ml[r].x - mx) * ml[r].y;
+      const float m_own = own_ml[head].x;
+      f = (L > 0.f && m_own != -INFINITY) ? exp2f(m_own - mx) * g / L : 0.f;
+    }
+    head_f[head] = f;
+  }
+  __syncthreads();
+  if (warp < kProducerWarps || warp > kMmaWarp) {
+    // Eight warps read O^T out of TMEM: warp w reads lane quarter w % 4; the
+    // producer warps take dim blocks 0-1, the softmax warps blocks 2-3.
+    // O^T block b: this lane holds dim 128 b + 32 quarter + lane for all 64 heads.
+    const int quarter = warp & 3;
+    const uint32_t lane_addr = static_cast<uint32_t>(quarter * 32) << 16;
+    const int blk0 = warp < kProducerWarps ? 0 : 2;
+    float* dst = S == 1 ? p.out + static_cast<size_t>(row) * kHeads * kDv : o_stage;
+    tc_fence_after();
+    for (int c = 0; c < 2; ++c) {
+      float hf[32];
+#pragma unroll
+      for (int i = 0; i < 32; ++i) hf[i] = head_f[c * 32 + i];
+      for (int blk = blk0; blk < blk0 + 2; ++blk) {
+        const int dim = 128 * blk + 32 * quarter + lane;
+        float o[32];
+        tmem_ld32(tmem + lane_addr + blk * kHeads + c * 32, o);
+        float* col = dst + static_cast<size_t>(c * 32) * kDv + dim;
+#pragma unroll
+        for (int i = 0; i < 32; ++i) col[static_cast<size_t>(i) * kDv] = o[i] * hf[i];
+      }
+    }
+  }
+  if (S > 1) {
+    cluster.sync();  // every split's scaled O staged
+    // this CTA sums and writes the float4 columns [v0, v1) of every head's 512 dims
+    const int v0 = (kDv / 4) * split / S, v1 = (kDv / 4) * (split + 1) / S;
+    const int vecs = v1 - v0;
+    float* orow = p.out + static_cast<size_t>(row) * kHeads * kDv;
+    constexpr int kUnroll = 4;  // elements per thread in flight
+    for (int e0 = threadIdx.x; e0 < kHeads * vecs; e0 += kUnroll * kThreads) {
+      float4 acc[kUnroll];
+      int off[kUnroll];
+#pragma unroll
+      for (int u = 0; u < kUnroll; ++u) {
+        const int e = e0 + u * kThreads;
+        const int h = e / vecs;
+        off[u] = h * kDv + 4 * (v0 + e - h * vecs);
+        acc[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+#pragma unroll
+      for (int r = 0; r < kMaxSplits; ++r) {
+        if (r < S) {
+#pragma unroll
+          for (int u = 0; u < kUnroll; ++u) {
+            if (e0 + u * kThreads < kHeads * vecs) {
+              const float4 x = *reinterpret_cast<const float4*>(cluster.map_shared_rank(o_stage + off[u], r));
+              acc[u].x += x.x;
+              acc[u].y += x.y;
+              acc[u].z += x.z;
+              acc[u].w += x.w;
+            }
+          }
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < kUnroll; ++u)
+        if (e0 + u * kThreads < kHeads * vecs) *reinterpret_cast<float4*>(orow + off[u]) = acc[u];
+    }
+    cluster.sync();  // no CTA leaves while another reads its staging
   }
 
   tc_fence_before();
@@ -464,57 +586,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-// Merges split partials: o = sum_s 2^(m_s - M) O_s / sum_s 2^(m_s - M) l_s, times sigmoid(g).
-__global__ void __launch_bounds__(128) sga_combine_kernel(const float* __restrict__ part_o,
-                                                          const float* __restrict__ part_ml,
-                                                          const uint16_t* __restrict__ gate, float* __restrict__ out,
-                                                          int splits) {
-  const int row = blockIdx.x / kHeads;
-  const int head = blockIdx.x % kHeads;
-  __shared__ float wts[64];
-  if (threadIdx.x < 32) {
-    float mx = -INFINITY;
-    for (int s = threadIdx.x; s < splits; s += 32)
-      mx = fmaxf(mx, part_ml[((static_cast<size_t>(row) * splits + s) * kHeads + head) * 2]);
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, o));
-    float lsum = 0.f;
-    for (int s = threadIdx.x; s < splits; s += 32) {
-      const size_t k = ((static_cast<size_t>(row) * splits + s) * kHeads + head) * 2;
-      const float ms = part_ml[k];
-      const float w = (ms == -INFINITY) ? 0.f : exp2f(ms - mx);
-      wts[s] = w;
-      lsum += w * part_ml[k + 1];
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) lsum += __shfl_xor_sync(0xFFFFFFFFu, lsum, o);
-    const float g = gate ? sigmoidf_(bf16_bits_to_float(gate[static_cast<size_t>(row) * kHeads + head])) : 1.f;
-    const float f = lsum > 0.f ? g / lsum : 0.f;
-    __syncwarp();
-    for (int s = threadIdx.x; s < splits; s += 32) wts[s] *= f;
-  }
-  __syncthreads();
-  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-  for (int s = 0; s < splits; ++s) {
-    const float w = wts[s];
-    const float4 v = __ldg(reinterpret_cast<const float4*>(
-                               part_o + ((static_cast<size_t>(row) * splits + s) * kHeads + head) * kDv) +
-                           threadIdx.x);
-    acc.x = fmaf(w, v.x, acc.x);
-    acc.y = fmaf(w, v.y, acc.y);
-    acc.z = fmaf(w, v.z, acc.z);
-    acc.w = fmaf(w, v.w, acc.w);
-  }
-  reinterpret_cast<float4*>(out + (static_cast<size_t>(row) * kHeads + head) * kDv)[threadIdx.x] = acc;
-}
-
 }  // namespace
 
-// Splits of the K slots per query so that rows * splits fills ~148 SMs once.
+// Splits of the K slots per query (at most kMaxSplits, the CTAs of one
+// cluster) so that rows * splits fills ~148 SMs once.
 int attend_splits(int rows, int top_k) {
   const int chunks = (top_k + kChunk - 1) / kChunk;
   int best = 1;
-  for (int s = 1; s <= chunks && s <= 64; ++s) {
+  for (int s = 1; s <= chunks && s <= kMaxSplits; ++s) {
     if (chunks % s == 0 && static_cast<long long>(rows) * s <= 148) best = s;
   }
   return best;
@@ -524,8 +603,11 @@ cudaError_t launch_attend(const AttendArgs& a, cudaStream_t stream) {
   const int rows = a.batch * a.n_q;
   if (rows == 0) return cudaSuccess;
   const int splits = attend_splits(rows, a.top_k);
-  CUtensorMap qmap;
+  CUtensorMap qmap, kvmap;
   cudaError_t e = make_tmap_bf16_2d(&qmap, a.q, kDq, static_cast<uint64_t>(rows) * kHeads, kDq * 2, 64, kHeads);
+  if (e != cudaSuccess) return e;
+  // every cache row of every sequence, one 64-dim box per row (gather4 takes four rows at a time)
+  e = make_tmap_bf16_2d(&kvmap, a.kv, kDq, static_cast<uint64_t>(a.batch) * a.kv_stride, kDq * 2, 64, 1);
   if (e != cudaSuccess) return e;
   e = cudaFuncSetAttribute(sga_attend_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            static_cast<int>(kSmemBytes));
@@ -535,8 +617,6 @@ cudaError_t launch_attend(const AttendArgs& a, cudaStream_t stream) {
   p.idx = a.idx;
   p.gate = a.gate;
   p.out = a.out;
-  p.part_o = a.part_o;
-  p.part_ml = a.part_ml;
   p.status = a.status;
   p.n_q = a.n_q;
   p.kv_stride = a.kv_stride;
@@ -544,11 +624,19 @@ cudaError_t launch_attend(const AttendArgs& a, cudaStream_t stream) {
   p.splits = splits;
   p.chunks_per_split = (a.top_k + kChunk - 1) / kChunk / splits;
   p.scale_log2 = static_cast<float>(0.07216878364870322 * 1.4426950408889634);
-  sga_attend_kernel<<<rows * splits, kThreads, kSmemBytes, stream>>>(qmap, p);
-  e = cudaGetLastError();
-  if (e != cudaSuccess || splits == 1) return e;
-  sga_combine_kernel<<<rows * kHeads, 128, 0, stream>>>(a.part_o, a.part_ml, a.gate, a.out, splits);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(rows * splits));
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = kSmemBytes;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = splits;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, sga_attend_kernel, qmap, kvmap, p);
 }
 
 }  // namespace sga

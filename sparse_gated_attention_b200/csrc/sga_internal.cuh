@@ -41,8 +41,6 @@ struct AttendArgs {
   const int32_t* idx;    // [rows][K]
   const uint16_t* gate;  // [rows][64] or null
   float* out;            // [rows][64][512]
-  float* part_o;         // [rows][splits][64][512] scratch (splits > 1)
-  float* part_ml;        // [rows][splits][64][2] scratch (splits > 1)
   int* status;
   int batch, n_q, kv_stride, top_k;
 };

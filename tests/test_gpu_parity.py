@@ -187,6 +187,7 @@ def random_idx(rng, B, T, L, K, holes=0.1, shuffle=True):
 @pytest.mark.parametrize("B,T,L,K,gated", [(1, 1, 3000, 2048, True), (4, 1, 5000, 2048, True),
                                            (2, 3, 2500, 2048, False), (32, 1, 4096, 2048, True),
                                            (3, 1, 700, 64, True), (1, 2, 900, 192, True),
+                                           (1, 1, 2000, 320, True), (2, 1, 3000, 448, False),
                                            (200, 1, 3000, 2048, True)])
 def test_attend_matches_oracle(B, T, L, K, gated):
     rng = np.random.default_rng(B * 1000 + L)
