@@ -38,8 +38,11 @@
  *     error is kept until sga_clear_device_status.
  *   - Workspace: caller-allocated device memory of at least
  *     sga_workspace_size(dims, op) bytes, 256-byte aligned.  A zero-filled
- *     workspace starts with a clear status.  Calls that share a workspace must
- *     be ordered on one stream.
+ *     workspace starts with a clear status.  sga_forward also keeps per-query
+ *     histograms in it: its workspace must be zero-filled before the first
+ *     call, and every call leaves them zeroed for the next one.  After a
+ *     device error, zero the whole workspace before using it again.  Calls
+ *     that share a workspace must be ordered on one stream.
  *   - No C++ exception crosses this interface.
  */
 #ifndef SGA_H_

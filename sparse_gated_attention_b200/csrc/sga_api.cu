@@ -204,12 +204,12 @@ sga_status_t sga_forward(const sga_dims_t* dims, const sga_bf16_t* q_idx, const 
   float* scores = at<float>(ws, l.scores);
   int32_t* idx = idx_out ? idx_out : at<int32_t>(ws, l.idx);
   const int rows = dims->batch * dims->n_q;
-  // The indexer counts the first radix level of the selection as it writes the scores.
+  // The indexer counts the first radix level of the selection as it writes the
+  // scores; the selection clears each histogram row after reading it, so a
+  // zero-filled workspace stays ready for the next call.
   uint32_t* hist = at<uint32_t>(ws, l.hist);
-  cudaError_t e = cudaMemsetAsync(hist, 0, static_cast<size_t>(rows) * 4096 * 4, s);
-  if (e != cudaSuccess) return SGA_ERR_CUDA;
   IndexArgs ia{q_idx, w, k_idx, q_pos, scores, hist, status, dims->batch, dims->n_q, dims->kv_stride};
-  e = launch_index_scores(ia, sms, s);
+  cudaError_t e = launch_index_scores(ia, sms, s);
   if (e != cudaSuccess) return SGA_ERR_CUDA;
   TopkArgs ta{scores, q_pos, idx, at<uint32_t>(ws, l.bitmap), hist, status, rows, dims->kv_stride, dims->top_k};
   e = launch_topk(ta, s);

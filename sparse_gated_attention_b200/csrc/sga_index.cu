@@ -116,6 +116,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  // Set-up above overlaps the previous kernel on the stream; inputs are read below.
+  grid_dependency_wait();
+  grid_launch_dependents();
 
   const long long j0 = p.total_tiles * blockIdx.x / gridDim.x;
   const long long j1 = p.total_tiles * (blockIdx.x + 1) / gridDim.x;
@@ -326,8 +329,17 @@ cudaError_t launch_index_scores(const IndexArgs& a, int num_sms, cudaStream_t st
   p.tiles_per_row = tiles_per_row;
   p.total_tiles = total;
   const int grid = static_cast<int>(total < num_sms ? total : num_sms);
-  sga_index_kernel<<<grid, kThreads, kSmemBytes, stream>>>(kmap, qmap, p);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(grid));
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = kSmemBytes;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, sga_index_kernel, kmap, qmap, p);
 }
 
 }  // namespace sga

@@ -14,7 +14,7 @@ struct IndexArgs {
   const uint16_t* k_idx;  // [B][L][128]
   const int32_t* q_pos;   // [rows]
   float* scores;          // [rows][L]
-  uint32_t* hist;         // [rows][4096] first-level top-k histogram (zeroed by the caller) or null
+  uint32_t* hist;         // [rows][4096] first-level top-k histogram (all zero on entry) or null
   int* status;
   int batch, n_q, kv_stride;
 };
@@ -26,7 +26,7 @@ struct TopkArgs {
   const int32_t* q_pos;  // [rows]
   int32_t* idx;          // [rows][K]
   uint32_t* bitmap;      // [rows][words_per_row] scratch
-  const uint32_t* hist;  // [rows][4096] histogram of the top 12 order bits, or null
+  uint32_t* hist;        // [rows][4096] histogram of the top 12 order bits, or null; zeroed after use
   int* status;
   int rows, kv_stride, top_k;
 };

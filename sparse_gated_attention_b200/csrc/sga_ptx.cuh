@@ -71,6 +71,15 @@ __device__ __forceinline__ bool mbar_test_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
+// Programmatic dependent launch.  grid_dependency_wait returns once the grids
+// this one depends on have completed and their writes are visible (at once
+// when there are none); grid_launch_dependents lets the next grid on the
+// stream be scheduled early (it still waits in its own grid_dependency_wait).
+__device__ __forceinline__ void grid_dependency_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void grid_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // Waits for the phase with the given parity to complete.  Returns false when
 // the budget ran out or another thread of the CTA raised `abort_flag`.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag) {

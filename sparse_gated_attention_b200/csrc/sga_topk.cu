@@ -72,7 +72,7 @@ struct TopkParams {
   const int32_t* q_pos;
   int32_t* idx;
   uint32_t* bitmap;
-  const uint32_t* hist;
+  uint32_t* hist;  // first-level histograms from the indexer (or null); zeroed here after use
   int* status;
   int kv_stride, top_k;
   long long words_per_row;
@@ -286,18 +286,26 @@ __global__ void __launch_bounds__(kThreads, 1) sga_topk_stream_kernel(TopkParams
   const int tid = threadIdx.x, lane = tid & 31;
   const int K = p.top_k;
   int32_t* out = p.idx + static_cast<size_t>(row) * K;
+  grid_dependency_wait();  // scores, histograms and q_pos come from earlier kernels
+  grid_launch_dependents();
+  uint32_t* hist_row = p.hist ? p.hist + static_cast<size_t>(row) * kBins : nullptr;
   const int t = __ldg(p.q_pos + row);
   if (t < 0 || t >= p.kv_stride) {
     if (rank == 0) {
       if (tid == 0) record_status(p.status, kStatusDeviceArg);
       for (int j = tid; j < K; j += kThreads) out[j] = -1;
+      if (hist_row)
+        for (int b = tid; b < kBins; b += kThreads) hist_row[b] = 0;
     }
     return;
   }
   const int n = t + 1;
   if (n <= K) {
-    if (rank == 0)
+    if (rank == 0) {
       for (int j = tid; j < K; j += kThreads) out[j] = j < n ? j : -1;
+      if (hist_row)
+        for (int b = tid; b < kBins; b += kThreads) hist_row[b] = 0;
+    }
     return;
   }
   const float* sc = p.scores + static_cast<size_t>(row) * p.kv_stride;
@@ -343,8 +351,7 @@ __global__ void __launch_bounds__(kThreads, 1) sga_topk_stream_kernel(TopkParams
       if (kVec) {
         if (!mbar_wait(hist_bar, 0, &abort_flag)) record_status(p.status, kStatusTimeout);
       } else {
-        const uint32_t* hrow = p.hist + static_cast<size_t>(row) * kBins;
-        for (int b = tid; b < kBins; b += kThreads) ghist[b] = __ldg(hrow + b);
+        for (int b = tid; b < kBins; b += kThreads) ghist[b] = hist_row[b];
       }
       __syncthreads();
     } else {
@@ -516,7 +523,9 @@ __global__ void __launch_bounds__(kThreads, 1) sga_topk_stream_kernel(TopkParams
     sel_all += a;
     tie_all += b;
   }
-  cluster.sync();  // every CTA has read every count
+  cluster.sync();  // every CTA has read every count (and its copy of the histogram row)
+  if (rank == 0 && hist_row)  // ready for the next call
+    for (int b = tid; b < kBins; b += kThreads) hist_row[b] = 0;
   const uint32_t take_all = static_cast<uint32_t>(K) > sel_all ? static_cast<uint32_t>(K) - sel_all : 0u;
   if (rank == 0 && tid == 0 &&
       (sel_all > static_cast<uint32_t>(K) || sel_all + tie_all < static_cast<uint32_t>(K)))
@@ -600,18 +609,26 @@ __global__ void __launch_bounds__(kThreads, 1) sga_topk_resident_kernel(TopkPara
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int K = p.top_k;
   int32_t* out = p.idx + static_cast<size_t>(row) * K;
+  grid_dependency_wait();  // scores, histograms and q_pos come from earlier kernels
+  grid_launch_dependents();
+  uint32_t* hist_row = p.hist ? p.hist + static_cast<size_t>(row) * kBins : nullptr;
   const int t = __ldg(p.q_pos + row);
   if (t < 0 || t >= p.kv_stride) {
     if (rank == 0) {
       if (tid == 0) record_status(p.status, kStatusDeviceArg);
       for (int j = tid; j < K; j += kThreads) out[j] = -1;
+      if (hist_row)
+        for (int b = tid; b < kBins; b += kThreads) hist_row[b] = 0;
     }
     return;
   }
   const int n = t + 1;
   if (n <= K) {
-    if (rank == 0)
+    if (rank == 0) {
       for (int j = tid; j < K; j += kThreads) out[j] = j < n ? j : -1;
+      if (hist_row)
+        for (int b = tid; b < kBins; b += kThreads) hist_row[b] = 0;
+    }
     return;
   }
   // The host picks C with C * kResSeg >= kv_stride, so every segment fits.
@@ -633,7 +650,7 @@ __global__ void __launch_bounds__(kThreads, 1) sga_topk_resident_kernel(TopkPara
     if (tid == 0) {
       if (p.hist) {
         mbar_arrive_expect_tx(hist_bar, kBins * 4);
-        bulk_load(smem_u32(ghist), p.hist + static_cast<size_t>(row) * kBins, kBins * 4, hist_bar);
+        bulk_load(smem_u32(ghist), hist_row, kBins * 4, hist_bar);
       }
       for (int c = 0; c < nch; ++c) {
         const int cnt = min(kChunk, len - c * kChunk);
@@ -646,8 +663,7 @@ __global__ void __launch_bounds__(kThreads, 1) sga_topk_resident_kernel(TopkPara
   } else {
     for (int i = tid; i < len; i += kThreads) seg[i] = __ldg(sc + s0 + i);
     if (p.hist) {
-      const uint32_t* hrow = p.hist + static_cast<size_t>(row) * kBins;
-      for (int b = tid; b < kBins; b += kThreads) ghist[b] = __ldg(hrow + b);
+      for (int b = tid; b < kBins; b += kThreads) ghist[b] = hist_row[b];
     }
     __syncthreads();
   }
@@ -790,9 +806,12 @@ __global__ void __launch_bounds__(kThreads, 1) sga_topk_resident_kernel(TopkPara
       dst[1] = tot_t;
     }
   }
-  // Every count delivered.  No CTA touches another's shared memory after this
-  // barrier, so none has to wait for the others before exiting.
+  // Every count delivered (and every CTA's copy of the histogram row taken).
+  // No CTA touches another's shared memory after this barrier, so none has to
+  // wait for the others before exiting.
   cluster.sync();
+  if (rank == 0 && hist_row)  // ready for the next call
+    for (int b = tid; b < kBins; b += kThreads) hist_row[b] = 0;
   uint32_t sel_before = 0, tie_before = 0, sel_all = 0, tie_all = 0;
   for (int r = 0; r < C; ++r) {
     const uint32_t a = peer_counts[r][0], b = peer_counts[r][1];
@@ -862,13 +881,15 @@ cudaError_t launch_topk(const TopkArgs& a, cudaStream_t stream) {
   cfg.blockDim = dim3(kThreads);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = C;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 2;
   return cudaLaunchKernelEx(&cfg, kernel, p);
 }
 

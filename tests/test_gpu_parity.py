@@ -254,6 +254,31 @@ def test_forward_matches_oracle(B, T, L, pos):
     assert_close(out.cpu().numpy(), want_out, "forward")
 
 
+def test_forward_reuses_its_workspace():
+    """The selection clears the indexer's histograms after reading them, on
+    every exit (full selection, t + 1 <= K, bad position), so one zero-filled
+    workspace serves consecutive calls."""
+    B, L = 3, 6000
+    x = gen_small(B, 1, L, [[5999], [1000], [L + 5]])
+    ws = sga.alloc_workspace(sga.make_dims(B, 1, L), sga.OP_FORWARD)
+    idx, out = sga.forward(x["q_idx"], x["w"], x["k_idx"], x["q"], x["kv"], x["gate"], x["q_pos"], ws=ws)
+    assert sga.device_status(ws) == 6  # the bad position is reported
+    sub = {k: v[:2] for k, v in x.items()}
+    want_idx, want_out = oracle.forward(sub["q_idx"], sub["w"], sub["k_idx"], sub["q"], sub["kv"], sub["gate"],
+                                        sub["q_pos"].cpu())
+    np.testing.assert_array_equal(idx[:2].cpu().numpy(), want_idx)
+    assert_close(out[:2].cpu().numpy(), want_out, "forward, first call")
+    sga.clear_device_status(ws)
+    for pos in ([[1500], [5999], [4500]], [[5999], [2047], [3000]]):
+        x["q_pos"] = torch.as_tensor(np.asarray(pos, dtype=np.int32), device="cuda")
+        idx, out = sga.forward(x["q_idx"], x["w"], x["k_idx"], x["q"], x["kv"], x["gate"], x["q_pos"], ws=ws)
+        check_status(ws)
+        want_idx, want_out = oracle.forward(x["q_idx"], x["w"], x["k_idx"], x["q"], x["kv"], x["gate"],
+                                            x["q_pos"].cpu())
+        np.testing.assert_array_equal(idx.cpu().numpy(), want_idx)
+        assert_close(out.cpu().numpy(), want_out, f"forward, positions {pos}")
+
+
 def test_device_status_reports_bad_arguments():
     B, L = 2, 3000
     x = gen_small(B, 1, L, [[L - 1], [L - 1]])
