@@ -54,15 +54,29 @@ struct IndexParams {
   long long total_tiles;
 };
 
-// Work item j -> (query row, first key).  Returns false for tiles that lie past
-// the query position (or rows whose position is invalid).
-__device__ __forceinline__ bool tile_info(const IndexParams& p, long long j, int& row, int& key0, int& t) {
-  row = static_cast<int>(j / p.tiles_per_row);
-  key0 = static_cast<int>(j % p.tiles_per_row) * kKeys;
-  t = __ldg(p.q_pos + row);
-  if (t < 0 || t >= p.kv_stride) return false;
-  return key0 <= t;
-}
+// Walks work items j = (query row, 128-key tile) in order: one division at
+// the start, then a key step per item; the query position is read only when
+// the row changes.
+struct TileCursor {
+  int row, key0, t;
+  __device__ __forceinline__ void start(const IndexParams& p, long long j) {
+    row = static_cast<int>(j / p.tiles_per_row);
+    key0 = static_cast<int>(j % p.tiles_per_row) * kKeys;
+    t = __ldg(p.q_pos + row);
+  }
+  // Moves to item j + 1; `more` is false after the last item of the range.
+  __device__ __forceinline__ void next(const IndexParams& p, bool more) {
+    key0 += kKeys;
+    if (key0 >= p.tiles_per_row * kKeys) {
+      key0 = 0;
+      ++row;
+      if (more) t = __ldg(p.q_pos + row);
+    }
+  }
+  __device__ __forceinline__ bool bad_position(const IndexParams& p) const { return t < 0 || t >= p.kv_stride; }
+  // False for tiles past the query position or rows whose position is invalid.
+  __device__ __forceinline__ bool live(const IndexParams& p) const { return !bad_position(p) && key0 <= t; }
+};
 
 __global__ void __launch_bounds__(kThreads, 1)
     sga_index_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap qmap,
@@ -131,12 +145,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       long long n = 0, qc = 0;
       int cur_row = -1;
       bool ok = true;
-      for (long long j = j0; j < j1; ++j) {
-        int row, key0, t;
-        if (!tile_info(p, j, row, key0, t)) {
-          if (t < 0 || t >= p.kv_stride) record_status(p.status, kStatusDeviceArg);
+      TileCursor cur;
+      if (j0 < j1) cur.start(p, j0);
+      for (long long j = j0; j < j1; cur.next(p, ++j < j1)) {
+        if (!cur.live(p)) {
+          if (cur.bad_position(p)) record_status(p.status, kStatusDeviceArg);
           continue;
         }
+        const int row = cur.row, key0 = cur.key0;
         if (row != cur_row) {
           const int slot = static_cast<int>(qc & 1);
           if (!mbar_wait(qempty(slot), static_cast<uint32_t>((qc >> 1) & 1) ^ 1u, abort_flag)) {
@@ -178,9 +194,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       long long n = 0, qc = 0, an = 0;
       int cur_row = -1, cur_q = 0;
       bool ok = true;
-      for (long long j = j0; j < j1 && ok; ++j) {
-        int row, key0, t;
-        if (!tile_info(p, j, row, key0, t)) continue;
+      TileCursor cur;
+      if (j0 < j1) cur.start(p, j0);
+      for (long long j = j0; j < j1 && ok; cur.next(p, ++j < j1)) {
+        if (!cur.live(p)) continue;
+        const int row = cur.row;
         if (row != cur_row) {
           if (cur_row >= 0) mma_commit(qempty(cur_q));  // frees the previous query's buffer
           const int slot = static_cast<int>(qc & 1);
@@ -248,9 +266,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int b = et; b < kTopkHistBins; b += kEpiThreads) hist_s[b] = 0;
       named_barrier(1, kEpiThreads);
     }
-    for (long long j = j0; j < j1; ++j) {
-      int row, key0, t;
-      if (!tile_info(p, j, row, key0, t)) continue;
+    TileCursor cur;
+    if (j0 < j1) cur.start(p, j0);
+    for (long long j = j0; j < j1; cur.next(p, ++j < j1)) {
+      if (!cur.live(p)) continue;
+      const int row = cur.row, key0 = cur.key0, t = cur.t;
       if (row != cur_row) {
         if (with_hist && cur_row >= 0) flush_hist(cur_row);
         const uint4* wp = reinterpret_cast<const uint4*>(p.w + static_cast<size_t>(row) * kHeads);
@@ -279,11 +299,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       tmem_ld32(taddr + 32, v1);
       tc_fence_before();
       mbar_arrive(accempty(acc));
-      float s = 0.f;
+      // head sum as four independent chains (one warp per scheduler: the chain
+      // latency, not issue, bounds the epilogue); integer-valued inputs keep
+      // every partial sum exact, so the order does not change the score
+      float ps[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-      for (int h = 0; h < 32; ++h) s = fmaf(wv[h], fmaxf(v0[h], 0.f), s);
+      for (int h = 0; h < 32; ++h) ps[h & 3] = fmaf(wv[h], fmaxf(v0[h], 0.f), ps[h & 3]);
 #pragma unroll
-      for (int h = 0; h < 32; ++h) s = fmaf(wv[32 + h], fmaxf(v1[h], 0.f), s);
+      for (int h = 0; h < 32; ++h) ps[h & 3] = fmaf(wv[32 + h], fmaxf(v1[h], 0.f), ps[h & 3]);
+      const float s = (ps[0] + ps[1]) + (ps[2] + ps[3]);
       const int key = key0 + quarter * 32 + lane;
       if (key <= t) {
         p.scores[static_cast<size_t>(row) * p.kv_stride + key] = s;
