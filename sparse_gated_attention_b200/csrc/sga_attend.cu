@@ -24,12 +24,15 @@
 //     slot that is freed right after QK^T.  QK^T(j+1) is issued before PV(j),
 //     so the softmax of chunk j overlaps the next QK^T and chunk j+2 streams in
 //     while chunk j's values wait for P.
-//   * Warps 0-3 gather with TMA tile::gather4 (four cache rows x one 64-dim
-//     box per instruction, written by the TMA straight into the
-//     128-byte-swizzled layout); each warp gathers 16 rows of every chunk,
-//     so four warps keep the TMA unit busy.  An empty slot gathers the
-//     sequence's row 0 and is masked out of the softmax.  Warp 0 also
-//     publishes the validity mask of each chunk and loads Q.
+//   * Warps 0-3 gather each chunk through both of the SM's copy paths at
+//     once: value pairs 1-3 with TMA tile::gather4 (four cache rows x one
+//     64-dim box per instruction, written by the TMA straight into the
+//     128-byte-swizzled layout; each warp takes 16 rows), the rope box and
+//     value pair 0 with 16-byte cp.async from all 128 threads (swizzled by
+//     hand, empty slots zero-filled without a read).  An empty slot in a
+//     gather4 quad gathers the sequence's row 0 and is masked out of the
+//     softmax.  Warp 0 also publishes the validity mask of each chunk and
+//     loads Q.
 //     Warp 4 issues the MMAs without blocking on any one operand: it polls
 //     the barriers and issues PV(j) as soon as P_j is written, between the
 //     value pairs of QK^T(j+1), so value slots are released (and refilled)
@@ -70,6 +73,7 @@ constexpr int kQBytes = 9 * kQBox;
 constexpr int kPBytes = kHeads * kChunk * 2;  // 64 heads x 64 rows bf16
 constexpr int kMaskRing = 4;
 constexpr int kProducerWarps = 4;          // warps 0-3
+constexpr int kProducers = 32 * kProducerWarps;
 constexpr int kMmaWarp = 4;
 constexpr int kSoftmaxThreads = 128;        // warps 5-8
 constexpr int kThreads = 288;
@@ -152,10 +156,12 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kPairRing; ++s) {
-      mbar_init(pair_full(s), kProducerWarps);  // one expect_tx arrival per producer warp
+      // pair 0 of a chunk (slots 0 and 4) arrives by cp.async from every producer
+      // thread; pairs 1-3 by one gather4 expect_tx per producer warp
+      mbar_init(pair_full(s), s % kPairsPerChunk == 0 ? kProducers : kProducerWarps);
       mbar_init(pair_empty(s), 1);
     }
-    mbar_init(rope_full, kProducerWarps);
+    mbar_init(rope_full, kProducers);
     mbar_init(rope_empty, 1);
     mbar_init(q_full, 1);
     for (int b = 0; b < 2; ++b) {
@@ -197,6 +203,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int ptid = threadIdx.x;
     const int g = lane & 3;             // this lane's group of 4 rows within the warp's 16
     const int grow = 16 * warp + 4 * g;  // first chunk row of that group
+    const int part = ptid & 7;          // cp.async: 16-byte piece of a 128-byte row strip
+    const int rsub = ptid >> 3;         // cp.async: rows rsub + 16 i, i = 0..3
+    const uint16_t* kv_b = p.kv + static_cast<size_t>(b) * p.kv_stride * kDq;
     bool ok = true;
     if (ptid == 0) {
       mbar_arrive_expect_tx(q_full, kQBytes);
@@ -231,7 +240,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         ok = __shfl_sync(0xFFFFFFFFu, ok ? 1 : 0, 0) != 0;
         if (!ok) break;
       }
-      // cache rows of this lane's group (empty or invalid slots -> row 0, masked above)
+      // gather4: cache rows of this lane's quad (empty or invalid slots -> row 0, masked above)
       int y[4];
       {
         const int sidx = first + grow;  // a multiple of 4: one 16-byte load
@@ -241,15 +250,30 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int i = 0; i < 4; ++i) y[i] = row0 + ((e[i] >= 0 && e[i] < p.kv_stride) ? e[i] : 0);
       }
-      // rope dims 512..575 -> the rope slot (lanes 0-3: one group each)
+      // cp.async: this thread's four rows of the chunk (empty slots zero-filled)
+      const uint16_t* src[4];
+      uint32_t nbytes[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int sidx = first + rsub + 16 * i;
+        int sv = -1;
+        if (sidx < p.top_k) sv = __ldg(idx_row + sidx);
+        const bool valid = sv >= 0 && sv < p.kv_stride;
+        src[i] = kv_b + static_cast<size_t>(valid ? sv : 0) * kDq + part * 8;
+        nbytes[i] = valid ? 16u : 0u;
+      }
+      // rope dims 512..575 -> the rope slot (cp.async)
       if (!mbar_wait(rope_empty, static_cast<uint32_t>(j & 1) ^ 1u, abort_flag)) {
         ok = false;
         break;
       }
-      if (lane == 0) mbar_arrive_expect_tx(rope_full, 16 * 128);
-      __syncwarp();
-      if (lane < 4) tma_gather4(rope + grow * 128, &kvmap, rope_full, kDv, y[0], y[1], y[2], y[3]);
-      // value dims 128 q .. 128 q + 127 -> pair slot (4 j + q) mod 8 (lanes 0-7: group x box)
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int r = rsub + 16 * i;
+        cp_async_16(rope + r * 128 + ((part ^ (r & 7)) << 4), src[i] + kDv, nbytes[i]);
+      }
+      cp_async_arrive_noinc(rope_full);
+      // value dims 128 q .. 128 q + 127 -> pair slot (4 j + q) mod 8
       for (int q = 0; q < kPairsPerChunk; ++q) {
         const int n = j * kPairsPerChunk + q;
         const int slot = n % kPairRing;
@@ -258,15 +282,27 @@ __global__ void __launch_bounds__(kThreads, 1)
           break;
         }
         const uint32_t base = pairs + slot * kPairBytes;
-        if (lane == 0) mbar_arrive_expect_tx(pair_full(slot), 16 * 2 * 128);
-        __syncwarp();
-        if (lane < 8) {
-          const int bx = lane >> 2;
-          tma_gather4(base + bx * kBoxBytes + grow * 128, &kvmap, pair_full(slot), 128 * q + 64 * bx, y[0], y[1], y[2],
-                      y[3]);
+        if (q == 0) {  // cp.async from every producer thread
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const int r = rsub + 16 * i;
+            const uint32_t dst = base + r * 128 + ((part ^ (r & 7)) << 4);
+            cp_async_16(dst, src[i], nbytes[i]);
+            cp_async_16(dst + kBoxBytes, src[i] + 64, nbytes[i]);
+          }
+          cp_async_arrive_noinc(pair_full(slot));
+        } else {  // gather4 (lanes 0-7: quad x box)
+          if (lane == 0) mbar_arrive_expect_tx(pair_full(slot), 16 * 2 * 128);
+          __syncwarp();
+          if (lane < 8) {
+            const int bx = lane >> 2;
+            tma_gather4(base + bx * kBoxBytes + grow * 128, &kvmap, pair_full(slot), 128 * q + 64 * bx, y[0], y[1],
+                        y[2], y[3]);
+          }
         }
       }
     }
+    asm volatile("cp.async.wait_all;" ::: "memory");
     // On a timeout the waits above have run for about a second, long after any
     // gather issued before them has landed.
     if (!ok) {
@@ -374,74 +410,83 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
   } else {
-    // ------------------------------------------------------------ softmax + epilogue
+    // ------------------------------------------------------------ softmax
+    // S is read with the 16-lane x 256-bit TMEM shape, which matches the M = 64
+    // accumulator (16 rows per lane quarter): thread t of the warp holds rows
+    // t/4 and 8 + t/4 of its quarter, columns 8k + 2(t%4) and 8k + 2(t%4) + 1
+    // for k = 0..7.  The four threads of a row combine its max and sum with two
+    // shuffles, so every lane works on 32 scores per chunk.
     const int quarter = warp & 3;
-    const int head = quarter * 16 + (lane & 15);  // lanes 0-15 own this head's S row
-    const bool owner = lane < 16;
     const uint32_t lane_addr = static_cast<uint32_t>(quarter * 32) << 16;
-    float m_ref = -INFINITY, l_run = 0.f;
+    const int m4 = lane & 3;
+    const int hrow[2] = {quarter * 16 + (lane >> 2), quarter * 16 + 8 + (lane >> 2)};  // this thread's two heads
+    float m_ref[2] = {-INFINITY, -INFINITY}, l_run[2] = {0.f, 0.f};
     bool ok = true;
     for (int j = 0; j < nchunks; ++j) {
       const int sb = j & 1;
       if (!(ok = mbar_wait(s_full(sb), static_cast<uint32_t>((j >> 1) & 1), abort_flag))) break;
       tc_fence_after();
-      float s[64];
-      {
-        float a0[32], a1[32];
-        tmem_ld32(tmem + lane_addr + kSCol + sb * kChunk, a0);
-        tmem_ld32(tmem + lane_addr + kSCol + sb * kChunk + 32, a1);
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          s[i] = a0[i];
-          s[32 + i] = a1[i];
-        }
-      }
+      float r[32];
+      tmem_ld_16x256b_x8(tmem + lane_addr + kSCol + sb * kChunk, r);
       tc_fence_before();
       mbar_arrive(s_free(sb));
       const int mb = j % kMaskRing;
       if (!(ok = mbar_wait(mask_full(mb), static_cast<uint32_t>((j / kMaskRing) & 1), abort_flag))) break;
       const uint64_t mk = masks[mb];
       mbar_arrive(mask_empty(mb));
-      // row max as eight independent chains (one warp per scheduler: latency, not issue, bounds this)
-      float mp[8];
+      // x[i][2k + e] = score of row i at column 8k + 2 m4 + e (masked slots -> -inf)
+      float x[2][16];
 #pragma unroll
-      for (int k = 0; k < 8; ++k) mp[k] = -INFINITY;
+      for (int k = 0; k < 8; ++k) {
 #pragma unroll
-      for (int i = 0; i < 64; ++i) {
-        s[i] = ((mk >> i) & 1ull) ? s[i] * p.scale_log2 : -INFINITY;
-        mp[i & 7] = fmaxf(mp[i & 7], s[i]);
-      }
-      const float mt = fmaxf(fmaxf(fmaxf(mp[0], mp[1]), fmaxf(mp[2], mp[3])),
-                             fmaxf(fmaxf(mp[4], mp[5]), fmaxf(mp[6], mp[7])));
-      float alpha = 1.f;
-      bool resc = false;
-      if (m_ref == -INFINITY) {
-        m_ref = mt;  // nothing accumulated yet (all earlier weights were zero)
-      } else if (mt > m_ref + kRescaleThreshold) {
-        alpha = exp2f(m_ref - mt);
-        m_ref = mt;
-        resc = true;
-      }
-      float ps[8];
-#pragma unroll
-      for (int k = 0; k < 8; ++k) ps[k] = 0.f;
-      if (m_ref == -INFINITY) {  // every slot so far is empty: all weights are zero
-#pragma unroll
-        for (int i = 0; i < 64; ++i) s[i] = 0.f;
-      } else {
-#pragma unroll
-        for (int i = 0; i < 64; ++i) {
-          s[i] = fast_exp2(s[i] - m_ref);
-          ps[i & 7] += s[i];
+        for (int e = 0; e < 2; ++e) {
+          const bool valid = (mk >> (8 * k + 2 * m4 + e)) & 1ull;
+          x[0][2 * k + e] = valid ? r[4 * k + e] * p.scale_log2 : -INFINITY;
+          x[1][2 * k + e] = valid ? r[4 * k + 2 + e] * p.scale_log2 : -INFINITY;
         }
       }
-      const float psum = ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7]));
-      l_run = l_run * alpha + psum;
+      float alpha[2];
+      bool resc = false;
+#pragma unroll
+      for (int i = 0; i < 2; ++i) {
+        float mp[4];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) mp[c] = fmaxf(fmaxf(x[i][4 * c], x[i][4 * c + 1]), fmaxf(x[i][4 * c + 2], x[i][4 * c + 3]));
+        float mt = fmaxf(fmaxf(mp[0], mp[1]), fmaxf(mp[2], mp[3]));
+        mt = fmaxf(mt, __shfl_xor_sync(0xFFFFFFFFu, mt, 1));
+        mt = fmaxf(mt, __shfl_xor_sync(0xFFFFFFFFu, mt, 2));
+        alpha[i] = 1.f;
+        if (m_ref[i] == -INFINITY) {
+          m_ref[i] = mt;  // nothing accumulated yet (all earlier weights were zero)
+        } else if (mt > m_ref[i] + kRescaleThreshold) {
+          alpha[i] = exp2f(m_ref[i] - mt);
+          m_ref[i] = mt;
+          resc = true;
+        }
+        float ps[4] = {0.f, 0.f, 0.f, 0.f};
+        if (m_ref[i] == -INFINITY) {  // every slot so far is empty: all weights are zero
+#pragma unroll
+          for (int c = 0; c < 16; ++c) x[i][c] = 0.f;
+        } else {
+#pragma unroll
+          for (int c = 0; c < 16; ++c) {
+            x[i][c] = fast_exp2(x[i][c] - m_ref[i]);
+            ps[c & 3] += x[i][c];
+          }
+        }
+        float psum = (ps[0] + ps[1]) + (ps[2] + ps[3]);
+        psum += __shfl_xor_sync(0xFFFFFFFFu, psum, 1);
+        psum += __shfl_xor_sync(0xFFFFFFFFu, psum, 2);
+        l_run[i] = l_run[i] * alpha[i] + psum;
+      }
       // PV_{j-1} must be done before P and O are touched.
       if (!(ok = mbar_wait(p_free, static_cast<uint32_t>(j & 1) ^ 1u, abort_flag))) break;
       tc_fence_after();
-      if (owner) head_f[head] = alpha;
-      if (named_barrier_or(1, kSoftmaxThreads, owner && resc)) {
+      if (m4 == 0) {
+        head_f[hrow[0]] = alpha[0];
+        head_f[hrow[1]] = alpha[1];
+      }
+      if (named_barrier_or(1, kSoftmaxThreads, resc)) {
         // O^T[dim][head] *= alpha[head]: every lane holds one dim of each block
         for (int blk = 0; blk < 4; ++blk) {
           for (int c = 0; c < 2; ++c) {
@@ -454,22 +499,21 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         named_barrier(1, kSoftmaxThreads);
       }
-      if (owner) {
-        // P[head][row] in the 128-byte-swizzled K-major layout (8 heads per 1 KB atom)
-        const uint32_t rbase = (head >> 3) * 1024 + (head & 7) * 128;
+      // P[head][row] in the 128-byte-swizzled K-major layout (8 heads per 1 KB
+      // atom); this thread writes the bf16 pairs of columns 8k + 2 m4, +1.
 #pragma unroll
-        for (int c8 = 0; c8 < 8; ++c8) {
-          uint32_t hi[4], lo[4];
+      for (int i = 0; i < 2; ++i) {
+        const int h = hrow[i];
+        const uint32_t rbase = (h >> 3) * 1024 + (h & 7) * 128 + 4 * m4;
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const float x0 = s[8 * c8 + 2 * e], x1 = s[8 * c8 + 2 * e + 1];
-            hi[e] = pack_bf16(x0, x1);
-            const float h0 = __uint_as_float(hi[e] << 16), h1 = __uint_as_float(hi[e] & 0xFFFF0000u);
-            lo[e] = pack_bf16(x0 - h0, x1 - h1);
-          }
-          const uint32_t off = rbase + ((c8 ^ (head & 7)) << 4);
-          *reinterpret_cast<uint4*>(p_hi_ptr + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
-          *reinterpret_cast<uint4*>(p_hi_ptr + kPBytes + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+        for (int k = 0; k < 8; ++k) {
+          const float x0 = x[i][2 * k], x1 = x[i][2 * k + 1];
+          const uint32_t hi = pack_bf16(x0, x1);
+          const float h0 = __uint_as_float(hi << 16), h1 = __uint_as_float(hi & 0xFFFF0000u);
+          const uint32_t lo = pack_bf16(x0 - h0, x1 - h1);
+          const uint32_t off = rbase + ((k ^ (h & 7)) << 4);
+          *reinterpret_cast<uint32_t*>(p_hi_ptr + off) = hi;
+          *reinterpret_cast<uint32_t*>(p_hi_ptr + kPBytes + off) = lo;
         }
       }
       fence_proxy_async_smem();
@@ -481,7 +525,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       record_status(p.status, kStatusTimeout);
       *abort_flag = 1;
     }
-    if (owner) own_ml[head] = make_float2(m_ref, l_run);
+    if (m4 == 0) {
+      own_ml[hrow[0]] = make_float2(m_ref[0], l_run[0]);
+      own_ml[hrow[1]] = make_float2(m_ref[1], l_run[1]);
+    }
   }
 
   // ---- split merge: out = g / L * sum_r 2^(m_r - M) O_r with M = max_r m_r and
