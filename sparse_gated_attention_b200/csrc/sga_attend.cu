@@ -33,13 +33,12 @@
 //     gather4 quad gathers the sequence's row 0 and is masked out of the
 //     softmax.  Warp 0 also publishes the validity mask of each chunk and
 //     loads Q.
-//     Warp 4 issues the MMAs without blocking on any one operand: it polls
-//     the barriers and issues PV(j) as soon as P_j is written, between the
-//     value pairs of QK^T(j+1), so value slots are released (and refilled)
-//     as early as the softmax allows.  Warps 5-8 (one per TMEM lane quarter,
+//     Warp 4 issues QK^T, polling its barriers so it never waits on one
+//     operand while another is ready.  Warps 5-8 (one per TMEM lane quarter,
 //     16 heads each) run the softmax in the log2 domain with a lazy running
-//     max (O is rescaled only when the max grows by more than 2^8) and the
-//     epilogue.
+//     max (O is rescaled only when the max grows by more than 2^8); once P_j
+//     is written, one of their threads issues PV(j) itself, so value slots
+//     are released (and refilled) without a round trip through the MMA warp.
 //   * TMEM (512 columns): O^T in columns 0..255 (dim block b at 64 b, all
 //     lanes), S buffers at columns 256 and 320 (M = 64 layout: lanes 0-15 of
 //     each quarter).
@@ -76,11 +75,12 @@ constexpr int kProducerWarps = 4;          // warps 0-3
 constexpr int kProducers = 32 * kProducerWarps;
 constexpr int kMmaWarp = 4;
 constexpr int kSoftmaxThreads = 128;        // warps 5-8
+constexpr int kPvThread = (4 + 1) * 32;     // the softmax thread that issues PV
 constexpr int kThreads = 288;
 constexpr int kTmemCols = 512;
 constexpr int kSCol = 256;
 // barriers: pair_full[8] pair_empty[8] rope_full rope_empty q_full s_full[2] s_free[2]
-//           p_full p_free o_full mask_full[4] mask_empty[4]
+//           qk_done p_free o_full mask_full[4] mask_empty[4]
 constexpr int kNumBars = 2 * kPairRing + 2 + 1 + 2 + 2 + 3 + 2 * kMaskRing;
 constexpr int kMaxSplits = 8;               // splits of a query = CTAs of its cluster
 constexpr size_t kSmemBytes = 1024 + kPairRing * kPairBytes + kBoxBytes + kQBytes + 2 * kPBytes + kNumBars * 8 +
@@ -135,7 +135,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t q_full = rope_full + 16u;
   auto s_full = [&](int b) { return q_full + 8u * (1 + b); };
   auto s_free = [&](int b) { return q_full + 8u * (3 + b); };
-  const uint32_t p_full = q_full + 8u * 5;
+  const uint32_t qk_done = q_full + 8u * 5;  // every QK^T MMA of the MMA warp has finished
   const uint32_t p_free = q_full + 8u * 6;
   const uint32_t o_full = q_full + 8u * 7;
   auto mask_full = [&](int b) { return q_full + 8u * (8 + b); };
@@ -168,7 +168,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(s_full(b), 1);
       mbar_init(s_free(b), kSoftmaxThreads);
     }
-    mbar_init(p_full, kSoftmaxThreads);
+    mbar_init(qk_done, 1);
     mbar_init(p_free, 1);
     mbar_init(o_full, 1);
     for (int b = 0; b < kMaskRing; ++b) {
@@ -317,80 +317,52 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       constexpr uint32_t idesc_qk = idesc_bf16_f32(kHeads, kChunk, false, false);
-      constexpr uint32_t idesc_pv = idesc_bf16_f32(128, kHeads, true, false);
       bool ok = mbar_wait(q_full, 0, abort_flag);
-      // PV(j): O^T[dims 128 q ..][heads] += V_j^T (P_hi + P_lo)^T, one accumulator block per value pair
-      auto issue_pv = [&](int j) {
-        for (int q = 0; q < kPairsPerChunk; ++q) {
-          const int slot = (j * kPairsPerChunk + q) % kPairRing;
-          const uint32_t base = pairs + slot * kPairBytes;
-          const uint32_t d = tmem + q * kHeads;
-#pragma unroll
-          for (int kk = 0; kk < 4; ++kk) {
-            // A = V^T: M = 128 dims over the pair's two boxes, K = rows 16 kk ..
-            const uint64_t adesc = sdesc_sw128(base + kk * 2048, kBoxBytes, 1024);
-#pragma unroll
-            for (int part = 0; part < 2; ++part) {
-              const uint64_t bdesc = sdesc_sw128((part ? p_lo : p_hi) + kk * 32, 16, 1024);
-              mma_bf16(d, adesc, bdesc, idesc_pv, (j > 0 || kk > 0 || part > 0) ? 1u : 0u);
-            }
-          }
-          mma_commit(pair_empty(slot));
-        }
-        mma_commit(p_free);
-      };
-      // Non-blocking issue: PV(pv_j) as soon as P is written, else the next
-      // piece of QK^T(qk_j) (part 0: rope box once S buffer and rope slot are
-      // ready; parts 1-4: one value pair each).
-      int qk_j = 0, qk_part = 0, pv_j = 0;
+      // Non-blocking issue of QK^T(qk_j), piece by piece: part 0 is the rope
+      // box (once the S buffer and the rope slot are ready), parts 1-4 one
+      // value pair each.
+      int qk_j = 0, qk_part = 0;
       long long idle_since = clock64();
-      while (ok && pv_j < nchunks) {
+      while (ok && qk_j < nchunks) {
         bool did = false;
-        if (pv_j < qk_j && mbar_test_wait(p_full, static_cast<uint32_t>(pv_j & 1))) {
-          tc_fence_after();
-          issue_pv(pv_j);
-          ++pv_j;
-          did = true;
-        } else if (qk_j < nchunks) {
-          const int sb = qk_j & 1;
-          const uint32_t d = tmem + kSCol + sb * kChunk;
-          if (qk_part == 0) {
-            if (mbar_test_wait(s_free(sb), static_cast<uint32_t>((qk_j >> 1) & 1) ^ 1u) &&
-                mbar_test_wait(rope_full, static_cast<uint32_t>(qk_j & 1))) {
-              fence_proxy_async_smem();  // written by cp.async (generic proxy)
-              tc_fence_after();
+        const int sb = qk_j & 1;
+        const uint32_t d = tmem + kSCol + sb * kChunk;
+        if (qk_part == 0) {
+          if (mbar_test_wait(s_free(sb), static_cast<uint32_t>((qk_j >> 1) & 1) ^ 1u) &&
+              mbar_test_wait(rope_full, static_cast<uint32_t>(qk_j & 1))) {
+            fence_proxy_async_smem();  // written by cp.async (generic proxy)
+            tc_fence_after();
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+              mma_bf16(d, sdesc_sw128(q_s + 8 * kQBox + kk * 32, 16, 1024), sdesc_sw128(rope + kk * 32, 16, 1024),
+                       idesc_qk, kk > 0 ? 1u : 0u);
+            mma_commit(rope_empty);  // rope dims are not needed for P V
+            qk_part = 1;
+            did = true;
+          }
+        } else {
+          const int q = qk_part - 1;
+          const int n = qk_j * kPairsPerChunk + q;
+          const int slot = n % kPairRing;
+          if (mbar_test_wait(pair_full(slot), static_cast<uint32_t>((n / kPairRing) & 1))) {
+            fence_proxy_async_smem();
+            tc_fence_after();
+            const uint32_t base = pairs + slot * kPairBytes;
+#pragma unroll
+            for (int bx = 0; bx < 2; ++bx) {
 #pragma unroll
               for (int kk = 0; kk < 4; ++kk)
-                mma_bf16(d, sdesc_sw128(q_s + 8 * kQBox + kk * 32, 16, 1024), sdesc_sw128(rope + kk * 32, 16, 1024),
-                         idesc_qk, kk > 0 ? 1u : 0u);
-              mma_commit(rope_empty);  // rope dims are not needed for P V
-              qk_part = 1;
-              did = true;
+                mma_bf16(d, sdesc_sw128(q_s + (2 * q + bx) * kQBox + kk * 32, 16, 1024),
+                         sdesc_sw128(base + bx * kBoxBytes + kk * 32, 16, 1024), idesc_qk, 1u);
             }
-          } else {
-            const int q = qk_part - 1;
-            const int n = qk_j * kPairsPerChunk + q;
-            const int slot = n % kPairRing;
-            if (mbar_test_wait(pair_full(slot), static_cast<uint32_t>((n / kPairRing) & 1))) {
-              fence_proxy_async_smem();
-              tc_fence_after();
-              const uint32_t base = pairs + slot * kPairBytes;
-#pragma unroll
-              for (int bx = 0; bx < 2; ++bx) {
-#pragma unroll
-                for (int kk = 0; kk < 4; ++kk)
-                  mma_bf16(d, sdesc_sw128(q_s + (2 * q + bx) * kQBox + kk * 32, 16, 1024),
-                           sdesc_sw128(base + bx * kBoxBytes + kk * 32, 16, 1024), idesc_qk, 1u);
-              }
-              if (qk_part == kPairsPerChunk) {
-                mma_commit(s_full(sb));
-                ++qk_j;
-                qk_part = 0;
-              } else {
-                ++qk_part;
-              }
-              did = true;
+            if (qk_part == kPairsPerChunk) {
+              mma_commit(s_full(sb));
+              ++qk_j;
+              qk_part = 0;
+            } else {
+              ++qk_part;
             }
+            did = true;
           }
         }
         if (did) {
@@ -403,11 +375,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         record_status(p.status, kStatusTimeout);
         *abort_flag = 1;
       }
-      mma_commit(o_full);
-      if (!ok) {
-        volatile int never = 0;
-        mbar_wait(o_full, 0, &never);
-      }
+      mma_commit(qk_done);
+      volatile int never = 0;
+      mbar_wait(qk_done, 0, &never);  // every MMA this thread issued has finished
     }
   } else {
     // ------------------------------------------------------------ softmax
@@ -421,17 +391,20 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int m4 = lane & 3;
     const int hrow[2] = {quarter * 16 + (lane >> 2), quarter * 16 + 8 + (lane >> 2)};  // this thread's two heads
     float m_ref[2] = {-INFINITY, -INFINITY}, l_run[2] = {0.f, 0.f};
+    // Every softmax thread runs every iteration, even after a wait ran out
+    // (the abort flag then makes each later wait return at once), so the
+    // named barriers below always see all 128 threads.
     bool ok = true;
     for (int j = 0; j < nchunks; ++j) {
       const int sb = j & 1;
-      if (!(ok = mbar_wait(s_full(sb), static_cast<uint32_t>((j >> 1) & 1), abort_flag))) break;
+      ok = ok && mbar_wait(s_full(sb), static_cast<uint32_t>((j >> 1) & 1), abort_flag);
       tc_fence_after();
       float r[32];
       tmem_ld_16x256b_x8(tmem + lane_addr + kSCol + sb * kChunk, r);
       tc_fence_before();
       mbar_arrive(s_free(sb));
       const int mb = j % kMaskRing;
-      if (!(ok = mbar_wait(mask_full(mb), static_cast<uint32_t>((j / kMaskRing) & 1), abort_flag))) break;
+      ok = ok && mbar_wait(mask_full(mb), static_cast<uint32_t>((j / kMaskRing) & 1), abort_flag);
       const uint64_t mk = masks[mb];
       mbar_arrive(mask_empty(mb));
       // x[i][2k + e] = score of row i at column 8k + 2 m4 + e (masked slots -> -inf)
@@ -480,7 +453,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         l_run[i] = l_run[i] * alpha[i] + psum;
       }
       // PV_{j-1} must be done before P and O are touched.
-      if (!(ok = mbar_wait(p_free, static_cast<uint32_t>(j & 1) ^ 1u, abort_flag))) break;
+      ok = ok && mbar_wait(p_free, static_cast<uint32_t>(j & 1) ^ 1u, abort_flag);
       tc_fence_after();
       if (m4 == 0) {
         head_f[hrow[0]] = alpha[0];
@@ -518,12 +491,39 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       fence_proxy_async_smem();
       tc_fence_before();
-      mbar_arrive(p_full);
+      named_barrier(2, kSoftmaxThreads);  // P_j (and any rescale of O) complete
+      if (threadIdx.x == kPvThread) {
+        // PV(j): O^T[dims 128 q ..][heads] += V_j^T (P_hi + P_lo)^T, one accumulator block per value pair
+        constexpr uint32_t idesc_pv = idesc_bf16_f32(128, kHeads, true, false);
+        tc_fence_after();
+        for (int q = 0; q < kPairsPerChunk; ++q) {
+          const int slot = (j * kPairsPerChunk + q) % kPairRing;
+          const uint32_t base = pairs + slot * kPairBytes;
+          const uint32_t d = tmem + q * kHeads;
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk) {
+            // A = V^T: M = 128 dims over the pair's two boxes, K = rows 16 kk ..
+            const uint64_t adesc = sdesc_sw128(base + kk * 2048, kBoxBytes, 1024);
+#pragma unroll
+            for (int part = 0; part < 2; ++part) {
+              const uint64_t bdesc = sdesc_sw128((part ? p_lo : p_hi) + kk * 32, 16, 1024);
+              mma_bf16(d, adesc, bdesc, idesc_pv, (j > 0 || kk > 0 || part > 0) ? 1u : 0u);
+            }
+          }
+          mma_commit(pair_empty(slot));
+        }
+        mma_commit(p_free);
+      }
     }
+    if (threadIdx.x == kPvThread) mma_commit(o_full);  // every PV this thread issued
     const bool have_o = ok && mbar_wait(o_full, 0, abort_flag);
     if (!have_o) {
       record_status(p.status, kStatusTimeout);
       *abort_flag = 1;
+      if (threadIdx.x == kPvThread) {  // its MMAs must be done before TMEM is freed
+        volatile int never = 0;
+        mbar_wait(o_full, 0, &never);
+      }
     }
     if (m4 == 0) {
       own_ml[hrow[0]] = make_float2(m_ref[0], l_run[0]);
