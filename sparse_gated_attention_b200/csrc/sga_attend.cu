@@ -88,7 +88,10 @@ constexpr size_t kSmemBytes = 1024 + kPairRing * kPairBytes + kBoxBytes + kQByte
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 
 static_assert(kSmemBytes <= 232448, "shared memory budget");
-static_assert(kPairRing * kPairBytes == kHeads * kDv * 4, "the value ring stages one CTA's O for the split merge");
+// the split merge's receive buffer ([S][64][4 ceil(128 / S)] fp32, at most 136 KB for S <= 8, largest at
+// S = 7) lies over the value ring, the rope slot and the Q buffer, which are contiguous and idle once every
+// MMA has finished
+static_assert(kPairRing * kPairBytes + kBoxBytes + kQBytes >= 7 * kHeads * 76 * 4, "split merge receive buffer");
 
 struct AttendParams {
   const uint16_t* kv;
@@ -535,7 +538,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   // L = sum_r 2^(m_r - M) l_r (per head).  Every thread of the cluster takes
   // part in its barriers, on every path.
   const int S = p.splits;
-  float* o_stage = reinterpret_cast<float*>(smem);  // [64][512] fp32 in the value ring
+  float* o_stage = reinterpret_cast<float*>(smem);  // value ring + rope slot + Q buffer, idle after the MMAs
   if (S > 1) {
     cluster.sync();  // every split's (m, l) published; all MMAs of every CTA done
   } else {
@@ -567,6 +570,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     head_f[head] = f;
   }
   __syncthreads();
+  // With several splits, CTA r owns the float4 columns [v0(r), v0(r+1)) of
+  // every head's 512 dims, v0(r) = 128 r / S.  Every CTA pushes its scaled O
+  // for those dims into the owner's receive buffer with remote stores (a
+  // warp writes 32 consecutive dims of one head: one 128-byte line per
+  // store), laid out [source split][head][kStride] fp32 over the owner's idle
+  // value ring, rope slot and Q buffer; after one cluster barrier each owner
+  // sums its S buffers locally.  No CTA reads another's shared memory after
+  // that barrier.
+  const int kStride = 4 * ((kDv / 4 + S - 1) / S);  // floats per (source, head) row: the widest slice
+  float* recv = o_stage;
   if (warp < kProducerWarps || warp > kMmaWarp) {
     // Eight warps read O^T out of TMEM: warp w reads lane quarter w % 4; the
     // producer warps take dim blocks 0-1, the softmax warps blocks 2-3.
@@ -574,7 +587,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int quarter = warp & 3;
     const uint32_t lane_addr = static_cast<uint32_t>(quarter * 32) << 16;
     const int blk0 = warp < kProducerWarps ? 0 : 2;
-    float* dst = S == 1 ? p.out + static_cast<size_t>(row) * kHeads * kDv : o_stage;
     tc_fence_after();
     for (int c = 0; c < 2; ++c) {
       float hf[32];
@@ -584,49 +596,39 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int dim = 128 * blk + 32 * quarter + lane;
         float o[32];
         tmem_ld32(tmem + lane_addr + blk * kHeads + c * 32, o);
-        float* col = dst + static_cast<size_t>(c * 32) * kDv + dim;
+        float* col;
+        if (S == 1) {
+          col = p.out + static_cast<size_t>(row) * kHeads * kDv + static_cast<size_t>(c * 32) * kDv + dim;
 #pragma unroll
-        for (int i = 0; i < 32; ++i) col[static_cast<size_t>(i) * kDv] = o[i] * hf[i];
+          for (int i = 0; i < 32; ++i) col[static_cast<size_t>(i) * kDv] = o[i] * hf[i];
+        } else {
+          const int v = dim >> 2;
+          const int owner = ((v + 1) * S - 1) / (kDv / 4);  // the r with v0(r) <= v < v0(r + 1)
+          const int dl = dim - 4 * ((kDv / 4) * owner / S);
+          col = cluster.map_shared_rank(recv + (split * kHeads + c * 32) * kStride + dl, owner);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) col[i * kStride] = o[i] * hf[i];
+        }
       }
     }
   }
   if (S > 1) {
-    cluster.sync();  // every split's scaled O staged
-    // this CTA sums and writes the float4 columns [v0, v1) of every head's 512 dims
+    cluster.sync();  // every split's scaled O delivered to its owners
     const int v0 = (kDv / 4) * split / S, v1 = (kDv / 4) * (split + 1) / S;
     const int vecs = v1 - v0;
     float* orow = p.out + static_cast<size_t>(row) * kHeads * kDv;
-    constexpr int kUnroll = 4;  // elements per thread in flight
-    for (int e0 = threadIdx.x; e0 < kHeads * vecs; e0 += kUnroll * kThreads) {
-      float4 acc[kUnroll];
-      int off[kUnroll];
-#pragma unroll
-      for (int u = 0; u < kUnroll; ++u) {
-        const int e = e0 + u * kThreads;
-        const int h = e / vecs;
-        off[u] = h * kDv + 4 * (v0 + e - h * vecs);
-        acc[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int e = threadIdx.x; e < kHeads * vecs; e += kThreads) {
+      const int h = e / vecs, dv = e - h * vecs;
+      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int r = 0; r < S; ++r) {
+        const float4 x = *reinterpret_cast<const float4*>(recv + (r * kHeads + h) * kStride + 4 * dv);
+        acc.x += x.x;
+        acc.y += x.y;
+        acc.z += x.z;
+        acc.w += x.w;
       }
-#pragma unroll
-      for (int r = 0; r < kMaxSplits; ++r) {
-        if (r < S) {
-#pragma unroll
-          for (int u = 0; u < kUnroll; ++u) {
-            if (e0 + u * kThreads < kHeads * vecs) {
-              const float4 x = *reinterpret_cast<const float4*>(cluster.map_shared_rank(o_stage + off[u], r));
-              acc[u].x += x.x;
-              acc[u].y += x.y;
-              acc[u].z += x.z;
-              acc[u].w += x.w;
-            }
-          }
-        }
-      }
-#pragma unroll
-      for (int u = 0; u < kUnroll; ++u)
-        if (e0 + u * kThreads < kHeads * vecs) *reinterpret_cast<float4*>(orow + off[u]) = acc[u];
+      *reinterpret_cast<float4*>(orow + h * kDv + 4 * (v0 + dv)) = acc;
     }
-    cluster.sync();  // no CTA leaves while another reads its staging
   }
 
   tc_fence_before();
