@@ -46,15 +46,15 @@ def parse_args():
     return ap.parse_args()
 
 
-def algorithmic_bytes_per_query(ctx: int, top_k: int = 2048) -> dict:
+def algorithmic_bytes_per_query(ctx: int, top_k: int = 2048, key_bytes: int = 2) -> dict:
     """Bytes the method must move per decode query (intermediate scores excluded).
 
-    k_idx: every causal key once (ctx * 128 * 2), q_idx 64*128*2, w 64*2,
-    gathered latent rows top_k * 576 * 2, q 64*576*2, gate 64*2, out 64*512*4,
-    idx top_k * 4.
+    k_idx: every causal key once (ctx * 128 * key_bytes: 2 for bf16, 1 for E4M3),
+    q_idx 64*128*key_bytes, w 64*2, gathered latent rows top_k * 576 * 2,
+    q 64*576*2, gate 64*2, out 64*512*4, idx top_k * 4.
     """
-    parts = dict(k_idx=ctx * 256, q_idx=16384, w=128, kv_rows=top_k * 1152, q=73728, gate=128, out=131072,
-                 idx=top_k * 4)
+    parts = dict(k_idx=ctx * 128 * key_bytes, q_idx=8192 * key_bytes, w=128, kv_rows=top_k * 1152, q=73728,
+                 gate=128, out=131072, idx=top_k * 4)
     parts["total"] = sum(parts.values())
     parts["indexer"] = parts["k_idx"] + parts["q_idx"] + parts["w"]
     return parts
@@ -249,7 +249,8 @@ def main():
     out = torch.empty((B, T, 64, 512), dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream(dev)
     att_ws_bytes = sga.workspace_size(dims, sga.OP_SPARSE_MLA_ATTEND)
-    launches_per_step = 3 + (1 if att_ws_bytes > 256 else 0)  # indexer, top-k, attention (+ split combine)
+    launches_per_step = 3  # indexer, top-k, attention (the attention needs no workspace beyond the status word)
+    assert att_ws_bytes == 256
 
     def fwd_step():
         sga.forward(x["q_idx"], x["w"], x["k_idx"], x["q"], x["kv"], x["gate"], x["q_pos"], top_k=K, idx_out=idx,
@@ -334,6 +335,35 @@ def main():
     if sga.device_status(ws_all) != 0:
         raise RuntimeError("device status set during the end-to-end run")
 
+    # ---- the E4M3 indexer-key variant (a separate configuration, reported beside
+    # the headline): the same workload with q_idx and k_idx stored as E4M3
+    # (exact for the integer-valued inputs), timed like the main region.
+    xf = {"q_idx": synth.to_e4m3(x["q_idx"]), "k_idx": synth.to_e4m3(x["k_idx"])}
+
+    def fp8_step():
+        sga.forward_fp8(xf["q_idx"], x["w"], xf["k_idx"], x["q"], x["kv"], x["gate"], x["q_pos"], top_k=K,
+                        idx_out=idx, out=out, ws=ws_all, stream=stream)
+
+    for _ in range(max(args.warmup, 3)):
+        fp8_step()
+    torch.cuda.synchronize(dev)
+    if dist is not None:
+        dist.barrier()
+    s3, e3 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s3.record(stream)
+    for _ in range(args.steps):
+        fp8_step()
+    e3.record(stream)
+    torch.cuda.synchronize(dev)
+    fp8_ms = s3.elapsed_time(e3)
+    if dist is not None:
+        t = torch.tensor([fp8_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        fp8_ms = float(t.item())
+    if sga.device_status(ws_all) != 0:
+        raise RuntimeError("device status set during the E4M3 variant run")
+    del xf
+
     if dist is not None:
         dist.barrier()
         dist.destroy_process_group()
@@ -353,6 +383,16 @@ def main():
     if counters and counters.get("workload") == wl.name:
         traffic = counters.get("dram_bytes_per_launch")
     path_gbs = ab["total"] * rows / (ms_per_step * 1e-3) / 1e9
+
+    ab8 = algorithmic_bytes_per_query(L, K, key_bytes=1)
+    fp8_step_ms = fp8_ms / args.steps
+    fp8_gbs = ab8["total"] * rows / (fp8_step_ms * 1e-3) / 1e9
+    variants = {"fp8_index_keys": {
+        "value": total_queries / (fp8_ms / 1e3), "unit": UNIT, "ms_per_step": fp8_step_ms,
+        "config": f"{wl.name} with q_idx and k_idx stored as E4M3 (exact for the integer-valued inputs)",
+        "path_roofline": {"achieved_gbs": fp8_gbs, "frac_of_8tbs": fp8_gbs / NOMINAL_HBM_GBS,
+                          "frac_of_measured": fp8_gbs / peak, "bytes_per_query": ab8["total"]},
+        "gpu_launches": launches_per_step * args.steps}}
 
     cpu = None
     if not args.no_cpu_baseline and world == 1:
@@ -376,6 +416,7 @@ def main():
                 "d2h_bytes_per_step": d2h},
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clk.summary(),
+        "variants": variants,
     }
     print(json.dumps(line), flush=True)
 

@@ -62,6 +62,8 @@ extern "C" {
 #endif
 
 typedef uint16_t sga_bf16_t; /* bfloat16 bit pattern */
+typedef uint8_t sga_fp8_e4m3_t; /* FP8 E4M3 bit pattern: 1 sign, 4 exponent (bias 7), 3 mantissa bits;
+                                  no infinities, 0x7F / 0xFF are NaN, largest finite 448 */
 typedef void* sga_stream_t;  /* cudaStream_t */
 
 typedef enum {
@@ -156,6 +158,22 @@ SGA_API sga_status_t sga_forward(const sga_dims_t* dims, const sga_bf16_t* q_idx
                          const sga_bf16_t* k_idx, const sga_bf16_t* q, const sga_bf16_t* kv,
                          const sga_bf16_t* gate, const int32_t* q_pos, int32_t* idx_out, float* out, void* ws,
                          size_t ws_bytes, sga_stream_t stream);
+
+/* The indexer and the whole path with an E4M3 indexer-key cache (archdb "A.X
+ * K2": the indexer key is the 128 values per token cached beside the KV;
+ * its pretraining-precision field gives E4M3 matmuls; nlp.com.ai "A.X K2 FP8"
+ * releases the model in FP8).  q_idx [B][T][64][128] and k_idx [B][L][128]
+ * hold E4M3 bytes, used as their exact values with no block scale (so a key
+ * row is 128 B instead of 256 B); everything else, the workspace and the
+ * results are as for sga_index_scores / sga_forward.  Products of E4M3 values
+ * are exact in fp32, and integer-valued inputs keep exact scores. */
+SGA_API sga_status_t sga_index_scores_fp8(const sga_dims_t* dims, const sga_fp8_e4m3_t* q_idx, const sga_bf16_t* w,
+                                  const sga_fp8_e4m3_t* k_idx, const int32_t* q_pos, float* scores, void* ws,
+                                  size_t ws_bytes, sga_stream_t stream);
+SGA_API sga_status_t sga_forward_fp8(const sga_dims_t* dims, const sga_fp8_e4m3_t* q_idx, const sga_bf16_t* w,
+                             const sga_fp8_e4m3_t* k_idx, const sga_bf16_t* q, const sga_bf16_t* kv,
+                             const sga_bf16_t* gate, const int32_t* q_pos, int32_t* idx_out, float* out, void* ws,
+                             size_t ws_bytes, sga_stream_t stream);
 
 /* Synchronises `stream` and returns in *device_status the first device-side
  * error recorded in the workspace (an sga_status_t value, SGA_OK if none). */

@@ -20,6 +20,12 @@ Each function follows one step of the method:
   "A.X K2" attention fields: 64 heads, qk head dim 192, latent 512 + rope 64)
   followed by the head-specific sigmoid output gate (archdb "A.X K2" gate field).
 * ``forward`` - the three in sequence.
+* ``e4m3_to_float64`` / ``index_scores_e4m3`` / ``forward_e4m3`` - the same
+  path with an FP8 (E4M3) indexer-key cache (archdb "A.X K2": E4M3 matmuls in
+  its pretraining-precision field; nlp.com.ai "A.X K2 FP8"), reading each
+  E4M3 code as its exact value with no block scale.  Every finite E4M3 value is
+  a bf16 value, so the codes are converted exactly and the bf16 oracle runs
+  unchanged.
 
 Pins: every function is checked in ``tests/test_oracle_pins.py`` against closed
 forms, invariants, a hand-worked fixture and library routines (numpy matmul,
@@ -118,6 +124,48 @@ def index_scores(q_idx, w, k_idx, q_pos, n_threads: int = 0) -> np.ndarray:
     return out
 
 
+def e4m3_to_float64(codes) -> np.ndarray:
+    """FP8 E4M3 bit patterns -> exact values.
+
+    The format: 1 sign bit, 4 exponent bits (bias 7), 3 mantissa bits.  An
+    exponent field e > 0 gives (1 + m/8) * 2^(e-7); e = 0 is subnormal,
+    (m/8) * 2^-6.  There are no infinities; S.1111.111 is NaN, so the largest
+    finite value is 1.75 * 2^8 = 448.
+    """
+    c = np.asarray(codes, dtype=np.uint8).astype(np.int64)
+    sign = np.where(c & 0x80, -1.0, 1.0)
+    e = (c >> 3) & 0xF
+    m = (c & 0x7).astype(np.float64)
+    mag = np.where(e == 0, (m / 8.0) * 2.0 ** -6, (1.0 + m / 8.0) * np.exp2((e - 7).astype(np.float64)))
+    return np.where((e == 15) & (c & 0x7 == 7), np.nan, sign * mag)
+
+
+def e4m3_to_bf16_bits(codes) -> np.ndarray:
+    """FP8 E4M3 codes -> bf16 bit patterns of the same values.  Exact: a finite
+    E4M3 value has at most 4 significant bits and an exponent in [-9, 8]."""
+    v = e4m3_to_float64(codes).astype(np.float32)
+    return (v.view(np.uint32) >> 16).astype(np.uint16)
+
+
+def _codes(a) -> np.ndarray:
+    if hasattr(a, "cpu"):
+        a = a.detach().cpu().contiguous()
+        if str(a.dtype) == "torch.float8_e4m3fn":
+            import torch
+
+            a = a.view(torch.uint8)
+        a = a.numpy()
+    arr = np.ascontiguousarray(a)
+    if arr.dtype != np.uint8:
+        raise TypeError(f"expected E4M3 codes (uint8), got {arr.dtype}")
+    return arr
+
+
+def index_scores_e4m3(q_idx, w, k_idx, q_pos, n_threads: int = 0) -> np.ndarray:
+    """index_scores with E4M3 indexer queries [B,T,Hi,Di] and keys [B,L,Di] (codes)."""
+    return index_scores(e4m3_to_bf16_bits(_codes(q_idx)), w, e4m3_to_bf16_bits(_codes(k_idx)), q_pos, n_threads)
+
+
 def topk(scores, q_pos, k: int = TOP_K, n_threads: int = 0) -> np.ndarray:
     """Top-k positions per row (ties -> lower position), ascending, -1 padded.
 
@@ -175,3 +223,10 @@ def forward(q_idx, w, k_idx, q, kv, gate, q_pos, k: int = TOP_K, scale: float = 
     if rc:
         raise ValueError("oracle_forward: bad arguments")
     return idx, out
+
+
+def forward_e4m3(q_idx, w, k_idx, q, kv, gate, q_pos, k: int = TOP_K, scale: float = SCALE, v_dim: int = V_DIM,
+                 n_threads: int = 0):
+    """forward with E4M3 indexer queries and keys (codes); returns (idx, out) as forward does."""
+    return forward(e4m3_to_bf16_bits(_codes(q_idx)), w, e4m3_to_bf16_bits(_codes(k_idx)), q, kv, gate, q_pos, k=k,
+                   scale=scale, v_dim=v_dim, n_threads=n_threads)

@@ -22,7 +22,9 @@ from ._binding import (  # noqa: F401
     clear_device_status,
     device_status,
     forward,
+    forward_fp8,
     index_scores,
+    index_scores_fp8,
     load_library,
     make_dims,
     sparse_mla_attend,

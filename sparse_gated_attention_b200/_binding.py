@@ -29,7 +29,7 @@ STATUS_NAMES = {0: "SGA_OK", 1: "SGA_ERR_INVALID_ARG", 2: "SGA_ERR_UNSUPPORTED",
 
 EXPORTED = ["sga_abi_version", "sga_status_string", "sga_workspace_size", "sga_index_scores", "sga_topk_select",
             "sga_sparse_mla_attend", "sga_forward", "sga_get_device_status", "sga_clear_device_status",
-            "sga_topk_select_noalloc"]
+            "sga_topk_select_noalloc", "sga_index_scores_fp8", "sga_forward_fp8"]
 NOALLOC_SCRATCH_BYTES = 256 + 4 * 1024 * 1024
 
 
@@ -68,6 +68,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "sga_get_device_status": (ctypes.c_int, [P, P, ctypes.POINTER(i32)]),
         "sga_clear_device_status": (ctypes.c_int, [P, P]),
         "sga_topk_select_noalloc": (ctypes.c_int, [D, P, P, P, P]),
+        "sga_index_scores_fp8": (ctypes.c_int, [D, P, P, P, P, P, P, sz, P]),
+        "sga_forward_fp8": (ctypes.c_int, [D, P, P, P, P, P, P, P, P, P, P, sz, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -104,6 +106,13 @@ def _need(t, name, dtype, shape=None):
     if shape is not None and tuple(t.shape) != tuple(shape):
         raise ValueError(f"{name}: expected shape {tuple(shape)}, got {tuple(t.shape)}")
     return t
+
+
+def _need_fp8(t, name, shape):
+    """An E4M3 tensor (torch.float8_e4m3fn, or its bytes as uint8), returned as uint8."""
+    if isinstance(t, torch.Tensor) and t.dtype == torch.float8_e4m3fn:
+        t = t.view(torch.uint8)
+    return _need(t, name, torch.uint8, shape)
 
 
 def make_dims(batch: int, n_q: int, kv_stride: int, top_k: int = TOP_K) -> Dims:
@@ -147,6 +156,26 @@ def index_scores(q_idx, w, k_idx, q_pos, scores=None, ws=None, stream=None):
     if ws is None:
         ws = alloc_workspace(dims, OP_INDEX_SCORES, q_idx.device)
     _check("sga_index_scores", load_library().sga_index_scores(
+        ctypes.byref(dims), _ptr(q_idx), _ptr(w), _ptr(k_idx), _ptr(q_pos), _ptr(scores), _ptr(ws), ws.numel(),
+        _stream(stream)))
+    return scores
+
+
+def index_scores_fp8(q_idx, w, k_idx, q_pos, scores=None, ws=None, stream=None):
+    """Indexer scores [B,T,L] fp32 with E4M3 indexer queries and keys (see sga_index_scores_fp8)."""
+    B, T = q_idx.shape[0], q_idx.shape[1]
+    L = k_idx.shape[1]
+    q_idx = _need_fp8(q_idx, "q_idx", (B, T, INDEX_HEADS, INDEX_DIM))
+    k_idx = _need_fp8(k_idx, "k_idx", (B, L, INDEX_DIM))
+    _need(w, "w", torch.bfloat16, (B, T, INDEX_HEADS))
+    _need(q_pos, "q_pos", torch.int32, (B, T))
+    dims = make_dims(B, T, L)
+    if scores is None:
+        scores = torch.empty((B, T, L), dtype=torch.float32, device=q_idx.device)
+    _need(scores, "scores", torch.float32, (B, T, L))
+    if ws is None:
+        ws = alloc_workspace(dims, OP_INDEX_SCORES, q_idx.device)
+    _check("sga_index_scores_fp8", load_library().sga_index_scores_fp8(
         ctypes.byref(dims), _ptr(q_idx), _ptr(w), _ptr(k_idx), _ptr(q_pos), _ptr(scores), _ptr(ws), ws.numel(),
         _stream(stream)))
     return scores
@@ -228,6 +257,35 @@ def forward(q_idx, w, k_idx, q, kv, gate, q_pos, top_k: int = TOP_K, idx_out=Non
     if ws is None:
         ws = alloc_workspace(dims, OP_FORWARD, q.device)
     _check("sga_forward", load_library().sga_forward(
+        ctypes.byref(dims), _ptr(q_idx), _ptr(w), _ptr(k_idx), _ptr(q), _ptr(kv), _ptr(gate), _ptr(q_pos),
+        _ptr(idx_out), _ptr(out), _ptr(ws), ws.numel(), _stream(stream)))
+    return idx_out, out
+
+
+def forward_fp8(q_idx, w, k_idx, q, kv, gate, q_pos, top_k: int = TOP_K, idx_out=None, out=None, ws=None,
+                stream=None, return_idx: bool = True):
+    """The whole path with E4M3 indexer queries and keys (see sga_forward_fp8)."""
+    B, T = q_idx.shape[0], q_idx.shape[1]
+    L = k_idx.shape[1]
+    q_idx = _need_fp8(q_idx, "q_idx", (B, T, INDEX_HEADS, INDEX_DIM))
+    k_idx = _need_fp8(k_idx, "k_idx", (B, L, INDEX_DIM))
+    _need(w, "w", torch.bfloat16, (B, T, INDEX_HEADS))
+    _need(q, "q", torch.bfloat16, (B, T, HEADS, QK_DIM))
+    _need(kv, "kv", torch.bfloat16, (B, L, QK_DIM))
+    if gate is not None:
+        _need(gate, "gate", torch.bfloat16, (B, T, HEADS))
+    _need(q_pos, "q_pos", torch.int32, (B, T))
+    dims = make_dims(B, T, L, top_k)
+    if idx_out is None and return_idx:
+        idx_out = torch.empty((B, T, top_k), dtype=torch.int32, device=q.device)
+    if idx_out is not None:
+        _need(idx_out, "idx_out", torch.int32, (B, T, top_k))
+    if out is None:
+        out = torch.empty((B, T, HEADS, V_DIM), dtype=torch.float32, device=q.device)
+    _need(out, "out", torch.float32, (B, T, HEADS, V_DIM))
+    if ws is None:
+        ws = alloc_workspace(dims, OP_FORWARD, q.device)
+    _check("sga_forward_fp8", load_library().sga_forward_fp8(
         ctypes.byref(dims), _ptr(q_idx), _ptr(w), _ptr(k_idx), _ptr(q), _ptr(kv), _ptr(gate), _ptr(q_pos),
         _ptr(idx_out), _ptr(out), _ptr(ws), ws.numel(), _stream(stream)))
     return idx_out, out

@@ -93,8 +93,9 @@ T* at(void* ws, size_t off) {
 
 }  // namespace
 
-cudaError_t make_tmap_bf16_2d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer,
-                              uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer) {
+// 2-D tiled tensor map with the 128-byte swizzle over a row-major [outer][inner] array.
+cudaError_t make_tmap_2d(CUtensorMap* map, bool bytes, const void* base, uint64_t inner, uint64_t outer,
+                         uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer) {
   std::call_once(g_encode_once, []() {
     void* fn = nullptr;
     cudaDriverEntryPointQueryResult q;
@@ -108,15 +109,73 @@ cudaError_t make_tmap_bf16_2d(CUtensorMap* map, const void* base, uint64_t inner
   const cuuint64_t strides[1] = {row_bytes};
   const cuuint32_t box[2] = {box_inner, box_outer};
   const cuuint32_t estr[2] = {1, 1};
-  const CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
-                              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  const CUresult r = g_encode(map, bytes ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+                              const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                              CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+cudaError_t make_tmap_bf16_2d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer,
+                              uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer) {
+  return make_tmap_2d(map, false, base, inner, outer, row_bytes, box_inner, box_outer);
 }
 
 }  // namespace sga
 
 using namespace sga;
+
+namespace {
+
+// The indexer with bf16 or E4M3 (fp8) queries and keys; the rest of the path is shared.
+sga_status_t index_scores_impl(const sga_dims_t* dims, const void* q_idx, const sga_bf16_t* w, const void* k_idx,
+                               const int32_t* q_pos, float* scores, void* ws, size_t ws_bytes, sga_stream_t stream,
+                               bool fp8) {
+  if (!dims_ok(dims)) return SGA_ERR_INVALID_ARG;
+  if (!aligned(q_idx, 16) || !aligned(w, 16) || !aligned(k_idx, 16) || !aligned(q_pos, 4) || !aligned(scores, 16))
+    return SGA_ERR_INVALID_ARG;
+  Layout l;
+  sga_status_t st = check_ws(ws, ws_bytes, *dims, SGA_OP_INDEX_SCORES, &l);
+  if (st != SGA_OK) return st;
+  int sms = 0;
+  if ((st = device_info(&sms)) != SGA_OK) return st;
+  IndexArgs a{q_idx, w, k_idx, q_pos, scores, nullptr, at<int>(ws, 0), dims->batch, dims->n_q, dims->kv_stride, fp8};
+  return from_cuda(launch_index_scores(a, sms, static_cast<cudaStream_t>(stream)));
+}
+
+sga_status_t forward_impl(const sga_dims_t* dims, const void* q_idx, const sga_bf16_t* w, const void* k_idx,
+                          const sga_bf16_t* q, const sga_bf16_t* kv, const sga_bf16_t* gate, const int32_t* q_pos,
+                          int32_t* idx_out, float* out, void* ws, size_t ws_bytes, sga_stream_t stream, bool fp8) {
+  if (!dims_ok(dims)) return SGA_ERR_INVALID_ARG;
+  if (!aligned(q_idx, 16) || !aligned(w, 16) || !aligned(k_idx, 16) || !aligned(q, 16) || !aligned(kv, 16) ||
+      !aligned(q_pos, 4) || !aligned(out, 16) || (gate && !aligned(gate, 2)) || (idx_out && !aligned(idx_out, 16)))
+    return SGA_ERR_INVALID_ARG;
+  Layout l;
+  sga_status_t st = check_ws(ws, ws_bytes, *dims, SGA_OP_FORWARD, &l);
+  if (st != SGA_OK) return st;
+  int sms = 0;
+  if ((st = device_info(&sms)) != SGA_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int* status = at<int>(ws, 0);
+  float* scores = at<float>(ws, l.scores);
+  int32_t* idx = idx_out ? idx_out : at<int32_t>(ws, l.idx);
+  const int rows = dims->batch * dims->n_q;
+  // The indexer counts the first radix level of the selection as it writes the
+  // scores; the selection clears each histogram row after reading it, so a
+  // zero-filled workspace stays ready for the next call.
+  uint32_t* hist = at<uint32_t>(ws, l.hist);
+  IndexArgs ia{q_idx, w, k_idx, q_pos, scores, hist, status, dims->batch, dims->n_q, dims->kv_stride, fp8};
+  cudaError_t e = launch_index_scores(ia, sms, s);
+  if (e != cudaSuccess) return SGA_ERR_CUDA;
+  TopkArgs ta{scores, q_pos, idx, at<uint32_t>(ws, l.bitmap), hist, status, rows, dims->kv_stride, dims->top_k};
+  e = launch_topk(ta, s);
+  if (e != cudaSuccess) return SGA_ERR_CUDA;
+  AttendArgs aa{q, kv, idx, gate, out, status, dims->batch, dims->n_q, dims->kv_stride, dims->top_k};
+  return from_cuda(launch_attend(aa, s));
+}
+
+}  // namespace
+
 
 extern "C" {
 
@@ -141,19 +200,17 @@ sga_status_t sga_workspace_size(const sga_dims_t* dims, sga_op_t op, size_t* byt
   return SGA_OK;
 }
 
+
 sga_status_t sga_index_scores(const sga_dims_t* dims, const sga_bf16_t* q_idx, const sga_bf16_t* w,
                               const sga_bf16_t* k_idx, const int32_t* q_pos, float* scores, void* ws,
                               size_t ws_bytes, sga_stream_t stream) {
-  if (!dims_ok(dims)) return SGA_ERR_INVALID_ARG;
-  if (!aligned(q_idx, 16) || !aligned(w, 16) || !aligned(k_idx, 16) || !aligned(q_pos, 4) || !aligned(scores, 16))
-    return SGA_ERR_INVALID_ARG;
-  Layout l;
-  sga_status_t st = check_ws(ws, ws_bytes, *dims, SGA_OP_INDEX_SCORES, &l);
-  if (st != SGA_OK) return st;
-  int sms = 0;
-  if ((st = device_info(&sms)) != SGA_OK) return st;
-  IndexArgs a{q_idx, w, k_idx, q_pos, scores, nullptr, at<int>(ws, 0), dims->batch, dims->n_q, dims->kv_stride};
-  return from_cuda(launch_index_scores(a, sms, static_cast<cudaStream_t>(stream)));
+  return index_scores_impl(dims, q_idx, w, k_idx, q_pos, scores, ws, ws_bytes, stream, false);
+}
+
+sga_status_t sga_index_scores_fp8(const sga_dims_t* dims, const sga_fp8_e4m3_t* q_idx, const sga_bf16_t* w,
+                                  const sga_fp8_e4m3_t* k_idx, const int32_t* q_pos, float* scores, void* ws,
+                                  size_t ws_bytes, sga_stream_t stream) {
+  return index_scores_impl(dims, q_idx, w, k_idx, q_pos, scores, ws, ws_bytes, stream, true);
 }
 
 sga_status_t sga_topk_select(const sga_dims_t* dims, const float* scores, const int32_t* q_pos, int32_t* idx,
@@ -186,36 +243,19 @@ sga_status_t sga_sparse_mla_attend(const sga_dims_t* dims, const sga_bf16_t* q, 
   return from_cuda(launch_attend(a, static_cast<cudaStream_t>(stream)));
 }
 
+
 sga_status_t sga_forward(const sga_dims_t* dims, const sga_bf16_t* q_idx, const sga_bf16_t* w,
                          const sga_bf16_t* k_idx, const sga_bf16_t* q, const sga_bf16_t* kv,
                          const sga_bf16_t* gate, const int32_t* q_pos, int32_t* idx_out, float* out, void* ws,
                          size_t ws_bytes, sga_stream_t stream) {
-  if (!dims_ok(dims)) return SGA_ERR_INVALID_ARG;
-  if (!aligned(q_idx, 16) || !aligned(w, 16) || !aligned(k_idx, 16) || !aligned(q, 16) || !aligned(kv, 16) ||
-      !aligned(q_pos, 4) || !aligned(out, 16) || (gate && !aligned(gate, 2)) || (idx_out && !aligned(idx_out, 16)))
-    return SGA_ERR_INVALID_ARG;
-  Layout l;
-  sga_status_t st = check_ws(ws, ws_bytes, *dims, SGA_OP_FORWARD, &l);
-  if (st != SGA_OK) return st;
-  int sms = 0;
-  if ((st = device_info(&sms)) != SGA_OK) return st;
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
-  int* status = at<int>(ws, 0);
-  float* scores = at<float>(ws, l.scores);
-  int32_t* idx = idx_out ? idx_out : at<int32_t>(ws, l.idx);
-  const int rows = dims->batch * dims->n_q;
-  // The indexer counts the first radix level of the selection as it writes the
-  // scores; the selection clears each histogram row after reading it, so a
-  // zero-filled workspace stays ready for the next call.
-  uint32_t* hist = at<uint32_t>(ws, l.hist);
-  IndexArgs ia{q_idx, w, k_idx, q_pos, scores, hist, status, dims->batch, dims->n_q, dims->kv_stride};
-  cudaError_t e = launch_index_scores(ia, sms, s);
-  if (e != cudaSuccess) return SGA_ERR_CUDA;
-  TopkArgs ta{scores, q_pos, idx, at<uint32_t>(ws, l.bitmap), hist, status, rows, dims->kv_stride, dims->top_k};
-  e = launch_topk(ta, s);
-  if (e != cudaSuccess) return SGA_ERR_CUDA;
-  AttendArgs aa{q, kv, idx, gate, out, status, dims->batch, dims->n_q, dims->kv_stride, dims->top_k};
-  return from_cuda(launch_attend(aa, s));
+  return forward_impl(dims, q_idx, w, k_idx, q, kv, gate, q_pos, idx_out, out, ws, ws_bytes, stream, false);
+}
+
+sga_status_t sga_forward_fp8(const sga_dims_t* dims, const sga_fp8_e4m3_t* q_idx, const sga_bf16_t* w,
+                             const sga_fp8_e4m3_t* k_idx, const sga_bf16_t* q, const sga_bf16_t* kv,
+                             const sga_bf16_t* gate, const int32_t* q_pos, int32_t* idx_out, float* out, void* ws,
+                             size_t ws_bytes, sga_stream_t stream) {
+  return forward_impl(dims, q_idx, w, k_idx, q, kv, gate, q_pos, idx_out, out, ws, ws_bytes, stream, true);
 }
 
 sga_status_t sga_get_device_status(const void* ws, sga_stream_t stream, int32_t* device_status) {

@@ -3,23 +3,27 @@
 //
 //   scores[row, s] = sum_j w[row, j] * max(0, q_idx[row, j, :] . k_idx[b, s, :]),  s <= t
 //
-// Design (decode is HBM-bound: the 256 B index key of every past token is read
-// once and is ~93% of the bytes of the whole path at 128K context):
+// Design (decode is HBM-bound: the index key of every past token is read once
+// and is ~93% of the bytes of the whole path at 128K context):
 //   * A persistent grid, one CTA per SM, walks a contiguous range of
 //     (query, 128-key tile) work items.
-//   * Warp 0 streams 128-key x 128-dim bf16 tiles of k_idx with TMA (128-byte
-//     swizzle, L2 evict-first) through a 5-stage shared-memory ring, and the
-//     query's 64 x 128 indexer matrix into a double buffer when the query
-//     changes.
+//   * Warp 0 streams 128-key x 128-dim tiles of k_idx with TMA (128-byte
+//     swizzle, L2 evict-first) through a shared-memory ring, and the query's
+//     64 x 128 indexer matrix into a double buffer when the query changes.
+//     bf16 keys: 32 KB tiles in a 5-stage ring.  E4M3 keys (the FP8 cache of
+//     archdb "A.X K2", pretraining-precision field; nlp.com.ai "A.X K2 FP8"):
+//     16 KB tiles in a 10-stage ring, the same bytes in flight.
 //   * Warp 1 issues tcgen05.mma (M = 128 keys, N = 64 heads, K = 128 dims in 8
-//     steps of 16) into one of four 64-column TMEM accumulators.
-//   * Warps 2-5 (one per TMEM lane quarter) read a key's 64 head dots with
-//     tcgen05.ld, apply ReLU, the per-head weight and the head sum in fp32,
-//     mask s > t and store the score (32 consecutive keys per warp: one
-//     128-byte store).  When the caller asks for it, they also count each
-//     score's top 12 order bits into a per-query shared-memory histogram that
-//     is added to global memory when the query changes: the first level of
-//     the top-k radix select, computed while the scores are still in registers.
+//     kind::f16 steps of 16, or 4 kind::f8f6f4 steps of 32) into one of four
+//     64-column TMEM accumulators.
+//   * Warps 2-9, two groups of four that take alternate tiles (one warp per
+//     TMEM lane quarter in each), read a key's 64 head dots with tcgen05.ld,
+//     apply ReLU, the per-head weight and the head sum in fp32, mask s > t and
+//     store the score (32 consecutive keys per warp: one 128-byte store).
+//     When the caller asks for it, they also count each score's top 12 order
+//     bits into a per-query shared-memory histogram (one per group) that is
+//     added to global memory when the query changes: the first level of the
+//     top-k radix select, computed while the scores are still in registers.
 #include "sga_internal.cuh"
 #include "sga_ptx.cuh"
 
@@ -29,20 +33,32 @@ namespace {
 constexpr int kKeys = 128;    // keys per tile: MMA M
 constexpr int kDim = 128;     // indexer dim: MMA K
 constexpr int kHeads = 64;    // indexer heads: MMA N
-constexpr int kStages = 5;
-constexpr int kABox = kKeys * 64 * 2;  // one 128-byte-wide column strip of a tile
-constexpr int kAStage = 2 * kABox;     // 32 KB
-constexpr int kQBox = kHeads * 64 * 2;
-constexpr int kQBuf = 2 * kQBox;       // 16 KB
+constexpr int kABox = kKeys * 128;  // one 128-byte-wide column strip of a tile (16 KB)
+constexpr int kQBox = kHeads * 128;  // one 128-byte-wide column strip of a query's matrix (8 KB)
 constexpr int kAcc = 4;
 constexpr int kTmemCols = kAcc * kHeads;  // 256
-constexpr int kThreads = 192;
-constexpr int kNumBars = 2 * kStages + 4 + 2 * kAcc + 1;
+constexpr int kEpiGroups = 2;   // epilogue warp groups, taking alternate tiles
+constexpr int kThreads = 64 + kEpiGroups * 128;
 constexpr int kHistBytes = kTopkHistBins * 4;
 constexpr int kEpiThreads = 128;
-constexpr size_t kSmemBytes = 1024 + kStages * kAStage + 2 * kQBuf + kHistBytes + kNumBars * 8 + 16;
 
-static_assert(kDim == 2 * 64, "two 128-byte strips per key row");
+// bf16 keys: a key row is 256 B, two 128-byte strips; K = 128 in 8 MMA steps of 16.
+// E4M3 keys: a key row is one 128-byte strip; K = 128 in 4 MMA steps of 32.  The
+// E4M3 ring has twice the stages so the bytes in flight stay the same.
+template <bool kFp8>
+struct IndexCfg {
+  static constexpr int kStrips = kFp8 ? 1 : 2;        // 128-byte strips per key (and query) row
+  static constexpr int kStripElems = kFp8 ? 128 : 64;  // elements per strip
+  static constexpr int kStages = kFp8 ? 10 : 5;
+  static constexpr int kAStage = kStrips * kABox;
+  static constexpr int kQBuf = kStrips * kQBox;
+  static constexpr int kKSteps = kFp8 ? 4 : 8;         // 32-byte K steps per tile
+  static constexpr int kNumBars = 2 * kStages + 4 + 2 * kAcc + 1;
+  static constexpr size_t kSmemBytes =
+      1024 + kStages * kAStage + 2 * kQBuf + kEpiGroups * kHistBytes + kNumBars * 8 + 16;
+  static constexpr uint32_t kIdesc = kFp8 ? idesc_e4m3_f32(kKeys, kHeads) : idesc_bf16_f32(kKeys, kHeads, false, false);
+};
+static_assert(IndexCfg<false>::kSmemBytes <= 232448 && IndexCfg<true>::kSmemBytes <= 232448, "shared memory budget");
 
 struct IndexParams {
   const uint16_t* w;
@@ -78,15 +94,18 @@ struct TileCursor {
   __device__ __forceinline__ bool live(const IndexParams& p) const { return !bad_position(p) && key0 <= t; }
 };
 
+template <bool kFp8>
 __global__ void __launch_bounds__(kThreads, 1)
     sga_index_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap qmap,
                      IndexParams p) {
+  using C = IndexCfg<kFp8>;
+  constexpr int kStages = C::kStages, kAStage = C::kAStage, kQBuf = C::kQBuf, kNumBars = C::kNumBars;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t a_base = smem_u32(smem);
   const uint32_t q_base = a_base + kStages * kAStage;
   uint32_t* hist_s = reinterpret_cast<uint32_t*>(smem + kStages * kAStage + 2 * kQBuf);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kStages * kAStage + 2 * kQBuf + kHistBytes);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kStages * kAStage + 2 * kQBuf + kEpiGroups * kHistBytes);
   const uint32_t bar0 = smem_u32(bars);
   auto full = [&](int s) { return bar0 + 8u * s; };
   auto empty = [&](int s) { return bar0 + 8u * (kStages + s); };
@@ -160,8 +179,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             break;
           }
           mbar_arrive_expect_tx(qfull(slot), kQBuf);
-          tma_load_2d(q_base + slot * kQBuf, &qmap, qfull(slot), 0, row * kHeads, pol_keep);
-          tma_load_2d(q_base + slot * kQBuf + kQBox, &qmap, qfull(slot), 64, row * kHeads, pol_keep);
+#pragma unroll
+          for (int b = 0; b < C::kStrips; ++b)
+            tma_load_2d(q_base + slot * kQBuf + b * kQBox, &qmap, qfull(slot), b * C::kStripElems, row * kHeads,
+                        pol_keep);
           ++qc;
           cur_row = row;
         }
@@ -172,8 +193,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         mbar_arrive_expect_tx(full(st), kAStage);
         const int y = (row / p.n_q) * p.kv_stride + key0;
-        tma_load_2d(a_base + st * kAStage, &kmap, full(st), 0, y, pol_stream);
-        tma_load_2d(a_base + st * kAStage + kABox, &kmap, full(st), 64, y, pol_stream);
+#pragma unroll
+        for (int b = 0; b < C::kStrips; ++b)
+          tma_load_2d(a_base + st * kAStage + b * kABox, &kmap, full(st), b * C::kStripElems, y, pol_stream);
         ++n;
       }
       if (!ok) {
@@ -190,7 +212,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      constexpr uint32_t idesc = idesc_bf16_f32(kKeys, kHeads, false, false);
+      constexpr uint32_t idesc = C::kIdesc;
       long long n = 0, qc = 0, an = 0;
       int cur_row = -1, cur_q = 0;
       bool ok = true;
@@ -223,10 +245,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         const uint32_t d = tmem_base + static_cast<uint32_t>(acc * kHeads);
 #pragma unroll
-        for (int k = 0; k < kDim / 16; ++k) {
+        for (int k = 0; k < C::kKSteps; ++k) {
+          // 32-byte K steps: four per 128-byte strip
           const uint32_t a_addr = a_base + st * kAStage + (k >> 2) * kABox + (k & 3) * 32;
           const uint32_t b_addr = q_base + cur_q * kQBuf + (k >> 2) * kQBox + (k & 3) * 32;
-          mma_bf16(d, sdesc_sw128(a_addr, 16, 1024), sdesc_sw128(b_addr, 16, 1024), idesc, k > 0 ? 1u : 0u);
+          if constexpr (kFp8)
+            mma_e4m3(d, sdesc_sw128(a_addr, 16, 1024), sdesc_sw128(b_addr, 16, 1024), idesc, k > 0 ? 1u : 0u);
+          else
+            mma_bf16(d, sdesc_sw128(a_addr, 16, 1024), sdesc_sw128(b_addr, 16, 1024), idesc, k > 0 ? 1u : 0u);
         }
         mma_commit(empty(st));
         mma_commit(accfull(acc));
@@ -244,32 +270,42 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     // ------------------------------------------------------------ epilogue
+    // Two groups of four warps take alternate tiles (group g reads accumulators
+    // g and g + 2), each with its own histogram, so a group has two tile
+    // periods per tile.
+    const int group = (warp - 2) >> 2;
     const int quarter = warp & 3;  // TMEM lanes 32*quarter .. +31 (warp % 4 rule)
-    const int et = threadIdx.x - 64;
+    const int et = threadIdx.x - 64 - kEpiThreads * group;
+    const int bar_id = 1 + group;
+    uint32_t* hist_g = hist_s + group * kTopkHistBins;
     const bool with_hist = p.hist != nullptr;
     long long an = 0;
     int cur_row = -1;
     float wv[kHeads];
     // Adds the shared histogram of `r` to global memory and clears it.
     auto flush_hist = [&](int r) {
-      named_barrier(1, kEpiThreads);
+      named_barrier(bar_id, kEpiThreads);
       for (int b = et; b < kTopkHistBins; b += kEpiThreads) {
-        const uint32_t v = hist_s[b];
+        const uint32_t v = hist_g[b];
         if (v) {
           atomicAdd(p.hist + static_cast<size_t>(r) * kTopkHistBins + b, v);
-          hist_s[b] = 0;
+          hist_g[b] = 0;
         }
       }
-      named_barrier(1, kEpiThreads);
+      named_barrier(bar_id, kEpiThreads);
     };
     if (with_hist) {
-      for (int b = et; b < kTopkHistBins; b += kEpiThreads) hist_s[b] = 0;
-      named_barrier(1, kEpiThreads);
+      for (int b = et; b < kTopkHistBins; b += kEpiThreads) hist_g[b] = 0;
+      named_barrier(bar_id, kEpiThreads);
     }
     TileCursor cur;
     if (j0 < j1) cur.start(p, j0);
     for (long long j = j0; j < j1; cur.next(p, ++j < j1)) {
       if (!cur.live(p)) continue;
+      if ((an & 1) != group) {  // the other group's tile
+        ++an;
+        continue;
+      }
       const int row = cur.row, key0 = cur.key0, t = cur.t;
       if (row != cur_row) {
         if (with_hist && cur_row >= 0) flush_hist(cur_row);
@@ -311,7 +347,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int key = key0 + quarter * 32 + lane;
       if (key <= t) {
         p.scores[static_cast<size_t>(row) * p.kv_stride + key] = s;
-        if (with_hist) atomicAdd(hist_s + (order_bits(s) >> (32 - kTopkHistBits)), 1u);
+        if (with_hist) atomicAdd(hist_g + (order_bits(s) >> (32 - kTopkHistBits)), 1u);
       }
       ++an;
     }
@@ -333,14 +369,17 @@ cudaError_t launch_index_scores(const IndexArgs& a, int num_sms, cudaStream_t st
   const int tiles_per_row = (a.kv_stride + kKeys - 1) / kKeys;
   const long long total = static_cast<long long>(rows) * tiles_per_row;
   if (total == 0) return cudaSuccess;
+  const int esize = a.fp8 ? 1 : 2;
+  const uint32_t strip = a.fp8 ? 128 : 64;  // elements per 128-byte strip
   CUtensorMap kmap, qmap;
-  cudaError_t e = make_tmap_bf16_2d(&kmap, a.k_idx, kDim, static_cast<uint64_t>(a.batch) * a.kv_stride, kDim * 2,
-                                    64, kKeys);
+  cudaError_t e = make_tmap_2d(&kmap, a.fp8, a.k_idx, kDim, static_cast<uint64_t>(a.batch) * a.kv_stride,
+                               kDim * esize, strip, kKeys);
   if (e != cudaSuccess) return e;
-  e = make_tmap_bf16_2d(&qmap, a.q_idx, kDim, static_cast<uint64_t>(rows) * kHeads, kDim * 2, 64, kHeads);
+  e = make_tmap_2d(&qmap, a.fp8, a.q_idx, kDim, static_cast<uint64_t>(rows) * kHeads, kDim * esize, strip, kHeads);
   if (e != cudaSuccess) return e;
-  e = cudaFuncSetAttribute(sga_index_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           static_cast<int>(kSmemBytes));
+  auto kernel = a.fp8 ? sga_index_kernel<true> : sga_index_kernel<false>;
+  const size_t smem = a.fp8 ? IndexCfg<true>::kSmemBytes : IndexCfg<false>::kSmemBytes;
+  e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   IndexParams p;
   p.w = a.w;
@@ -356,14 +395,14 @@ cudaError_t launch_index_scores(const IndexArgs& a, int num_sms, cudaStream_t st
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(grid));
   cfg.blockDim = dim3(kThreads);
-  cfg.dynamicSmemBytes = kSmemBytes;
+  cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, sga_index_kernel, kmap, qmap, p);
+  return cudaLaunchKernelEx(&cfg, kernel, kmap, qmap, p);
 }
 
 }  // namespace sga

@@ -9,14 +9,15 @@ namespace sga {
 
 // ---- indexer (step 1) --------------------------------------------------------
 struct IndexArgs {
-  const uint16_t* q_idx;  // [rows][64][128]
+  const void* q_idx;      // [rows][64][128] bf16, or E4M3 bytes when fp8
   const uint16_t* w;      // [rows][64]
-  const uint16_t* k_idx;  // [B][L][128]
+  const void* k_idx;      // [B][L][128] bf16, or E4M3 bytes when fp8
   const int32_t* q_pos;   // [rows]
   float* scores;          // [rows][L]
   uint32_t* hist;         // [rows][4096] first-level top-k histogram (all zero on entry) or null
   int* status;
   int batch, n_q, kv_stride;
+  bool fp8;               // indexer queries and keys in E4M3
 };
 cudaError_t launch_index_scores(const IndexArgs& a, int num_sms, cudaStream_t stream);
 
@@ -52,5 +53,8 @@ cudaError_t launch_attend(const AttendArgs& a, cudaStream_t stream);
 // apart, box {box_inner, box_outer}, 128-byte swizzle.
 cudaError_t make_tmap_bf16_2d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer,
                               uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer);
+// Same, over bytes (E4M3 values) when `bytes`, else bf16.
+cudaError_t make_tmap_2d(CUtensorMap* map, bool bytes, const void* base, uint64_t inner, uint64_t outer,
+                         uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer);
 
 }  // namespace sga

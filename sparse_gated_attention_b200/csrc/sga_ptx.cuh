@@ -189,6 +189,21 @@ __device__ __forceinline__ void mma_commit(uint32_t bar) {
 }
 
 // Instruction descriptor, kind::f16 with bf16 A/B and fp32 D.
+// tcgen05.mma kind::f8f6f4 with both operands E4M3 (format code 0), f32 accumulator, K-major A and B.
+__device__ __forceinline__ void mma_e4m3(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                         uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+__host__ __device__ constexpr uint32_t idesc_e4m3_f32(int M, int N) {
+  return (1u << 4)                     // D format: f32 (A and B format fields 0: E4M3)
+         | ((uint32_t)(N >> 3) << 17)  // N / 8
+         | ((uint32_t)(M >> 4) << 24);  // M / 16
+}
 __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, bool a_mn_major, bool b_mn_major) {
   return (1u << 4)                              // D format: f32
          | (1u << 7)                            // A format: bf16

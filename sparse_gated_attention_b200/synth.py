@@ -114,6 +114,20 @@ def make_inputs(wl: Workload, device="cpu", seed: int = 0) -> dict:
     return dict(q_idx=q_idx, w=w, k_idx=k_idx, q=q, kv=kv, gate=gate, q_pos=q_pos)
 
 
+def to_e4m3(x: torch.Tensor) -> torch.Tensor:
+    """bf16 tensor -> float8_e4m3fn storage (exact for the integer-valued indexer inputs)."""
+    return x.to(torch.float8_e4m3fn)
+
+
+def make_inputs_fp8(wl: Workload, device="cpu", seed: int = 0) -> dict:
+    """The inputs of ``make_inputs`` with the indexer queries and keys stored as E4M3
+    (the FP8 indexer-key cache variant); the integer values in [-3, 3] are kept exactly."""
+    x = make_inputs(wl, device, seed)
+    x["q_idx"] = to_e4m3(x["q_idx"])
+    x["k_idx"] = to_e4m3(x["k_idx"])
+    return x
+
+
 def input_bytes(wl: Workload) -> dict:
     """Bytes of each input tensor (for reporting)."""
     B, T, L = wl.batch, wl.n_q, wl.ctx

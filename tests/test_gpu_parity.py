@@ -338,3 +338,74 @@ def test_workload_sampled_parity(name, count):
                                             x["kv"][b:b + 1].cpu(), sel(x["gate"]), sel(x["q_pos"]))
         np.testing.assert_array_equal(idx[b, ts].cpu().numpy(), want_idx[0])
         assert_close(out[b, ts].cpu().numpy(), want_out[0], f"{name} seq {b}")
+
+
+# ----------------------------------------------------------------------------- E4M3 indexer-key variant
+# sga_index_scores_fp8 / sga_forward_fp8 read the indexer queries and keys as
+# E4M3 codes; the oracle decodes each code to its exact value.
+
+
+@pytest.mark.parametrize("B,T,L,pos", INDEX_CASES)
+def test_index_scores_fp8_bit_exact(B, T, L, pos):
+    x = gen_small(B, T, L, pos)
+    qf, kf = synth.to_e4m3(x["q_idx"]), synth.to_e4m3(x["k_idx"])
+    scores = torch.full((B, T, L), float("nan"), device="cuda")
+    ws = sga.alloc_workspace(sga.make_dims(B, T, L), sga.OP_INDEX_SCORES)
+    sga.index_scores_fp8(qf, x["w"], kf, x["q_pos"], scores=scores, ws=ws)
+    check_status(ws)
+    want = oracle.index_scores_e4m3(qf, x["w"], kf, x["q_pos"].cpu())
+    got = scores.cpu().numpy().astype(np.float64)
+    pos = np.asarray(pos)
+    for b in range(B):
+        for t in range(T):
+            p = pos[b, t]
+            np.testing.assert_array_equal(got[b, t, : p + 1], want[b, t, : p + 1])
+
+
+def test_index_scores_fp8_general_codes():
+    """Random finite E4M3 codes (magnitudes 2^-9 .. 448, both signs): every
+    product is exact in fp32, only the order of the fp32 sums differs."""
+    B, T, L = 2, 2, 3000
+    g = torch.Generator(device="cuda").manual_seed(3)
+    codes = lambda shape: torch.randint(0, 0x7F, shape, generator=g, device="cuda", dtype=torch.int32)  # noqa: E731
+    sign = lambda shape: torch.randint(0, 2, shape, generator=g, device="cuda", dtype=torch.int32) * 0x80  # noqa: E731
+    qf = (codes((B, T, 64, 128)) | sign((B, T, 64, 128))).to(torch.uint8)
+    kf = (codes((B, L, 128)) | sign((B, L, 128))).to(torch.uint8)
+    w = torch.rand((B, T, 64), generator=g, device="cuda").to(torch.bfloat16)
+    q_pos = torch.tensor([[L - 1, 1000], [2999, 17]], dtype=torch.int32, device="cuda")
+    scores = sga.index_scores_fp8(qf, w, kf, q_pos)
+    want = oracle.index_scores_e4m3(qf, w, kf, q_pos.cpu())
+    got = scores.cpu().numpy().astype(np.float64)
+    for b in range(B):
+        for t in range(T):
+            p = int(q_pos[b, t])
+            err = np.abs(got[b, t, : p + 1] - want[b, t, : p + 1])
+            assert err.max() <= 1e-5 * max(np.abs(want[b, t, : p + 1]).max(), 1.0)
+
+
+@pytest.mark.parametrize("B,T,L,pos", [(2, 1, 1500, [[1499], [700]]), (2, 2, 6000, [[5999, 3000], [2500, 2047]])])
+def test_forward_fp8_matches_oracle(B, T, L, pos):
+    x = gen_small(B, T, L, pos)
+    qf, kf = synth.to_e4m3(x["q_idx"]), synth.to_e4m3(x["k_idx"])
+    ws = sga.alloc_workspace(sga.make_dims(B, T, L), sga.OP_FORWARD)
+    idx, out = sga.forward_fp8(qf, x["w"], kf, x["q"], x["kv"], x["gate"], x["q_pos"], ws=ws)
+    check_status(ws)
+    want_idx, want_out = oracle.forward_e4m3(qf, x["w"], kf, x["q"], x["kv"], x["gate"], x["q_pos"].cpu())
+    np.testing.assert_array_equal(idx.cpu().numpy(), want_idx)
+    assert_close(out.cpu().numpy(), want_out, "forward fp8")
+
+
+def test_workload_fp8_sampled_parity():
+    """The 128K decode workload with an E4M3 indexer-key cache, as the bench runs it."""
+    wl = synth.WORKLOADS["decode_b32_ctx128k"]
+    x = synth.make_inputs_fp8(wl, device="cuda", seed=0)
+    ws = sga.alloc_workspace(sga.make_dims(wl.batch, wl.n_q, wl.ctx, wl.top_k), sga.OP_FORWARD)
+    idx, out = sga.forward_fp8(x["q_idx"], x["w"], x["k_idx"], x["q"], x["kv"], x["gate"], x["q_pos"], ws=ws)
+    torch.cuda.synchronize()
+    check_status(ws)
+    for b in sampled_rows(wl, 3):
+        sel = lambda t: t[b:b + 1].contiguous().cpu()  # noqa: E731
+        want_idx, want_out = oracle.forward_e4m3(sel(x["q_idx"]), sel(x["w"]), sel(x["k_idx"]), sel(x["q"]),
+                                                 sel(x["kv"]), sel(x["gate"]), sel(x["q_pos"]))
+        np.testing.assert_array_equal(idx[b].cpu().numpy(), want_idx[0])
+        assert_close(out[b].cpu().numpy(), want_out[0], f"fp8 workload seq {b}")

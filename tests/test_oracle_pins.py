@@ -348,3 +348,53 @@ def test_forward_equals_steps(oracle_mod):
         chosen = np.zeros(len(s), bool)
         chosen[idx[0, t]] = True
         assert s[chosen].min() >= s[~chosen].max()
+
+
+# ----------------------------------------------------------------------------- the E4M3 indexer-key variant
+# The fp8 oracle reads each E4M3 code as its exact value (1 sign, 4 exponent bits
+# with bias 7, 3 mantissa bits; exponent 0 subnormal; S.1111.111 NaN) and runs the
+# bf16 oracle on the same values.  The decoder is pinned to the format definition
+# (hand-worked codes) and to torch's float8_e4m3fn conversion.
+
+E4M3_HAND = [
+    (0x00, 0.0), (0x80, -0.0), (0x38, 1.0), (0xB8, -1.0), (0x3C, 1.5), (0x30, 0.5), (0x40, 2.0),
+    (0x44, 3.0), (0xC4, -3.0), (0x7E, 448.0), (0xFE, -448.0), (0x08, 2.0 ** -6), (0x01, 2.0 ** -9),
+    (0x07, 7 * 2.0 ** -9), (0x77, 240.0),
+]
+
+
+def test_e4m3_hand_worked_codes(oracle_mod):
+    for code, want in E4M3_HAND:
+        got = oracle_mod.e4m3_to_float64([code])[0]
+        assert got == want and np.signbit(got) == np.signbit(want), (hex(code), got, want)
+    assert np.isnan(oracle_mod.e4m3_to_float64([0x7F, 0xFF])).all()
+
+
+def test_e4m3_matches_torch_for_every_code(oracle_mod):
+    codes = np.arange(256, dtype=np.uint8)
+    ref = torch.from_numpy(codes.copy()).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    got = oracle_mod.e4m3_to_float64(codes)
+    nan = np.isnan(ref)
+    assert (np.isnan(got) == nan).all()
+    np.testing.assert_array_equal(got[~nan], ref[~nan])
+
+
+def test_e4m3_to_bf16_is_exact(oracle_mod):
+    codes = np.arange(256, dtype=np.uint8)
+    v = oracle_mod.e4m3_to_float64(codes)
+    back = (oracle_mod.e4m3_to_bf16_bits(codes).astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    fin = np.isfinite(v)
+    np.testing.assert_array_equal(back[fin], v[fin])
+
+
+def test_index_scores_e4m3_equals_bf16_on_integer_inputs(oracle_mod):
+    # integers in [-3, 3] are exact in both formats, so both caches give the same scores
+    rng = np.random.default_rng(5)
+    q = rng.integers(-3, 4, size=(1, 2, 64, 128)).astype(np.float32)
+    k = rng.integers(-3, 4, size=(1, 300, 128)).astype(np.float32)
+    w = torch.from_numpy(rng.integers(0, 4, size=(1, 2, 64)).astype(np.float32)).to(torch.bfloat16)
+    pos = np.array([[299, 150]], dtype=np.int32)
+    qt, kt = torch.from_numpy(q), torch.from_numpy(k)
+    want = oracle_mod.index_scores(qt.to(torch.bfloat16), w, kt.to(torch.bfloat16), pos)
+    got = oracle_mod.index_scores_e4m3(qt.to(torch.float8_e4m3fn), w, kt.to(torch.float8_e4m3fn), pos)
+    np.testing.assert_array_equal(got, want)
