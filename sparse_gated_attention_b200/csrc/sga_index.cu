@@ -14,7 +14,7 @@
 //     archdb "A.X K2", pretraining-precision field; nlp.com.ai "A.X K2 FP8"):
 //     16 KB tiles in a 10-stage ring, the same bytes in flight.
 //   * Warp 1 issues tcgen05.mma (M = 128 keys, N = 64 heads, K = 128 dims in 8
-//     kind::f16 steps of 16, or 4 kind::f8f6f4 steps of 32) into one of four
+//     kind::f16 steps of 16, or 4 kind::f8f6f4 steps of 32) into one of eight
 //     64-column TMEM accumulators.
 //   * Warps 2-9, two groups of four that take alternate tiles (one warp per
 //     TMEM lane quarter in each), read a key's 64 head dots with tcgen05.ld,
@@ -35,8 +35,8 @@ constexpr int kDim = 128;     // indexer dim: MMA K
 constexpr int kHeads = 64;    // indexer heads: MMA N
 constexpr int kABox = kKeys * 128;  // one 128-byte-wide column strip of a tile (16 KB)
 constexpr int kQBox = kHeads * 128;  // one 128-byte-wide column strip of a query's matrix (8 KB)
-constexpr int kAcc = 4;
-constexpr int kTmemCols = kAcc * kHeads;  // 256
+constexpr int kAcc = 8;  // TMEM accumulators (all 512 columns): the MMA runs up to 8 tiles ahead of the epilogue
+constexpr int kTmemCols = kAcc * kHeads;  // 512
 constexpr int kEpiGroups = 2;   // epilogue warp groups, taking alternate tiles
 constexpr int kThreads = 64 + kEpiGroups * 128;
 constexpr int kHistBytes = kTopkHistBins * 4;
@@ -270,9 +270,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     // ------------------------------------------------------------ epilogue
-    // Two groups of four warps take alternate tiles (group g reads accumulators
-    // g and g + 2), each with its own histogram, so a group has two tile
-    // periods per tile.
+    // Two groups of four warps take alternate tiles (group g reads the
+    // accumulators of its parity), each with its own histogram, so a group has
+    // two tile periods per tile.
     const int group = (warp - 2) >> 2;
     const int quarter = warp & 3;  // TMEM lanes 32*quarter .. +31 (warp % 4 rule)
     const int et = threadIdx.x - 64 - kEpiThreads * group;
@@ -329,10 +329,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         break;
       }
       tc_fence_after();
-      float v0[32], v1[32];
+      float v[64];
       const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + static_cast<uint32_t>(acc * kHeads);
-      tmem_ld32(taddr, v0);
-      tmem_ld32(taddr + 32, v1);
+      tmem_ld64(taddr, v);
       tc_fence_before();
       mbar_arrive(accempty(acc));
       // head sum as four independent chains (one warp per scheduler: the chain
@@ -340,9 +339,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       // every partial sum exact, so the order does not change the score
       float ps[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-      for (int h = 0; h < 32; ++h) ps[h & 3] = fmaf(wv[h], fmaxf(v0[h], 0.f), ps[h & 3]);
-#pragma unroll
-      for (int h = 0; h < 32; ++h) ps[h & 3] = fmaf(wv[32 + h], fmaxf(v1[h], 0.f), ps[h & 3]);
+      for (int h = 0; h < 64; ++h) ps[h & 3] = fmaf(wv[h], fmaxf(v[h], 0.f), ps[h & 3]);
       const float s = (ps[0] + ps[1]) + (ps[2] + ps[3]);
       const int key = key0 + quarter * 32 + lane;
       if (key <= t) {
