@@ -36,6 +36,7 @@ constexpr int kHeads = 64;    // indexer heads: MMA N
 constexpr int kABox = kKeys * 128;  // one 128-byte-wide column strip of a tile (16 KB)
 constexpr int kQBox = kHeads * 128;  // one 128-byte-wide column strip of a query's matrix (8 KB)
 constexpr int kAcc = 8;  // TMEM accumulators (all 512 columns): the MMA runs up to 8 tiles ahead of the epilogue
+static_assert((kAcc & (kAcc - 1)) == 0, "the epilogue indexes accumulators with a mask");
 constexpr int kTmemCols = kAcc * kHeads;  // 512
 constexpr int kEpiGroups = 2;   // epilogue warp groups, taking alternate tiles
 constexpr int kThreads = 64 + kEpiGroups * 128;
@@ -162,6 +163,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint64_t pol_stream = policy_evict_first();
       const uint64_t pol_keep = policy_evict_last();
       long long n = 0, qc = 0;
+      int st = 0;         // ring stage of tile n
+      uint32_t ph = 0;    // phase parity of that stage's current use
       int cur_row = -1;
       bool ok = true;
       TileCursor cur;
@@ -186,8 +189,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           ++qc;
           cur_row = row;
         }
-        const int st = static_cast<int>(n % kStages);
-        if (!mbar_wait(empty(st), static_cast<uint32_t>((n / kStages) & 1) ^ 1u, abort_flag)) {
+        if (!mbar_wait(empty(st), ph ^ 1u, abort_flag)) {
           ok = false;
           break;
         }
@@ -197,6 +199,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int b = 0; b < C::kStrips; ++b)
           tma_load_2d(a_base + st * kAStage + b * kABox, &kmap, full(st), b * C::kStripElems, y, pol_stream);
         ++n;
+        if (++st == kStages) {
+          st = 0;
+          ph ^= 1u;
+        }
       }
       if (!ok) {
         record_status(p.status, kStatusTimeout);
@@ -213,7 +219,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       constexpr uint32_t idesc = C::kIdesc;
-      long long n = 0, qc = 0, an = 0;
+      // Descriptors are built once and stepped: the start-address field is
+      // address / 16, so adding (offset / 16) moves a descriptor by offset bytes.
+      const uint64_t a_desc0 = sdesc_sw128(a_base, 16, 1024);
+      const uint64_t q_desc0 = sdesc_sw128(q_base, 16, 1024);
+      long long qc = 0;
+      int st = 0, acc = 0;            // ring stage and TMEM accumulator of the next tile
+      uint32_t ph = 0, aph = 0;       // their phase parities
       int cur_row = -1, cur_q = 0;
       bool ok = true;
       TileCursor cur;
@@ -232,32 +244,38 @@ __global__ void __launch_bounds__(kThreads, 1)
           ++qc;
           cur_row = row;
         }
-        const int acc = static_cast<int>(an % kAcc);
-        if (!mbar_wait(accempty(acc), static_cast<uint32_t>((an / kAcc) & 1) ^ 1u, abort_flag)) {
+        if (!mbar_wait(accempty(acc), aph ^ 1u, abort_flag)) {
           ok = false;
           break;
         }
-        const int st = static_cast<int>(n % kStages);
-        if (!mbar_wait(full(st), static_cast<uint32_t>((n / kStages) & 1), abort_flag)) {
+        if (!mbar_wait(full(st), ph, abort_flag)) {
           ok = false;
           break;
         }
         tc_fence_after();
         const uint32_t d = tmem_base + static_cast<uint32_t>(acc * kHeads);
+        const uint64_t a_desc = a_desc0 + static_cast<uint64_t>((st * kAStage) >> 4);
+        const uint64_t b_desc = q_desc0 + static_cast<uint64_t>((cur_q * kQBuf) >> 4);
 #pragma unroll
         for (int k = 0; k < C::kKSteps; ++k) {
           // 32-byte K steps: four per 128-byte strip
-          const uint32_t a_addr = a_base + st * kAStage + (k >> 2) * kABox + (k & 3) * 32;
-          const uint32_t b_addr = q_base + cur_q * kQBuf + (k >> 2) * kQBox + (k & 3) * 32;
+          const uint64_t a_off = static_cast<uint64_t>(((k >> 2) * kABox + (k & 3) * 32) >> 4);
+          const uint64_t b_off = static_cast<uint64_t>(((k >> 2) * kQBox + (k & 3) * 32) >> 4);
           if constexpr (kFp8)
-            mma_e4m3(d, sdesc_sw128(a_addr, 16, 1024), sdesc_sw128(b_addr, 16, 1024), idesc, k > 0 ? 1u : 0u);
+            mma_e4m3(d, a_desc + a_off, b_desc + b_off, idesc, k > 0 ? 1u : 0u);
           else
-            mma_bf16(d, sdesc_sw128(a_addr, 16, 1024), sdesc_sw128(b_addr, 16, 1024), idesc, k > 0 ? 1u : 0u);
+            mma_bf16(d, a_desc + a_off, b_desc + b_off, idesc, k > 0 ? 1u : 0u);
         }
         mma_commit(empty(st));
         mma_commit(accfull(acc));
-        ++n;
-        ++an;
+        if (++st == kStages) {
+          st = 0;
+          ph ^= 1u;
+        }
+        if (++acc == kAcc) {
+          acc = 0;
+          aph ^= 1u;
+        }
       }
       if (!ok) {
         record_status(p.status, kStatusTimeout);
@@ -279,7 +297,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int bar_id = 1 + group;
     uint32_t* hist_g = hist_s + group * kTopkHistBins;
     const bool with_hist = p.hist != nullptr;
-    long long an = 0;
+    int an = 0;  // live tiles seen (both groups' ones): accumulator an % kAcc
     int cur_row = -1;
     float wv[kHeads];
     // Adds the shared histogram of `r` to global memory and clears it.
@@ -322,8 +340,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         cur_row = row;
       }
-      const int acc = static_cast<int>(an % kAcc);
-      if (!mbar_wait(accfull(acc), static_cast<uint32_t>((an / kAcc) & 1), abort_flag)) {
+      const int acc = an & (kAcc - 1);
+      if (!mbar_wait(accfull(acc), static_cast<uint32_t>(an / kAcc) & 1u, abort_flag)) {
         record_status(p.status, kStatusTimeout);
         *abort_flag = 1;
         break;
