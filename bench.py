@@ -2,13 +2,18 @@
 
 One step = one pass of the whole path over one batch of queries: the indexer
 over every cached position, top-2048 selection, sparse latent attention and the
-head gate.  The three C-ABI calls issued per step (sga_index_scores,
-sga_topk_select, sga_sparse_mla_attend) are exactly the launches sga_forward
-makes; they are issued separately so CUDA events on the same stream can time
-each kernel inside the timed region.
+head gate, as one sga_forward call (three kernel launches).  The timed region
+is K such steps between CUDA events on the launching stream.  Each kernel is
+then timed alone in its own event-timed loop of the matching C-ABI call
+(sga_index_scores, sga_topk_select, sga_sparse_mla_attend) for the roofline of
+the dominant kernel; an end-to-end region repeats the step with the query-side
+inputs copied from pinned host memory and the results copied back; the E4M3
+index-key variant is timed like the main region.
 
-Prints one JSON line (rank 0).  `--impl reference` times the fp64 CPU oracle
-on the host cores instead (a bounded sample of the same workload).
+Under torchrun every rank is an independent replica with its own batch (weak
+scaling); each timed region starts after a barrier and its time is the maximum
+over ranks.  Prints one JSON line (rank 0).  `--impl reference` times the fp64
+CPU oracle on the host cores instead (a bounded sample of the same workload).
 """
 from __future__ import annotations
 
@@ -199,6 +204,21 @@ def run_reference(args, wl, rank):
     print(json.dumps(line), flush=True)
 
 
+def max_over_ranks(dist, device, ms: float) -> float:
+    """The slowest rank's time for a timed region (every rank calls this in the same order)."""
+    if dist is None:
+        return ms
+    t = torch.tensor([ms], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_rate(rows_per_rank: int, steps: int, world: int, elapsed_ms: float) -> float:
+    """Queries per second over all replicas: every rank decodes its own batch of rows_per_rank
+    queries per step (weak scaling), timed by the slowest rank."""
+    return rows_per_rank * steps * world / (elapsed_ms / 1e3)
+
+
 def config_of(wl):
     return {"workload": wl.name, "batch": wl.batch, "queries_per_seq": wl.n_q, "ctx": wl.ctx, "top_k": wl.top_k,
             "heads": 64, "latent": 576, "index_heads": 64, "index_dim": 128,
@@ -285,11 +305,7 @@ def main():
             fwd_step()
         stop.record(stream)
         torch.cuda.synchronize(dev)
-    elapsed_ms = start.elapsed_time(stop)
-    if dist is not None:
-        t = torch.tensor([elapsed_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        elapsed_ms = float(t.item())
+    elapsed_ms = max_over_ranks(dist, dev, start.elapsed_time(stop))
     if sga.device_status(ws_all) != 0:
         raise RuntimeError("device status set during the timed region")
 
@@ -327,11 +343,7 @@ def main():
         e2e_step()
     e2.record(stream)
     torch.cuda.synchronize(dev)
-    e2e_ms = s2.elapsed_time(e2)
-    if dist is not None:
-        t = torch.tensor([e2e_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = max_over_ranks(dist, dev, s2.elapsed_time(e2))
     if sga.device_status(ws_all) != 0:
         raise RuntimeError("device status set during the end-to-end run")
 
@@ -355,11 +367,7 @@ def main():
         fp8_step()
     e3.record(stream)
     torch.cuda.synchronize(dev)
-    fp8_ms = s3.elapsed_time(e3)
-    if dist is not None:
-        t = torch.tensor([fp8_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        fp8_ms = float(t.item())
+    fp8_ms = max_over_ranks(dist, dev, s3.elapsed_time(e3))
     if sga.device_status(ws_all) != 0:
         raise RuntimeError("device status set during the E4M3 variant run")
     del xf
@@ -371,8 +379,7 @@ def main():
         return
 
     ms_per_step = elapsed_ms / args.steps
-    total_queries = rows * args.steps * world
-    value = total_queries / (elapsed_ms / 1e3)
+    value = whole_job_rate(rows, args.steps, world, elapsed_ms)
     ab = algorithmic_bytes_per_query(L, K)
     peak, peak_kind = measured_peaks()
     k1_ms = statistics.mean(k1)
@@ -388,7 +395,7 @@ def main():
     fp8_step_ms = fp8_ms / args.steps
     fp8_gbs = ab8["total"] * rows / (fp8_step_ms * 1e-3) / 1e9
     variants = {"fp8_index_keys": {
-        "value": total_queries / (fp8_ms / 1e3), "unit": UNIT, "ms_per_step": fp8_step_ms,
+        "value": whole_job_rate(rows, args.steps, world, fp8_ms), "unit": UNIT, "ms_per_step": fp8_step_ms,
         "config": f"{wl.name} with q_idx and k_idx stored as E4M3 (exact for the integer-valued inputs)",
         "path_roofline": {"achieved_gbs": fp8_gbs, "frac_of_8tbs": fp8_gbs / NOMINAL_HBM_GBS,
                           "frac_of_measured": fp8_gbs / peak, "bytes_per_query": ab8["total"]},
@@ -412,7 +419,7 @@ def main():
                       "note": "each call timed alone; inside sga_forward the indexer also builds the top-k "
                               "first-level histogram and the top-k skips its histogram pass"},
         "cpu_baseline": cpu,
-        "e2e": {"value": total_queries / (e2e_ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+        "e2e": {"value": whole_job_rate(rows, args.steps, world, e2e_ms), "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h},
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clk.summary(),
