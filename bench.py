@@ -45,6 +45,8 @@ def parse_args():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=None, help="workload name (default: decode_b32_ctx128k)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-layer", dest="layer", action="store_false",
+                    help="skip the whole-layer variant (the projections either side of the path)")
     ap.add_argument("--cpu-sample-queries", type=int, default=0, help="oracle sample size (0 = auto)")
     ap.add_argument("--batch", type=int, default=0, help="custom decode workload: sequences (with --ctx)")
     ap.add_argument("--ctx", type=int, default=0, help="custom decode workload: context length (with --batch)")
@@ -372,6 +374,40 @@ def main():
         raise RuntimeError("device status set during the E4M3 variant run")
     del xf
 
+    # ---- one whole SGA layer (a separate configuration): h -> projections ->
+    # the path -> W_UV, o_proj, on the same caches (the new tokens' rows are
+    # rewritten at their positions every step), timed like the main region.
+    layer = None
+    if args.layer:
+        lw_t = synth.make_layer_weights(device=dev, seed=rank)
+        lw = sga.layer_weights(lw_t)
+        gl = torch.Generator(device=dev).manual_seed(rank + 99)
+        h = torch.randn((B, T, synth.D_MODEL), generator=gl, device=dev).to(torch.bfloat16)
+        ws_layer = sga.alloc_layer_workspace(dims, lw, sga.LAYER_FORWARD, dev)
+        y = torch.empty((B, T, synth.D_MODEL), dtype=torch.float32, device=dev)
+
+        def layer_step():
+            sga.layer_forward(lw_t, h, x["q_pos"], x["kv"], x["k_idx"], top_k=K, idx_out=idx, y=y, ws=ws_layer,
+                              stream=stream)
+
+        for _ in range(max(args.warmup, 3)):
+            layer_step()
+        torch.cuda.synchronize(dev)
+        if dist is not None:
+            dist.barrier()
+        s4, e4 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s4.record(stream)
+        for _ in range(args.steps):
+            layer_step()
+        e4.record(stream)
+        torch.cuda.synchronize(dev)
+        layer_ms = max_over_ranks(dist, dev, s4.elapsed_time(e4))
+        if sga.device_status(ws_layer) != 0:
+            raise RuntimeError("device status set during the layer variant run")
+        weight_bytes = sum(t.numel() * t.element_size() for t in lw_t.values())
+        layer = {"ms": layer_ms, "weight_bytes": weight_bytes,
+                 "act_bytes": h.numel() * 2 + y.numel() * 4}
+
     if dist is not None:
         dist.barrier()
         dist.destroy_process_group()
@@ -400,6 +436,19 @@ def main():
         "path_roofline": {"achieved_gbs": fp8_gbs, "frac_of_8tbs": fp8_gbs / NOMINAL_HBM_GBS,
                           "frac_of_measured": fp8_gbs / peak, "bytes_per_query": ab8["total"]},
         "gpu_launches": launches_per_step * args.steps}}
+    if layer is not None:
+        layer_step_ms = layer["ms"] / args.steps
+        layer_bytes = ab["total"] * rows + layer["weight_bytes"] + layer["act_bytes"]
+        layer_gbs = layer_bytes / (layer_step_ms * 1e-3) / 1e9
+        variants["sga_layer"] = {
+            "value": whole_job_rate(rows, args.steps, world, layer["ms"]), "unit": UNIT, "ms_per_step": layer_step_ms,
+            "config": f"{wl.name} as one whole SGA layer: d_model 7168, q rank 1536, projections in cuBLAS "
+                      f"(bf16, fp32 accumulation), bf16 activations between contractions",
+            "path_roofline": {"achieved_gbs": layer_gbs, "frac_of_8tbs": layer_gbs / NOMINAL_HBM_GBS,
+                              "frac_of_measured": layer_gbs / peak, "bytes_per_step": layer_bytes,
+                              "weight_bytes": layer["weight_bytes"]},
+            # own kernels per step: two projection preps, three bf16 conversions, the path's three
+            "gpu_launches": 8 * args.steps}
 
     cpu = None
     if not args.no_cpu_baseline and world == 1:

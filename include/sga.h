@@ -208,6 +208,94 @@ SGA_API sga_status_t sga_clear_device_status(void* ws, sga_stream_t stream);
 SGA_API sga_status_t sga_topk_select_noalloc(const sga_dims_t* dims, const float* scores, const int32_t* q_pos,
                                              int32_t* idx, sga_stream_t stream);
 
+/* ------------------------------------------------------------------------
+ * One SGA attention layer: the projections either side of the path.
+ * Sources: archdb "A.X K2", attention fields (64 heads; qk head dim 192 = 128
+ * nope + 64 rope; v head dim 128; KV latent 512; q low-rank width 1536; a
+ * 64-dim decoupled RoPE key shared across heads; partial RoPE with base 1e6;
+ * no per-head QK norm; no projection bias), gate field (head-specific sigmoid
+ * gate on the attention output before o_proj, projected jointly with the
+ * query) and token-selection field (DSA-style indexer, 64 heads of dim 128).
+ * For new tokens h [B][T][D] at positions q_pos:
+ *   c_q = W_DQ h;  [q_nope_h, q_rope_h] = W_UQ_h c_q;  g = W_G c_q
+ *   [c_kv, k_rope] = W_DKV h;  k_idx = W_IK h;  w = W_IW h;  q_idx = W_IQ c_q
+ *   q_rope, k_rope rotated by RoPE at the token's position: interleaved pairs
+ *     (2i, 2i+1), angle q_pos * 1e6^(-i/32), i < 32 (no YaRN factor)
+ *   q_h = [W_UK_h^T q_nope_h, q_rope_h]   (W_UK absorbed into the query)
+ *   kv_cache[b, q_pos] = [c_kv, k_rope];  k_idx_cache[b, q_pos] = k_idx
+ *   idx, out = sga_forward(q_idx, w, k_idx_cache, q, kv_cache, g, q_pos)
+ *   o_h = W_UV_h out_h;  y = W_O [o_1; ...; o_64]
+ * Every activation between two contractions is rounded to bf16 (to nearest,
+ * ties to even); the contractions accumulate in fp32; y is fp32.  The GEMMs
+ * run in cuBLAS (bf16 inputs, fp32 accumulation); the first call on each
+ * device creates the library's cuBLAS handle, so make it outside stream
+ * capture; the handle lives until the process exits.  Calls on one device
+ * share that handle and must be ordered on one stream.
+ *
+ * Weights: bf16, row-major, `out = W in` (torch Linear layout), packed so the
+ * projections that read the same input are one GEMM:
+ *   w_hq [R + 768][D]:        rows W_DQ (R) | W_DKV (576: c_kv then k_rope)
+ *                             | W_IK (128) | W_IW (64)
+ *   w_cq [20544][R]:          rows W_UQ (head h: rows 192h .. 192h+191, the 128
+ *                             nope rows first) | W_G (64) | W_IQ (head j: rows
+ *                             12352 + 128j ..)
+ *   w_uk [64][128][512]:      k_nope_h = w_uk[h] c_kv
+ *   w_uv [64][128][512]:      o_h = w_uv[h] out_h
+ *   w_o  [D][8192]
+ * D = d_model (7168 in A.X K2) and R = q_rank (1536) are multiples of 8; every
+ * weight pointer is 16-byte aligned.  The new tokens of one sequence must
+ * have distinct positions.                                                   */
+
+typedef struct {
+  int32_t d_model; /* D */
+  int32_t q_rank;  /* R */
+  const sga_bf16_t* w_hq;
+  const sga_bf16_t* w_cq;
+  const sga_bf16_t* w_uk;
+  const sga_bf16_t* w_uv;
+  const sga_bf16_t* w_o;
+} sga_layer_weights_t;
+
+typedef enum {
+  SGA_LAYER_PROJECT = 0, /* sga_layer_project */
+  SGA_LAYER_OUTPUT = 1,  /* sga_layer_output */
+  SGA_LAYER_FORWARD = 2  /* sga_layer_forward (covers both) */
+} sga_layer_op_t;
+
+/* Bytes of workspace a layer call needs (256-byte aligned, zero-filled before
+ * the first sga_layer_forward, as for sga_forward; the layer's status word is
+ * at its start).  Depends on dims and on weights->d_model / q_rank only.
+ * SGA_ERR_INVALID_ARG for bad dims, sizes or a null `bytes`. */
+SGA_API sga_status_t sga_layer_workspace_size(const sga_dims_t* dims, const sga_layer_weights_t* weights,
+                                              sga_layer_op_t op, size_t* bytes);
+
+/* The projections in front of the path for new tokens:
+ *   h      [B][T][D] bf16              q_pos [B][T] int32, 0 <= q_pos < L
+ *   kv_cache [B][L][576] bf16, k_idx_cache [B][L][128] bf16: the rows at
+ *          (b, q_pos[b,i]) are overwritten with the new tokens' rows; no
+ *          other row is touched
+ *   q [B][T][64][576], gate [B][T][64], q_idx [B][T][64][128], w [B][T][64]
+ *          bf16 (outputs): the inputs sga_forward takes for these tokens
+ * Device error: a position outside [0, L) (that token's cache rows are not
+ * written). */
+SGA_API sga_status_t sga_layer_project(const sga_dims_t* dims, const sga_layer_weights_t* weights,
+                                       const sga_bf16_t* h, const int32_t* q_pos, sga_bf16_t* kv_cache,
+                                       sga_bf16_t* k_idx_cache, sga_bf16_t* q, sga_bf16_t* gate, sga_bf16_t* q_idx,
+                                       sga_bf16_t* w, void* ws, size_t ws_bytes, sga_stream_t stream);
+
+/* The projections after the path: out [B][T][64][512] fp32 (the gated
+ * attention output sga_forward writes) -> y [B][T][D] fp32. */
+SGA_API sga_status_t sga_layer_output(const sga_dims_t* dims, const sga_layer_weights_t* weights, const float* out,
+                                      float* y, void* ws, size_t ws_bytes, sga_stream_t stream);
+
+/* The whole layer: sga_layer_project -> sga_forward -> sga_layer_output, with
+ * every intermediate in the workspace.  idx_out [B][T][K] int32 may be NULL;
+ * dims->top_k as for sga_forward. */
+SGA_API sga_status_t sga_layer_forward(const sga_dims_t* dims, const sga_layer_weights_t* weights,
+                                       const sga_bf16_t* h, const int32_t* q_pos, sga_bf16_t* kv_cache,
+                                       sga_bf16_t* k_idx_cache, int32_t* idx_out, float* y, void* ws, size_t ws_bytes,
+                                       sga_stream_t stream);
+
 #ifdef __cplusplus
 } /* extern "C" */
 #endif

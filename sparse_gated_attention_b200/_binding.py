@@ -24,12 +24,18 @@ V_DIM = 512
 TOP_K = 2048
 
 OP_INDEX_SCORES, OP_TOPK_SELECT, OP_SPARSE_MLA_ATTEND, OP_FORWARD = 0, 1, 2, 3
+LAYER_PROJECT, LAYER_OUTPUT, LAYER_FORWARD = 0, 1, 2
+# packed layer weights (see sga_layer_weights_t): rows of w_hq after W_DQ, rows of w_cq
+HQ_EXTRA = QK_DIM + INDEX_DIM + INDEX_HEADS  # 768
+CQ_ROWS = HEADS * 192 + HEADS + INDEX_HEADS * INDEX_DIM  # 20,544
+V_HEAD = 128
 STATUS_NAMES = {0: "SGA_OK", 1: "SGA_ERR_INVALID_ARG", 2: "SGA_ERR_UNSUPPORTED", 3: "SGA_ERR_WORKSPACE",
                 4: "SGA_ERR_CUDA", 5: "SGA_ERR_TIMEOUT", 6: "SGA_ERR_DEVICE_ARG"}
 
 EXPORTED = ["sga_abi_version", "sga_status_string", "sga_workspace_size", "sga_index_scores", "sga_topk_select",
             "sga_sparse_mla_attend", "sga_forward", "sga_get_device_status", "sga_clear_device_status",
-            "sga_topk_select_noalloc", "sga_index_scores_fp8", "sga_forward_fp8"]
+            "sga_topk_select_noalloc", "sga_index_scores_fp8", "sga_forward_fp8", "sga_layer_workspace_size",
+            "sga_layer_project", "sga_layer_output", "sga_layer_forward"]
 NOALLOC_SCRATCH_BYTES = 256 + 4 * 1024 * 1024
 
 
@@ -42,6 +48,12 @@ class SGAError(RuntimeError):
 class Dims(ctypes.Structure):
     _fields_ = [("batch", ctypes.c_int32), ("n_q", ctypes.c_int32), ("kv_stride", ctypes.c_int32),
                 ("top_k", ctypes.c_int32)]
+
+
+class LayerWeights(ctypes.Structure):
+    _fields_ = [("d_model", ctypes.c_int32), ("q_rank", ctypes.c_int32), ("w_hq", ctypes.c_void_p),
+                ("w_cq", ctypes.c_void_p), ("w_uk", ctypes.c_void_p), ("w_uv", ctypes.c_void_p),
+                ("w_o", ctypes.c_void_p)]
 
 
 _lib = None
@@ -70,6 +82,11 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "sga_topk_select_noalloc": (ctypes.c_int, [D, P, P, P, P]),
         "sga_index_scores_fp8": (ctypes.c_int, [D, P, P, P, P, P, P, sz, P]),
         "sga_forward_fp8": (ctypes.c_int, [D, P, P, P, P, P, P, P, P, P, P, sz, P]),
+        "sga_layer_workspace_size": (ctypes.c_int, [D, ctypes.POINTER(LayerWeights), ctypes.c_int,
+                                                    ctypes.POINTER(sz)]),
+        "sga_layer_project": (ctypes.c_int, [D, ctypes.POINTER(LayerWeights), P, P, P, P, P, P, P, P, P, sz, P]),
+        "sga_layer_output": (ctypes.c_int, [D, ctypes.POINTER(LayerWeights), P, P, P, sz, P]),
+        "sga_layer_forward": (ctypes.c_int, [D, ctypes.POINTER(LayerWeights), P, P, P, P, P, P, P, sz, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -289,3 +306,97 @@ def forward_fp8(q_idx, w, k_idx, q, kv, gate, q_pos, top_k: int = TOP_K, idx_out
         ctypes.byref(dims), _ptr(q_idx), _ptr(w), _ptr(k_idx), _ptr(q), _ptr(kv), _ptr(gate), _ptr(q_pos),
         _ptr(idx_out), _ptr(out), _ptr(ws), ws.numel(), _stream(stream)))
     return idx_out, out
+
+
+# ----------------------------------------------------------------------------- one SGA layer
+def layer_weights(wts: dict) -> LayerWeights:
+    """The C struct for packed bf16 weights {w_hq, w_cq, w_uk, w_uv, w_o} (see sga_layer_weights_t).
+    The tensors must stay alive while the struct is in use."""
+    w_hq, w_cq, w_o = wts["w_hq"], wts["w_cq"], wts["w_o"]
+    D = w_hq.shape[1]
+    R = w_hq.shape[0] - HQ_EXTRA
+    _need(w_hq, "w_hq", torch.bfloat16, (R + HQ_EXTRA, D))
+    _need(w_cq, "w_cq", torch.bfloat16, (CQ_ROWS, R))
+    _need(wts["w_uk"], "w_uk", torch.bfloat16, (HEADS, 128, V_DIM))
+    _need(wts["w_uv"], "w_uv", torch.bfloat16, (HEADS, V_HEAD, V_DIM))
+    _need(w_o, "w_o", torch.bfloat16, (D, HEADS * V_HEAD))
+    return LayerWeights(int(D), int(R), w_hq.data_ptr(), w_cq.data_ptr(), wts["w_uk"].data_ptr(),
+                        wts["w_uv"].data_ptr(), w_o.data_ptr())
+
+
+def layer_workspace_size(dims: Dims, lw: LayerWeights, op: int = LAYER_FORWARD) -> int:
+    out = ctypes.c_size_t(0)
+    _check("sga_layer_workspace_size", load_library().sga_layer_workspace_size(
+        ctypes.byref(dims), ctypes.byref(lw), int(op), ctypes.byref(out)))
+    return int(out.value)
+
+
+def alloc_layer_workspace(dims: Dims, lw: LayerWeights, op: int = LAYER_FORWARD, device=None) -> torch.Tensor:
+    """A zero-filled layer workspace (ready for the first sga_layer_forward)."""
+    return torch.zeros(layer_workspace_size(dims, lw, op), dtype=torch.uint8, device=device or "cuda")
+
+
+def _layer_common(wts, h, q_pos, kv_cache, k_idx_cache):
+    lw = layer_weights(wts)
+    B, T, D = h.shape
+    L = kv_cache.shape[1]
+    _need(h, "h", torch.bfloat16, (B, T, lw.d_model))
+    _need(q_pos, "q_pos", torch.int32, (B, T))
+    _need(kv_cache, "kv_cache", torch.bfloat16, (B, L, QK_DIM))
+    _need(k_idx_cache, "k_idx_cache", torch.bfloat16, (B, L, INDEX_DIM))
+    return lw, B, T, L
+
+
+def layer_project(wts, h, q_pos, kv_cache, k_idx_cache, ws=None, stream=None):
+    """The projections in front of the path (sga_layer_project).  Writes the new tokens'
+    rows into the caches in place; returns dict(q, gate, q_idx, w), bf16."""
+    lw, B, T, L = _layer_common(wts, h, q_pos, kv_cache, k_idx_cache)
+    dev = h.device
+    q = torch.empty((B, T, HEADS, QK_DIM), dtype=torch.bfloat16, device=dev)
+    gate = torch.empty((B, T, HEADS), dtype=torch.bfloat16, device=dev)
+    q_idx = torch.empty((B, T, INDEX_HEADS, INDEX_DIM), dtype=torch.bfloat16, device=dev)
+    w = torch.empty((B, T, INDEX_HEADS), dtype=torch.bfloat16, device=dev)
+    dims = make_dims(B, T, L)
+    if ws is None:
+        ws = alloc_layer_workspace(dims, lw, LAYER_PROJECT, dev)
+    _check("sga_layer_project", load_library().sga_layer_project(
+        ctypes.byref(dims), ctypes.byref(lw), _ptr(h), _ptr(q_pos), _ptr(kv_cache), _ptr(k_idx_cache), _ptr(q),
+        _ptr(gate), _ptr(q_idx), _ptr(w), _ptr(ws), ws.numel(), _stream(stream)))
+    return {"q": q, "gate": gate, "q_idx": q_idx, "w": w}
+
+
+def layer_output(wts, out, y=None, ws=None, stream=None):
+    """The projections after the path (sga_layer_output): out [B,T,64,512] fp32 -> y [B,T,D] fp32."""
+    lw = layer_weights(wts)
+    B, T = out.shape[0], out.shape[1]
+    _need(out, "out", torch.float32, (B, T, HEADS, V_DIM))
+    if y is None:
+        y = torch.empty((B, T, lw.d_model), dtype=torch.float32, device=out.device)
+    _need(y, "y", torch.float32, (B, T, lw.d_model))
+    dims = make_dims(B, T, 1)
+    if ws is None:
+        ws = alloc_layer_workspace(dims, lw, LAYER_OUTPUT, out.device)
+    _check("sga_layer_output", load_library().sga_layer_output(
+        ctypes.byref(dims), ctypes.byref(lw), _ptr(out), _ptr(y), _ptr(ws), ws.numel(), _stream(stream)))
+    return y
+
+
+def layer_forward(wts, h, q_pos, kv_cache, k_idx_cache, top_k: int = TOP_K, idx_out=None, y=None, ws=None,
+                  stream=None, return_idx: bool = True):
+    """One SGA layer (sga_layer_forward).  Writes the new tokens' cache rows in place;
+    returns (idx [B,T,K] or None, y [B,T,D] fp32)."""
+    lw, B, T, L = _layer_common(wts, h, q_pos, kv_cache, k_idx_cache)
+    dims = make_dims(B, T, L, top_k)
+    if idx_out is None and return_idx:
+        idx_out = torch.empty((B, T, top_k), dtype=torch.int32, device=h.device)
+    if idx_out is not None:
+        _need(idx_out, "idx_out", torch.int32, (B, T, top_k))
+    if y is None:
+        y = torch.empty((B, T, lw.d_model), dtype=torch.float32, device=h.device)
+    _need(y, "y", torch.float32, (B, T, lw.d_model))
+    if ws is None:
+        ws = alloc_layer_workspace(dims, lw, LAYER_FORWARD, h.device)
+    _check("sga_layer_forward", load_library().sga_layer_forward(
+        ctypes.byref(dims), ctypes.byref(lw), _ptr(h), _ptr(q_pos), _ptr(kv_cache), _ptr(k_idx_cache),
+        _ptr(idx_out), _ptr(y), _ptr(ws), ws.numel(), _stream(stream)))
+    return idx_out, y

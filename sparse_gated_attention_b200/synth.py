@@ -18,6 +18,19 @@ memory stays at one sequence's worth of fp32 temporaries):
 * ``q_pos``  [B,T] int32   decode: L-1 (one query at the last position);
                            chunked prefill: first_pos .. first_pos+T-1
 
+One SGA layer around the path (``make_layer_inputs``) adds, from a second
+generator seeded with ``seed + LAYER_SEED_OFFSET`` and drawn in this order:
+
+* ``h``      [B,T,D]       the new tokens' hidden states, N(0,1) rounded to bf16
+* the packed projection weights (the layout of ``sga_layer_weights_t``), each
+  N(0,1) / sqrt(fan_in) rounded to bf16 so activations stay O(1):
+  ``w_hq`` [R+768, D] (fan_in D), ``w_cq`` [20544, R] (fan_in R),
+  ``w_uk`` [64,128,512] and ``w_uv`` [64,128,512] (fan_in 512), ``w_o`` [D, 8192]
+  (fan_in 8192); D = 7168 and R = 1536 are the archdb "A.X K2" residual width
+  and q low-rank width.
+The caches (``kv``, ``k_idx``) and ``q_pos`` are those of ``make_inputs``; the
+layer overwrites the rows at ``q_pos`` with the new tokens' projected rows.
+
 Integer indexer inputs make every indexer score an exact integer in fp32, so
 the selected positions can be compared bit for bit.  The shapes follow the
 indexer and attention fields of the archdb "A.X K2" page (64 indexer heads of
@@ -133,3 +146,41 @@ def input_bytes(wl: Workload) -> dict:
     B, T, L = wl.batch, wl.n_q, wl.ctx
     return dict(q_idx=B * T * INDEX_HEADS * INDEX_DIM * 2, w=B * T * INDEX_HEADS * 2, k_idx=B * L * INDEX_DIM * 2,
                 q=B * T * HEADS * QK_DIM * 2, kv=B * L * QK_DIM * 2, gate=B * T * HEADS * 2, q_pos=B * T * 4)
+
+
+D_MODEL = 7168
+Q_RANK = 1536
+LAYER_SEED_OFFSET = 0x5EED
+HQ_EXTRA = QK_DIM + INDEX_DIM + INDEX_HEADS  # rows of w_hq after W_DQ
+CQ_ROWS = HEADS * 192 + HEADS + INDEX_HEADS * INDEX_DIM
+
+
+def _scaled(g, shape, fan_in, device):
+    return (torch.randn(shape, generator=g, device=device, dtype=torch.float32) * fan_in ** -0.5).to(torch.bfloat16)
+
+
+def make_layer_weights(d_model: int = D_MODEL, q_rank: int = Q_RANK, device="cpu", seed: int = 0) -> dict:
+    """Packed bf16 projection weights of one layer (see the module docstring)."""
+    device = torch.device(device)
+    g = torch.Generator(device=device)
+    g.manual_seed(seed + LAYER_SEED_OFFSET)
+    return {
+        "w_hq": _scaled(g, (q_rank + HQ_EXTRA, d_model), d_model, device),
+        "w_cq": _scaled(g, (CQ_ROWS, q_rank), q_rank, device),
+        "w_uk": _scaled(g, (HEADS, 128, V_DIM), V_DIM, device),
+        "w_uv": _scaled(g, (HEADS, 128, V_DIM), V_DIM, device),
+        "w_o": _scaled(g, (d_model, HEADS * 128), HEADS * 128, device),
+    }
+
+
+def make_layer_inputs(wl: Workload, d_model: int = D_MODEL, q_rank: int = Q_RANK, device="cpu",
+                      seed: int = 0) -> dict:
+    """The workload's caches and positions, the new tokens' hidden states h and
+    the layer's packed weights (see the module docstring)."""
+    x = make_inputs(wl, device, seed)
+    device = torch.device(device)
+    g = torch.Generator(device=device)
+    g.manual_seed(seed + 2 * LAYER_SEED_OFFSET)
+    h = torch.randn((wl.batch, wl.n_q, d_model), generator=g, device=device, dtype=torch.float32).to(torch.bfloat16)
+    return {"h": h, "q_pos": x["q_pos"], "kv": x["kv"], "k_idx": x["k_idx"],
+            "weights": make_layer_weights(d_model, q_rank, device, seed)}
