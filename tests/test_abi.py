@@ -109,3 +109,66 @@ def test_binding_fails_loudly_without_library(tmp_path):
             _binding.load_library(str(tmp_path / "missing.so"))
     finally:
         _binding._lib = saved
+
+
+# ----------------------------------------------------------------------------- one SGA layer
+def _layer_weights(d_model=7168, q_rank=1536, w_hq=0x300000, w_cq=0x400000, w_uk=0x500000, w_uv=0x600000,
+                   w_o=0x700000):
+    return sga.LayerWeights(d_model, q_rank, w_hq, w_cq, w_uk, w_uv, w_o)
+
+
+def test_layer_workspace_sizes(lib):
+    d = sga.make_dims(32, 1, 131072)
+    lw = _layer_weights()
+    proj = sga.layer_workspace_size(d, lw, sga.LAYER_PROJECT)
+    outp = sga.layer_workspace_size(d, lw, sga.LAYER_OUTPUT)
+    fwd = sga.layer_workspace_size(d, lw, sga.LAYER_FORWARD)
+    cublas = 32 << 20
+    rows = 32
+    # the projections keep both GEMM outputs in fp32, c_q and q_nope in bf16, q_lat in fp32
+    assert proj >= 256 + cublas + rows * 4 * (1536 + 768 + 20544 + 64 * 512) + rows * 2 * (1536 + 64 * 128)
+    # the output side keeps out and o in bf16 and o in fp32
+    assert outp >= 256 + cublas + rows * (2 * 64 * 512 + 6 * 8192)
+    # the whole layer also holds the path's workspace and the path's inputs and output
+    assert fwd >= sga.workspace_size(d, sga.OP_FORWARD) + proj - 256 + outp - 256 - cublas
+    # sizes depend on q_rank, not on d_model
+    assert sga.layer_workspace_size(d, _layer_weights(d_model=4096), sga.LAYER_FORWARD) == fwd
+    assert sga.layer_workspace_size(d, _layer_weights(q_rank=1024), sga.LAYER_FORWARD) < fwd
+
+
+@pytest.mark.parametrize("d_model,q_rank", [(7170, 1536), (7168, 1530), (0, 1536), (7168, 0)])
+def test_layer_bad_widths_rejected(lib, d_model, q_rank):
+    d = sga.make_dims(2, 1, 1000)
+    out = ctypes.c_size_t(0)
+    lw = _layer_weights(d_model=d_model, q_rank=q_rank)
+    assert lib.sga_layer_workspace_size(ctypes.byref(d), ctypes.byref(lw), sga.LAYER_FORWARD, ctypes.byref(out)) == 1
+
+
+def test_layer_bad_arguments_rejected_on_host(lib):
+    d = sga.make_dims(2, 1, 1000)
+    P = ctypes.c_void_p
+    good, odd, ws = P(0x100000), P(0x100002), P(0x20000000)
+    big = 1 << 30
+    out = ctypes.c_size_t(0)
+    lw = _layer_weights()
+    assert lib.sga_layer_workspace_size(ctypes.byref(d), ctypes.byref(lw), 7, ctypes.byref(out)) == 1
+    assert lib.sga_layer_workspace_size(ctypes.byref(d), None, sga.LAYER_FORWARD, ctypes.byref(out)) == 1
+    # null or misaligned weights and activations
+    for bad in (_layer_weights(w_hq=0), _layer_weights(w_cq=0x400002), _layer_weights(w_uk=0)):
+        assert lib.sga_layer_project(ctypes.byref(d), ctypes.byref(bad), good, good, good, good, good, good, good,
+                                     good, ws, big, None) == 1
+    for bad in (_layer_weights(w_uv=0), _layer_weights(w_o=0x700008)):
+        assert lib.sga_layer_output(ctypes.byref(d), ctypes.byref(bad), good, good, ws, big, None) == 1
+    assert lib.sga_layer_project(ctypes.byref(d), ctypes.byref(lw), odd, good, good, good, good, good, good, good,
+                                 ws, big, None) == 1
+    assert lib.sga_layer_forward(ctypes.byref(d), ctypes.byref(lw), good, good, good, good, None, odd, ws, big,
+                                 None) == 1
+    # workspace: null, misaligned, too small
+    assert lib.sga_layer_output(ctypes.byref(d), ctypes.byref(lw), good, good, None, big, None) == 3
+    assert lib.sga_layer_output(ctypes.byref(d), ctypes.byref(lw), good, good, P(0x20000010), big, None) == 3
+    assert lib.sga_layer_forward(ctypes.byref(d), ctypes.byref(lw), good, good, good, good, None, good, ws, 4096,
+                                 None) == 3
+    # the whole layer checks the path's top_k too
+    bad_k = sga.make_dims(2, 1, 1000, 100)
+    assert lib.sga_layer_workspace_size(ctypes.byref(bad_k), ctypes.byref(lw), sga.LAYER_FORWARD,
+                                        ctypes.byref(out)) == 1
