@@ -27,9 +27,23 @@ Each function follows one step of the method:
   a bf16 value, so the codes are converted exactly and the bf16 oracle runs
   unchanged.
 
-Pins: every function is checked in ``tests/test_oracle_pins.py`` against closed
-forms, invariants, a hand-worked fixture and library routines (numpy matmul,
-torch SDPA in fp64, Python's sort), not against itself.
+Two modules build on these steps in plain numpy fp64:
+
+* ``oracle.layer`` - one SGA attention layer: the projections either side of
+  the path (q low-rank path, decoupled RoPE, the gate projected with the query,
+  W_UK absorption, the cache update, W_UV and o_proj; archdb "A.X K2"
+  attention and gate fields).
+* ``oracle.warmup`` - the indexer's sparse warm-up objective (a KL divergence
+  from the frozen attention's distribution over the indexer's own top-k) and
+  its gradients (arXiv abstract "A.X K2 Technical Report": the indexer is
+  optimised against its own sparse top-k selection).
+
+Pins: every function is checked against closed forms, invariants, a
+hand-worked fixture and library routines (numpy matmul, torch SDPA and softmax
+in fp64, torch's bf16 conversion, Python's sort, finite differences), not
+against itself: ``tests/test_oracle_pins.py``, ``tests/test_layer_oracle.py``
+and ``tests/test_warmup_oracle.py``, with planted mistakes in the
+``*_mutants.py`` tests.
 """
 from __future__ import annotations
 
