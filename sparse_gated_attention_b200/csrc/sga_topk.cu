@@ -21,14 +21,20 @@
 //      same bin.  Levels stop when that bin fits a candidate list (4096 keys)
 //      or is a single key.  Under sga_forward the indexer has already counted
 //      the first level, so that pass is skipped.
-//   2. If the bin is wider than one key: one ballot pass collects the keys in
-//      the bin into the CTA's candidate list; every CTA copies all lists over
-//      distributed shared memory and narrows them to K* itself (no leader).
-//   3. One ballot pass builds, per 32 positions, a selection word (key > K*)
-//      and a tie word (key == K*); lane j keeps the words of step j.  Warp and
-//      block scans of their popcounts plus the other CTAs' two counts give
-//      each set bit its output slot; ties are taken in position order until
-//      the K slots are full.
+//   2. One ballot pass builds, per 32 positions, an "above" word (keys whose
+//      bin lies above the selected bin: selected whatever K* is) and an
+//      in-bin word; lane j keeps the words of step j.  If the bin is wider
+//      than one key, its keys are listed in the CTA's candidate list (one
+//      atomic per warp), each CTA pushes its list length to every CTA with a
+//      remote store, and after one cluster barrier every CTA copies the other
+//      lists over distributed shared memory and narrows them to K* itself (no
+//      leader).
+//   3. The in-bin bits are split against K* from the resident scores into
+//      selected (key > K*) and tie (key == K*) bits.  Warp and block scans of
+//      the word popcounts, plus the (selected, ties) counts every CTA pushes
+//      to the others, give each set bit its output slot; ties are taken in
+//      position order until the K slots are full.  Two cluster barriers follow
+//      the radix levels and none precedes the exit.
 // Streaming kernel (longer rows): the segment streams through a 3-slot ring of
 // 32 KB bulk copies once per pass; the second step records selection / tie
 // words (shared memory up to 65536 positions, else the workspace) and stages
