@@ -296,6 +296,31 @@ SGA_API sga_status_t sga_layer_forward(const sga_dims_t* dims, const sga_layer_w
                                        sga_bf16_t* k_idx_cache, int32_t* idx_out, float* y, void* ws, size_t ws_bytes,
                                        sga_stream_t stream);
 
+/* ------------------------------------------------------------------------
+ * The indexer's sparse warm-up objective and its gradients (arXiv abstract
+ * "A.X K2 Technical Report": the indexer is optimised against its own sparse
+ * top-k selection rather than the dense attention distribution; archdb
+ * "A.X K2", stage notes: indexer-only training with the backbone frozen).
+ * The pages give no formula; the reading, for query t with its selection S =
+ * the valid entries of idx[b,i,:] (as sga_forward returns them):
+ *   p(s)  = (1/64) sum_h softmax_{s in S}((q[b,i,h,:] . kv[b,s,:]) * 192^-0.5)
+ *           the frozen attention's distribution (a target: no gradient)
+ *   r(s)  = softmax_{s in S}(score(s)), score as in sga_index_scores
+ *   loss[b,i] = KL(p || r)
+ * and the gradients of the loss with respect to the indexer's inputs:
+ *   grad_q_idx [B][T][64][128] fp32, grad_w [B][T][64] fp32 (overwritten);
+ *   grad_k_idx [B][L][128] fp32: ADDED to (zero it before the first call;
+ *   a position selected by several queries receives all their terms).
+ * The ReLU passes no gradient at 0.  Inputs as for sga_forward; loss [B][T]
+ * fp32.  Workspace: sga_indexer_warmup_workspace_size bytes, 256-byte aligned,
+ * its status word at the start (zero-filled before the first call).  B*T is
+ * at most 65535.  Device error: an index outside [-1, L) (treated as empty). */
+SGA_API sga_status_t sga_indexer_warmup_workspace_size(const sga_dims_t* dims, size_t* bytes);
+SGA_API sga_status_t sga_indexer_warmup(const sga_dims_t* dims, const sga_bf16_t* q_idx, const sga_bf16_t* w,
+                                        const sga_bf16_t* k_idx, const sga_bf16_t* q, const sga_bf16_t* kv,
+                                        const int32_t* idx, float* loss, float* grad_q_idx, float* grad_w,
+                                        float* grad_k_idx, void* ws, size_t ws_bytes, sga_stream_t stream);
+
 #ifdef __cplusplus
 } /* extern "C" */
 #endif

@@ -35,7 +35,8 @@ STATUS_NAMES = {0: "SGA_OK", 1: "SGA_ERR_INVALID_ARG", 2: "SGA_ERR_UNSUPPORTED",
 EXPORTED = ["sga_abi_version", "sga_status_string", "sga_workspace_size", "sga_index_scores", "sga_topk_select",
             "sga_sparse_mla_attend", "sga_forward", "sga_get_device_status", "sga_clear_device_status",
             "sga_topk_select_noalloc", "sga_index_scores_fp8", "sga_forward_fp8", "sga_layer_workspace_size",
-            "sga_layer_project", "sga_layer_output", "sga_layer_forward"]
+            "sga_layer_project", "sga_layer_output", "sga_layer_forward", "sga_indexer_warmup_workspace_size",
+            "sga_indexer_warmup"]
 NOALLOC_SCRATCH_BYTES = 256 + 4 * 1024 * 1024
 
 
@@ -87,6 +88,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "sga_layer_project": (ctypes.c_int, [D, ctypes.POINTER(LayerWeights), P, P, P, P, P, P, P, P, P, sz, P]),
         "sga_layer_output": (ctypes.c_int, [D, ctypes.POINTER(LayerWeights), P, P, P, sz, P]),
         "sga_layer_forward": (ctypes.c_int, [D, ctypes.POINTER(LayerWeights), P, P, P, P, P, P, P, sz, P]),
+        "sga_indexer_warmup_workspace_size": (ctypes.c_int, [D, ctypes.POINTER(sz)]),
+        "sga_indexer_warmup": (ctypes.c_int, [D, P, P, P, P, P, P, P, P, P, P, P, sz, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -400,3 +403,40 @@ def layer_forward(wts, h, q_pos, kv_cache, k_idx_cache, top_k: int = TOP_K, idx_
         ctypes.byref(dims), ctypes.byref(lw), _ptr(h), _ptr(q_pos), _ptr(kv_cache), _ptr(k_idx_cache),
         _ptr(idx_out), _ptr(y), _ptr(ws), ws.numel(), _stream(stream)))
     return idx_out, y
+
+
+# ----------------------------------------------------------------------------- indexer warm-up objective
+def indexer_warmup_workspace_size(dims: Dims) -> int:
+    out = ctypes.c_size_t(0)
+    _check("sga_indexer_warmup_workspace_size",
+           load_library().sga_indexer_warmup_workspace_size(ctypes.byref(dims), ctypes.byref(out)))
+    return int(out.value)
+
+
+def indexer_warmup(q_idx, w, k_idx, q, kv, idx, grad_k_idx=None, ws=None, stream=None):
+    """The indexer's sparse warm-up objective over the selection idx (sga_indexer_warmup).
+    Returns dict(loss [B,T], grad_q_idx [B,T,64,128], grad_w [B,T,64], grad_k_idx [B,L,128]),
+    fp32; grad_k_idx is added to (a zero-filled tensor is made when none is passed)."""
+    B, T = q_idx.shape[0], q_idx.shape[1]
+    L = k_idx.shape[1]
+    K = idx.shape[-1]
+    _need(q_idx, "q_idx", torch.bfloat16, (B, T, INDEX_HEADS, INDEX_DIM))
+    _need(w, "w", torch.bfloat16, (B, T, INDEX_HEADS))
+    _need(k_idx, "k_idx", torch.bfloat16, (B, L, INDEX_DIM))
+    _need(q, "q", torch.bfloat16, (B, T, HEADS, QK_DIM))
+    _need(kv, "kv", torch.bfloat16, (B, L, QK_DIM))
+    _need(idx, "idx", torch.int32, (B, T, K))
+    dev = q_idx.device
+    dims = make_dims(B, T, L, K)
+    loss = torch.empty((B, T), dtype=torch.float32, device=dev)
+    grad_q_idx = torch.empty((B, T, INDEX_HEADS, INDEX_DIM), dtype=torch.float32, device=dev)
+    grad_w = torch.empty((B, T, INDEX_HEADS), dtype=torch.float32, device=dev)
+    if grad_k_idx is None:
+        grad_k_idx = torch.zeros((B, L, INDEX_DIM), dtype=torch.float32, device=dev)
+    _need(grad_k_idx, "grad_k_idx", torch.float32, (B, L, INDEX_DIM))
+    if ws is None:
+        ws = torch.zeros(indexer_warmup_workspace_size(dims), dtype=torch.uint8, device=dev)
+    _check("sga_indexer_warmup", load_library().sga_indexer_warmup(
+        ctypes.byref(dims), _ptr(q_idx), _ptr(w), _ptr(k_idx), _ptr(q), _ptr(kv), _ptr(idx), _ptr(loss),
+        _ptr(grad_q_idx), _ptr(grad_w), _ptr(grad_k_idx), _ptr(ws), ws.numel(), _stream(stream)))
+    return {"loss": loss, "grad_q_idx": grad_q_idx, "grad_w": grad_w, "grad_k_idx": grad_k_idx}

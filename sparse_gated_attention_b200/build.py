@@ -10,7 +10,7 @@ PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libsga.so")
-SOURCES = ["sga_api.cu", "sga_index.cu", "sga_topk.cu", "sga_attend.cu", "sga_layer.cu"]
+SOURCES = ["sga_api.cu", "sga_index.cu", "sga_topk.cu", "sga_attend.cu", "sga_layer.cu", "sga_warmup.cu"]
 DEPS = SOURCES + ["sga_ptx.cuh", "sga_internal.cuh"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 

@@ -172,3 +172,32 @@ def test_layer_bad_arguments_rejected_on_host(lib):
     bad_k = sga.make_dims(2, 1, 1000, 100)
     assert lib.sga_layer_workspace_size(ctypes.byref(bad_k), ctypes.byref(lw), sga.LAYER_FORWARD,
                                         ctypes.byref(out)) == 1
+
+
+# ----------------------------------------------------------------------------- indexer warm-up objective
+def test_warmup_workspace_size(lib):
+    d = sga.make_dims(2, 3, 5000, 2048)
+    rows, K = 6, 2048
+    # status block, then z and a ([rows][64][K] fp32 each), the scores and g ([rows][K] fp32 each)
+    assert sga.indexer_warmup_workspace_size(d) == 256 + 2 * rows * 64 * K * 4 + 2 * rows * K * 4
+
+
+@pytest.mark.parametrize("dims", [(1, 1, 100, 100), (1, 1, 100, 0), (70000, 1, 100, 2048), (0, 1, 100, 2048)])
+def test_warmup_bad_dims_rejected(lib, dims):
+    d = sga.make_dims(*dims)
+    out = ctypes.c_size_t(0)
+    assert lib.sga_indexer_warmup_workspace_size(ctypes.byref(d), ctypes.byref(out)) == 1
+
+
+def test_warmup_bad_arguments_rejected_on_host(lib):
+    d = sga.make_dims(2, 1, 1000, 2048)
+    P = ctypes.c_void_p
+    g, odd, ws = P(0x100000), P(0x100002), P(0x20000000)
+    big = 1 << 30
+    call = lib.sga_indexer_warmup
+    assert call(ctypes.byref(d), None, g, g, g, g, g, g, g, g, g, ws, big, None) == 1   # q_idx null
+    assert call(ctypes.byref(d), g, g, g, odd, g, g, g, g, g, g, ws, big, None) == 1    # q misaligned
+    assert call(ctypes.byref(d), g, g, g, g, g, g, g, g, g, None, ws, big, None) == 1   # grad_k_idx null
+    assert call(ctypes.byref(d), g, g, g, g, g, g, g, g, g, g, None, big, None) == 3    # workspace null
+    assert call(ctypes.byref(d), g, g, g, g, g, g, g, g, g, g, P(0x20000010), big, None) == 3
+    assert call(ctypes.byref(d), g, g, g, g, g, g, g, g, g, g, ws, 1024, None) == 3      # too small
