@@ -1,0 +1,50 @@
+"""GPU parity of sga_indexer_warmup against the warm-up oracle.
+
+Not collected yet (the file name does not start with test_): the warm-up
+kernels have not run on a GPU.  Renamed to test_gpu_warmup.py once they have,
+it joins the GPU suite.  Tolerances: the loss within 1e-4 relative, each
+gradient within rel-L2 1e-3 (fp32 sums of bf16 products against fp64); the
+selection is the oracle's, which the path reproduces bit for bit on these
+integer-valued indexer inputs."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from oracle import warmup as W
+import sparse_gated_attention_b200 as sga
+from sparse_gated_attention_b200 import synth
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _device():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from sparse_gated_attention_b200 import build
+    build.build()
+    sga.load_library()
+    oracle.build()
+
+
+def rel_l2(got, want):
+    return np.linalg.norm(got - want) / max(np.linalg.norm(want), 1e-30)
+
+
+@pytest.mark.parametrize("B,T,L,pos", [(2, 2, 3000, [[2998, 2999], [1200, 2047]]), (1, 1, 500, [[499]]),
+                                       (3, 1, 9000, [[8999], [4500], [100]])])
+def test_indexer_warmup_matches_oracle(B, T, L, pos):
+    wl = synth.custom(batch=B, n_q=T, ctx=L, first_pos=int(np.min(pos)))
+    x = synth.make_inputs(wl, device="cuda", seed=5)
+    q_pos = torch.as_tensor(np.asarray(pos, dtype=np.int32), device="cuda")
+    want = W.warmup_loss(x["q_idx"], x["w"], x["k_idx"], x["q"], x["kv"], q_pos.cpu())
+    idx = torch.as_tensor(want["idx"], device="cuda")  # the oracle's selection (bit-exact with the path's)
+    ws = torch.zeros(sga.indexer_warmup_workspace_size(sga.make_dims(B, T, L)), dtype=torch.uint8, device="cuda")
+    got = sga.indexer_warmup(x["q_idx"], x["w"], x["k_idx"], x["q"], x["kv"], idx, ws=ws)
+    torch.cuda.synchronize()
+    assert sga.device_status(ws) == 0
+    np.testing.assert_allclose(got["loss"].cpu().numpy(), want["per_query"], rtol=1e-4)
+    for k in ("grad_q_idx", "grad_w", "grad_k_idx"):
+        r = rel_l2(got[k].cpu().numpy().astype(np.float64), want[k])
+        assert r <= 1e-3, (k, r)
