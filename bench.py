@@ -35,6 +35,7 @@ METRIC = "SGA decode queries/s at 128K ctx; achieved HBM GB/s vs 8 TB/s roofline
 UNIT = "queries/s"
 NOMINAL_HBM_GBS = 8000.0
 FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
 
 
 def parse_args():
@@ -45,6 +46,8 @@ def parse_args():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=None, help="workload name (default: decode_b32_ctx128k)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-prefill", dest="prefill", action="store_false",
+                    help="skip the chunked-prefill variant (4096 queries over a 128K cache)")
     ap.add_argument("--no-layer", dest="layer", action="store_false",
                     help="skip the whole-layer variant (the projections either side of the path)")
     ap.add_argument("--cpu-sample-queries", type=int, default=0, help="oracle sample size (0 = auto)")
@@ -75,6 +78,22 @@ def measured_peaks():
         return float(d["hbm_gbs"]), "measured"
     except Exception:
         return FALLBACK_HBM_GBS, "fallback"
+
+
+def measured_tensor_peak():
+    """Dense bf16 TFLOP/s measured on this machine (burst: a kernel timed in isolation)."""
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return float(json.load(f)["bf16_tflops"]), "measured"
+    except Exception:
+        return FALLBACK_BF16_TFLOPS, "fallback"
+
+
+def causal_index_flops(positions) -> float:
+    """Multiply-adds of the indexer over every causal key of each query, 2 flops each:
+    2 * 64 heads * 128 dims * (t + 1) per query."""
+    return float(2 * 64 * 128 * sum(int(t) + 1 for t in positions))
 
 
 def kernel_counters(kernel_file: str):
@@ -259,6 +278,59 @@ def config_of(wl):
             "heads": 64, "latent": 576, "index_heads": 64, "index_dim": 128,
             "l2": "inputs larger than L2 (k_idx+kv rows ~1.16 GB/step vs 126 MB L2), no flush",
             "parallelism": "replicas"}
+
+
+def prefill_variant(sga, synth, args, dev, stream, dist, rank) -> dict:
+    """Times sga_forward and the indexer alone on the chunked-prefill workload."""
+    wl = synth.WORKLOADS["prefill_t4096_ctx128k"]
+    x = synth.make_inputs(wl, device=dev, seed=rank)
+    B, T, L, K = wl.batch, wl.n_q, wl.ctx, wl.top_k
+    dims = sga.make_dims(B, T, L, K)
+    ws = sga.alloc_workspace(dims, sga.OP_FORWARD, dev)
+    ws_i = sga.alloc_workspace(dims, sga.OP_INDEX_SCORES, dev)
+    scores = torch.empty((B, T, L), dtype=torch.float32, device=dev)
+    idx = torch.empty((B, T, K), dtype=torch.int32, device=dev)
+    out = torch.empty((B, T, 64, 512), dtype=torch.float32, device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+
+    def forward():
+        sga.forward(x["q_idx"], x["w"], x["k_idx"], x["q"], x["kv"], x["gate"], x["q_pos"], top_k=K, idx_out=idx,
+                    out=out, ws=ws, stream=stream)
+
+    def indexer():
+        sga.index_scores(x["q_idx"], x["w"], x["k_idx"], x["q_pos"], scores=scores, ws=ws_i, stream=stream)
+
+    def per_iteration_ms(fn, n):
+        for _ in range(max(args.warmup, 3)):
+            fn()
+        torch.cuda.synchronize(dev)
+        if dist is not None:
+            dist.barrier()
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n)]
+        for a, b in evs:
+            flush.zero_()
+            a.record(stream)
+            fn()
+            b.record(stream)
+        torch.cuda.synchronize(dev)
+        return [a.elapsed_time(b) for a, b in evs]
+
+    n = max(5, min(args.steps, 20))
+    chunk_ms = max_over_ranks(dist, dev, statistics.median(per_iteration_ms(forward, n)))
+    k1_ms = max_over_ranks(dist, dev, statistics.median(per_iteration_ms(indexer, n)))
+    if sga.device_status(ws) != 0 or sga.device_status(ws_i) != 0:
+        raise RuntimeError("device status set during the prefill variant")
+    positions = x["q_pos"].flatten().tolist()
+    flops = causal_index_flops(positions)
+    peak_tf, peak_kind = measured_tensor_peak()
+    world = dist.get_world_size() if dist is not None else 1
+    k1_tf = flops / (k1_ms * 1e-3) / 1e12
+    return {"value": B * T * world / (chunk_ms * 1e-3), "unit": "queries/s", "ms_per_chunk": chunk_ms,
+            "config": f"{wl.name}: {T} new queries at positions {positions[0]}..{positions[-1]} over a "
+                      f"{L}-row cache, top_k {K}; median of {n} iterations, L2 flushed (256 MB memset) before each",
+            "indexer": {"ms": k1_ms, "tflops": k1_tf, "flops_per_launch": flops, "peak_tflops": peak_tf,
+                        "peak_kind": peak_kind, "frac": k1_tf / peak_tf, "bound": "tensor"},
+            "gpu_launches": 3}
 
 
 def main():
@@ -474,6 +546,19 @@ def main():
         weight_bytes = sum(t.numel() * t.element_size() for t in lw_t.values())
         layer = {"ms": layer_ms, "weight_bytes": weight_bytes,
                  "act_bytes": h.numel() * 2 + y.numel() * 4}
+        del lw_t, ws_layer
+
+    # ---- chunked prefill (a separate configuration): 4096 new queries over a 128K cache.
+    # The indexer is a dense causal contraction here, so it is reported in TFLOP/s against
+    # the bf16 tensor peak, with the whole chunk's time.  L2 is flushed (256 MB memset)
+    # before every timed iteration, outside its events.
+    prefill = None
+    if args.prefill:
+        try:
+            prefill = prefill_variant(sga, synth, args, dev, stream, dist, rank)
+        except (RuntimeError, TypeError, ValueError) as exc:
+            torch.cuda.synchronize(dev)
+            prefill = {"error": f"{type(exc).__name__}: {exc}"}
 
     if dist is not None:
         dist.barrier()
@@ -503,6 +588,8 @@ def main():
         "path_roofline": {"achieved_gbs": fp8_gbs, "frac_of_8tbs": fp8_gbs / NOMINAL_HBM_GBS,
                           "frac_of_measured": fp8_gbs / peak, "bytes_per_query": ab8["total"]},
         "gpu_launches": launches_per_step * args.steps}}
+    if prefill is not None:
+        variants["prefill_t4096_ctx128k"] = prefill
     if layer is not None:
         layer_step_ms = layer["ms"] / args.steps
         layer_bytes = ab["total"] * rows + layer["weight_bytes"] + layer["act_bytes"]

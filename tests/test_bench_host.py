@@ -73,3 +73,18 @@ def test_traffic_is_reported_only_for_the_source_it_was_taken_on(tmp_path, monke
     src.write_text("kernel v2")
     assert bench.kernel_counters("k.cu") is None
     assert bench.kernel_counters("missing.cu") is None
+
+
+def test_causal_indexer_flops_of_the_prefill_chunk():
+    # 4096 queries at positions 126,976..131,071: 2 * 64 * 128 * sum(t + 1) = 8.66 TFLOP
+    positions = range(126976, 131072)
+    assert bench.causal_index_flops(positions) == 2 * 64 * 128 * 4096 * (126977 + 131072) / 2
+    assert abs(bench.causal_index_flops(positions) / 1e12 - 8.659) < 1e-3
+    assert bench.causal_index_flops([0]) == 2 * 64 * 128
+
+
+def test_tensor_peak_from_the_measured_file_else_the_fallback(tmp_path, monkeypatch):
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    assert bench.measured_tensor_peak() == (bench.FALLBACK_BF16_TFLOPS, "fallback")
+    (tmp_path / "MEASURED_PEAKS.json").write_text(json.dumps({"hbm_gbs": 6554.6, "bf16_tflops": 1591.5}))
+    assert bench.measured_tensor_peak() == (1591.5, "measured")
