@@ -104,7 +104,8 @@ def kernel_counters(kernel_file: str):
         with open(path) as f:
             d = json.load(f)
         entry = d[kernel_file]
-        sha = hashlib.sha256(open(src, "rb").read()).hexdigest()
+        with open(src, "rb") as f:
+            sha = hashlib.sha256(f.read()).hexdigest()
         if entry.get("source_sha256") != sha:
             return None
         return entry

@@ -20,7 +20,8 @@ def lib():
 
 
 def declared_symbols():
-    text = open(os.path.join(ROOT, "include", "sga.h")).read()
+    with open(os.path.join(ROOT, "include", "sga.h")) as f:
+        text = f.read()
     return sorted(set(re.findall(r"SGA_API\s+[\w\s\*]+?\b(sga_\w+)\s*\(", text)))
 
 

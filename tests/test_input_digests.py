@@ -16,7 +16,8 @@ def test_input_recipe_bytes_are_unchanged():
                                                   os.path.join(HERE, "golden", "make_input_digests.py"))
     mod = importlib.util.module_from_spec(spec)
     spec.loader.exec_module(mod)
-    stored = json.load(open(os.path.join(HERE, "golden", "input_digests.json")))
+    with open(os.path.join(HERE, "golden", "input_digests.json")) as f:
+        stored = json.load(f)
     if stored["torch"].split("+")[0] != torch.__version__.split("+")[0]:
         pytest.skip(f"digests written with torch {stored['torch']}, running {torch.__version__}")
     assert mod.cases() == stored["digests"]

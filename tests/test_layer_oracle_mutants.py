@@ -28,7 +28,8 @@ MUTANTS = {
 
 
 def _mutant(old: str, new: str) -> types.ModuleType:
-    src = open(SRC).read()
+    with open(SRC) as f:
+        src = f.read()
     assert src.count(old) == 1, old
     mod = types.ModuleType("oracle.layer_mutant")
     mod.__package__ = "oracle"

@@ -52,12 +52,14 @@ PIN_CALLS = [
 
 
 def _compile_mutant(name, edits, tmpdir):
-    src = open(os.path.join(os.path.dirname(oracle.__file__), "sga_oracle.cpp")).read()
+    with open(os.path.join(os.path.dirname(oracle.__file__), "sga_oracle.cpp")) as f:
+        src = f.read()
     for old, new in edits:
         assert src.count(old) == 1, f"{name}: edit target not found exactly once: {old!r}"
         src = src.replace(old, new)
     path = os.path.join(tmpdir, f"{name}.cpp")
-    open(path, "w").write(src)
+    with open(path, "w") as f:
+        f.write(src)
     so = os.path.join(tmpdir, f"lib{name}.so")
     subprocess.check_call(["g++", "-O1", "-std=c++17", "-shared", "-fPIC", "-pthread", path, "-o", so])
     return so

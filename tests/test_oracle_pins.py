@@ -38,7 +38,8 @@ def f64(t):
 
 
 def test_indexer_worked_example(oracle_mod):
-    g = json.load(open(os.path.join(GOLDEN, "indexer_worked_example.json")))
+    with open(os.path.join(GOLDEN, "indexer_worked_example.json")) as f:
+        g = json.load(f)
     q_idx = bf(g["q_idx"])[None, None]
     w = bf(g["w"])[None, None]
     k_idx = bf(g["k_idx"])[None]
@@ -176,7 +177,8 @@ def test_topk_invariants_random(oracle_mod):
 
 
 def test_attention_worked_example(oracle_mod):
-    g = json.load(open(os.path.join(GOLDEN, "attention_worked_example.json")))
+    with open(os.path.join(GOLDEN, "attention_worked_example.json")) as f:
+        g = json.load(f)
     q = bf(g["q"])[None, None, None]
     kv = bf(g["kv"])[None]
     for case in g["cases"]:

@@ -26,7 +26,8 @@ MUTANTS = {
 
 
 def _mutant(old, new):
-    src = open(SRC).read()
+    with open(SRC) as f:
+        src = f.read()
     assert src.count(old) == 1, old
     mod = types.ModuleType("oracle.warmup_mutant")
     mod.__package__ = "oracle"
