@@ -202,3 +202,44 @@ def test_warmup_bad_arguments_rejected_on_host(lib):
     assert call(ctypes.byref(d), g, g, g, g, g, g, g, g, g, g, None, big, None) == 3    # workspace null
     assert call(ctypes.byref(d), g, g, g, g, g, g, g, g, g, g, P(0x20000010), big, None) == 3
     assert call(ctypes.byref(d), g, g, g, g, g, g, g, g, g, g, ws, 1024, None) == 3      # too small
+
+
+C_CLIENT = r"""
+#include <stdio.h>
+#include <string.h>
+#include "sga.h"
+
+int main(void) {
+  sga_dims_t d = {32, 1, 131072, 2048};
+  size_t fwd = 0, att = 0, warm = 0, layer = 0;
+  sga_layer_weights_t lw = {7168, 1536, 0, 0, 0, 0, 0};
+  if (sga_abi_version() != 1) return 1;
+  if (strcmp(sga_status_string(SGA_OK), "SGA_OK") != 0) return 2;
+  if (sga_workspace_size(&d, SGA_OP_FORWARD, &fwd) != SGA_OK || fwd == 0) return 3;
+  if (sga_workspace_size(&d, SGA_OP_SPARSE_MLA_ATTEND, &att) != SGA_OK || att != 256) return 4;
+  if (sga_indexer_warmup_workspace_size(&d, &warm) != SGA_OK || warm == 0) return 5;
+  if (sga_layer_workspace_size(&d, &lw, SGA_LAYER_FORWARD, &layer) != SGA_OK || layer <= fwd) return 6;
+  /* rejected on the host, before any device call */
+  if (sga_index_scores(&d, NULL, NULL, NULL, NULL, NULL, NULL, 0, NULL) != SGA_ERR_INVALID_ARG) return 7;
+  d.top_k = 100;
+  if (sga_workspace_size(&d, SGA_OP_FORWARD, &fwd) != SGA_ERR_INVALID_ARG) return 8;
+  printf("ok %zu %zu %zu\n", att, warm, layer);
+  return 0;
+}
+"""
+
+
+def test_the_header_is_a_c_abi(lib, tmp_path):
+    """A C99 program includes include/sga.h, links libsga.so and calls the host-only entry points."""
+    import subprocess
+
+    src = tmp_path / "client.c"
+    src.write_text(C_CLIENT)
+    exe = tmp_path / "client"
+    libdir = os.path.dirname(sga.LIB_PATH)
+    subprocess.check_call(["gcc", "-std=c99", "-Wall", "-Werror", "-pedantic", "-I", os.path.join(ROOT, "include"),
+                           str(src), "-o", str(exe), os.path.join(libdir, "libsga.so"),
+                           "-Wl,-rpath," + libdir])
+    out = subprocess.run([str(exe)], capture_output=True, text=True, timeout=120)
+    assert out.returncode == 0, (out.returncode, out.stdout, out.stderr)
+    assert out.stdout.startswith("ok 256 ")
