@@ -11,7 +11,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libsga.so")
 SOURCES = ["sga_api.cu", "sga_index.cu", "sga_topk.cu", "sga_attend.cu", "sga_layer.cu", "sga_warmup.cu"]
-DEPS = SOURCES + ["sga_ptx.cuh", "sga_internal.cuh"]
+DEPS = SOURCES + ["sga_ptx.cuh", "sga_internal.cuh", "sga_host.h"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 

@@ -8,15 +8,17 @@
 #include <mutex>
 
 #include "../../include/sga.h"
+#include "sga_host.h"
 #include "sga_internal.cuh"
 
 namespace sga {
 namespace {
 
-constexpr size_t kAlign = 256;
-constexpr size_t kStatusBytes = 256;
-
-size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+using host::align_up;
+using host::aligned;
+using host::at;
+using host::kStatusBytes;
+constexpr size_t kAlign = host::kWsAlign;
 
 struct Layout {
   size_t bitmap = 0, scores = 0, idx = 0, hist = 0, total = 0;
@@ -54,8 +56,6 @@ Layout make_layout(const sga_dims_t& d, sga_op_t op) {
   return l;
 }
 
-bool aligned(const void* p, size_t a) { return p && (reinterpret_cast<uintptr_t>(p) % a) == 0; }
-
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
 std::once_flag g_encode_once;
 
@@ -85,11 +85,6 @@ sga_status_t check_ws(void* ws, size_t ws_bytes, const sga_dims_t& d, sga_op_t o
 }
 
 sga_status_t from_cuda(cudaError_t e) { return e == cudaSuccess ? SGA_OK : SGA_ERR_CUDA; }
-
-template <class T>
-T* at(void* ws, size_t off) {
-  return reinterpret_cast<T*>(static_cast<uint8_t*>(ws) + off);
-}
 
 }  // namespace
 

@@ -1,0 +1,26 @@
+// Host-side helpers shared by the C-ABI entry points: workspace alignment,
+// the status block at the start of every workspace, pointer checks.
+#pragma once
+
+#include <stddef.h>
+#include <stdint.h>
+
+namespace sga {
+namespace host {
+
+constexpr size_t kWsAlign = 256;      // every workspace region starts on this boundary
+constexpr size_t kStatusBytes = 256;  // the status block at the start of a workspace
+
+inline size_t align_up(size_t x) { return (x + kWsAlign - 1) / kWsAlign * kWsAlign; }
+
+// Non-null and a multiple of `a` bytes.
+inline bool aligned(const void* p, size_t a) { return p && (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+// The region of the workspace `off` bytes from its start.
+template <class T>
+T* at(void* ws, size_t off) {
+  return reinterpret_cast<T*>(static_cast<uint8_t*>(ws) + off);
+}
+
+}  // namespace host
+}  // namespace sga

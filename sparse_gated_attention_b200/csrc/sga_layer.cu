@@ -37,6 +37,7 @@
 #include <mutex>
 
 #include "../../include/sga.h"
+#include "sga_host.h"
 
 namespace {
 
@@ -54,12 +55,13 @@ constexpr int kHqExtra = kKvDim + kIdxDim + kIdxHeads;            // 768
 constexpr int kOWidth = kHeads * kVHead;                          // 8,192
 constexpr double kRopeBase = 1.0e6;
 
-constexpr size_t kAlign = 256;
-constexpr size_t kStatusBytes = 256;
+using sga::host::align_up;
+using sga::host::aligned;
+using sga::host::at;
+using sga::host::kStatusBytes;
+constexpr size_t kAlign = sga::host::kWsAlign;
 constexpr size_t kCublasWs = 32u << 20;
 
-size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
-bool aligned(const void* p, size_t a) { return p && (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
 __device__ __forceinline__ float round_bf16(float x) { return __bfloat162float(__float2bfloat16_rn(x)); }
 __device__ __forceinline__ uint16_t bf16_bits(float x) { return __bfloat16_as_ushort(__float2bfloat16_rn(x)); }
@@ -262,11 +264,6 @@ sga_status_t layer_layout(const sga_dims_t& d, int q_rank, sga_layer_op_t op, La
   }
   l->total = off;
   return SGA_OK;
-}
-
-template <class T>
-T* at(void* ws, size_t off) {
-  return reinterpret_cast<T*>(static_cast<uint8_t*>(ws) + off);
 }
 
 bool weights_ok(const sga_layer_weights_t* W, bool front, bool back) {

@@ -31,6 +31,7 @@
 #include <mutex>
 
 #include "../../include/sga.h"
+#include "sga_host.h"
 
 namespace {
 
@@ -43,8 +44,11 @@ constexpr int kThreads = 256;
 constexpr int kRowPad = kDq + 8;            // staged q / kv row: 584 bf16 (1168 B)
 constexpr int kIdxPad = kIdxDim + 8;        // staged q_idx / k_idx row: 136 bf16 (272 B)
 constexpr float kScale = static_cast<float>(SGA_SOFTMAX_SCALE);
-constexpr size_t kAlign = 256;
-constexpr size_t kStatusBytes = 256;
+using sga::host::align_up;
+using sga::host::aligned;
+using sga::host::at;
+using sga::host::kStatusBytes;
+constexpr size_t kAlign = sga::host::kWsAlign;
 
 // kernel A: q, kv rows, q_idx, k rows (bf16, padded), a (fp32)
 constexpr size_t kLogitsSmem = (2 * kHeads * kRowPad + 2 * kChunk * kIdxPad) * 2 + kIdxHeads * kChunk * 4;
@@ -324,8 +328,6 @@ __global__ void __launch_bounds__(kThreads) warmup_grad_kernel(WarmupArgs p) {
   }
 }
 
-size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
-bool aligned(const void* p, size_t a) { return p && (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
 struct WarmupLayout {
   size_t z = 0, a = 0, score = 0, g = 0, total = 0;
@@ -352,11 +354,6 @@ WarmupLayout warmup_layout(const sga_dims_t& d) {
   off += align_up(rows * K * 4);
   l.total = off;
   return l;
-}
-
-template <class T>
-T* at(void* ws, size_t off) {
-  return reinterpret_cast<T*>(static_cast<uint8_t*>(ws) + off);
 }
 
 }  // namespace
