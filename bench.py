@@ -48,6 +48,8 @@ def parse_args():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-prefill", dest="prefill", action="store_false",
                     help="skip the chunked-prefill variant (4096 queries over a 128K cache)")
+    ap.add_argument("--no-decode-variants", dest="decode_variants", action="store_false",
+                    help="skip the other decode workloads (8K x 4, 32K x 64, 256K x 8 with ties)")
     ap.add_argument("--no-layer", dest="layer", action="store_false",
                     help="skip the whole-layer variant (the projections either side of the path)")
     ap.add_argument("--cpu-sample-queries", type=int, default=0, help="oracle sample size (0 = auto)")
@@ -281,6 +283,58 @@ def config_of(wl):
             "parallelism": "replicas"}
 
 
+def per_iteration_ms(fn, n, flush, warmup, dev, stream, dist):
+    """CUDA-event times of n calls of fn on `stream`, each after an L2 flush (a
+    memset of `flush`, outside its events), after `warmup` untimed calls."""
+    for _ in range(max(warmup, 3)):
+        fn()
+    torch.cuda.synchronize(dev)
+    if dist is not None:
+        dist.barrier()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n)]
+    with torch.cuda.stream(stream):
+        for a, b in evs:
+            flush.zero_()
+            a.record(stream)
+            fn()
+            b.record(stream)
+    torch.cuda.synchronize(dev)
+    return [a.elapsed_time(b) for a, b in evs]
+
+
+def decode_variant(sga, synth, name, args, dev, stream, dist, rank, peak) -> dict:
+    """One sga_forward step of another decode workload, timed per iteration with
+    L2 flushed (256 MB memset) before each; the median is reported."""
+    wl = synth.WORKLOADS[name]
+    x = synth.make_inputs(wl, device=dev, seed=rank)
+    B, T, L, K = wl.batch, wl.n_q, wl.ctx, wl.top_k
+    dims = sga.make_dims(B, T, L, K)
+    ws = sga.alloc_workspace(dims, sga.OP_FORWARD, dev)
+    idx = torch.empty((B, T, K), dtype=torch.int32, device=dev)
+    out = torch.empty((B, T, 64, 512), dtype=torch.float32, device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+
+    def forward():
+        sga.forward(x["q_idx"], x["w"], x["k_idx"], x["q"], x["kv"], x["gate"], x["q_pos"], top_k=K, idx_out=idx,
+                    out=out, ws=ws, stream=stream)
+
+    n = max(5, min(args.steps, 20))
+    ms = max_over_ranks(dist, dev, statistics.median(per_iteration_ms(forward, n, flush, args.warmup, dev, stream,
+                                                                      dist)))
+    if sga.device_status(ws) != 0:
+        raise RuntimeError(f"device status set during the {name} variant")
+    rows = B * T
+    world = dist.get_world_size() if dist is not None else 1
+    ab = algorithmic_bytes_per_query(L, K)
+    gbs = ab["total"] * rows / (ms * 1e-3) / 1e9
+    return {"value": rows * world / (ms * 1e-3), "unit": UNIT, "ms_per_step": ms,
+            "config": f"{name}: {B} sequences x {T} query at position {L - 1}, top_k {K}; median of {n} "
+                      f"iterations, L2 flushed (256 MB memset) before each",
+            "path_roofline": {"achieved_gbs": gbs, "frac_of_8tbs": gbs / NOMINAL_HBM_GBS,
+                              "frac_of_measured": gbs / peak, "bytes_per_query": ab["total"]},
+            "gpu_launches": 3}
+
+
 def prefill_variant(sga, synth, args, dev, stream, dist, rank) -> dict:
     """Times sga_forward and the indexer alone on the chunked-prefill workload."""
     wl = synth.WORKLOADS["prefill_t4096_ctx128k"]
@@ -301,24 +355,11 @@ def prefill_variant(sga, synth, args, dev, stream, dist, rank) -> dict:
     def indexer():
         sga.index_scores(x["q_idx"], x["w"], x["k_idx"], x["q_pos"], scores=scores, ws=ws_i, stream=stream)
 
-    def per_iteration_ms(fn, n):
-        for _ in range(max(args.warmup, 3)):
-            fn()
-        torch.cuda.synchronize(dev)
-        if dist is not None:
-            dist.barrier()
-        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n)]
-        for a, b in evs:
-            flush.zero_()
-            a.record(stream)
-            fn()
-            b.record(stream)
-        torch.cuda.synchronize(dev)
-        return [a.elapsed_time(b) for a, b in evs]
-
     n = max(5, min(args.steps, 20))
-    chunk_ms = max_over_ranks(dist, dev, statistics.median(per_iteration_ms(forward, n)))
-    k1_ms = max_over_ranks(dist, dev, statistics.median(per_iteration_ms(indexer, n)))
+    chunk_ms = max_over_ranks(dist, dev, statistics.median(per_iteration_ms(forward, n, flush, args.warmup, dev,
+                                                                            stream, dist)))
+    k1_ms = max_over_ranks(dist, dev, statistics.median(per_iteration_ms(indexer, n, flush, args.warmup, dev,
+                                                                         stream, dist)))
     if sga.device_status(ws) != 0 or sga.device_status(ws_i) != 0:
         raise RuntimeError("device status set during the prefill variant")
     positions = x["q_pos"].flatten().tolist()
@@ -549,6 +590,18 @@ def main():
                  "act_bytes": h.numel() * 2 + y.numel() * 4}
         del lw_t, ws_layer
 
+    # ---- the other decode workloads (separate configurations, one line each in `variants`)
+    decode_lines = {}
+    if args.decode_variants and args.workload is None and not (args.batch and args.ctx):
+        peak_gbs, _ = measured_peaks()
+        for name in ("decode_b4_ctx8k", "decode_b64_ctx32k", "decode_b8_ctx256k_ties"):
+            try:
+                decode_lines[name] = decode_variant(sga, synth, name, args, dev, stream, dist, rank, peak_gbs)
+            except (RuntimeError, TypeError, ValueError) as exc:
+                torch.cuda.synchronize(dev)
+                decode_lines[name] = {"error": f"{type(exc).__name__}: {exc}"}
+            torch.cuda.empty_cache()
+
     # ---- chunked prefill (a separate configuration): 4096 new queries over a 128K cache.
     # The indexer is a dense causal contraction here, so it is reported in TFLOP/s against
     # the bf16 tensor peak, with the whole chunk's time.  L2 is flushed (256 MB memset)
@@ -589,6 +642,7 @@ def main():
         "path_roofline": {"achieved_gbs": fp8_gbs, "frac_of_8tbs": fp8_gbs / NOMINAL_HBM_GBS,
                           "frac_of_measured": fp8_gbs / peak, "bytes_per_query": ab8["total"]},
         "gpu_launches": launches_per_step * args.steps}}
+    variants.update(decode_lines)
     if prefill is not None:
         variants["prefill_t4096_ctx128k"] = prefill
     if layer is not None:

@@ -132,7 +132,10 @@ SGA_API sga_status_t sga_index_scores(const sga_dims_t* dims, const sga_bf16_t* 
  * followed by -1 in unused slots.
  *   scores [B][T][L] fp32 (entries s > t are not read)   q_pos [B][T] int32
  *   idx    [B][T][K] int32 (output)
- * NaN scores give an unspecified selection.  Device error: t outside [0, L). */
+ * NaN scores give an unspecified selection.  Device error: t outside [0, L):
+ * that row's idx is all -1, the error goes only to the workspace status word
+ * and the call itself still returns SGA_OK, so read the status (or validate
+ * q_pos on the host) before trusting a row of -1. */
 SGA_API sga_status_t sga_topk_select(const sga_dims_t* dims, const float* scores, const int32_t* q_pos, int32_t* idx,
                              void* ws, size_t ws_bytes, sga_stream_t stream);
 
@@ -182,6 +185,22 @@ SGA_API sga_status_t sga_get_device_status(const void* ws, sga_stream_t stream, 
 /* Clears the workspace status word (asynchronously on `stream`). */
 SGA_API sga_status_t sga_clear_device_status(void* ws, sga_stream_t stream);
 
+/* Diagnostic of the device-side failure path; no counterpart on the pages.
+ * Every wait inside the kernels of this library gives up after a cycle
+ * budget: the waiting thread writes SGA_ERR_TIMEOUT to the workspace status
+ * word and raises an abort flag that releases every other wait of its thread
+ * block, which then frees its tensor memory and exits, leaving the CUDA
+ * context usable.  This call runs that sequence in one small kernel on a
+ * shared-memory barrier that nothing completes (no copy is in flight): one
+ * thread waits `budget_cycles` SM clock cycles, a second waits with the
+ * kernels' own budget (about one second) and is released by the abort flag.
+ * Afterwards the status word holds SGA_ERR_TIMEOUT and the second 32-bit word
+ * of the workspace holds the number of waits that gave up (2; it is added to,
+ * so zero it first).  budget_cycles in [1, 2^31); ws: at least 256 bytes,
+ * 256-byte aligned.  Asynchronous on `stream`. */
+SGA_API sga_status_t sga_selftest_bounded_wait(int64_t budget_cycles, void* ws, size_t ws_bytes,
+                                               sga_stream_t stream);
+
 /* Bytes of device memory inside the library that sga_topk_select_noalloc uses
  * as its scratch (a status word plus the selection bitmaps). */
 #define SGA_NOALLOC_SCRATCH_BYTES (256 + 4 * 1024 * 1024)
@@ -203,8 +222,11 @@ SGA_API sga_status_t sga_clear_device_status(void* ws, sga_stream_t stream);
  * what must start at zero (the status word; the kernel zeroes its bitmap
  * words before use).  Calls that overlap on the GPU race on the array, so
  * order them on one stream.  Device-side errors are not reported (the status
- * word is private to the library); all other arguments, results and errors
- * are as for sga_topk_select. */
+ * word is private to the library): a row whose q_pos lies outside [0, L)
+ * comes back as all -1 while the call returns SGA_OK, so validate q_pos on the
+ * host.  All other arguments, results and errors are as for sga_topk_select.
+ * A failed look-up of the array's address returns SGA_ERR_CUDA, and the next
+ * call on that device looks it up again. */
 SGA_API sga_status_t sga_topk_select_noalloc(const sga_dims_t* dims, const float* scores, const int32_t* q_pos,
                                              int32_t* idx, sga_stream_t stream);
 

@@ -36,7 +36,7 @@ EXPORTED = ["sga_abi_version", "sga_status_string", "sga_workspace_size", "sga_i
             "sga_sparse_mla_attend", "sga_forward", "sga_get_device_status", "sga_clear_device_status",
             "sga_topk_select_noalloc", "sga_index_scores_fp8", "sga_forward_fp8", "sga_layer_workspace_size",
             "sga_layer_project", "sga_layer_output", "sga_layer_forward", "sga_indexer_warmup_workspace_size",
-            "sga_indexer_warmup"]
+            "sga_indexer_warmup", "sga_selftest_bounded_wait"]
 NOALLOC_SCRATCH_BYTES = 256 + 4 * 1024 * 1024
 
 
@@ -90,6 +90,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "sga_layer_forward": (ctypes.c_int, [D, ctypes.POINTER(LayerWeights), P, P, P, P, P, P, P, sz, P]),
         "sga_indexer_warmup_workspace_size": (ctypes.c_int, [D, ctypes.POINTER(sz)]),
         "sga_indexer_warmup": (ctypes.c_int, [D, P, P, P, P, P, P, P, P, P, P, P, sz, P]),
+        "sga_selftest_bounded_wait": (ctypes.c_int, [ctypes.c_int64, P, sz, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -440,3 +441,11 @@ def indexer_warmup(q_idx, w, k_idx, q, kv, idx, grad_k_idx=None, ws=None, stream
         ctypes.byref(dims), _ptr(q_idx), _ptr(w), _ptr(k_idx), _ptr(q), _ptr(kv), _ptr(idx), _ptr(loss),
         _ptr(grad_q_idx), _ptr(grad_w), _ptr(grad_k_idx), _ptr(ws), ws.numel(), _stream(stream)))
     return {"loss": loss, "grad_q_idx": grad_q_idx, "grad_w": grad_w, "grad_k_idx": grad_k_idx}
+
+
+def selftest_bounded_wait(budget_cycles: int, ws: torch.Tensor, stream=None) -> None:
+    """Runs the bounded-wait diagnostic (sga_selftest_bounded_wait) on ``ws``
+    (a uint8 device tensor of at least 256 bytes); asynchronous on the stream."""
+    _need(ws, "ws", torch.uint8)
+    _check("sga_selftest_bounded_wait", load_library().sga_selftest_bounded_wait(
+        int(budget_cycles), _ptr(ws), ws.numel(), _stream(stream)))

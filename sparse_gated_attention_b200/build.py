@@ -10,7 +10,8 @@ PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libsga.so")
-SOURCES = ["sga_api.cu", "sga_index.cu", "sga_topk.cu", "sga_attend.cu", "sga_layer.cu", "sga_warmup.cu"]
+SOURCES = ["sga_api.cu", "sga_index.cu", "sga_topk.cu", "sga_attend.cu", "sga_layer.cu", "sga_warmup.cu",
+           "sga_diag.cu"]
 DEPS = SOURCES + ["sga_ptx.cuh", "sga_internal.cuh", "sga_host.h"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 

@@ -84,7 +84,14 @@ sga_status_t check_ws(void* ws, size_t ws_bytes, const sga_dims_t& d, sga_op_t o
   return SGA_OK;
 }
 
-sga_status_t from_cuda(cudaError_t e) { return e == cudaSuccess ? SGA_OK : SGA_ERR_CUDA; }
+// A failed launch or runtime call also leaves the error as the thread's last
+// CUDA error; it is cleared here so that it does not surface in the caller's
+// next, unrelated error check.
+sga_status_t from_cuda(cudaError_t e) {
+  if (e == cudaSuccess) return SGA_OK;
+  cudaGetLastError();
+  return SGA_ERR_CUDA;
+}
 
 }  // namespace
 
@@ -134,6 +141,7 @@ sga_status_t index_scores_impl(const sga_dims_t* dims, const void* q_idx, const 
   if (st != SGA_OK) return st;
   int sms = 0;
   if ((st = device_info(&sms)) != SGA_OK) return st;
+  host::NvtxRange range("sga.index_scores");
   IndexArgs a{q_idx, w, k_idx, q_pos, scores, nullptr, at<int>(ws, 0), dims->batch, dims->n_q, dims->kv_stride, fp8};
   return from_cuda(launch_index_scores(a, sms, static_cast<cudaStream_t>(stream)));
 }
@@ -159,12 +167,20 @@ sga_status_t forward_impl(const sga_dims_t* dims, const void* q_idx, const sga_b
   // scores; the selection clears each histogram row after reading it, so a
   // zero-filled workspace stays ready for the next call.
   uint32_t* hist = at<uint32_t>(ws, l.hist);
-  IndexArgs ia{q_idx, w, k_idx, q_pos, scores, hist, status, dims->batch, dims->n_q, dims->kv_stride, fp8};
-  cudaError_t e = launch_index_scores(ia, sms, s);
-  if (e != cudaSuccess) return SGA_ERR_CUDA;
-  TopkArgs ta{scores, q_pos, idx, at<uint32_t>(ws, l.bitmap), hist, status, rows, dims->kv_stride, dims->top_k};
-  e = launch_topk(ta, s);
-  if (e != cudaSuccess) return SGA_ERR_CUDA;
+  cudaError_t e;
+  {
+    host::NvtxRange range("sga.index_scores");
+    IndexArgs ia{q_idx, w, k_idx, q_pos, scores, hist, status, dims->batch, dims->n_q, dims->kv_stride, fp8};
+    e = launch_index_scores(ia, sms, s);
+  }
+  if (e != cudaSuccess) return from_cuda(e);
+  {
+    host::NvtxRange range("sga.topk_select");
+    TopkArgs ta{scores, q_pos, idx, at<uint32_t>(ws, l.bitmap), hist, status, rows, dims->kv_stride, dims->top_k};
+    e = launch_topk(ta, s);
+  }
+  if (e != cudaSuccess) return from_cuda(e);
+  host::NvtxRange range("sga.sparse_mla_attend");
   AttendArgs aa{q, kv, idx, gate, out, status, dims->batch, dims->n_q, dims->kv_stride, dims->top_k};
   return from_cuda(launch_attend(aa, s));
 }
@@ -217,6 +233,7 @@ sga_status_t sga_topk_select(const sga_dims_t* dims, const float* scores, const 
   if (st != SGA_OK) return st;
   int sms = 0;
   if ((st = device_info(&sms)) != SGA_OK) return st;
+  host::NvtxRange range("sga.topk_select");
   TopkArgs a{scores,          q_pos, idx, at<uint32_t>(ws, l.bitmap), nullptr, at<int>(ws, 0),
              dims->batch * dims->n_q, dims->kv_stride, dims->top_k};
   return from_cuda(launch_topk(a, static_cast<cudaStream_t>(stream)));
@@ -234,6 +251,7 @@ sga_status_t sga_sparse_mla_attend(const sga_dims_t* dims, const sga_bf16_t* q, 
   if (st != SGA_OK) return st;
   int sms = 0;
   if ((st = device_info(&sms)) != SGA_OK) return st;
+  host::NvtxRange range("sga.sparse_mla_attend");
   AttendArgs a{q, kv, idx, gate, out, at<int>(ws, 0), dims->batch, dims->n_q, dims->kv_stride, dims->top_k};
   return from_cuda(launch_attend(a, static_cast<cudaStream_t>(stream)));
 }
@@ -277,13 +295,27 @@ sga_status_t sga_clear_device_status(void* ws, sga_stream_t stream) {
 // Scratch of sga_topk_select_noalloc: a status word then the selection bitmaps.  It
 // lives in the library for callers that cannot allocate device memory.  In host
 // code the symbol is only a host-side stand-in, so the device address is looked
-// up once per device (with that device current) and passed to the kernel.
+// up per device (with that device current) and passed to the kernel.  A lookup
+// that fails is not remembered: the next call on that device tries again.
 namespace {
 constexpr int kNoallocMaxDevices = 64;
 static __device__ __align__(256) unsigned char g_noalloc_scratch[SGA_NOALLOC_SCRATCH_BYTES];
 void* g_noalloc_ptr[kNoallocMaxDevices] = {};
-cudaError_t g_noalloc_err[kNoallocMaxDevices] = {};
-std::once_flag g_noalloc_once[kNoallocMaxDevices];
+std::mutex g_noalloc_mu;
+
+// The scratch array's device address on device `dev` (the current device), or null.
+void* noalloc_scratch(int dev) {
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (!g_noalloc_ptr[dev]) {
+    void* ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) == cudaSuccess) {
+      g_noalloc_ptr[dev] = ptr;
+    } else {
+      cudaGetLastError();
+    }
+  }
+  return g_noalloc_ptr[dev];
+}
 }  // namespace
 
 extern "C" {
@@ -303,15 +335,11 @@ sga_status_t sga_topk_select_noalloc(const sga_dims_t* dims, const float* scores
     cudaGetLastError();
     return SGA_ERR_UNSUPPORTED;
   }
-  std::call_once(g_noalloc_once[dev], [dev]() {
-    void* ptr = nullptr;
-    g_noalloc_err[dev] = cudaGetSymbolAddress(&ptr, g_noalloc_scratch);
-    if (g_noalloc_err[dev] == cudaSuccess) g_noalloc_ptr[dev] = ptr;
-  });
-  if (g_noalloc_err[dev] != cudaSuccess || !g_noalloc_ptr[dev]) return SGA_ERR_CUDA;
-  void* scratch = g_noalloc_ptr[dev];
+  void* scratch = noalloc_scratch(dev);
+  if (!scratch) return SGA_ERR_CUDA;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (cudaMemsetAsync(scratch, 0, kStatusBytes, s) != cudaSuccess) return SGA_ERR_CUDA;  // status word
+  cudaError_t e = cudaMemsetAsync(scratch, 0, kStatusBytes, s);  // status word
+  if (e != cudaSuccess) return from_cuda(e);
   TopkArgs a{scores,   q_pos, idx, at<uint32_t>(scratch, kStatusBytes), nullptr, at<int>(scratch, 0),
              static_cast<int>(rows), dims->kv_stride, dims->top_k};
   return from_cuda(launch_topk(a, s));

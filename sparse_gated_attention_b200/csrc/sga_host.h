@@ -2,6 +2,7 @@
 // the status block at the start of every workspace, pointer checks.
 #pragma once
 
+#include <nvtx3/nvToolsExt.h>
 #include <stddef.h>
 #include <stdint.h>
 
@@ -21,6 +22,15 @@ template <class T>
 T* at(void* ws, size_t off) {
   return reinterpret_cast<T*>(static_cast<uint8_t*>(ws) + off);
 }
+
+// One NVTX range (named after the stage it brackets) for the lifetime of the
+// object: the host-side launch of that stage shows as a range in profilers.
+struct NvtxRange {
+  explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+  NvtxRange(const NvtxRange&) = delete;
+  NvtxRange& operator=(const NvtxRange&) = delete;
+};
 
 }  // namespace host
 }  // namespace sga

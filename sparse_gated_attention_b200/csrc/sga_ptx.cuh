@@ -81,14 +81,15 @@ __device__ __forceinline__ void grid_launch_dependents() {
 }
 
 // Waits for the phase with the given parity to complete.  Returns false when
-// the budget ran out or another thread of the CTA raised `abort_flag`.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag) {
+// the budget (cycles) ran out or another thread of the CTA raised `abort_flag`.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                          long long budget = kWaitBudgetCycles) {
   if (mbar_try_wait(bar, parity)) return true;
   const long long start = clock64();
   while (true) {
     if (mbar_try_wait(bar, parity)) return true;
     if (*abort_flag) return false;
-    if (clock64() - start > kWaitBudgetCycles) return false;
+    if (clock64() - start > budget) return false;
   }
 }
 

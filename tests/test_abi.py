@@ -88,6 +88,12 @@ def test_null_and_misaligned_pointers_rejected_on_host(lib):
     assert lib.sga_topk_select(ctypes.byref(d), good, good, good, ws, 64, None) == 3
     assert lib.sga_get_device_status(None, None, None) == 1
     assert lib.sga_clear_device_status(None, None) == 1
+    # the bounded-wait diagnostic: budget out of range, workspace null / misaligned / too small
+    assert lib.sga_selftest_bounded_wait(0, ws, 256, None) == 1
+    assert lib.sga_selftest_bounded_wait(1 << 31, ws, 256, None) == 1
+    assert lib.sga_selftest_bounded_wait(1000, None, 256, None) == 3
+    assert lib.sga_selftest_bounded_wait(1000, P(0x200010), 256, None) == 3
+    assert lib.sga_selftest_bounded_wait(1000, ws, 128, None) == 3
 
 
 def test_binding_refuses_cpu_tensors():

@@ -150,10 +150,15 @@ def test_topk_sizes(L, K, t):
 # Rows of up to 8 x 32768 positions are selected with each CTA's segment held
 # in shared memory; longer rows stream.  A row stride that is not a multiple
 # of 4 takes plain loads instead of bulk copies.  Many rows with a long stride
-# give clusters of 3 and 5 CTAs.
+# give clusters of 3 and 5 CTAs.  The streaming kernel keeps a CTA's selection
+# and tie words in shared memory while its segment spans at most 65,536
+# positions, i.e. rows up to 8 x 65,536; longer rows (600,001 and up) keep them
+# in the workspace.
 @pytest.mark.parametrize("rows,L,kind", [(2, 100001, "int"), (2, 100001, "ties"), (100, 70000, "int"),
                                          (40, 131075, "ties"), (2, 300000, "int"), (2, 300000, "ties"),
-                                         (3, 300003, "int"), (1, 262145, "float")])
+                                         (3, 300003, "int"), (1, 262145, "float"),
+                                         (2, 600004, "int"), (2, 600001, "ties"), (2, 600001, "int"),
+                                         (2, 600004, "ties"), (1, 700000, "float")])
 def test_topk_kernel_paths(rows, L, kind):
     rng = np.random.default_rng(rows * 7 + L)
     if kind == "int":
@@ -164,6 +169,8 @@ def test_topk_kernel_paths(rows, L, kind):
         sc = rng.normal(size=(rows, L)).astype(np.float32).astype(np.float64)
     pos = rng.integers(2048, L, size=rows)
     pos[0] = L - 1
+    if L > 8 * 65536 and rows > 1:
+        pos[1] = L - 2  # every row of the long cases takes the workspace words
     got, want = run_topk(sc, pos, 2048)
     np.testing.assert_array_equal(got, want)
 

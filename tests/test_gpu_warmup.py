@@ -1,11 +1,10 @@
 """GPU parity of sga_indexer_warmup against the warm-up oracle.
 
-Not collected yet (the file name does not start with test_): the warm-up
-kernels have not run on a GPU.  Renamed to test_gpu_warmup.py once they have,
-it joins the GPU suite.  Tolerances: the loss within 1e-4 relative, each
-gradient within rel-L2 1e-3 (fp32 sums of bf16 products against fp64); the
-selection is the oracle's, which the path reproduces bit for bit on these
-integer-valued indexer inputs."""
+Tolerances: the loss within 1e-4 relative, each gradient within rel-L2 1e-3
+(fp32 sums of bf16 products against fp64; the key gradient is accumulated with
+float atomics, so its rounding depends on the order in which the queries'
+terms arrive); the selection is the oracle's, which the path reproduces bit for
+bit on these integer-valued indexer inputs."""
 import numpy as np
 import pytest
 import torch

@@ -4,10 +4,13 @@ Some callers cannot allocate device memory, such as a custom operator inside
 another inference engine that is handed only its input and output buffers.
 sga_topk_select_noalloc serves them from a static scratch array inside the
 library.  This file checks, through the C ABI, that it selects exactly what
-sga_topk_select (with a caller workspace) selects, on two different calls in a
-row, so the second call also shows that state left behind by the first does not
-leak into its result.  It sits last in collection order so that a failure here
-comes after every other test has run.
+sga_topk_select (with a caller workspace) and the fp64 oracle select, on two
+different calls in a row, so the second call also shows that state left behind
+by the first does not leak into its result.  Rows longer than 8 x 65,536
+positions keep their selection and tie bitmaps in the scratch array itself
+(shorter rows keep them in shared memory and use only its status word), so the
+long cases exercise the array.  The file sits last in collection order so that
+a failure here comes after every other test has run.
 """
 import ctypes
 
@@ -15,6 +18,7 @@ import numpy as np
 import pytest
 import torch
 
+import oracle
 import sparse_gated_attention_b200 as sga
 
 pytestmark = pytest.mark.gpu
@@ -27,6 +31,7 @@ def lib():
     from sparse_gated_attention_b200 import build
 
     build.build()
+    oracle.build()
     return sga.load_library()
 
 
@@ -49,13 +54,33 @@ def case(seed, B, L, hi, k=2048):
     return scores, q_pos
 
 
+def check_against_both(lib, scores, q_pos, k=2048):
+    got = call_noalloc(lib, scores, q_pos, k)
+    want = sga.topk_select(scores, q_pos, top_k=k)
+    torch.cuda.synchronize()
+    got_np = got.cpu().numpy()
+    np.testing.assert_array_equal(got_np, want.cpu().numpy())
+    B, T, L = scores.shape
+    ref = oracle.topk(scores.cpu().numpy().astype(np.float64).reshape(B * T, L),
+                      q_pos.cpu().numpy().reshape(B * T), k=k)
+    np.testing.assert_array_equal(got_np.reshape(B * T, k), ref)
+
+
 def test_noalloc_matches_workspace_entry_point_on_two_calls(lib):
     for seed, B, L, hi in [(1, 12, 100000, 40), (2, 5, 131072, 5000)]:
         scores, q_pos = case(seed, B, L, hi)
-        got = call_noalloc(lib, scores, q_pos, 2048)
-        want = sga.topk_select(scores, q_pos, top_k=2048)
-        torch.cuda.synchronize()
-        np.testing.assert_array_equal(got.cpu().numpy(), want.cpu().numpy())
+        check_against_both(lib, scores, q_pos)
+
+
+@pytest.mark.parametrize("L", [600004, 600001])
+def test_noalloc_bitmaps_in_the_scratch_array_on_two_calls(lib, L):
+    """Two rows of ~600K positions: 2 x 2 x 18,751 words x 4 B = 300 KB of
+    bitmaps in the library's array.  The second call (other seed, other
+    positions) reuses the words the first one left behind."""
+    for seed, hi in [(11, 9), (12, 3000)]:
+        scores, q_pos = case(seed, 2, L, hi)
+        q_pos[1, 0] = L - 2 - seed  # both rows long enough for the array
+        check_against_both(lib, scores, q_pos)
 
 
 def test_noalloc_rejects_sizes_beyond_its_scratch(lib):
