@@ -166,7 +166,7 @@ sga_status_t forward_impl(const sga_dims_t* dims, const void* q_idx, const sga_b
   // The indexer counts the first radix level of the selection as it writes the
   // scores; the selection clears each histogram row after reading it, so a
   // zero-filled workspace stays ready for the next call.
-  uint32_t* hist = at<uint32_t>(ws, l.hist);
+  uint32_t* hist = index_uses_prefill(dims->n_q) ? nullptr : at<uint32_t>(ws, l.hist);
   cudaError_t e;
   {
     host::NvtxRange range("sga.index_scores");

@@ -377,6 +377,429 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
+// ============================================================================ prefill
+// Many queries per sequence (chunked prefill): a work item is (query block,
+// 128-key tile), a block being kQB = 8 consecutive queries of one sequence.
+// The tensor core computes D[key, (query, head)] for the block as two N = 256
+// halves (4 queries x 64 heads) into two 256-column TMEM accumulators; the
+// epilogue drains one half while the tensor core fills the other.  The block's
+// queries (the B operand: 128 KB in bf16, 64 KB in E4M3) stay in shared memory
+// for all of its tiles, so every key tile serves 8 queries; keys arrive as
+// 16 KB strips (128 keys x 128 bytes) through a ring, with an L2 evict-last
+// policy because every CTA sweeps the same sequence's keys.  No first-level
+// selection histogram is counted here.
+constexpr int kQB = 8;                            // queries per block
+constexpr int kHalfQ = 4;                         // queries per accumulator
+constexpr int kPfN = kHalfQ * kHeads;             // MMA N: 256
+constexpr int kPfEpiWarps = 8;                    // two per TMEM lane quarter
+constexpr int kPfThreads = 64 + 32 * kPfEpiWarps;  // 320
+
+template <bool kFp8>
+struct PrefillCfg {
+  static constexpr int kStrips = kFp8 ? 1 : 2;  // 128-byte strips per key / query row
+  static constexpr int kStripElems = kFp8 ? 128 : 64;
+  static constexpr int kStages = kFp8 ? 8 : 5;  // ring of key strips (16 KB each)
+  static constexpr int kQStrip = kPfN * 128;    // one strip of a half's 256 query rows: 32 KB
+  static constexpr int kQHalf = kStrips * kQStrip;
+  static constexpr int kQBytes = 2 * kQHalf;
+  static constexpr int kKSteps = kFp8 ? 4 : 8;
+  static constexpr int kWFloats = kHalfQ * kHeads;  // each epilogue warp's four queries' weights
+  static constexpr int kWBytes = kPfEpiWarps * kWFloats * 4;
+  static constexpr int kNumBars = 2 * kStages + 2 + 4 + 1;
+  static constexpr size_t kSmemBytes = 1024 + kStages * kABox + kQBytes + kWBytes + kNumBars * 8 + 16;
+  static constexpr uint32_t kIdesc = kFp8 ? idesc_e4m3_f32(kKeys, kPfN) : idesc_bf16_f32(kKeys, kPfN, false, false);
+};
+static_assert(PrefillCfg<false>::kSmemBytes <= 232448 && PrefillCfg<true>::kSmemBytes <= 232448,
+              "shared memory budget");
+
+struct PrefillParams {
+  const uint16_t* w;
+  const int32_t* q_pos;
+  float* scores;
+  int* status;
+  int n_q, kv_stride, tiles_per_block, blocks_per_seq;
+  long long total_items;
+};
+
+// Walks work items j = (query block, 128-key tile) in order, re-reading the
+// block's positions only when the block changes.  tmax is the largest valid
+// position of the block (-1 if none); tiles past it are dead.
+struct BlockCursor {
+  int blk, key0, seq, row0, nrows, tmax;
+  bool bad;  // some row of the block has a position outside [0, L)
+  __device__ __forceinline__ void load(const PrefillParams& p) {
+    seq = blk / p.blocks_per_seq;
+    const int i = blk - seq * p.blocks_per_seq;
+    row0 = seq * p.n_q + i * kQB;
+    nrows = min(kQB, p.n_q - i * kQB);
+    tmax = -1;
+    bad = false;
+    for (int r = 0; r < nrows; ++r) {
+      const int t = __ldg(p.q_pos + row0 + r);
+      if (t >= 0 && t < p.kv_stride) {
+        tmax = max(tmax, t);
+      } else {
+        bad = true;
+      }
+    }
+  }
+  __device__ __forceinline__ void start(const PrefillParams& p, long long j) {
+    blk = static_cast<int>(j / p.tiles_per_block);
+    key0 = static_cast<int>(j % p.tiles_per_block) * kKeys;
+    load(p);
+  }
+  __device__ __forceinline__ void next(const PrefillParams& p, bool more) {
+    key0 += kKeys;
+    if (key0 >= p.tiles_per_block * kKeys) {
+      key0 = 0;
+      ++blk;
+      if (more) load(p);
+    }
+  }
+  __device__ __forceinline__ bool live() const { return key0 <= tmax; }
+};
+
+// acc += a * b on two fp32 lanes at once (one packed instruction).
+__device__ __forceinline__ void ffma2(float2& acc, float a0, float a1, float b0, float b1) {
+  asm("{\n\t.reg .b64 x, y, z;\n\t"
+      "mov.b64 x, {%2, %3};\n\t"
+      "mov.b64 y, {%4, %5};\n\t"
+      "mov.b64 z, {%0, %1};\n\t"
+      "fma.rn.f32x2 z, x, y, z;\n\t"
+      "mov.b64 {%0, %1}, z;\n\t}"
+      : "+f"(acc.x), "+f"(acc.y)
+      : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
+}
+
+// sum_j w[j] * max(0, v[j]) over 64 heads, as four independent pairs of
+// chains (exact for integer-valued inputs, whatever the order).
+__device__ __forceinline__ float weighted_relu_sum(const float (&v)[64], const float* w) {
+  const float4* wq = reinterpret_cast<const float4*>(w);
+  float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+#pragma unroll
+  for (int c = 0; c < kHeads / 4; ++c) {
+    const float4 wv = wq[c];
+    ffma2(acc[(2 * c) & 3], wv.x, wv.y, fmaxf(v[4 * c], 0.f), fmaxf(v[4 * c + 1], 0.f));
+    ffma2(acc[(2 * c + 1) & 3], wv.z, wv.w, fmaxf(v[4 * c + 2], 0.f), fmaxf(v[4 * c + 3], 0.f));
+  }
+  return ((acc[0].x + acc[0].y) + (acc[1].x + acc[1].y)) + ((acc[2].x + acc[2].y) + (acc[3].x + acc[3].y));
+}
+
+// Score store that should not displace the keys every CTA keeps re-reading from L2.
+__device__ __forceinline__ void st_evict_first(float* addr, float v, uint64_t policy) {
+  asm volatile("st.global.L2::cache_hint.f32 [%0], %1, %2;" ::"l"(addr), "f"(v), "l"(policy) : "memory");
+}
+
+template <bool kFp8>
+__global__ void __launch_bounds__(kPfThreads, 1)
+    sga_index_prefill_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap qmap,
+                             PrefillParams p) {
+  using C = PrefillCfg<kFp8>;
+  constexpr int kStages = C::kStages;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t a_base = smem_u32(smem);
+  const uint32_t q_base = a_base + kStages * kABox;
+  float* w_s = reinterpret_cast<float*>(smem + kStages * kABox + C::kQBytes);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kStages * kABox + C::kQBytes + C::kWBytes);
+  const uint32_t bar0 = smem_u32(bars);
+  auto full = [&](int s) { return bar0 + 8u * s; };
+  auto empty = [&](int s) { return bar0 + 8u * (kStages + s); };
+  const uint32_t qfull = bar0 + 8u * (2 * kStages);
+  const uint32_t qempty = qfull + 8u;
+  auto accfull = [&](int h) { return qfull + 8u * (2 + h); };
+  auto accempty = [&](int h) { return qfull + 8u * (4 + h); };
+  const uint32_t done_bar = qfull + 8u * 6;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::kNumBars);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(full(s), 1);
+      mbar_init(empty(s), 1);
+    }
+    mbar_init(qfull, 1);
+    mbar_init(qempty, 1);
+    for (int h = 0; h < 2; ++h) {
+      mbar_init(accfull(h), 1);
+      mbar_init(accempty(h), kPfEpiWarps);
+    }
+    mbar_init(done_bar, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tmap(&kmap);
+    prefetch_tmap(&qmap);
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_slot), 2 * kPfN);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  grid_dependency_wait();
+  grid_launch_dependents();
+
+  const long long j0 = p.total_items * blockIdx.x / gridDim.x;
+  const long long j1 = p.total_items * (blockIdx.x + 1) / gridDim.x;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      const uint64_t pol_keys = policy_evict_last();
+      const uint64_t pol_q = policy_evict_first();
+      long long n = 0;  // strips issued
+      int st = 0, qc = 0, seen_blk = -1, q_blk = -1;
+      uint32_t ph = 0;
+      bool ok = true;
+      BlockCursor cur;
+      if (j0 < j1) cur.start(p, j0);
+      for (long long j = j0; j < j1; cur.next(p, ++j < j1)) {
+        if (cur.blk != seen_blk) {
+          if (cur.bad) record_status(p.status, kStatusDeviceArg);
+          seen_blk = cur.blk;
+        }
+        if (!cur.live()) continue;
+        if (cur.blk != q_blk) {  // the block's queries, once its previous user has finished
+          if (!mbar_wait(qempty, static_cast<uint32_t>(qc & 1) ^ 1u, abort_flag)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(qfull, static_cast<uint32_t>(cur.nrows * C::kStrips * kQBox));
+          for (int r = 0; r < cur.nrows; ++r)
+#pragma unroll
+            for (int b = 0; b < C::kStrips; ++b)
+              tma_load_2d(q_base + (r / kHalfQ) * C::kQHalf + b * C::kQStrip + (r % kHalfQ) * kQBox, &qmap, qfull,
+                          b * C::kStripElems, (cur.row0 + r) * kHeads, pol_q);
+          ++qc;
+          q_blk = cur.blk;
+        }
+        const int y = cur.seq * p.kv_stride + cur.key0;
+#pragma unroll
+        for (int b = 0; b < C::kStrips; ++b) {
+          if (!mbar_wait(empty(st), ph ^ 1u, abort_flag)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(full(st), kABox);
+          tma_load_2d(a_base + st * kABox, &kmap, full(st), b * C::kStripElems, y, pol_keys);
+          ++n;
+          if (++st == kStages) {
+            st = 0;
+            ph ^= 1u;
+          }
+        }
+        if (!ok) break;
+      }
+      if (!ok) {
+        record_status(p.status, kStatusTimeout);
+        *abort_flag = 1;
+        // Let the copies already issued land before the CTA retires.
+        volatile int never = 0;
+        for (long long m = (n > kStages ? n - kStages : 0); m < n; ++m)
+          mbar_wait(full(static_cast<int>(m % kStages)), static_cast<uint32_t>((m / kStages) & 1), &never);
+        if (qc > 0) mbar_wait(qfull, static_cast<uint32_t>((qc - 1) & 1), &never);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc = C::kIdesc;
+      const uint64_t a_desc0 = sdesc_sw128(a_base, 16, 1024);
+      const uint64_t q_desc0 = sdesc_sw128(q_base, 16, 1024);
+      int st = 0, qc = 0, q_blk = -1;
+      uint32_t ph = 0;
+      long long tiles = 0;
+      bool ok = true;
+      BlockCursor cur;
+      if (j0 < j1) cur.start(p, j0);
+      for (long long j = j0; j < j1 && ok; cur.next(p, ++j < j1)) {
+        if (!cur.live()) continue;
+        if (cur.blk != q_blk) {
+          if (q_blk >= 0) mma_commit(qempty);  // the previous block's queries are free once its MMAs finish
+          if (!mbar_wait(qfull, static_cast<uint32_t>(qc & 1), abort_flag)) {
+            ok = false;
+            break;
+          }
+          ++qc;
+          q_blk = cur.blk;
+        }
+        int sst[C::kStrips];
+#pragma unroll
+        for (int b = 0; b < C::kStrips; ++b) {
+          if (!mbar_wait(full(st), ph, abort_flag)) ok = false;
+          sst[b] = st;
+          if (++st == kStages) {
+            st = 0;
+            ph ^= 1u;
+          }
+        }
+        if (!ok) break;
+        const uint32_t tpar = static_cast<uint32_t>(tiles & 1);
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          if (!mbar_wait(accempty(h), tpar ^ 1u, abort_flag)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t d = tmem_base + static_cast<uint32_t>(h * kPfN);
+#pragma unroll
+          for (int k = 0; k < C::kKSteps; ++k) {
+            // 32-byte K steps: four per 128-byte strip
+            const int b = k >> 2;
+            const uint64_t a_desc = a_desc0 + static_cast<uint64_t>((sst[b] * kABox + (k & 3) * 32) >> 4);
+            const uint64_t b_desc = q_desc0 + static_cast<uint64_t>((h * C::kQHalf + b * C::kQStrip + (k & 3) * 32) >> 4);
+            if constexpr (kFp8)
+              mma_e4m3(d, a_desc, b_desc, idesc, k > 0 ? 1u : 0u);
+            else
+              mma_bf16(d, a_desc, b_desc, idesc, k > 0 ? 1u : 0u);
+          }
+          mma_commit(accfull(h));
+        }
+        if (!ok) break;
+#pragma unroll
+        for (int b = 0; b < C::kStrips; ++b) mma_commit(empty(sst[b]));
+        ++tiles;
+      }
+      if (!ok) {
+        record_status(p.status, kStatusTimeout);
+        *abort_flag = 1;
+      }
+      mma_commit(done_bar);
+      volatile int never = 0;
+      mbar_wait(done_bar, 0, &never);
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    // Eight warps, two per TMEM lane quarter: in each half, the first warp of a
+    // quarter takes the half's queries 0-1, the second queries 2-3.  Thread =
+    // one key (TMEM lane); each warp keeps its four queries' weights in shared
+    // memory as fp32.
+    const int e = warp - 2;
+    const int quarter = warp & 3;
+    const int sub = e >> 2;
+    float* w_mine = w_s + e * C::kWFloats;  // [h * 2 + qq][64]
+    const uint64_t pol_scores = policy_evict_first();
+    long long tiles = 0;
+    int cur_blk = -1;
+    int trow[4] = {-1, -1, -1, -1};
+    int rrow[4] = {0, 0, 0, 0};
+    BlockCursor cur;
+    if (j0 < j1) cur.start(p, j0);
+    for (long long j = j0; j < j1; cur.next(p, ++j < j1)) {
+      if (!cur.live()) continue;
+      if (cur.blk != cur_blk) {
+        __syncwarp();
+        for (int i = lane; i < C::kWFloats; i += 32) {
+          const int s = i >> 6, qi = (s >> 1) * kHalfQ + sub * 2 + (s & 1);
+          w_mine[i] = qi < cur.nrows
+                          ? bf16_bits_to_float(__ldg(p.w + static_cast<size_t>(cur.row0 + qi) * kHeads + (i & 63)))
+                          : 0.f;
+        }
+#pragma unroll
+        for (int s = 0; s < 4; ++s) {
+          const int qi = (s >> 1) * kHalfQ + sub * 2 + (s & 1);
+          int t = -1;
+          if (qi < cur.nrows) {
+            t = __ldg(p.q_pos + cur.row0 + qi);
+            if (t < 0 || t >= p.kv_stride) t = -1;
+          }
+          trow[s] = t;
+          rrow[s] = cur.row0 + qi;
+        }
+        __syncwarp();
+        cur_blk = cur.blk;
+      }
+      const uint32_t tpar = static_cast<uint32_t>(tiles & 1);
+      const int key = cur.key0 + quarter * 32 + lane;
+      bool ok = true;
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        if (!mbar_wait(accfull(h), tpar, abort_flag)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        // one query's 64 head dots at a time (registers: three of the ten
+        // warps share a sub-partition, which caps a thread at 168)
+        float v[64];
+        const uint32_t taddr =
+            tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + static_cast<uint32_t>(h * kPfN + sub * 2 * kHeads);
+        tmem_ld64(taddr, v);
+        const float s0 = weighted_relu_sum(v, w_mine + (h * 2) * kHeads);
+        tmem_ld64(taddr + kHeads, v);
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(accempty(h));
+        const float s1 = weighted_relu_sum(v, w_mine + (h * 2 + 1) * kHeads);
+        if (key <= trow[h * 2])
+          st_evict_first(p.scores + static_cast<size_t>(rrow[h * 2]) * p.kv_stride + key, s0, pol_scores);
+        if (key <= trow[h * 2 + 1])
+          st_evict_first(p.scores + static_cast<size_t>(rrow[h * 2 + 1]) * p.kv_stride + key, s1, pol_scores);
+      }
+      if (!ok) {
+        record_status(p.status, kStatusTimeout);
+        *abort_flag = 1;
+        break;
+      }
+      ++tiles;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, 2 * kPfN);
+  }
+}
+
+}  // namespace
+
+bool index_uses_prefill(int n_q) { return n_q >= kQB; }
+
+namespace {
+
+cudaError_t launch_prefill(const IndexArgs& a, int num_sms, cudaStream_t stream, const CUtensorMap& kmap,
+                           const CUtensorMap& qmap) {
+  const int blocks_per_seq = (a.n_q + kQB - 1) / kQB;
+  const int tiles_per_block = (a.kv_stride + kKeys - 1) / kKeys;
+  const long long total = static_cast<long long>(a.batch) * blocks_per_seq * tiles_per_block;
+  auto kernel = a.fp8 ? sga_index_prefill_kernel<true> : sga_index_prefill_kernel<false>;
+  const size_t smem = a.fp8 ? PrefillCfg<true>::kSmemBytes : PrefillCfg<false>::kSmemBytes;
+  cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  PrefillParams p;
+  p.w = a.w;
+  p.q_pos = a.q_pos;
+  p.scores = a.scores;
+  p.status = a.status;
+  p.n_q = a.n_q;
+  p.kv_stride = a.kv_stride;
+  p.tiles_per_block = tiles_per_block;
+  p.blocks_per_seq = blocks_per_seq;
+  p.total_items = total;
+  const int grid = static_cast<int>(total < num_sms ? total : num_sms);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(grid));
+  cfg.blockDim = dim3(kPfThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, kmap, qmap, p);
+}
+
 }  // namespace
 
 cudaError_t launch_index_scores(const IndexArgs& a, int num_sms, cudaStream_t stream) {
@@ -392,6 +815,7 @@ cudaError_t launch_index_scores(const IndexArgs& a, int num_sms, cudaStream_t st
   if (e != cudaSuccess) return e;
   e = make_tmap_2d(&qmap, a.fp8, a.q_idx, kDim, static_cast<uint64_t>(rows) * kHeads, kDim * esize, strip, kHeads);
   if (e != cudaSuccess) return e;
+  if (index_uses_prefill(a.n_q)) return launch_prefill(a, num_sms, stream, kmap, qmap);
   auto kernel = a.fp8 ? sga_index_kernel<true> : sga_index_kernel<false>;
   const size_t smem = a.fp8 ? IndexCfg<true>::kSmemBytes : IndexCfg<false>::kSmemBytes;
   e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));

@@ -19,7 +19,10 @@ struct IndexArgs {
   int batch, n_q, kv_stride;
   bool fp8;               // indexer queries and keys in E4M3
 };
+// n_q >= 8 queries per sequence take the prefill kernel (query blocks x key
+// tiles), which counts no histogram: `hist` is then ignored.
 cudaError_t launch_index_scores(const IndexArgs& a, int num_sms, cudaStream_t stream);
+bool index_uses_prefill(int n_q);
 
 // ---- top-k (step 2) ------------------------------------------------------------
 struct TopkArgs {

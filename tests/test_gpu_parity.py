@@ -87,6 +87,66 @@ def test_index_scores_bit_exact(B, T, L, pos):
             np.testing.assert_array_equal(got[b, t, : p + 1], want[b, t, : p + 1])
 
 
+# Eight or more queries per sequence take the prefill indexer (blocks of 8
+# queries share each key tile).  Cases: one exact block over whole tiles; a
+# ragged block (13 = 8 + 5) over a ragged last tile; a block of one row;
+# positions out of order inside a block, including 0 and small ones.
+def _prefill_positions(B, T, L, seed):
+    rng = np.random.default_rng(seed)
+    pos = rng.integers(0, L, size=(B, T))
+    pos[0, 0] = L - 1
+    pos[-1, -1] = 0
+    if T > 2:
+        pos[0, 1] = 5
+    return pos.tolist()
+
+
+PREFILL_INDEX_CASES = [
+    (1, 8, 1024, [list(range(1016, 1024))]),
+    (2, 13, 3001, _prefill_positions(2, 13, 3001, 1)),
+    (3, 9, 700, _prefill_positions(3, 9, 700, 2)),
+    (1, 40, 5000, _prefill_positions(1, 40, 5000, 3)),
+    (1, 64, 8192, [list(range(8128, 8192))]),
+]
+
+
+@pytest.mark.parametrize("B,T,L,pos", PREFILL_INDEX_CASES)
+def test_index_scores_prefill_bit_exact(B, T, L, pos):
+    x = gen_small(B, T, L, pos)
+    scores = torch.full((B, T, L), float("nan"), device="cuda")
+    ws = sga.alloc_workspace(sga.make_dims(B, T, L), sga.OP_INDEX_SCORES)
+    sga.index_scores(x["q_idx"], x["w"], x["k_idx"], x["q_pos"], scores=scores, ws=ws)
+    check_status(ws)
+    want = oracle.index_scores(x["q_idx"], x["w"], x["k_idx"], x["q_pos"].cpu())
+    got = scores.cpu().numpy().astype(np.float64)
+    pos = np.asarray(pos)
+    for b in range(B):
+        for t in range(T):
+            p = pos[b, t]
+            np.testing.assert_array_equal(got[b, t, : p + 1], want[b, t, : p + 1])
+            assert np.all(np.isnan(got[b, t, p + 1:])), "entries past the position are left unwritten"
+
+
+def test_index_scores_prefill_bad_position():
+    """A row of a block with a position outside [0, L) is skipped and reported;
+    the other rows of its block are exact."""
+    B, T, L = 1, 10, 1000
+    pos = [[999, 500, 1005, 3, 998, 997, 996, 995, 994, 993]]
+    x = gen_small(B, T, L, pos)
+    scores = torch.full((B, T, L), float("nan"), device="cuda")
+    ws = sga.alloc_workspace(sga.make_dims(B, T, L), sga.OP_INDEX_SCORES)
+    sga.index_scores(x["q_idx"], x["w"], x["k_idx"], x["q_pos"], scores=scores, ws=ws)
+    assert sga.device_status(ws) == 6
+    got = scores.cpu().numpy().astype(np.float64)
+    assert np.all(np.isnan(got[0, 2]))
+    good = [t for t in range(T) if t != 2]
+    qp = x["q_pos"][:, good].contiguous()
+    want = oracle.index_scores(x["q_idx"][:, good].contiguous(), x["w"][:, good].contiguous(), x["k_idx"], qp.cpu())
+    for i, t in enumerate(good):
+        p = pos[0][t]
+        np.testing.assert_array_equal(got[0, t, : p + 1], want[0, i, : p + 1])
+
+
 def test_index_scores_ties_workload_exact():
     x = gen_small(2, 1, 20000, [[19999], [12345]], k_range=1)
     scores = sga.index_scores(x["q_idx"], x["w"], x["k_idx"], x["q_pos"])
@@ -250,7 +310,9 @@ def test_attend_permutation_invariance_and_gate():
 
 @pytest.mark.parametrize("B,T,L,pos", [(2, 1, 1500, [[1499], [700]]),  # ctx <= 2048: dense
                                        (2, 2, 6000, [[2047, 2048], [5999, 3000]]),
-                                       (4, 1, 8192, [[8191]] * 4)])
+                                       (4, 1, 8192, [[8191]] * 4),
+                                       (2, 12, 6000, _prefill_positions(2, 12, 6000, 4)),  # prefill indexer
+                                       (1, 16, 9000, [list(range(8984, 9000))])])
 def test_forward_matches_oracle(B, T, L, pos):
     x = gen_small(B, T, L, pos)
     ws = sga.alloc_workspace(sga.make_dims(B, T, L), sga.OP_FORWARD)
@@ -354,6 +416,23 @@ def test_workload_sampled_parity(name, count):
 
 @pytest.mark.parametrize("B,T,L,pos", INDEX_CASES)
 def test_index_scores_fp8_bit_exact(B, T, L, pos):
+    x = gen_small(B, T, L, pos)
+    qf, kf = synth.to_e4m3(x["q_idx"]), synth.to_e4m3(x["k_idx"])
+    scores = torch.full((B, T, L), float("nan"), device="cuda")
+    ws = sga.alloc_workspace(sga.make_dims(B, T, L), sga.OP_INDEX_SCORES)
+    sga.index_scores_fp8(qf, x["w"], kf, x["q_pos"], scores=scores, ws=ws)
+    check_status(ws)
+    want = oracle.index_scores_e4m3(qf, x["w"], kf, x["q_pos"].cpu())
+    got = scores.cpu().numpy().astype(np.float64)
+    pos = np.asarray(pos)
+    for b in range(B):
+        for t in range(T):
+            p = pos[b, t]
+            np.testing.assert_array_equal(got[b, t, : p + 1], want[b, t, : p + 1])
+
+
+@pytest.mark.parametrize("B,T,L,pos", PREFILL_INDEX_CASES)
+def test_index_scores_prefill_fp8_bit_exact(B, T, L, pos):
     x = gen_small(B, T, L, pos)
     qf, kf = synth.to_e4m3(x["q_idx"]), synth.to_e4m3(x["k_idx"])
     scores = torch.full((B, T, L), float("nan"), device="cuda")
