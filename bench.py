@@ -52,6 +52,10 @@ def parse_args():
                     help="skip the other decode workloads (8K x 4, 32K x 64, 256K x 8 with ties)")
     ap.add_argument("--no-layer", dest="layer", action="store_false",
                     help="skip the whole-layer variant (the projections either side of the path)")
+    ap.add_argument("--prefill-only", action="store_true",
+                    help="run only the chunked-prefill variant and print it (a profiling case)")
+    ap.add_argument("--prefill-queries", type=int, default=0, help="prefill variant: new queries (default 4096)")
+    ap.add_argument("--prefill-ctx", type=int, default=0, help="prefill variant: cache rows (default 131072)")
     ap.add_argument("--cpu-sample-queries", type=int, default=0, help="oracle sample size (0 = auto)")
     ap.add_argument("--batch", type=int, default=0, help="custom decode workload: sequences (with --ctx)")
     ap.add_argument("--ctx", type=int, default=0, help="custom decode workload: context length (with --batch)")
@@ -336,8 +340,14 @@ def decode_variant(sga, synth, name, args, dev, stream, dist, rank, peak) -> dic
 
 
 def prefill_variant(sga, synth, args, dev, stream, dist, rank) -> dict:
-    """Times sga_forward and the indexer alone on the chunked-prefill workload."""
+    """Times sga_forward and the indexer alone on the chunked-prefill workload
+    (4096 queries over a 128K cache unless --prefill-queries / --prefill-ctx say
+    otherwise: the last queries of the context, one sequence)."""
     wl = synth.WORKLOADS["prefill_t4096_ctx128k"]
+    if args.prefill_queries or args.prefill_ctx:
+        T = args.prefill_queries or wl.n_q
+        L = args.prefill_ctx or wl.ctx
+        wl = synth.custom(batch=1, n_q=T, ctx=L, first_pos=L - T, name=f"prefill_t{T}_ctx{L // 1024}k")
     x = synth.make_inputs(wl, device=dev, seed=rank)
     B, T, L, K = wl.batch, wl.n_q, wl.ctx, wl.top_k
     dims = sga.make_dims(B, T, L, K)
@@ -367,7 +377,7 @@ def prefill_variant(sga, synth, args, dev, stream, dist, rank) -> dict:
     peak_tf, peak_kind = measured_tensor_peak()
     world = dist.get_world_size() if dist is not None else 1
     k1_tf = flops / (k1_ms * 1e-3) / 1e12
-    return {"value": B * T * world / (chunk_ms * 1e-3), "unit": "queries/s", "ms_per_chunk": chunk_ms,
+    return {"name": wl.name, "value": B * T * world / (chunk_ms * 1e-3), "unit": "queries/s", "ms_per_chunk": chunk_ms,
             "config": f"{wl.name}: {T} new queries at positions {positions[0]}..{positions[-1]} over a "
                       f"{L}-row cache, top_k {K}; median of {n} iterations, L2 flushed (256 MB memset) before each",
             "indexer": {"ms": k1_ms, "tflops": k1_tf, "flops_per_launch": flops, "peak_tflops": peak_tf,
@@ -404,6 +414,14 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
     dev = torch.device("cuda", local_rank)
     sga.load_library()
+    if args.prefill_only:
+        res = prefill_variant(sga, synth, args, dev, torch.cuda.current_stream(dev), dist, rank)
+        if dist is not None:
+            dist.barrier()
+            dist.destroy_process_group()
+        if rank == 0:
+            print(json.dumps({"variant": res.pop("name"), **res}), flush=True)
+        return
 
     x = synth.make_inputs(wl, device=dev, seed=rank)
     B, T, L, K = wl.batch, wl.n_q, wl.ctx, wl.top_k
@@ -417,9 +435,7 @@ def main():
     idx = torch.empty((B, T, K), dtype=torch.int32, device=dev)
     out = torch.empty((B, T, 64, 512), dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream(dev)
-    att_ws_bytes = sga.workspace_size(dims, sga.OP_SPARSE_MLA_ATTEND)
-    launches_per_step = 3  # indexer, top-k, attention (the attention needs no workspace beyond the status word)
-    assert att_ws_bytes == 256
+    launches_per_step = 3  # indexer, top-k, attention (the attention's split merge needs no combine kernel)
 
     def fwd_step():
         sga.forward(x["q_idx"], x["w"], x["k_idx"], x["q"], x["kv"], x["gate"], x["q_pos"], top_k=K, idx_out=idx,
@@ -644,7 +660,7 @@ def main():
         "gpu_launches": launches_per_step * args.steps}}
     variants.update(decode_lines)
     if prefill is not None:
-        variants["prefill_t4096_ctx128k"] = prefill
+        variants[prefill.pop("name", "prefill_t4096_ctx128k")] = prefill
     if layer is not None:
         layer_step_ms = layer["ms"] / args.steps
         layer_bytes = ab["total"] * rows + layer["weight_bytes"] + layer["act_bytes"]
