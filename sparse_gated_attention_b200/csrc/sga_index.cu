@@ -7,17 +7,19 @@
 // and is ~93% of the bytes of the whole path at 128K context):
 //   * A persistent grid, one CTA per SM, walks a contiguous range of
 //     (query, 128-key tile) work items.
-//   * Warp 0 streams 128-key x 128-dim tiles of k_idx with TMA (128-byte
-//     swizzle, L2 evict-first) through a shared-memory ring, and the query's
+//   * Warp 0 streams 32 KB tiles of k_idx with TMA (128-byte swizzle, L2
+//     evict-first) through a 5-stage shared-memory ring, and the query's
 //     64 x 128 indexer matrix into a double buffer when the query changes.
-//     bf16 keys: 32 KB tiles in a 5-stage ring.  E4M3 keys (the FP8 cache of
+//     bf16 keys: a tile is 128 keys x 128 dims.  E4M3 keys (the FP8 cache of
 //     archdb "A.X K2", pretraining-precision field; nlp.com.ai "A.X K2 FP8"):
-//     16 KB tiles in a 10-stage ring, the same bytes in flight.
+//     a tile is 256 keys (two M = 128 halves), so one barrier round trip per
+//     stage covers as many bytes as in bf16.
 //   * Warp 1 issues tcgen05.mma (M = 128 keys, N = 64 heads, K = 128 dims in 8
-//     kind::f16 steps of 16, or 4 kind::f8f6f4 steps of 32) into one of eight
-//     64-column TMEM accumulators.
+//     kind::f16 steps of 16, or 4 kind::f8f6f4 steps of 32 per half) into one
+//     of eight 64-column (bf16) or four 128-column (E4M3) TMEM accumulators.
 //   * Warps 2-9, two groups of four that take alternate tiles (one warp per
-//     TMEM lane quarter in each), read a key's 64 head dots with tcgen05.ld,
+//     TMEM lane quarter in each; a thread takes one key per 128-key half),
+//     read a key's 64 head dots with tcgen05.ld,
 //     apply ReLU, the per-head weight and the head sum in fp32, mask s > t and
 //     store the score (32 consecutive keys per warp: one 128-byte store).
 //     When the caller asks for it, they also count each score's top 12 order
@@ -35,25 +37,29 @@ constexpr int kDim = 128;     // indexer dim: MMA K
 constexpr int kHeads = 64;    // indexer heads: MMA N
 constexpr int kABox = kKeys * 128;  // one 128-byte-wide column strip of a tile (16 KB)
 constexpr int kQBox = kHeads * 128;  // one 128-byte-wide column strip of a query's matrix (8 KB)
-constexpr int kAcc = 8;  // TMEM accumulators (all 512 columns): the MMA runs up to 8 tiles ahead of the epilogue
-static_assert((kAcc & (kAcc - 1)) == 0, "the epilogue indexes accumulators with a mask");
-constexpr int kTmemCols = kAcc * kHeads;  // 512
+constexpr int kTmemCols = 512;  // TMEM accumulators fill all 512 columns
 constexpr int kEpiGroups = 2;   // epilogue warp groups, taking alternate tiles
 constexpr int kThreads = 64 + kEpiGroups * 128;
 constexpr int kHistBytes = kTopkHistBins * 4;
 constexpr int kEpiThreads = 128;
 
-// bf16 keys: a key row is 256 B, two 128-byte strips; K = 128 in 8 MMA steps of 16.
-// E4M3 keys: a key row is one 128-byte strip; K = 128 in 4 MMA steps of 32.  The
-// E4M3 ring has twice the stages so the bytes in flight stay the same.
+// bf16 keys: a key row is 256 B, two 128-byte strips; K = 128 in 8 MMA steps of
+// 16; a tile is 128 keys.  E4M3 keys: a key row is one 128-byte strip; K = 128
+// in 4 MMA steps of 32; a tile is 256 keys (two M = 128 halves), so both tiles
+// are 32 KB and one barrier round trip per stage covers the same bytes.
 template <bool kFp8>
 struct IndexCfg {
   static constexpr int kStrips = kFp8 ? 1 : 2;        // 128-byte strips per key (and query) row
   static constexpr int kStripElems = kFp8 ? 128 : 64;  // elements per strip
-  static constexpr int kStages = kFp8 ? 10 : 5;
-  static constexpr int kAStage = kStrips * kABox;
+  static constexpr int kHalves = kFp8 ? 2 : 1;         // 128-key halves per tile (one MMA M each)
+  static constexpr int kTileKeys = kKeys * kHalves;
+  static constexpr int kStages = 5;
+  static constexpr int kAStage = kStrips * kABox * kHalves;  // 32 KB
   static constexpr int kQBuf = kStrips * kQBox;
   static constexpr int kKSteps = kFp8 ? 4 : 8;         // 32-byte K steps per tile
+  static constexpr int kAccCols = kHeads * kHalves;    // one tile's accumulator
+  static constexpr int kAcc = kTmemCols / kAccCols;    // 8 (bf16) or 4 (E4M3) tiles in flight
+  static_assert((kAcc & (kAcc - 1)) == 0, "the epilogue indexes accumulators with a mask");
   static constexpr int kNumBars = 2 * kStages + 4 + 2 * kAcc + 1;
   static constexpr size_t kSmemBytes =
       1024 + kStages * kAStage + 2 * kQBuf + kEpiGroups * kHistBytes + kNumBars * 8 + 16;
@@ -74,17 +80,18 @@ struct IndexParams {
 // Walks work items j = (query row, 128-key tile) in order: one division at
 // the start, then a key step per item; the query position is read only when
 // the row changes.
+template <int kTileKeys>
 struct TileCursor {
   int row, key0, t;
   __device__ __forceinline__ void start(const IndexParams& p, long long j) {
     row = static_cast<int>(j / p.tiles_per_row);
-    key0 = static_cast<int>(j % p.tiles_per_row) * kKeys;
+    key0 = static_cast<int>(j % p.tiles_per_row) * kTileKeys;
     t = __ldg(p.q_pos + row);
   }
   // Moves to item j + 1; `more` is false after the last item of the range.
   __device__ __forceinline__ void next(const IndexParams& p, bool more) {
-    key0 += kKeys;
-    if (key0 >= p.tiles_per_row * kKeys) {
+    key0 += kTileKeys;
+    if (key0 >= p.tiles_per_row * kTileKeys) {
       key0 = 0;
       ++row;
       if (more) t = __ldg(p.q_pos + row);
@@ -101,6 +108,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                      IndexParams p) {
   using C = IndexCfg<kFp8>;
   constexpr int kStages = C::kStages, kAStage = C::kAStage, kQBuf = C::kQBuf, kNumBars = C::kNumBars;
+  constexpr int kAcc = C::kAcc;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t a_base = smem_u32(smem);
@@ -167,7 +175,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t ph = 0;    // phase parity of that stage's current use
       int cur_row = -1;
       bool ok = true;
-      TileCursor cur;
+      TileCursor<C::kTileKeys> cur;
       if (j0 < j1) cur.start(p, j0);
       for (long long j = j0; j < j1; cur.next(p, ++j < j1)) {
         if (!cur.live(p)) {
@@ -198,6 +206,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int b = 0; b < C::kStrips; ++b)
           tma_load_2d(a_base + st * kAStage + b * kABox, &kmap, full(st), b * C::kStripElems, y, pol_stream);
+        // (an E4M3 tile is one box of 256 key rows: both halves, 16 KB apart)
         ++n;
         if (++st == kStages) {
           st = 0;
@@ -228,7 +237,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t ph = 0, aph = 0;       // their phase parities
       int cur_row = -1, cur_q = 0;
       bool ok = true;
-      TileCursor cur;
+      TileCursor<C::kTileKeys> cur;
       if (j0 < j1) cur.start(p, j0);
       for (long long j = j0; j < j1 && ok; cur.next(p, ++j < j1)) {
         if (!cur.live(p)) continue;
@@ -253,18 +262,21 @@ __global__ void __launch_bounds__(kThreads, 1)
           break;
         }
         tc_fence_after();
-        const uint32_t d = tmem_base + static_cast<uint32_t>(acc * kHeads);
-        const uint64_t a_desc = a_desc0 + static_cast<uint64_t>((st * kAStage) >> 4);
         const uint64_t b_desc = q_desc0 + static_cast<uint64_t>((cur_q * kQBuf) >> 4);
 #pragma unroll
-        for (int k = 0; k < C::kKSteps; ++k) {
-          // 32-byte K steps: four per 128-byte strip
-          const uint64_t a_off = static_cast<uint64_t>(((k >> 2) * kABox + (k & 3) * 32) >> 4);
-          const uint64_t b_off = static_cast<uint64_t>(((k >> 2) * kQBox + (k & 3) * 32) >> 4);
-          if constexpr (kFp8)
-            mma_e4m3(d, a_desc + a_off, b_desc + b_off, idesc, k > 0 ? 1u : 0u);
-          else
-            mma_bf16(d, a_desc + a_off, b_desc + b_off, idesc, k > 0 ? 1u : 0u);
+        for (int hh = 0; hh < C::kHalves; ++hh) {
+          const uint32_t d = tmem_base + static_cast<uint32_t>(acc * C::kAccCols + hh * kHeads);
+          const uint64_t a_desc = a_desc0 + static_cast<uint64_t>((st * kAStage + hh * kABox) >> 4);
+#pragma unroll
+          for (int k = 0; k < C::kKSteps; ++k) {
+            // 32-byte K steps: four per 128-byte strip
+            const uint64_t a_off = static_cast<uint64_t>(((k >> 2) * kABox + (k & 3) * 32) >> 4);
+            const uint64_t b_off = static_cast<uint64_t>(((k >> 2) * kQBox + (k & 3) * 32) >> 4);
+            if constexpr (kFp8)
+              mma_e4m3(d, a_desc + a_off, b_desc + b_off, idesc, k > 0 ? 1u : 0u);
+            else
+              mma_bf16(d, a_desc + a_off, b_desc + b_off, idesc, k > 0 ? 1u : 0u);
+          }
         }
         mma_commit(empty(st));
         mma_commit(accfull(acc));
@@ -316,7 +328,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int b = et; b < kTopkHistBins; b += kEpiThreads) hist_g[b] = 0;
       named_barrier(bar_id, kEpiThreads);
     }
-    TileCursor cur;
+    TileCursor<C::kTileKeys> cur;
     if (j0 < j1) cur.start(p, j0);
     for (long long j = j0; j < j1; cur.next(p, ++j < j1)) {
       if (!cur.live(p)) continue;
@@ -347,22 +359,28 @@ __global__ void __launch_bounds__(kThreads, 1)
         break;
       }
       tc_fence_after();
-      float v[64];
-      const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + static_cast<uint32_t>(acc * kHeads);
-      tmem_ld64(taddr, v);
-      tc_fence_before();
-      mbar_arrive(accempty(acc));
-      // head sum as four independent chains (one warp per scheduler: the chain
-      // latency, not issue, bounds the epilogue); integer-valued inputs keep
-      // every partial sum exact, so the order does not change the score
-      float ps[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-      for (int h = 0; h < 64; ++h) ps[h & 3] = fmaf(wv[h], fmaxf(v[h], 0.f), ps[h & 3]);
-      const float s = (ps[0] + ps[1]) + (ps[2] + ps[3]);
-      const int key = key0 + quarter * 32 + lane;
-      if (key <= t) {
-        p.scores[static_cast<size_t>(row) * p.kv_stride + key] = s;
-        if (with_hist) atomicAdd(hist_g + (order_bits(s) >> (32 - kTopkHistBits)), 1u);
+      for (int hh = 0; hh < C::kHalves; ++hh) {
+        float v[64];
+        const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
+                               static_cast<uint32_t>(acc * C::kAccCols + hh * kHeads);
+        tmem_ld64(taddr, v);
+        if (hh == C::kHalves - 1) {
+          tc_fence_before();
+          mbar_arrive(accempty(acc));
+        }
+        // head sum as four independent chains (one warp per scheduler: the chain
+        // latency, not issue, bounds the epilogue); integer-valued inputs keep
+        // every partial sum exact, so the order does not change the score
+        float ps[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int h = 0; h < 64; ++h) ps[h & 3] = fmaf(wv[h], fmaxf(v[h], 0.f), ps[h & 3]);
+        const float s = (ps[0] + ps[1]) + (ps[2] + ps[3]);
+        const int key = key0 + hh * kKeys + quarter * 32 + lane;
+        if (key <= t) {
+          p.scores[static_cast<size_t>(row) * p.kv_stride + key] = s;
+          if (with_hist) atomicAdd(hist_g + (order_bits(s) >> (32 - kTopkHistBits)), 1u);
+        }
       }
       ++an;
     }
@@ -804,18 +822,21 @@ cudaError_t launch_prefill(const IndexArgs& a, int num_sms, cudaStream_t stream,
 
 cudaError_t launch_index_scores(const IndexArgs& a, int num_sms, cudaStream_t stream) {
   const int rows = a.batch * a.n_q;
-  const int tiles_per_row = (a.kv_stride + kKeys - 1) / kKeys;
+  const bool prefill = index_uses_prefill(a.n_q);
+  // decode E4M3 tiles are 256 keys: one box of 256 rows
+  const int tile_keys = (a.fp8 && !prefill) ? IndexCfg<true>::kTileKeys : kKeys;
+  const int tiles_per_row = (a.kv_stride + tile_keys - 1) / tile_keys;
   const long long total = static_cast<long long>(rows) * tiles_per_row;
   if (total == 0) return cudaSuccess;
   const int esize = a.fp8 ? 1 : 2;
   const uint32_t strip = a.fp8 ? 128 : 64;  // elements per 128-byte strip
   CUtensorMap kmap, qmap;
   cudaError_t e = make_tmap_2d(&kmap, a.fp8, a.k_idx, kDim, static_cast<uint64_t>(a.batch) * a.kv_stride,
-                               kDim * esize, strip, kKeys);
+                               kDim * esize, strip, static_cast<uint32_t>(tile_keys));
   if (e != cudaSuccess) return e;
   e = make_tmap_2d(&qmap, a.fp8, a.q_idx, kDim, static_cast<uint64_t>(rows) * kHeads, kDim * esize, strip, kHeads);
   if (e != cudaSuccess) return e;
-  if (index_uses_prefill(a.n_q)) return launch_prefill(a, num_sms, stream, kmap, qmap);
+  if (prefill) return launch_prefill(a, num_sms, stream, kmap, qmap);
   auto kernel = a.fp8 ? sga_index_kernel<true> : sga_index_kernel<false>;
   const size_t smem = a.fp8 ? IndexCfg<true>::kSmemBytes : IndexCfg<false>::kSmemBytes;
   e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));

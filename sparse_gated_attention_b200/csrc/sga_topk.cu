@@ -11,8 +11,8 @@
 // contiguous segment of positions (a multiple of 128).
 //
 // Resident kernel (segments of at most 32768 positions, i.e. rows up to
-// 8 x 32768): the whole segment is copied once into shared memory (four 32 KB
-// bulk copies) and every pass reads it there.  Warp w owns 1024 consecutive
+// 8 x 32768): the whole segment is copied once into shared memory (eight
+// 16-byte loads per thread, all in flight at once) and every pass reads it there.  Warp w owns 1024 consecutive
 // positions of the segment and walks them 32 at a time, so a ballot over one
 // step is the 32-position word of that step in position order.
 //   1. MSD radix select over the score key, 12/12/8 bits per level: each CTA
@@ -69,8 +69,7 @@ constexpr size_t kSmemBytes =
 constexpr int kResSeg = 32768;                  // positions per CTA held in shared memory (128 KB)
 constexpr int kResWarpSpan = kResSeg / kWarps;  // 1024 consecutive positions per warp
 constexpr int kResSteps = kResWarpSpan / 32;    // 32 ballot steps per warp and pass
-constexpr int kResChunks = kResSeg / kChunk;    // 4 bulk copies
-constexpr size_t kResSmemBytes = kResSeg * 4 + 2 * kBins * 4 + kCandCap * 8 + (kResChunks + 1) * 8;
+constexpr size_t kResSmemBytes = kResSeg * 4 + 2 * kBins * 4 + kCandCap * 8;
 static_assert(kResSteps == 32, "lane j keeps the words of step j");
 
 struct TopkParams {
@@ -144,31 +143,68 @@ __device__ __forceinline__ Narrow find_bin(const uint32_t* hist, uint32_t need, 
 }
 
 // Narrows the first nc candidates (key << 32 | ~position), all in the bin
-// (prefix, mask, shift), to the exact K-th key with the radix levels of the
-// main selection.  Returns K* in the high 32 bits (kmask then covers all of
-// them); `need` becomes the number of ties at K* still to take.
+// (prefix, mask, shift), to the exact K-th key with 8-bit radix levels: every
+// thread counts into a 256-bin histogram in `ghist`, then one warp finds the
+// bin with a warp scan (8 bins per lane) and publishes it, so a level costs
+// three block barriers and no block-wide scan.  Every thread must call it after
+// the list is complete.  Returns K* in the high 32 bits (kmask then covers all
+// of them); `need` becomes the number of ties at K* still to take.
 __device__ __noinline__ uint64_t refine_candidates(const uint64_t* cand, uint32_t nc, uint32_t* ghist, uint32_t prefix,
                                                    uint32_t mask, int shift, uint32_t& need, uint32_t* warp_buf,
                                                    Narrow* narrow, uint64_t& kmask) {
-  const int tid = threadIdx.x;
+  (void)warp_buf;
+  constexpr int kDigit = 8;
+  const int tid = threadIdx.x, lane = tid & 31;
   kmask = static_cast<uint64_t>(mask) << 32;
   uint64_t kpref = static_cast<uint64_t>(prefix) << 32;
   while (shift > 0) {
-    const int width = shift >= kBits ? kBits : shift;
+    const int width = shift >= kDigit ? kDigit : shift;
     shift -= width;
-    const uint32_t dmask = (1u << width) - 1u;
-    for (int b = tid; b < kBins; b += kThreads) ghist[b] = 0;
+    const int nbins = 1 << width;
+    const uint32_t dmask = static_cast<uint32_t>(nbins - 1);
+    if (tid < (1 << kDigit)) ghist[tid] = 0;
     __syncthreads();
     for (uint32_t i = tid; i < nc; i += kThreads) {
       const uint64_t c = cand[i];
       if ((c & kmask) == kpref) atomicAdd(ghist + (static_cast<uint32_t>(c >> (32 + shift)) & dmask), 1u);
     }
     __syncthreads();
-    const Narrow nr = find_bin(ghist, need, warp_buf, narrow);
-    kpref |= static_cast<uint64_t>(nr.digit) << (32 + shift);
+    if (tid < 32) {
+      // lane l holds bins nbins-1-8l .. nbins-8-8l (descending keys)
+      uint32_t h[8], sum = 0;
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        const int b = nbins - 1 - (8 * lane + k);
+        h[k] = b >= 0 ? ghist[b] : 0u;
+        sum += h[k];
+      }
+      uint32_t incl = sum;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t y = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+        if (lane >= o) incl += y;
+      }
+      const uint32_t excl = incl - sum;
+      if (excl < need && need <= incl) {  // exactly one lane
+        uint32_t run = excl;
+        bool found = false;
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          if (!found && need <= run + h[k]) {
+            narrow->digit = static_cast<uint32_t>(nbins - 1 - (8 * lane + k));
+            narrow->above = run;
+            found = true;
+          }
+          run += h[k];
+        }
+      }
+    }
+    __syncthreads();
+    kpref |= static_cast<uint64_t>(narrow->digit) << (32 + shift);
     kmask |= static_cast<uint64_t>(dmask) << (32 + shift);
-    need -= nr.above;
+    need -= narrow->above;
   }
+  __syncthreads();  // every thread has read `narrow` and the histogram before either is reused
   return kpref;
 }
 
@@ -583,15 +619,6 @@ __global__ void __launch_bounds__(kThreads, 1) sga_topk_stream_kernel(TopkParams
   }
 }
 
-// Waits (once per warp) for the bulk copy that holds this warp's positions.
-__device__ __forceinline__ void wait_own_chunk(bool& have, int wbase, int len, uint32_t bar0, volatile int* abort_flag,
-                                               int* status) {
-  if (have) return;
-  have = true;
-  if (wbase < len && !mbar_wait(bar0 + 8u * static_cast<uint32_t>(wbase / kChunk), 0, abort_flag))
-    record_status(status, kStatusTimeout);
-}
-
 template <bool kVec>
 __global__ void __launch_bounds__(kThreads, 1) sga_topk_resident_kernel(TopkParams p) {
   extern __shared__ __align__(128) uint8_t smem_raw[];
@@ -599,14 +626,12 @@ __global__ void __launch_bounds__(kThreads, 1) sga_topk_resident_kernel(TopkPara
   uint32_t* lhist = reinterpret_cast<uint32_t*>(smem_raw + kResSeg * 4);
   uint32_t* ghist = lhist + kBins;
   uint64_t* cand = reinterpret_cast<uint64_t*>(ghist + kBins);
-  uint64_t* bars = cand + kCandCap;  // chunk[kResChunks], hist
   __shared__ uint32_t warp_buf[kWarps];
   __shared__ uint32_t wsel[kWarps], wtie[kWarps];  // per-warp exclusive prefixes of the word popcounts
   __shared__ Narrow narrow;
   __shared__ uint32_t cand_n;
   __shared__ uint32_t peer_n[kMaxCluster];          // candidate-list lengths, written by each CTA of the cluster
   __shared__ uint32_t peer_counts[kMaxCluster][2];  // (selected, ties) of each CTA's segment, written by that CTA
-  __shared__ int abort_flag;
 
   cg::cluster_group cluster = cg::this_cluster();
   const int C = static_cast<int>(cluster.num_blocks());
@@ -642,39 +667,37 @@ __global__ void __launch_bounds__(kThreads, 1) sga_topk_resident_kernel(TopkPara
   const int per = (((n + C - 1) / C) + 127) & ~127;
   const int s0 = min(rank * per, n), s1 = min(s0 + per, n);
   const int len = s1 - s0;
-  const int nch = (len + kChunk - 1) / kChunk;
-  const uint32_t bar0 = smem_u32(bars);
-  const uint32_t hist_bar = bar0 + 8u * kResChunks;
-  if (tid == 0) {
-    cand_n = 0;
-    abort_flag = 0;
-    for (int i = 0; i <= kResChunks; ++i) mbar_init(bar0 + 8u * i, 1);
-    fence_barrier_init();
-  }
-  __syncthreads();
+  if (tid == 0) cand_n = 0;
   if (kVec) {
-    if (tid == 0) {
-      if (p.hist) {
-        mbar_arrive_expect_tx(hist_bar, kBins * 4);
-        bulk_load(smem_u32(ghist), hist_row, kBins * 4, hist_bar);
-      }
-      for (int c = 0; c < nch; ++c) {
-        const int cnt = min(kChunk, len - c * kChunk);
-        // rows are 16-byte aligned and kv_stride % 4 == 0, so rounding up stays inside the row
-        const uint32_t bytes = static_cast<uint32_t>((cnt + 3) & ~3) * 4u;
-        mbar_arrive_expect_tx(bar0 + 8u * c, bytes);
-        bulk_load(smem_u32(seg + c * kChunk), sc + s0 + c * kChunk, bytes, bar0 + 8u * c);
-      }
+    // The whole segment with 16-byte loads from every thread, all in flight at
+    // once (rows are 16-byte aligned and kv_stride % 4 == 0, so rounding the
+    // length up to 4 stays inside the row), and the histogram row likewise.
+    constexpr int kPerThread = kResSeg / 4 / kThreads;  // 8 float4
+    const float4* src = reinterpret_cast<const float4*>(sc + s0);
+    const int n4 = (len + 3) >> 2;
+    float4 v[kPerThread];
+#pragma unroll
+    for (int k = 0; k < kPerThread; ++k) {
+      const int i = tid + k * kThreads;
+      if (i < n4) v[k] = __ldcg(src + i);
     }
+    uint4 hv = make_uint4(0u, 0u, 0u, 0u);
+    if (p.hist) hv = __ldcg(reinterpret_cast<const uint4*>(hist_row) + tid);
+#pragma unroll
+    for (int k = 0; k < kPerThread; ++k) {
+      const int i = tid + k * kThreads;
+      if (i < n4) reinterpret_cast<float4*>(seg)[i] = v[k];
+    }
+    if (p.hist) reinterpret_cast<uint4*>(ghist)[tid] = hv;
   } else {
     for (int i = tid; i < len; i += kThreads) seg[i] = __ldg(sc + s0 + i);
     if (p.hist) {
       for (int b = tid; b < kBins; b += kThreads) ghist[b] = hist_row[b];
     }
-    __syncthreads();
   }
+  __syncthreads();
+  static_assert(kBins == 4 * kThreads, "one uint4 of the histogram row per thread");
   const int wbase = warp * kResWarpSpan;  // this warp's first position within the segment
-  bool have_seg = !kVec;
 
   // ---- 1. radix levels on the score key until the bin fits the candidate list or is one key
   uint32_t prefix = 0, mask = 0;
@@ -687,11 +710,9 @@ __global__ void __launch_bounds__(kThreads, 1) sga_topk_resident_kernel(TopkPara
     shift -= width;
     const uint32_t dmask = (1u << width) - 1u;
     if (first && p.hist) {
-      if (kVec && !mbar_wait(hist_bar, 0, &abort_flag)) record_status(p.status, kStatusTimeout);
-      __syncthreads();
+      // the first level comes from the indexer's histogram, already in ghist
     } else {
       for (int b = tid; b < kBins; b += kThreads) lhist[b] = 0;
-      wait_own_chunk(have_seg, wbase, len, bar0, &abort_flag, p.status);
       __syncthreads();
 #pragma unroll 4
       for (int j = 0; j < kResSteps; ++j) {
@@ -722,7 +743,6 @@ __global__ void __launch_bounds__(kThreads, 1) sga_topk_resident_kernel(TopkPara
   // ---- 2. one pass: per 32 positions a word of keys above the bin and a word
   // of keys in it (lane j keeps the words of step j).  As floats, "above" is
   // f > f_hi and "in the bin" f_lo <= f <= f_hi.
-  wait_own_chunk(have_seg, wbase, len, bar0, &abort_flag, p.status);
   const float f_lo = key_to_float_lo(prefix), f_hi = key_to_float_hi(prefix | ~mask);
   uint32_t my_sel = 0, my_bin = 0;
 #pragma unroll 8
