@@ -52,6 +52,8 @@ def parse_args():
                     help="skip the other decode workloads (8K x 4, 32K x 64, 256K x 8 with ties)")
     ap.add_argument("--no-layer", dest="layer", action="store_false",
                     help="skip the whole-layer variant (the projections either side of the path)")
+    ap.add_argument("--layer-only", action="store_true",
+                    help="run only the whole-layer variant and print it (a profiling case)")
     ap.add_argument("--prefill-only", action="store_true",
                     help="run only the chunked-prefill variant and print it (a profiling case)")
     ap.add_argument("--prefill-queries", type=int, default=0, help="prefill variant: new queries (default 4096)")
@@ -385,6 +387,40 @@ def prefill_variant(sga, synth, args, dev, stream, dist, rank) -> dict:
             "gpu_launches": 3}
 
 
+def layer_variant(sga, synth, args, dev, stream, dist, rank, x, dims, idx) -> dict:
+    """One whole SGA layer (a separate configuration): h -> projections -> the path
+    -> W_UV, o_proj, on the workload's caches (the new tokens' rows are rewritten
+    at their positions every step), timed over K steps like the main region."""
+    B, T = x["q_pos"].shape
+    K = dims.top_k
+    lw_t = synth.make_layer_weights(device=dev, seed=rank)
+    gl = torch.Generator(device=dev).manual_seed(rank + 99)
+    h = torch.randn((B, T, synth.D_MODEL), generator=gl, device=dev).to(torch.bfloat16)
+    ws_layer = sga.alloc_layer_workspace(dims, sga.layer_weights(lw_t), sga.LAYER_FORWARD, dev)
+    y = torch.empty((B, T, synth.D_MODEL), dtype=torch.float32, device=dev)
+
+    def layer_step():
+        sga.layer_forward(lw_t, h, x["q_pos"], x["kv"], x["k_idx"], top_k=K, idx_out=idx, y=y, ws=ws_layer,
+                          stream=stream)
+
+    for _ in range(max(args.warmup, 3)):
+        layer_step()
+    torch.cuda.synchronize(dev)
+    if dist is not None:
+        dist.barrier()
+    s4, e4 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s4.record(stream)
+    for _ in range(args.steps):
+        layer_step()
+    e4.record(stream)
+    torch.cuda.synchronize(dev)
+    layer_ms = max_over_ranks(dist, dev, s4.elapsed_time(e4))
+    if sga.device_status(ws_layer) != 0:
+        raise RuntimeError("device status set during the layer variant run")
+    weight_bytes = sum(t.numel() * t.element_size() for t in lw_t.values())
+    return {"ms": layer_ms, "weight_bytes": weight_bytes, "act_bytes": h.numel() * 2 + y.numel() * 4}
+
+
 def main():
     args = parse_args()
     from sparse_gated_attention_b200 import synth
@@ -414,6 +450,16 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
     dev = torch.device("cuda", local_rank)
     sga.load_library()
+    if args.layer_only:
+        wl_l = synth.WORKLOADS[args.workload or synth.HEADLINE]
+        xl = synth.make_inputs(wl_l, device=dev, seed=rank)
+        dl = sga.make_dims(wl_l.batch, wl_l.n_q, wl_l.ctx, wl_l.top_k)
+        il = torch.empty((wl_l.batch, wl_l.n_q, wl_l.top_k), dtype=torch.int32, device=dev)
+        res = layer_variant(sga, synth, args, dev, torch.cuda.current_stream(dev), dist, rank, xl, dl, il)
+        if rank == 0:
+            print(json.dumps({"variant": "sga_layer", "ms_per_step": res["ms"] / args.steps,
+                              "weight_bytes": res["weight_bytes"]}), flush=True)
+        return
     if args.prefill_only:
         res = prefill_variant(sga, synth, args, dev, torch.cuda.current_stream(dev), dist, rank)
         if dist is not None:
@@ -574,37 +620,7 @@ def main():
     # ---- one whole SGA layer (a separate configuration): h -> projections ->
     # the path -> W_UV, o_proj, on the same caches (the new tokens' rows are
     # rewritten at their positions every step), timed like the main region.
-    layer = None
-    if args.layer:
-        lw_t = synth.make_layer_weights(device=dev, seed=rank)
-        lw = sga.layer_weights(lw_t)
-        gl = torch.Generator(device=dev).manual_seed(rank + 99)
-        h = torch.randn((B, T, synth.D_MODEL), generator=gl, device=dev).to(torch.bfloat16)
-        ws_layer = sga.alloc_layer_workspace(dims, lw, sga.LAYER_FORWARD, dev)
-        y = torch.empty((B, T, synth.D_MODEL), dtype=torch.float32, device=dev)
-
-        def layer_step():
-            sga.layer_forward(lw_t, h, x["q_pos"], x["kv"], x["k_idx"], top_k=K, idx_out=idx, y=y, ws=ws_layer,
-                              stream=stream)
-
-        for _ in range(max(args.warmup, 3)):
-            layer_step()
-        torch.cuda.synchronize(dev)
-        if dist is not None:
-            dist.barrier()
-        s4, e4 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        s4.record(stream)
-        for _ in range(args.steps):
-            layer_step()
-        e4.record(stream)
-        torch.cuda.synchronize(dev)
-        layer_ms = max_over_ranks(dist, dev, s4.elapsed_time(e4))
-        if sga.device_status(ws_layer) != 0:
-            raise RuntimeError("device status set during the layer variant run")
-        weight_bytes = sum(t.numel() * t.element_size() for t in lw_t.values())
-        layer = {"ms": layer_ms, "weight_bytes": weight_bytes,
-                 "act_bytes": h.numel() * 2 + y.numel() * 4}
-        del lw_t, ws_layer
+    layer = layer_variant(sga, synth, args, dev, stream, dist, rank, x, dims, idx) if args.layer else None
 
     # ---- the other decode workloads (separate configurations, one line each in `variants`)
     decode_lines = {}
@@ -667,13 +683,14 @@ def main():
         layer_gbs = layer_bytes / (layer_step_ms * 1e-3) / 1e9
         variants["sga_layer"] = {
             "value": whole_job_rate(rows, args.steps, world, layer["ms"]), "unit": UNIT, "ms_per_step": layer_step_ms,
-            "config": f"{wl.name} as one whole SGA layer: d_model 7168, q rank 1536, projections in cuBLAS "
-                      f"(bf16, fp32 accumulation), bf16 activations between contractions",
+            "config": f"{wl.name} as one whole SGA layer: d_model 7168, q rank 1536, projections in the library's "
+                      f"weight-streaming tcgen05 GEMM (bf16, fp32 accumulation), bf16 activations between contractions",
             "path_roofline": {"achieved_gbs": layer_gbs, "frac_of_8tbs": layer_gbs / NOMINAL_HBM_GBS,
                               "frac_of_measured": layer_gbs / peak, "bytes_per_step": layer_bytes,
                               "weight_bytes": layer["weight_bytes"]},
-            # own kernels per step: two projection preps, three bf16 conversions, the path's three
-            "gpu_launches": 8 * args.steps}
+            # own kernels per step: five GEMMs, two projection preps, the out conversion, the
+            # G5 partial sum, the path's three
+            "gpu_launches": 12 * args.steps}
 
     cpu = None
     if not args.no_cpu_baseline and world == 1:

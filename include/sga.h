@@ -249,10 +249,10 @@ SGA_API sga_status_t sga_topk_select_noalloc(const sga_dims_t* dims, const float
  *   o_h = W_UV_h out_h;  y = W_O [o_1; ...; o_64]
  * Every activation between two contractions is rounded to bf16 (to nearest,
  * ties to even); the contractions accumulate in fp32; y is fp32.  The GEMMs
- * run in cuBLAS (bf16 inputs, fp32 accumulation); the first call on each
- * device creates the library's cuBLAS handle, so make it outside stream
- * capture; the handle lives until the process exits.  Calls on one device
- * share that handle and must be ordered on one stream.
+ * are this library's tcgen05 kernels (the weights streamed once, the new
+ * tokens in the MMA's N dimension); when one splits K for parallelism its fp32
+ * partial sums are added in a fixed order, so results do not depend on the
+ * schedule.  Layer calls are thread-safe across distinct workspaces.
  *
  * Weights: bf16, row-major, `out = W in` (torch Linear layout), packed so the
  * projections that read the same input are one GEMM:

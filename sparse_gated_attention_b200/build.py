@@ -10,8 +10,8 @@ PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libsga.so")
-SOURCES = ["sga_api.cu", "sga_index.cu", "sga_topk.cu", "sga_attend.cu", "sga_layer.cu", "sga_warmup.cu",
-           "sga_diag.cu"]
+SOURCES = ["sga_api.cu", "sga_index.cu", "sga_topk.cu", "sga_attend.cu", "sga_gemm.cu", "sga_layer.cu",
+           "sga_warmup.cu", "sga_diag.cu"]
 DEPS = SOURCES + ["sga_ptx.cuh", "sga_internal.cuh", "sga_host.h"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
@@ -21,15 +21,6 @@ def nvcc_path() -> str:
     if not os.path.exists(cand):
         raise RuntimeError("nvcc not found: the CUDA toolkit is required to build libsga")
     return cand
-
-
-def cublas_link() -> list:
-    """Link flags for cuBLAS (the layer's projection GEMMs).  The soname
-    libcublas.so.12 resolves to the copy PyTorch has already loaded when the
-    binding opens the library after importing torch; the toolkit's directory
-    is the runpath for any other loader."""
-    lib = os.path.join(os.path.dirname(os.path.dirname(os.path.realpath(nvcc_path()))), "lib64")
-    return ["-L", lib, "-lcublas", "-Xlinker", "-rpath=" + lib]
 
 
 def _stale() -> bool:
@@ -47,7 +38,7 @@ def build(force: bool = False, verbose: bool = False) -> str:
     tmp = LIB + ".tmp"
     cmd = [nvcc_path(), "-std=c++17", "-O3", *ARCH, "-lineinfo", "-shared", "-Xcompiler", "-fPIC",
            "-Xcompiler", "-fvisibility=hidden", "-I", os.path.join(ROOT, "include"),
-           *[os.path.join(CSRC, f) for f in SOURCES], "-o", tmp, *cublas_link()]
+           *[os.path.join(CSRC, f) for f in SOURCES], "-o", tmp]
     if verbose:
         print(" ".join(cmd), file=sys.stderr)
     subprocess.check_call(cmd)

@@ -51,6 +51,26 @@ struct AttendArgs {
 int attend_splits(int rows, int top_k);
 cudaError_t launch_attend(const AttendArgs& a, cudaStream_t stream);
 
+// ---- the layer's projections: weight-streaming GEMM -----------------------------------
+// Y[b][n][m] = sum_k X[n][x_col_per_batch * b + k] W[b](m, k), W row-major
+// [batch][m][k] (K-major) or [batch][k][m] (MN-major), bf16 in, fp32 accumulate.
+constexpr int kGemmMaxN = 128;  // tokens per work item (more tokens: several items)
+struct GemmArgs {
+  const uint16_t* w;
+  const uint16_t* x;     // [n][x_ld] bf16 (x_ld * 2 bytes a multiple of 16)
+  int m, n, k, batch;
+  bool w_mn_major;
+  int x_ld, x_col_per_batch;
+  int splits;            // K splits: fp32 partials, added by the consumer in split order
+  float* part;           // fp32 output part[split][n][batch * m], or null
+  uint16_t* out;         // bf16 output out[col * out_ld + b * out_boff + m] (splits == 1), or null
+  int out_ld, out_boff;
+  int* status;
+};
+// K splits that keep `num_sms` SMs streaming when there are fewer tiles than SMs.
+int gemm_splits(int m, int n, int k, int batch, int num_sms);
+cudaError_t launch_gemm(const GemmArgs& a, int num_sms, cudaStream_t stream);
+
 // ---- tensor maps -------------------------------------------------------------------
 // 2-D bf16 tensor map: `inner` elements per row, `outer` rows, rows `row_bytes`
 // apart, box {box_inner, box_outer}, 128-byte swizzle.
