@@ -73,7 +73,8 @@ typedef enum {
   SGA_ERR_WORKSPACE = 3,   /* workspace null, misaligned or too small */
   SGA_ERR_CUDA = 4,        /* a CUDA runtime call or kernel launch failed */
   SGA_ERR_TIMEOUT = 5,     /* device: a bounded wait inside a kernel ran out */
-  SGA_ERR_DEVICE_ARG = 6   /* device: a position or index outside its range */
+  SGA_ERR_DEVICE_ARG = 6,  /* device: a position or index outside its range */
+  SGA_ERR_INTERNAL = 7     /* device: an internal invariant check failed (libsga_debug.so only) */
 } sga_status_t;
 
 typedef enum {

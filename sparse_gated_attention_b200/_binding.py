@@ -15,6 +15,9 @@ import torch
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libsga.so")
+# The SGA_DEBUG build (device invariant checks compiled in); load_library takes it
+# when the environment sets SGA_LIBRARY=debug.
+LIB_DEBUG_PATH = os.path.join(_PKG, "libsga_debug.so")
 
 INDEX_HEADS = 64
 INDEX_DIM = 128
@@ -30,7 +33,7 @@ HQ_EXTRA = QK_DIM + INDEX_DIM + INDEX_HEADS  # 768
 CQ_ROWS = HEADS * 192 + HEADS + INDEX_HEADS * INDEX_DIM  # 20,544
 V_HEAD = 128
 STATUS_NAMES = {0: "SGA_OK", 1: "SGA_ERR_INVALID_ARG", 2: "SGA_ERR_UNSUPPORTED", 3: "SGA_ERR_WORKSPACE",
-                4: "SGA_ERR_CUDA", 5: "SGA_ERR_TIMEOUT", 6: "SGA_ERR_DEVICE_ARG"}
+                4: "SGA_ERR_CUDA", 5: "SGA_ERR_TIMEOUT", 6: "SGA_ERR_DEVICE_ARG", 7: "SGA_ERR_INTERNAL"}
 
 EXPORTED = ["sga_abi_version", "sga_status_string", "sga_workspace_size", "sga_index_scores", "sga_topk_select",
             "sga_sparse_mla_attend", "sga_forward", "sga_get_device_status", "sga_clear_device_status",
@@ -60,11 +63,14 @@ class LayerWeights(ctypes.Structure):
 _lib = None
 
 
-def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
-    """Loads libsga.so (built in-tree by ``sparse_gated_attention_b200.build``)."""
+def load_library(path: str | None = None) -> ctypes.CDLL:
+    """Loads libsga.so (built in-tree by ``sparse_gated_attention_b200.build``), or
+    libsga_debug.so when the environment sets SGA_LIBRARY=debug."""
     global _lib
     if _lib is not None:
         return _lib
+    if path is None:
+        path = LIB_DEBUG_PATH if os.environ.get("SGA_LIBRARY") == "debug" else LIB_PATH
     if not os.path.exists(path):
         raise RuntimeError(f"libsga.so not found at {path}: build it with `python -m sparse_gated_attention_b200.build`")
     lib = ctypes.CDLL(path)

@@ -201,6 +201,7 @@ const char* sga_status_string(sga_status_t s) {
     case SGA_ERR_CUDA: return "SGA_ERR_CUDA";
     case SGA_ERR_TIMEOUT: return "SGA_ERR_TIMEOUT";
     case SGA_ERR_DEVICE_ARG: return "SGA_ERR_DEVICE_ARG";
+    case SGA_ERR_INTERNAL: return "SGA_ERR_INTERNAL";
   }
   return "SGA_ERR_UNKNOWN";
 }

@@ -254,7 +254,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (sidx < p.top_k) v = __ldg(reinterpret_cast<const int4*>(idx_row + sidx));
         const int e[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-        for (int i = 0; i < 4; ++i) y[i] = row0 + ((e[i] >= 0 && e[i] < p.kv_stride) ? e[i] : 0);
+        for (int i = 0; i < 4; ++i) {
+          y[i] = row0 + ((e[i] >= 0 && e[i] < p.kv_stride) ? e[i] : 0);
+          SGA_DCHECK(p.status, y[i] >= row0 && y[i] < row0 + p.kv_stride);
+        }
       }
       // cp.async: this thread's four rows of the chunk (empty slots zero-filled)
       const uint16_t* src[4];

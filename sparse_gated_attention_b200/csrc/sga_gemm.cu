@@ -55,7 +55,7 @@ struct Item {
   int b, t, nb, s, ks0, ks1;
 };
 
-__device__ __forceinline__ Item decode_item(const GemmParams& p, long long j) {
+__device__ __forceinline__ Item decode_item(const GemmParams& p, long long j, int* status) {
   Item it;
   it.s = static_cast<int>(j % p.splits);
   long long r = j / p.splits;
@@ -65,6 +65,7 @@ __device__ __forceinline__ Item decode_item(const GemmParams& p, long long j) {
   it.b = static_cast<int>(r / p.m_tiles);
   it.ks0 = static_cast<int>(static_cast<long long>(p.k_strips) * it.s / p.splits);
   it.ks1 = static_cast<int>(static_cast<long long>(p.k_strips) * (it.s + 1) / p.splits);
+  SGA_DCHECK(status, it.ks0 < it.ks1 && it.t * kGM < p.m && it.nb * kGemmMaxN < p.n && it.b < p.batch);
   return it;
 }
 
@@ -141,7 +142,7 @@ __global__ void __launch_bounds__(kGThreads, 1)
       int ks = 0;
       bool valid = j < p.items;
       if (valid) {
-        it = decode_item(p, j);
+        it = decode_item(p, j, status);
         ks = it.ks0;
       }
       auto advance = [&]() {
@@ -149,7 +150,7 @@ __global__ void __launch_bounds__(kGThreads, 1)
           j += gridDim.x;
           valid = j < p.items;
           if (valid) {
-            it = decode_item(p, j);
+            it = decode_item(p, j, status);
             ks = it.ks0;
           }
         }
@@ -206,7 +207,7 @@ __global__ void __launch_bounds__(kGThreads, 1)
       long long n_items = 0;
       bool ok = true;
       for (long long j = blockIdx.x; j < p.items && ok; j += gridDim.x) {
-        const Item it = decode_item(p, j);
+        const Item it = decode_item(p, j, status);
         const int acc = static_cast<int>(n_items & 1);
         if (!mbar_wait(accempty(acc), static_cast<uint32_t>((n_items >> 1) & 1) ^ 1u, abort_flag)) {
           ok = false;
@@ -253,7 +254,7 @@ __global__ void __launch_bounds__(kGThreads, 1)
     const int quarter = warp & 3;
     long long n_items = 0;
     for (long long j = blockIdx.x; j < p.items; j += gridDim.x) {
-      const Item it = decode_item(p, j);
+      const Item it = decode_item(p, j, status);
       const int acc = static_cast<int>(n_items & 1);
       if (!mbar_wait(accfull(acc), static_cast<uint32_t>((n_items >> 1) & 1), abort_flag)) {
         record_status(status, kStatusTimeout);

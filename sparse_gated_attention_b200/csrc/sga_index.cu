@@ -450,6 +450,7 @@ struct BlockCursor {
     const int i = blk - seq * p.blocks_per_seq;
     row0 = seq * p.n_q + i * kQB;
     nrows = min(kQB, p.n_q - i * kQB);
+    SGA_DCHECK(p.status, nrows > 0 && row0 + nrows <= (seq + 1) * p.n_q);
     tmax = -1;
     bad = false;
     for (int r = 0; r < nrows; ++r) {

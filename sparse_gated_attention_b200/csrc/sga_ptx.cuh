@@ -14,6 +14,21 @@ namespace sga {
 // Device status codes (values of sga_status_t).
 constexpr int kStatusTimeout = 5;
 constexpr int kStatusDeviceArg = 6;
+constexpr int kStatusInternal = 7;
+
+// Invariant checks of the SGA_DEBUG build: a failed check records
+// SGA_ERR_INTERNAL in the workspace status word (the kernel carries on; nothing
+// traps).  Release builds compile them away.
+#ifdef SGA_DEBUG
+#define SGA_DCHECK(status, cond)                                          \
+  do {                                                                    \
+    if (!(cond)) ::sga::record_status((status), ::sga::kStatusInternal); \
+  } while (0)
+#else
+#define SGA_DCHECK(status, cond) \
+  do {                           \
+  } while (0)
+#endif
 
 // ~1-2 s at the clocks a B200 runs under load.
 constexpr long long kWaitBudgetCycles = 2000000000LL;

@@ -850,6 +850,7 @@ __global__ void __launch_bounds__(kThreads, 1) sga_topk_resident_kernel(TopkPara
   }
   if (rank == 0 && tid == 0 && (sel_all + need != static_cast<uint32_t>(K) || tie_all < need))
     record_status(p.status, kStatusDeviceArg);
+  SGA_DCHECK(p.status, resolved || cand_n <= static_cast<uint32_t>(kCandCap));  // the bin fit the candidate list
   const uint32_t sel_base = sel_before + wsel[warp] + (is - cs);
   const uint32_t tie_base = tie_before + wtie[warp] + (it - ct);
   const int pos0 = s0 + lpos;
@@ -859,6 +860,7 @@ __global__ void __launch_bounds__(kThreads, 1) sga_topk_resident_kernel(TopkPara
     const uint32_t tr = tie_base + __popc(my_tie & below);
     if (((my_tie >> b) & 1u) && tr >= need) continue;
     const uint32_t slot = sel_base + __popc(my_sel & below) + min(tr, need);
+    SGA_DCHECK(p.status, slot < static_cast<uint32_t>(K) && pos0 + b <= t);
     if (slot < static_cast<uint32_t>(K)) out[slot] = pos0 + b;
   }
   if (rank == 0) {

@@ -42,7 +42,19 @@ def test_abi_version_and_status_strings(lib):
     assert lib.sga_abi_version() == 1
     assert lib.sga_status_string(0) == b"SGA_OK"
     assert lib.sga_status_string(5) == b"SGA_ERR_TIMEOUT"
+    assert lib.sga_status_string(7) == b"SGA_ERR_INTERNAL"
     assert lib.sga_status_string(99) == b"SGA_ERR_UNKNOWN"
+
+
+def test_debug_library_builds_and_exports_the_same_calls():
+    """libsga_debug.so: the same sources with the SGA_DEBUG invariant checks."""
+    path = sga_build.build(debug=True)
+    dbg = ctypes.CDLL(path)
+    for n in sga.EXPORTED:
+        assert hasattr(dbg, n), n
+    dbg.sga_status_string.restype = ctypes.c_char_p
+    dbg.sga_status_string.argtypes = [ctypes.c_int]
+    assert dbg.sga_status_string(7) == b"SGA_ERR_INTERNAL"
 
 
 def test_workspace_sizes(lib):
