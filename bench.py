@@ -50,6 +50,8 @@ def parse_args():
                     help="skip the chunked-prefill variant (4096 queries over a 128K cache)")
     ap.add_argument("--no-decode-variants", dest="decode_variants", action="store_false",
                     help="skip the other decode workloads (8K x 4, 32K x 64, 256K x 8 with ties)")
+    ap.add_argument("--no-warmup-objective", dest="warmup_objective", action="store_false",
+                    help="skip the indexer's sparse warm-up objective (a training-time variant)")
     ap.add_argument("--no-layer", dest="layer", action="store_false",
                     help="skip the whole-layer variant (the projections either side of the path)")
     ap.add_argument("--layer-only", action="store_true",
@@ -421,6 +423,50 @@ def layer_variant(sga, synth, args, dev, stream, dist, rank, x, dims, idx) -> di
     return {"ms": layer_ms, "weight_bytes": weight_bytes, "act_bytes": h.numel() * 2 + y.numel() * 4}
 
 
+def warmup_objective_variant(sga, args, dev, stream, dist, rank, x, dims, idx, peak) -> dict:
+    """The indexer's sparse warm-up objective and its gradients (a training-time
+    variant; sga_indexer_warmup) over the headline step's own selection, timed
+    over K steps like the main region.  The key gradient is added to one
+    [B][L][128] fp32 buffer every step, as an optimiser step would read it."""
+    B, T = x["q_pos"].shape
+    L, K = dims.kv_stride, dims.top_k
+    ws = torch.zeros(sga.indexer_warmup_workspace_size(dims), dtype=torch.uint8, device=dev)
+    gk = torch.zeros((B, L, 128), dtype=torch.float32, device=dev)
+
+    def step():
+        sga.indexer_warmup(x["q_idx"], x["w"], x["k_idx"], x["q"], x["kv"], idx, grad_k_idx=gk, ws=ws, stream=stream)
+
+    for _ in range(max(args.warmup, 3)):
+        step()
+    torch.cuda.synchronize(dev)
+    if dist is not None:
+        dist.barrier()
+    s0, e0 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e0.record(stream)
+    torch.cuda.synchronize(dev)
+    ms = max_over_ranks(dist, dev, s0.elapsed_time(e0))
+    if sga.device_status(ws) != 0:
+        raise RuntimeError("device status set during the warm-up objective variant")
+    rows = B * T
+    world = dist.get_world_size() if dist is not None else 1
+    # per query: the selected latent and key rows, q, q_idx, w, idx, the q_idx / w
+    # gradients and loss written, the key gradient rows read and written (the
+    # workspace's per-slot logits and dots are intermediates, not counted)
+    per_query = K * 1152 + K * 256 + 73728 + 16384 + 128 + K * 4 + 32768 + 256 + 4 + K * 128 * 4 * 2
+    step_ms = ms / args.steps
+    gbs = per_query * rows / (step_ms * 1e-3) / 1e9
+    return {"value": whole_job_rate(rows, args.steps, world, ms), "unit": UNIT, "ms_per_step": step_ms,
+            "config": f"{rows} queries of the headline workload: KL(attention target || indexer softmax) over each "
+                      f"query's 2048 selected positions and the gradients of q_idx, w and k_idx (three SIMT fp32 "
+                      f"kernels)",
+            "path_roofline": {"achieved_gbs": gbs, "frac_of_8tbs": gbs / NOMINAL_HBM_GBS, "frac_of_measured": gbs / peak,
+                              "bytes_per_query": per_query},
+            "gpu_launches": 3 * args.steps}
+
+
 def main():
     args = parse_args()
     from sparse_gated_attention_b200 import synth
@@ -622,6 +668,17 @@ def main():
     # rewritten at their positions every step), timed like the main region.
     layer = layer_variant(sga, synth, args, dev, stream, dist, rank, x, dims, idx) if args.layer else None
 
+    # ---- the indexer's sparse warm-up objective (a training-time variant) over this step's selection
+    warm = None
+    if args.warmup_objective:
+        try:
+            fwd_step()  # idx of the current inputs
+            warm = warmup_objective_variant(sga, args, dev, stream, dist, rank, x, dims, idx, measured_peaks()[0])
+        except (RuntimeError, TypeError, ValueError) as exc:
+            torch.cuda.synchronize(dev)
+            warm = {"error": f"{type(exc).__name__}: {exc}"}
+        torch.cuda.empty_cache()
+
     # ---- the other decode workloads (separate configurations, one line each in `variants`)
     decode_lines = {}
     if args.decode_variants and args.workload is None and not (args.batch and args.ctx):
@@ -675,6 +732,8 @@ def main():
                           "frac_of_measured": fp8_gbs / peak, "bytes_per_query": ab8["total"]},
         "gpu_launches": launches_per_step * args.steps}}
     variants.update(decode_lines)
+    if warm is not None:
+        variants["indexer_warmup"] = warm
     if prefill is not None:
         variants[prefill.pop("name", "prefill_t4096_ctx128k")] = prefill
     if layer is not None:
