@@ -323,6 +323,22 @@ def test_forward_matches_oracle(B, T, L, pos):
     assert_close(out.cpu().numpy(), want_out, "forward")
 
 
+@pytest.mark.parametrize("k_range,L", [(0, 9000), (1, 20000)])
+def test_forward_wide_threshold_bin(k_range, L):
+    """Index keys all zero (every score equal) or in {-1, 0, 1} (heavy ties): the
+    bin of the K-th score holds more keys than the candidate list, so the
+    selection narrows it with passes over its positions and takes the lowest
+    positions among the ties."""
+    B = 2
+    x = gen_small(B, 1, L, [[L - 1], [L // 2]], k_range=k_range, seed=7)
+    ws = sga.alloc_workspace(sga.make_dims(B, 1, L), sga.OP_FORWARD)
+    idx, out = sga.forward(x["q_idx"], x["w"], x["k_idx"], x["q"], x["kv"], x["gate"], x["q_pos"], ws=ws)
+    check_status(ws)
+    want_idx, want_out = oracle.forward(x["q_idx"], x["w"], x["k_idx"], x["q"], x["kv"], x["gate"], x["q_pos"].cpu())
+    np.testing.assert_array_equal(idx.cpu().numpy(), want_idx)
+    assert_close(out.cpu().numpy(), want_out, f"forward, k_range {k_range}")
+
+
 def test_forward_reuses_its_workspace():
     """The selection clears the indexer's histograms after reading them, on
     every exit (full selection, t + 1 <= K, bad position), so one zero-filled
