@@ -339,6 +339,29 @@ def test_forward_wide_threshold_bin(k_range, L):
     assert_close(out.cpu().numpy(), want_out, f"forward, k_range {k_range}")
 
 
+@pytest.mark.parametrize("order,L", [("rising", 20000), ("falling", 20000), ("rising", 70000)])
+def test_forward_monotone_scores(order, L):
+    """Scores that rise (or fall) with the position, in runs of equal values:
+    the top K are the last (or first) positions, the K-th key's run is split,
+    and its lowest positions are taken; the second call checks that the first
+    left the workspace's histograms cleared."""
+    B = 2
+    run = L // 250 + 1
+    x = gen_small(B, 1, L, [[L - 1], [L // 2]], seed=11)
+    c = torch.arange(L, device="cuda") // run
+    if order == "falling":
+        c = c.max() - c
+    x["k_idx"] = c.to(torch.bfloat16).view(1, L, 1).expand(B, L, 128).contiguous()
+    x["q_idx"] = torch.ones_like(x["q_idx"])
+    ws = sga.alloc_workspace(sga.make_dims(B, 1, L), sga.OP_FORWARD)
+    for _ in range(2):
+        idx, out = sga.forward(x["q_idx"], x["w"], x["k_idx"], x["q"], x["kv"], x["gate"], x["q_pos"], ws=ws)
+        check_status(ws)
+    want_idx, want_out = oracle.forward(x["q_idx"], x["w"], x["k_idx"], x["q"], x["kv"], x["gate"], x["q_pos"].cpu())
+    np.testing.assert_array_equal(idx.cpu().numpy(), want_idx)
+    assert_close(out.cpu().numpy(), want_out, f"forward, {order} scores")
+
+
 def test_forward_reuses_its_workspace():
     """The selection clears the indexer's histograms after reading them, on
     every exit (full selection, t + 1 <= K, bad position), so one zero-filled
