@@ -13,14 +13,17 @@
 //   dq_idx_j = sum_s g_s w_j [a_js > 0] k_idx_s
 //   dk_idx_s += sum_j g_s w_j [a_js > 0] q_idx_j        (summed over the queries that select s)
 //
-// Three kernels, all plain fp32 SIMT arithmetic on bf16 inputs:
-//   A  per (query, 64-slot chunk): gathers the chunk's latent and key rows,
-//      writes the 64 head logits z, the 64 indexer dots a and the score of
-//      every slot to the workspace (empty slots: z = -inf);
-//   B  per query: per-head softmax statistics, the target p, the indexer
-//      softmax r, the loss and g = r - p; zeroes the query's q_idx and w
-//      gradients;
-//   C  per (query, chunk): accumulates the gradients with atomic adds.
+// Kernels, in launch order:
+//   B  per query: clears the query's q_idx and w gradients;
+//   A  per (query, 64-slot chunk), on the tensor core: gathers the chunk's
+//      latent and key rows, writes the 64 head logits z, the 64 indexer dots
+//      a, the score of every slot (empty slots: z = -inf) and each head's
+//      (max, sum of exponentials) over the chunk to the workspace;
+//   C  per (query, chunk): the target's per-head statistics merged from the
+//      chunks', the indexer softmax's from all the query's scores; p, r,
+//      g = r - p and the loss terms of the chunk's slots; then the gradients,
+//      added with atomics;
+//   B  per query: the loss, the chunks' terms summed in chunk order.
 // Staged rows are padded by 16 bytes so that the rows a warp reads at once
 // start on different shared-memory banks.
 #include <cuda_bf16.h>
@@ -32,6 +35,7 @@
 
 #include "../../include/sga.h"
 #include "sga_host.h"
+#include "sga_ptx.cuh"
 
 namespace {
 
@@ -41,7 +45,6 @@ constexpr int kIdxHeads = SGA_INDEX_HEADS;  // 64
 constexpr int kIdxDim = SGA_INDEX_DIM;      // 128
 constexpr int kChunk = 64;                  // selected slots per CTA
 constexpr int kThreads = 256;
-constexpr int kRowPad = kDq + 8;            // staged q / kv row: 584 bf16 (1168 B)
 constexpr int kIdxPad = kIdxDim + 8;        // staged q_idx / k_idx row: 136 bf16 (272 B)
 constexpr float kScale = static_cast<float>(SGA_SOFTMAX_SCALE);
 using sga::host::align_up;
@@ -50,8 +53,11 @@ using sga::host::at;
 using sga::host::kStatusBytes;
 constexpr size_t kAlign = sga::host::kWsAlign;
 
-// kernel A: q, kv rows, q_idx, k rows (bf16, padded), a (fp32)
-constexpr size_t kLogitsSmem = (2 * kHeads * kRowPad + 2 * kChunk * kIdxPad) * 2 + kIdxHeads * kChunk * 4;
+// kernel A (tensor core): 22 swizzled boxes of 64 rows x 64 bf16, and the 1 KB alignment
+constexpr int kLogitThreads = 128;
+constexpr int kBox = 64 * 128;
+constexpr uint32_t kLogitTmemCols = 128;  // z at column 0, a at column 64
+constexpr size_t kLogitsSmem = 1024 + 22 * kBox;
 // kernel C: q_idx, k rows (bf16, padded), act and ReLU(a) (fp32)
 constexpr size_t kGradSmem = 2 * kChunk * kIdxPad * 2 + 2 * kIdxHeads * kChunk * 4;
 static_assert(kLogitsSmem <= 232448 && kGradSmem <= 232448, "shared memory");
@@ -70,7 +76,8 @@ struct WarmupArgs {
   float* z;               // workspace [rows][64][K]
   float* a;               // workspace [rows][64][K]
   float* score;           // workspace [rows][K]
-  float* g;               // workspace [rows][K]
+  float* loss_part;       // workspace [rows][K / 64]: each chunk's share of the loss
+  float2* stats;          // workspace [rows][64][K / 64]: each chunk's (max z, sum exp(z - max)) per head
   int* status;
   int n_q, kv_stride, top_k;
 };
@@ -133,95 +140,213 @@ __device__ void gather_rows(uint16_t* dst, int pad, const uint16_t* cache, int w
   }
 }
 
-// A: logits, indexer dots and scores of one chunk of selected slots.
-__global__ void __launch_bounds__(kThreads) warmup_logits_kernel(WarmupArgs p) {
-  extern __shared__ __align__(16) uint8_t smem[];
-  uint16_t* qs = reinterpret_cast<uint16_t*>(smem);  // [64][kRowPad]
-  uint16_t* kvs = qs + kHeads * kRowPad;               // [64][kRowPad]
-  uint16_t* qis = kvs + kChunk * kRowPad;              // [64][kIdxPad]
-  uint16_t* ks = qis + kIdxHeads * kIdxPad;            // [64][kIdxPad]
-  float* as = reinterpret_cast<float*>(ks + kChunk * kIdxPad);  // [64 j][64 s]
+// A: logits, indexer dots, scores and the chunk's softmax statistics of one
+// chunk of 64 selected slots, on the tensor core.  All 128 threads gather the
+// query's 64 x 576 latent query, the chunk's 64 latent rows, the 64 x 128
+// indexer query and the chunk's 64 key rows into 128-byte-swizzled boxes of 64
+// rows x 64 dims (16-byte cp.async; empty slots are zero-filled); one thread
+// issues z = Q C^T (M = 64 heads, N = 64 slots, K = 576) and a = Q_idx K^T
+// (M = 64 indexer heads, K = 128) into tensor memory; each warp then reads 16
+// rows of both with the 16-lane x 256-bit shape (thread t: rows t/4 and 8 + t/4
+// of its quarter, columns 8k + 2(t%4) and +1).
+__global__ void __launch_bounds__(kLogitThreads, 1) warmup_logits_kernel(WarmupArgs p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t q_s = sga::smem_u32(smem);    // 9 boxes: the query's 64 heads x 576
+  const uint32_t kv_s = q_s + 9 * kBox;         // 9 boxes: the chunk's 64 latent rows
+  const uint32_t qi_s = kv_s + 9 * kBox;        // 2 boxes: 64 indexer heads x 128
+  const uint32_t ki_s = qi_s + 2 * kBox;        // 2 boxes: the chunk's 64 key rows
   __shared__ int slot_row[kChunk];
+  __shared__ float sc_part[4][kChunk];
+  __shared__ __align__(8) uint64_t mma_bar;
+  __shared__ uint32_t tmem_slot;
+  __shared__ int abort_flag;
   const int c = blockIdx.x, row = blockIdx.y, b = row / p.n_q, t = threadIdx.x;
+  const int warp = t >> 5, lane = t & 31;
   const size_t seq_base = static_cast<size_t>(b) * p.kv_stride;
+  const int nch = p.top_k / kChunk;
+  if (t == 0) {
+    sga::mbar_init(sga::smem_u32(&mma_bar), 1);
+    abort_flag = 0;
+    sga::fence_barrier_init();
+  }
+  if (warp == 0) {
+    sga::tmem_alloc(sga::smem_u32(&tmem_slot), kLogitTmemCols);
+    sga::tmem_relinquish();
+  }
   load_slot_rows(p, row, c, slot_row);
-  stage_rows(qs, kRowPad, p.q + static_cast<size_t>(row) * kHeads * kDq, kDq, kHeads);
-  stage_rows(qis, kIdxPad, p.q_idx + static_cast<size_t>(row) * kIdxHeads * kIdxDim, kIdxDim, kIdxHeads);
+  sga::tc_fence_before();
   __syncthreads();
-  gather_rows(kvs, kRowPad, p.kv, kDq, seq_base, slot_row);
-  gather_rows(ks, kIdxPad, p.k_idx, kIdxDim, seq_base, slot_row);
-  __syncthreads();
-  const int h = t >> 2, s0 = t & 3;  // head (or indexer head) and first slot of this thread
+  sga::tc_fence_after();
+  const uint32_t tmem = tmem_slot;
   {
-    float acc[16];
+    // 16-byte pieces: a 576-wide row is 72 (box piece >> 3, part piece & 7); a 128-wide row 16
+    const uint16_t* qrow = p.q + static_cast<size_t>(row) * kHeads * kDq;
+    for (int e = t; e < kHeads * 72; e += kLogitThreads) {
+      const int r = e / 72, pc = e - r * 72;
+      sga::cp_async_16(q_s + (pc >> 3) * kBox + r * 128 + (((pc & 7) ^ (r & 7)) << 4), qrow + r * kDq + pc * 8, 16);
+    }
+    for (int e = t; e < kChunk * 72; e += kLogitThreads) {
+      const int r = e / 72, pc = e - r * 72, sr = slot_row[r];
+      const uint16_t* src = p.kv + (seq_base + (sr >= 0 ? sr : 0)) * kDq + pc * 8;
+      sga::cp_async_16(kv_s + (pc >> 3) * kBox + r * 128 + (((pc & 7) ^ (r & 7)) << 4), src, sr >= 0 ? 16u : 0u);
+    }
+    const uint16_t* qirow = p.q_idx + static_cast<size_t>(row) * kIdxHeads * kIdxDim;
+    for (int e = t; e < kIdxHeads * 16; e += kLogitThreads) {
+      const int r = e >> 4, pc = e & 15;
+      sga::cp_async_16(qi_s + (pc >> 3) * kBox + r * 128 + (((pc & 7) ^ (r & 7)) << 4), qirow + r * kIdxDim + pc * 8,
+                       16);
+    }
+    for (int e = t; e < kChunk * 16; e += kLogitThreads) {
+      const int r = e >> 4, pc = e & 15, sr = slot_row[r];
+      const uint16_t* src = p.k_idx + (seq_base + (sr >= 0 ? sr : 0)) * kIdxDim + pc * 8;
+      sga::cp_async_16(ki_s + (pc >> 3) * kBox + r * 128 + (((pc & 7) ^ (r & 7)) << 4), src, sr >= 0 ? 16u : 0u);
+    }
+    asm volatile("cp.async.wait_all;" ::: "memory");
+    sga::fence_proxy_async_smem();  // written by cp.async, read by the tensor core
+  }
+  __syncthreads();
+  if (t == 0) {
+    constexpr uint32_t idesc = sga::idesc_bf16_f32(kHeads, kChunk, false, false);
+    sga::tc_fence_after();
+    for (int bx = 0; bx < 9; ++bx)
 #pragma unroll
-    for (int i = 0; i < 16; ++i) acc[i] = 0.f;
-    const __nv_bfloat162* qh = reinterpret_cast<const __nv_bfloat162*>(qs + h * kRowPad);
-    for (int d2 = 0; d2 < kDq / 2; ++d2) {
-      const float2 qv = __bfloat1622float2(qh[d2]);
+      for (int kk = 0; kk < 4; ++kk)
+        sga::mma_bf16(tmem, sga::sdesc_sw128(q_s + bx * kBox + kk * 32, 16, 1024),
+                      sga::sdesc_sw128(kv_s + bx * kBox + kk * 32, 16, 1024), idesc, (bx | kk) ? 1u : 0u);
+    for (int bx = 0; bx < 2; ++bx)
 #pragma unroll
-      for (int i = 0; i < 16; ++i) {
-        const float2 kv2 =
-            __bfloat1622float2(reinterpret_cast<const __nv_bfloat162*>(kvs + (s0 + 4 * i) * kRowPad)[d2]);
-        acc[i] = fmaf(qv.x, kv2.x, acc[i]);
-        acc[i] = fmaf(qv.y, kv2.y, acc[i]);
+      for (int kk = 0; kk < 4; ++kk)
+        sga::mma_bf16(tmem + kChunk, sga::sdesc_sw128(qi_s + bx * kBox + kk * 32, 16, 1024),
+                      sga::sdesc_sw128(ki_s + bx * kBox + kk * 32, 16, 1024), idesc, (bx | kk) ? 1u : 0u);
+    sga::mma_commit(sga::smem_u32(&mma_bar));
+  }
+  bool ok = sga::mbar_wait(sga::smem_u32(&mma_bar), 0, &abort_flag);
+  if (!ok) {
+    atomicCAS(p.status, 0, static_cast<int>(SGA_ERR_TIMEOUT));
+    abort_flag = 1;
+  }
+  ok = __syncthreads_and(ok) != 0;  // the epilogue's shuffles need whole warps
+  sga::tc_fence_after();
+  if (ok) {
+    const uint32_t lane_addr = static_cast<uint32_t>(warp * 32) << 16;
+    float r[32], ra[32];
+    sga::tmem_ld_16x256b_x8(tmem + lane_addr, r);
+    sga::tmem_ld_16x256b_x8(tmem + lane_addr + kChunk, ra);
+    const int m4 = lane & 3;
+    const int hr[2] = {warp * 16 + (lane >> 2), warp * 16 + 8 + (lane >> 2)};  // this thread's two rows
+    const float wj[2] = {bf(p.w[static_cast<size_t>(row) * kIdxHeads + hr[0]]),
+                         bf(p.w[static_cast<size_t>(row) * kIdxHeads + hr[1]])};
+    float sc[16];  // this thread's score partials, columns 8k + 2 m4 + e
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+      float zz[16];
+      float m = -INFINITY;
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const int col = 8 * k + 2 * m4 + e;
+          zz[2 * k + e] = slot_row[col] >= 0 ? r[4 * k + 2 * i + e] * kScale : -INFINITY;
+          m = fmaxf(m, zz[2 * k + e]);
+        }
+      }
+      m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
+      m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 2));
+      float l = 0.f;
+      if (m != -INFINITY) {
+#pragma unroll
+        for (int k = 0; k < 16; ++k) l += expf(zz[k] - m);
+      }
+      l += __shfl_xor_sync(0xffffffffu, l, 1);
+      l += __shfl_xor_sync(0xffffffffu, l, 2);
+      const size_t zrow = (static_cast<size_t>(row) * kHeads + hr[i]) * p.top_k + static_cast<size_t>(c) * kChunk;
+      const size_t arow = (static_cast<size_t>(row) * kIdxHeads + hr[i]) * p.top_k + static_cast<size_t>(c) * kChunk;
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        const int col = 8 * k + 2 * m4;
+        *reinterpret_cast<float2*>(p.z + zrow + col) = make_float2(zz[2 * k], zz[2 * k + 1]);
+        *reinterpret_cast<float2*>(p.a + arow + col) = make_float2(ra[4 * k + 2 * i], ra[4 * k + 2 * i + 1]);
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const float v = wj[i] * fmaxf(ra[4 * k + 2 * i + e], 0.f);
+          sc[2 * k + e] = i == 0 ? v : sc[2 * k + e] + v;
+        }
+      }
+      if (m4 == 0)
+        p.stats[(static_cast<size_t>(row) * kHeads + hr[i]) * nch + c] = make_float2(m, l);
+    }
+    // the warp's 16 rows summed (lanes that share m4 hold the same columns)
+#pragma unroll
+    for (int k = 0; k < 16; ++k) {
+      sc[k] += __shfl_xor_sync(0xffffffffu, sc[k], 4);
+      sc[k] += __shfl_xor_sync(0xffffffffu, sc[k], 8);
+      sc[k] += __shfl_xor_sync(0xffffffffu, sc[k], 16);
+    }
+    if (lane < 4) {
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        sc_part[warp][8 * k + 2 * m4] = sc[2 * k];
+        sc_part[warp][8 * k + 2 * m4 + 1] = sc[2 * k + 1];
       }
     }
-    float* zr = p.z + (static_cast<size_t>(row) * kHeads + h) * p.top_k + static_cast<size_t>(c) * kChunk;
-#pragma unroll
-    for (int i = 0; i < 16; ++i) zr[s0 + 4 * i] = slot_row[s0 + 4 * i] >= 0 ? acc[i] * kScale : -INFINITY;
+  } else if (t == 0) {
+    volatile int never = 0;
+    sga::mbar_wait(sga::smem_u32(&mma_bar), 0, &never);  // its MMAs must finish before tensor memory is freed
   }
-  {
-    float acc[16];
-#pragma unroll
-    for (int i = 0; i < 16; ++i) acc[i] = 0.f;
-    const __nv_bfloat162* qj = reinterpret_cast<const __nv_bfloat162*>(qis + h * kIdxPad);
-    for (int d2 = 0; d2 < kIdxDim / 2; ++d2) {
-      const float2 qv = __bfloat1622float2(qj[d2]);
-#pragma unroll
-      for (int i = 0; i < 16; ++i) {
-        const float2 k2 = __bfloat1622float2(reinterpret_cast<const __nv_bfloat162*>(ks + (s0 + 4 * i) * kIdxPad)[d2]);
-        acc[i] = fmaf(qv.x, k2.x, acc[i]);
-        acc[i] = fmaf(qv.y, k2.y, acc[i]);
-      }
-    }
-#pragma unroll
-    for (int i = 0; i < 16; ++i) as[h * kChunk + s0 + 4 * i] = acc[i];
-  }
+  sga::tc_fence_before();
   __syncthreads();
-  for (int e = t; e < kIdxHeads * kChunk; e += kThreads) {
-    const int j = e / kChunk, s = e - j * kChunk;
-    p.a[(static_cast<size_t>(row) * kIdxHeads + j) * p.top_k + static_cast<size_t>(c) * kChunk + s] = as[e];
-  }
-  if (t < kChunk) {
-    float sc = 0.f;
-    for (int j = 0; j < kIdxHeads; ++j)
-      sc = fmaf(bf(p.w[static_cast<size_t>(row) * kIdxHeads + j]), fmaxf(as[j * kChunk + t], 0.f), sc);
-    p.score[static_cast<size_t>(row) * p.top_k + static_cast<size_t>(c) * kChunk + t] = sc;
+  if (ok && t < kChunk)
+    p.score[static_cast<size_t>(row) * p.top_k + static_cast<size_t>(c) * kChunk + t] =
+        (sc_part[0][t] + sc_part[1][t]) + (sc_part[2][t] + sc_part[3][t]);
+  if (warp == 0) {
+    sga::tc_fence_after();
+    sga::tmem_dealloc(tmem, kLogitTmemCols);
   }
 }
 
-// B: per query, the target p, the indexer softmax r, the loss and g = r - p.
-__global__ void __launch_bounds__(kThreads) warmup_objective_kernel(WarmupArgs p) {
-  __shared__ float hm[kHeads], hl[kHeads], red[kThreads / 32];
-  const int row = blockIdx.x, t = threadIdx.x, lane = t & 31, warp = t >> 5;
-  const int K = p.top_k;
-  const float* zr = p.z + static_cast<size_t>(row) * kHeads * K;
-  const float* sr = p.score + static_cast<size_t>(row) * K;
+// C: per (query, chunk), the objective for the chunk's slots, then their
+// gradients.  The target's per-head statistics come merged from every
+// chunk's (max, sum) pair, the indexer softmax's from all of the query's
+// scores; then for each slot p(s), r(s), g_s = r(s) - p(s) and its loss term
+// (the chunk's share goes to the workspace, summed in chunk order by kernel
+// B), and the gradients are added into the query's q_idx and w gradients and
+// the key gradients of the selected cache rows.
+__global__ void __launch_bounds__(kThreads) warmup_grad_kernel(WarmupArgs p) {
+  extern __shared__ __align__(16) uint8_t smem[];
+  uint16_t* qis = reinterpret_cast<uint16_t*>(smem);             // [64][kIdxPad]
+  uint16_t* ks = qis + kIdxHeads * kIdxPad;                        // [64][kIdxPad]
+  float* act = reinterpret_cast<float*>(ks + kChunk * kIdxPad);   // [64 j][64 s]: g_s w_j [a_js > 0]
+  float* relu = act + kIdxHeads * kChunk;                          // [64 j][64 s]: ReLU(a_js)
+  __shared__ int slot_row[kChunk];
+  __shared__ float gs[kChunk], wj[kIdxHeads], hm[kHeads], hinv[kHeads], red[kThreads / 32];
+  __shared__ float pp_part[kThreads / kChunk][kChunk];
+  const int c = blockIdx.x, row = blockIdx.y, b = row / p.n_q, t = threadIdx.x;
+  const int lane = t & 31, warp = t >> 5;
+  const int K = p.top_k, nch = K / kChunk;
+  const size_t seq_base = static_cast<size_t>(b) * p.kv_stride;
+  load_slot_rows(p, row, c, slot_row);
+  if (t < kIdxHeads) wj[t] = bf(p.w[static_cast<size_t>(row) * kIdxHeads + t]);
+  stage_rows(qis, kIdxPad, p.q_idx + static_cast<size_t>(row) * kIdxHeads * kIdxDim, kIdxDim, kIdxHeads);
+  // ---- the target's per-head statistics: the chunks' (max, sum) pairs merged
   for (int h = warp; h < kHeads; h += kThreads / 32) {
+    const float2* st = p.stats + (static_cast<size_t>(row) * kHeads + h) * nch;
     float m = -INFINITY;
-    for (int s = lane; s < K; s += 32) m = fmaxf(m, zr[static_cast<size_t>(h) * K + s]);
+    for (int cc = lane; cc < nch; cc += 32) m = fmaxf(m, st[cc].x);
     m = warp_max(m);
     float l = 0.f;
     if (m != -INFINITY)
-      for (int s = lane; s < K; s += 32) l += expf(zr[static_cast<size_t>(h) * K + s] - m);
+      for (int cc = lane; cc < nch; cc += 32)
+        if (st[cc].x != -INFINITY) l += st[cc].y * expf(st[cc].x - m);
     l = warp_sum(l);
     if (lane == 0) {
       hm[h] = m;
-      hl[h] = l;
+      hinv[h] = l > 0.f ? 1.f / l : 0.f;
     }
   }
-  // the indexer softmax over the valid slots (an empty slot has z = -inf in every head)
+  // ---- the indexer softmax over the query's valid slots (an empty slot has z = -inf in every head)
+  const float* zr = p.z + static_cast<size_t>(row) * kHeads * K;
+  const float* sr = p.score + static_cast<size_t>(row) * K;
   float smax = -INFINITY;
   for (int s = t; s < K; s += kThreads)
     if (zr[s] != -INFINITY) smax = fmaxf(smax, sr[s]);
@@ -230,45 +355,38 @@ __global__ void __launch_bounds__(kThreads) warmup_objective_kernel(WarmupArgs p
   if (smax != -INFINITY)
     for (int s = t; s < K; s += kThreads)
       if (zr[s] != -INFINITY) ssum += expf(sr[s] - smax);
-  ssum = block_reduce<false>(ssum, red);
-  const float log_ssum = logf(ssum);
-  float part = 0.f;
-  for (int s = t; s < K; s += kThreads) {
-    float gs = 0.f;
-    if (zr[s] != -INFINITY) {
-      float pp = 0.f;
-      for (int h = 0; h < kHeads; ++h) pp += expf(zr[static_cast<size_t>(h) * K + s] - hm[h]) / hl[h];
-      pp *= 1.f / kHeads;
-      const float log_r = sr[s] - smax - log_ssum;
-      if (pp > 0.f) part += pp * (logf(pp) - log_r);
-      gs = expf(log_r) - pp;
+  ssum = block_reduce<false>(ssum, red);  // (its barriers also publish hm, hinv, wj and slot_row)
+  // ---- p(s) for the chunk's slots: thread (slot s, head group hg) sums 16 heads
+  {
+    const int s = t & (kChunk - 1), hg = t / kChunk;
+    constexpr int kHeadsPerGroup = kHeads / (kThreads / kChunk);
+    const float* zc = zr + static_cast<size_t>(c) * kChunk + s;
+    float pp = 0.f;
+    if (slot_row[s] >= 0) {
+#pragma unroll 4
+      for (int h = hg * kHeadsPerGroup; h < (hg + 1) * kHeadsPerGroup; ++h)
+        pp += expf(zc[static_cast<size_t>(h) * K] - hm[h]) * hinv[h];
     }
-    p.g[static_cast<size_t>(row) * K + s] = gs;
+    pp_part[hg][s] = pp;
   }
-  part = block_reduce<false>(part, red);
-  if (t == 0) p.loss[row] = part;
-  for (int e = t; e < kIdxHeads * kIdxDim; e += kThreads)
-    p.grad_q_idx[static_cast<size_t>(row) * kIdxHeads * kIdxDim + e] = 0.f;
-  if (t < kIdxHeads) p.grad_w[static_cast<size_t>(row) * kIdxHeads + t] = 0.f;
-}
-
-// C: the gradients of one chunk, added into the query's q_idx and w gradients
-// and into the key gradients of the selected cache rows.
-__global__ void __launch_bounds__(kThreads) warmup_grad_kernel(WarmupArgs p) {
-  extern __shared__ __align__(16) uint8_t smem[];
-  uint16_t* qis = reinterpret_cast<uint16_t*>(smem);             // [64][kIdxPad]
-  uint16_t* ks = qis + kIdxHeads * kIdxPad;                        // [64][kIdxPad]
-  float* act = reinterpret_cast<float*>(ks + kChunk * kIdxPad);   // [64 j][64 s]: g_s w_j [a_js > 0]
-  float* relu = act + kIdxHeads * kChunk;                          // [64 j][64 s]: ReLU(a_js)
-  __shared__ int slot_row[kChunk];
-  __shared__ float gs[kChunk], wj[kIdxHeads];
-  const int c = blockIdx.x, row = blockIdx.y, b = row / p.n_q, t = threadIdx.x;
-  const size_t seq_base = static_cast<size_t>(b) * p.kv_stride;
-  load_slot_rows(p, row, c, slot_row);
-  if (t < kChunk) gs[t] = p.g[static_cast<size_t>(row) * p.top_k + static_cast<size_t>(c) * kChunk + t];
-  if (t < kIdxHeads) wj[t] = bf(p.w[static_cast<size_t>(row) * kIdxHeads + t]);
-  stage_rows(qis, kIdxPad, p.q_idx + static_cast<size_t>(row) * kIdxHeads * kIdxDim, kIdxDim, kIdxHeads);
   __syncthreads();
+  float term = 0.f;
+  if (t < kChunk) {
+    float g = 0.f;
+    if (slot_row[t] >= 0) {
+      float pp = 0.f;
+#pragma unroll
+      for (int hg = 0; hg < kThreads / kChunk; ++hg) pp += pp_part[hg][t];
+      pp *= 1.f / kHeads;
+      const float log_r = sr[static_cast<size_t>(c) * kChunk + t] - smax - logf(ssum);
+      if (pp > 0.f) term = pp * (logf(pp) - log_r);
+      g = expf(log_r) - pp;
+    }
+    gs[t] = g;
+  }
+  term = block_reduce<false>(term, red);  // (its barriers also publish gs)
+  if (t == 0) p.loss_part[static_cast<size_t>(row) * nch + c] = term;
+  // ---- the gradients of the chunk
   gather_rows(ks, kIdxPad, p.k_idx, kIdxDim, seq_base, slot_row);
   for (int e = t; e < kIdxHeads * kChunk; e += kThreads) {
     const int j = e / kChunk, s = e - j * kChunk;
@@ -329,8 +447,25 @@ __global__ void __launch_bounds__(kThreads) warmup_grad_kernel(WarmupArgs p) {
 }
 
 
+// B: per query, the loss (the chunks' terms summed in chunk order); also clears
+// the query's q_idx and w gradients, which the next call's kernel C adds into.
+__global__ void __launch_bounds__(kThreads) warmup_loss_kernel(WarmupArgs p, bool clear_grads) {
+  const int row = blockIdx.x, t = threadIdx.x;
+  const int nch = p.top_k / kChunk;
+  if (t == 0 && !clear_grads) {
+    float sum = 0.f;
+    for (int cc = 0; cc < nch; ++cc) sum += p.loss_part[static_cast<size_t>(row) * nch + cc];
+    p.loss[row] = sum;
+  }
+  if (clear_grads) {
+    for (int e = t; e < kIdxHeads * kIdxDim; e += kThreads)
+      p.grad_q_idx[static_cast<size_t>(row) * kIdxHeads * kIdxDim + e] = 0.f;
+    if (t < kIdxHeads) p.grad_w[static_cast<size_t>(row) * kIdxHeads + t] = 0.f;
+  }
+}
+
 struct WarmupLayout {
-  size_t z = 0, a = 0, score = 0, g = 0, total = 0;
+  size_t z = 0, a = 0, score = 0, stats = 0, loss_part = 0, total = 0;
 };
 
 bool warmup_dims_ok(const sga_dims_t* d) {
@@ -350,8 +485,10 @@ WarmupLayout warmup_layout(const sga_dims_t& d) {
   off += align_up(rows * kIdxHeads * K * 4);
   l.score = off;
   off += align_up(rows * K * 4);
-  l.g = off;
-  off += align_up(rows * K * 4);
+  l.stats = off;
+  off += align_up(rows * kHeads * (K / kChunk) * 8);
+  l.loss_part = off;
+  off += align_up(rows * (K / kChunk) * 4);
   l.total = off;
   return l;
 }
@@ -399,16 +536,19 @@ sga_status_t sga_indexer_warmup(const sga_dims_t* dims, const sga_bf16_t* q_idx,
     }
   }
   WarmupArgs a{q_idx, w, k_idx, q, kv, idx, loss, grad_q_idx, grad_w, grad_k_idx, at<float>(ws, l.z),
-               at<float>(ws, l.a), at<float>(ws, l.score), at<float>(ws, l.g), at<int>(ws, 0), dims->n_q,
+               at<float>(ws, l.a), at<float>(ws, l.score), at<float>(ws, l.loss_part), at<float2>(ws, l.stats),
+               at<int>(ws, 0), dims->n_q,
                dims->kv_stride, dims->top_k};
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const int rows = dims->batch * dims->n_q;
   const dim3 grid(dims->top_k / kChunk, rows);
-  warmup_logits_kernel<<<grid, kThreads, kLogitsSmem, s>>>(a);
+  warmup_loss_kernel<<<rows, kThreads, 0, s>>>(a, true);
   if (cudaGetLastError() != cudaSuccess) return SGA_ERR_CUDA;
-  warmup_objective_kernel<<<rows, kThreads, 0, s>>>(a);
+  warmup_logits_kernel<<<grid, kLogitThreads, kLogitsSmem, s>>>(a);
   if (cudaGetLastError() != cudaSuccess) return SGA_ERR_CUDA;
   warmup_grad_kernel<<<grid, kThreads, kGradSmem, s>>>(a);
+  if (cudaGetLastError() != cudaSuccess) return SGA_ERR_CUDA;
+  warmup_loss_kernel<<<rows, kThreads, 0, s>>>(a, false);
   return cudaGetLastError() == cudaSuccess ? SGA_OK : SGA_ERR_CUDA;
 }
 
