@@ -460,11 +460,11 @@ def warmup_objective_variant(sga, args, dev, stream, dist, rank, x, dims, idx, p
     gbs = per_query * rows / (step_ms * 1e-3) / 1e9
     return {"value": whole_job_rate(rows, args.steps, world, ms), "unit": UNIT, "ms_per_step": step_ms,
             "config": f"{rows} queries of the headline workload: KL(attention target || indexer softmax) over each "
-                      f"query's 2048 selected positions and the gradients of q_idx, w and k_idx (three SIMT fp32 "
-                      f"kernels)",
+                      f"query's 2048 selected positions and the gradients of q_idx, w and k_idx (logits, indexer dots "
+                      f"and gradient contractions on tcgen05, bf16 operands, fp32 accumulation)",
             "path_roofline": {"achieved_gbs": gbs, "frac_of_8tbs": gbs / NOMINAL_HBM_GBS, "frac_of_measured": gbs / peak,
                               "bytes_per_query": per_query},
-            "gpu_launches": 3 * args.steps}
+            "gpu_launches": 4 * args.steps}
 
 
 def main():

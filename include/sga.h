@@ -331,11 +331,14 @@ SGA_API sga_status_t sga_layer_forward(const sga_dims_t* dims, const sga_layer_w
  *   r(s)  = softmax_{s in S}(score(s)), score as in sga_index_scores
  *   loss[b,i] = KL(p || r)
  * and the gradients of the loss with respect to the indexer's inputs:
- *   grad_q_idx [B][T][64][128] fp32, grad_w [B][T][64] fp32 (overwritten);
- *   grad_k_idx [B][L][128] fp32: ADDED to (zero it before the first call;
- *   a position selected by several queries receives all their terms).
+ *   grad_q_idx [B][T][64][128] fp32 (8-byte aligned), grad_w [B][T][64]
+ *   fp32 (overwritten);
+ *   grad_k_idx [B][L][128] fp32 (8-byte aligned): ADDED to (zero it before
+ *   the first call; a position selected by several queries receives all
+ *   their terms).  The gradients are summed with float atomics, so their last
+ *   bits depend on the order in which the terms arrive.
  * The ReLU passes no gradient at 0.  Inputs as for sga_forward; loss [B][T]
- * fp32.  Workspace: sga_indexer_warmup_workspace_size bytes, 256-byte aligned,
+ * fp32 (its terms summed in a fixed order).  Workspace: sga_indexer_warmup_workspace_size bytes, 256-byte aligned,
  * its status word at the start (zero-filled before the first call).  B*T is
  * at most 65535.  Device error: an index outside [-1, L) (treated as empty). */
 SGA_API sga_status_t sga_indexer_warmup_workspace_size(const sga_dims_t* dims, size_t* bytes);

@@ -24,8 +24,6 @@
 //      g = r - p and the loss terms of the chunk's slots; then the gradients,
 //      added with atomics;
 //   B  per query: the loss, the chunks' terms summed in chunk order.
-// Staged rows are padded by 16 bytes so that the rows a warp reads at once
-// start on different shared-memory banks.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <math.h>
@@ -45,7 +43,6 @@ constexpr int kIdxHeads = SGA_INDEX_HEADS;  // 64
 constexpr int kIdxDim = SGA_INDEX_DIM;      // 128
 constexpr int kChunk = 64;                  // selected slots per CTA
 constexpr int kThreads = 256;
-constexpr int kIdxPad = kIdxDim + 8;        // staged q_idx / k_idx row: 136 bf16 (272 B)
 constexpr float kScale = static_cast<float>(SGA_SOFTMAX_SCALE);
 using sga::host::align_up;
 using sga::host::aligned;
@@ -58,8 +55,11 @@ constexpr int kLogitThreads = 128;
 constexpr int kBox = 64 * 128;
 constexpr uint32_t kLogitTmemCols = 128;  // z at column 0, a at column 64
 constexpr size_t kLogitsSmem = 1024 + 22 * kBox;
-// kernel C: q_idx, k rows (bf16, padded), act and ReLU(a) (fp32)
-constexpr size_t kGradSmem = 2 * kChunk * kIdxPad * 2 + 2 * kIdxHeads * kChunk * 4;
+// kernel C (tensor core): q_idx, the key rows and act's two parts in six boxes; the request
+// is sized so that at most two CTAs (256 tensor-memory columns each) share an SM
+constexpr uint32_t kGradTmemCols = 256;  // dq_idx at column 0, dk at column 128
+constexpr size_t kGradSmem = 80 * 1024;
+static_assert(kGradSmem >= 1024 + 6 * kBox && 3 * (kGradSmem + 4096) > 232448, "two CTAs per SM");
 static_assert(kLogitsSmem <= 232448 && kGradSmem <= 232448, "shared memory");
 
 struct WarmupArgs {
@@ -114,29 +114,6 @@ __device__ void load_slot_rows(const WarmupArgs& p, int row, int c, int* slot_ro
       s = -1;
     }
     slot_row[t] = s;
-  }
-}
-
-// Copies `rows` rows of `width` bf16 (16-byte aligned, width a multiple of 8) into padded shared rows.
-__device__ void stage_rows(uint16_t* dst, int pad, const uint16_t* src, int width, int rows) {
-  const int vecs = width / 8;
-  for (int e = threadIdx.x; e < rows * vecs; e += kThreads) {
-    const int r = e / vecs, v = e - r * vecs;
-    *reinterpret_cast<uint4*>(dst + r * pad + v * 8) =
-        reinterpret_cast<const uint4*>(src + static_cast<size_t>(r) * width)[v];
-  }
-}
-
-// Gathers the chunk's cache rows (zeros for empty slots) into padded shared rows.
-__device__ void gather_rows(uint16_t* dst, int pad, const uint16_t* cache, int width, size_t seq_base,
-                            const int* slot_row) {
-  const int vecs = width / 8;
-  for (int e = threadIdx.x; e < kChunk * vecs; e += kThreads) {
-    const int s = e / vecs, v = e - s * vecs;
-    const int r = slot_row[s];
-    uint4 val = make_uint4(0u, 0u, 0u, 0u);
-    if (r >= 0) val = reinterpret_cast<const uint4*>(cache + (seq_base + r) * width)[v];
-    *reinterpret_cast<uint4*>(dst + s * pad + v * 8) = val;
   }
 }
 
@@ -310,24 +287,64 @@ __global__ void __launch_bounds__(kLogitThreads, 1) warmup_logits_kernel(WarmupA
 // chunk's (max, sum) pair, the indexer softmax's from all of the query's
 // scores; then for each slot p(s), r(s), g_s = r(s) - p(s) and its loss term
 // (the chunk's share goes to the workspace, summed in chunk order by kernel
-// B), and the gradients are added into the query's q_idx and w gradients and
-// the key gradients of the selected cache rows.
-__global__ void __launch_bounds__(kThreads) warmup_grad_kernel(WarmupArgs p) {
-  extern __shared__ __align__(16) uint8_t smem[];
-  uint16_t* qis = reinterpret_cast<uint16_t*>(smem);             // [64][kIdxPad]
-  uint16_t* ks = qis + kIdxHeads * kIdxPad;                        // [64][kIdxPad]
-  float* act = reinterpret_cast<float*>(ks + kChunk * kIdxPad);   // [64 j][64 s]: g_s w_j [a_js > 0]
-  float* relu = act + kIdxHeads * kChunk;                          // [64 j][64 s]: ReLU(a_js)
+// B).  With act[j][s] = g_s w_j [a_js > 0], carried as two bf16 parts (hi +
+// lo, about 16 mantissa bits), the tensor core computes
+//   dq_idx[j][d] = sum_s act[j][s] k[s][d]   (M = 64 j, N = 128 d, K = 64 s;
+//                                              act K-major, k rows MN-major)
+//   dk[s][d]     = sum_j act[j][s] q_idx[j][d] (M = 64 s, N = 128 d, K = 64 j;
+//                                              act and q_idx MN-major)
+// into tensor memory (columns 0 and 128); eight warps read them back (warps
+// 0-3 dq_idx, 4-7 dk, one TMEM lane quarter each) and add them to the query's
+// q_idx gradient and the selected rows' key gradients with float2 atomics.
+// dw_j = sum_s g_s ReLU(a_js) is summed by the threads that build act.
+__global__ void __launch_bounds__(kThreads, 2) warmup_grad_kernel(WarmupArgs p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t qi_s = sga::smem_u32(smem);  // 2 boxes: q_idx [64 j][128 d]
+  const uint32_t ki_s = qi_s + 2 * kBox;       // 2 boxes: the chunk's key rows [64 s][128 d]
+  const uint32_t ah_s = ki_s + 2 * kBox;       // act, high bf16 part [64 j][64 s]
+  const uint32_t al_s = ah_s + kBox;           // act, low part
+  uint8_t* ah_ptr = smem + 4 * kBox;
   __shared__ int slot_row[kChunk];
   __shared__ float gs[kChunk], wj[kIdxHeads], hm[kHeads], hinv[kHeads], red[kThreads / 32];
   __shared__ float pp_part[kThreads / kChunk][kChunk];
+  __shared__ __align__(8) uint64_t mma_bar;
+  __shared__ uint32_t tmem_slot;
+  __shared__ int abort_flag;
   const int c = blockIdx.x, row = blockIdx.y, b = row / p.n_q, t = threadIdx.x;
   const int lane = t & 31, warp = t >> 5;
   const int K = p.top_k, nch = K / kChunk;
   const size_t seq_base = static_cast<size_t>(b) * p.kv_stride;
+  if (t == 0) {
+    sga::mbar_init(sga::smem_u32(&mma_bar), 1);
+    abort_flag = 0;
+    sga::fence_barrier_init();
+  }
+  if (warp == 0) {
+    sga::tmem_alloc(sga::smem_u32(&tmem_slot), kGradTmemCols);
+    sga::tmem_relinquish();
+  }
   load_slot_rows(p, row, c, slot_row);
   if (t < kIdxHeads) wj[t] = bf(p.w[static_cast<size_t>(row) * kIdxHeads + t]);
-  stage_rows(qis, kIdxPad, p.q_idx + static_cast<size_t>(row) * kIdxHeads * kIdxDim, kIdxDim, kIdxHeads);
+  sga::tc_fence_before();
+  __syncthreads();
+  sga::tc_fence_after();
+  const uint32_t tmem = tmem_slot;
+  {
+    // q_idx and the chunk's key rows into swizzled boxes (16-byte pieces; empty slots zero-filled);
+    // they land while the objective below is computed
+    const uint16_t* qirow = p.q_idx + static_cast<size_t>(row) * kIdxHeads * kIdxDim;
+    for (int e = t; e < kIdxHeads * 16; e += kThreads) {
+      const int r = e >> 4, pc = e & 15;
+      sga::cp_async_16(qi_s + (pc >> 3) * kBox + r * 128 + (((pc & 7) ^ (r & 7)) << 4), qirow + r * kIdxDim + pc * 8,
+                       16);
+    }
+    for (int e = t; e < kChunk * 16; e += kThreads) {
+      const int r = e >> 4, pc = e & 15, sr = slot_row[r];
+      const uint16_t* src = p.k_idx + (seq_base + (sr >= 0 ? sr : 0)) * kIdxDim + pc * 8;
+      sga::cp_async_16(ki_s + (pc >> 3) * kBox + r * 128 + (((pc & 7) ^ (r & 7)) << 4), src, sr >= 0 ? 16u : 0u);
+    }
+  }
   // ---- the target's per-head statistics: the chunks' (max, sum) pairs merged
   for (int h = warp; h < kHeads; h += kThreads / 32) {
     const float2* st = p.stats + (static_cast<size_t>(row) * kHeads + h) * nch;
@@ -355,7 +372,7 @@ __global__ void __launch_bounds__(kThreads) warmup_grad_kernel(WarmupArgs p) {
   if (smax != -INFINITY)
     for (int s = t; s < K; s += kThreads)
       if (zr[s] != -INFINITY) ssum += expf(sr[s] - smax);
-  ssum = block_reduce<false>(ssum, red);  // (its barriers also publish hm, hinv, wj and slot_row)
+  ssum = block_reduce<false>(ssum, red);  // (its barriers also publish hm and hinv)
   // ---- p(s) for the chunk's slots: thread (slot s, head group hg) sums 16 heads
   {
     const int s = t & (kChunk - 1), hg = t / kChunk;
@@ -386,66 +403,114 @@ __global__ void __launch_bounds__(kThreads) warmup_grad_kernel(WarmupArgs p) {
   }
   term = block_reduce<false>(term, red);  // (its barriers also publish gs)
   if (t == 0) p.loss_part[static_cast<size_t>(row) * nch + c] = term;
-  // ---- the gradients of the chunk
-  gather_rows(ks, kIdxPad, p.k_idx, kIdxDim, seq_base, slot_row);
-  for (int e = t; e < kIdxHeads * kChunk; e += kThreads) {
-    const int j = e / kChunk, s = e - j * kChunk;
-    const float av =
-        p.a[(static_cast<size_t>(row) * kIdxHeads + j) * p.top_k + static_cast<size_t>(c) * kChunk + s];
-    const bool on = slot_row[s] >= 0 && av > 0.f;
-    act[e] = on ? gs[s] * wj[j] : 0.f;
-    relu[e] = on ? av : 0.f;
+  // ---- act (two bf16 parts) and dw: thread (j, 16 slots from s0)
+  {
+    const int j = t >> 2, s0 = (t & 3) * 16;
+    const float4* ap = reinterpret_cast<const float4*>(
+        p.a + (static_cast<size_t>(row) * kIdxHeads + j) * K + static_cast<size_t>(c) * kChunk + s0);
+    float av[16];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float4 v = ap[i];
+      av[4 * i] = v.x;
+      av[4 * i + 1] = v.y;
+      av[4 * i + 2] = v.z;
+      av[4 * i + 3] = v.w;
+    }
+    float dw = 0.f;
+    uint32_t hi[8], lo[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      float x[2];
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const int s = s0 + 2 * i + e;
+        const bool on = slot_row[s] >= 0 && av[2 * i + e] > 0.f;
+        x[e] = on ? gs[s] * wj[j] : 0.f;
+        if (on) dw = fmaf(gs[s], av[2 * i + e], dw);
+      }
+      const __nv_bfloat162 h2 = __floats2bfloat162_rn(x[0], x[1]);
+      hi[i] = *reinterpret_cast<const uint32_t*>(&h2);
+      const float2 hf = __bfloat1622float2(h2);
+      const __nv_bfloat162 l2 = __floats2bfloat162_rn(x[0] - hf.x, x[1] - hf.y);
+      lo[i] = *reinterpret_cast<const uint32_t*>(&l2);
+    }
+    // row j of each act box: 16-byte pieces s0 / 8 and s0 / 8 + 1, swizzled
+#pragma unroll
+    for (int q = 0; q < 2; ++q) {
+      const int piece = (s0 >> 3) + q;
+      const uint32_t off = j * 128 + ((piece ^ (j & 7)) << 4);
+      *reinterpret_cast<uint4*>(ah_ptr + off) = make_uint4(hi[4 * q], hi[4 * q + 1], hi[4 * q + 2], hi[4 * q + 3]);
+      *reinterpret_cast<uint4*>(ah_ptr + kBox + off) =
+          make_uint4(lo[4 * q], lo[4 * q + 1], lo[4 * q + 2], lo[4 * q + 3]);
+    }
+    dw += __shfl_xor_sync(0xffffffffu, dw, 1);
+    dw += __shfl_xor_sync(0xffffffffu, dw, 2);
+    if ((t & 3) == 0) atomicAdd(&p.grad_w[static_cast<size_t>(row) * kIdxHeads + j], dw);
   }
+  asm volatile("cp.async.wait_all;" ::: "memory");
+  sga::fence_proxy_async_smem();  // cp.async and st.shared writes, read by the tensor core
   __syncthreads();
-  if (t < kIdxHeads) {
-    float acc = 0.f;
-    for (int s = 0; s < kChunk; ++s) acc = fmaf(gs[s], relu[t * kChunk + s], acc);
-    atomicAdd(&p.grad_w[static_cast<size_t>(row) * kIdxHeads + t], acc);
+  if (t == 0) {
+    constexpr uint32_t idesc_dq = sga::idesc_bf16_f32(kIdxHeads, kIdxDim, false, true);
+    constexpr uint32_t idesc_dk = sga::idesc_bf16_f32(kChunk, kIdxDim, true, true);
+    sga::tc_fence_after();
+#pragma unroll
+    for (int kk = 0; kk < 4; ++kk)
+#pragma unroll
+      for (int part = 0; part < 2; ++part)
+        sga::mma_bf16(tmem, sga::sdesc_sw128((part ? al_s : ah_s) + kk * 32, 16, 1024),
+                      sga::sdesc_sw128(ki_s + kk * 2048, kBox, 1024), idesc_dq, (kk | part) ? 1u : 0u);
+#pragma unroll
+    for (int kk = 0; kk < 4; ++kk)
+#pragma unroll
+      for (int part = 0; part < 2; ++part)
+        sga::mma_bf16(tmem + kIdxDim, sga::sdesc_sw128((part ? al_s : ah_s) + kk * 2048, kBox, 1024),
+                      sga::sdesc_sw128(qi_s + kk * 2048, kBox, 1024), idesc_dk, (kk | part) ? 1u : 0u);
+    sga::mma_commit(sga::smem_u32(&mma_bar));
   }
-  const int q4 = t >> 2, d0 = (t & 3) * 32;
-  {
-    // dq_idx[j][d0 .. d0+31], j = q4
-    float acc[32];
-#pragma unroll
-    for (int i = 0; i < 32; ++i) acc[i] = 0.f;
-    for (int s = 0; s < kChunk; ++s) {
-      const float av = act[q4 * kChunk + s];
-      const __nv_bfloat162* kr = reinterpret_cast<const __nv_bfloat162*>(ks + s * kIdxPad + d0);
-#pragma unroll
-      for (int i = 0; i < 16; ++i) {
-        const float2 k2 = __bfloat1622float2(kr[i]);
-        acc[2 * i] = fmaf(av, k2.x, acc[2 * i]);
-        acc[2 * i + 1] = fmaf(av, k2.y, acc[2 * i + 1]);
-      }
-    }
-    float* dst = p.grad_q_idx + (static_cast<size_t>(row) * kIdxHeads + q4) * kIdxDim + d0;
-#pragma unroll
-    for (int i = 0; i < 32; ++i) atomicAdd(dst + i, acc[i]);
+  bool ok = sga::mbar_wait(sga::smem_u32(&mma_bar), 0, &abort_flag);
+  if (!ok) {
+    atomicCAS(p.status, 0, static_cast<int>(SGA_ERR_TIMEOUT));
+    abort_flag = 1;
   }
-  {
-    // dk[s][d0 .. d0+31], s = q4
-    const int r = slot_row[q4];
-    if (r >= 0) {
-      float acc[32];
+  ok = __syncthreads_and(ok) != 0;  // the epilogue's loads need whole warps
+  sga::tc_fence_after();
+  if (ok) {
+    const int quarter = warp & 3, which = warp >> 2;  // 0: dq_idx, 1: dk
+    const uint32_t taddr = tmem + (static_cast<uint32_t>(quarter * 32) << 16) + which * kIdxDim;
+    const int m4 = lane & 3;
+    const int rr[2] = {quarter * 16 + (lane >> 2), quarter * 16 + 8 + (lane >> 2)};
+    for (int half = 0; half < 2; ++half) {
+      float v[32];
+      sga::tmem_ld_16x256b_x8(taddr + 64 * half, v);
 #pragma unroll
-      for (int i = 0; i < 32; ++i) acc[i] = 0.f;
-      for (int j = 0; j < kIdxHeads; ++j) {
-        const float av = act[j * kChunk + q4];
-        const __nv_bfloat162* qr = reinterpret_cast<const __nv_bfloat162*>(qis + j * kIdxPad + d0);
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const float2 q2 = __bfloat1622float2(qr[i]);
-          acc[2 * i] = fmaf(av, q2.x, acc[2 * i]);
-          acc[2 * i + 1] = fmaf(av, q2.y, acc[2 * i + 1]);
+      for (int i = 0; i < 2; ++i) {
+        float* dst;
+        if (which == 0) {
+          dst = p.grad_q_idx + (static_cast<size_t>(row) * kIdxHeads + rr[i]) * kIdxDim;
+        } else {
+          const int r = slot_row[rr[i]];
+          if (r < 0) continue;
+          dst = p.grad_k_idx + (seq_base + r) * kIdxDim;
         }
-      }
-      float* dst = p.grad_k_idx + (seq_base + r) * kIdxDim + d0;
 #pragma unroll
-      for (int i = 0; i < 32; ++i) atomicAdd(dst + i, acc[i]);
+        for (int k = 0; k < 8; ++k)
+          atomicAdd(reinterpret_cast<float2*>(dst + 64 * half + 8 * k + 2 * m4),
+                    make_float2(v[4 * k + 2 * i], v[4 * k + 2 * i + 1]));
+      }
     }
+  } else if (t == 0) {
+    volatile int never = 0;
+    sga::mbar_wait(sga::smem_u32(&mma_bar), 0, &never);  // its MMAs must finish before tensor memory is freed
+  }
+  sga::tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    sga::tc_fence_after();
+    sga::tmem_dealloc(tmem, kGradTmemCols);
   }
 }
-
 
 // B: per query, the loss (the chunks' terms summed in chunk order); also clears
 // the query's q_idx and w gradients, which the next call's kernel C adds into.
@@ -509,8 +574,8 @@ sga_status_t sga_indexer_warmup(const sga_dims_t* dims, const sga_bf16_t* q_idx,
                                 void* ws, size_t ws_bytes, sga_stream_t stream) {
   if (!warmup_dims_ok(dims)) return SGA_ERR_INVALID_ARG;
   if (!aligned(q_idx, 16) || !aligned(w, 2) || !aligned(k_idx, 16) || !aligned(q, 16) || !aligned(kv, 16) ||
-      !aligned(idx, 4) || !aligned(loss, 4) || !aligned(grad_q_idx, 4) || !aligned(grad_w, 4) ||
-      !aligned(grad_k_idx, 4))
+      !aligned(idx, 4) || !aligned(loss, 4) || !aligned(grad_q_idx, 8) || !aligned(grad_w, 4) ||
+      !aligned(grad_k_idx, 8))
     return SGA_ERR_INVALID_ARG;
   const WarmupLayout l = warmup_layout(*dims);
   if (!aligned(ws, kAlign) || ws_bytes < l.total) return SGA_ERR_WORKSPACE;
