@@ -18,7 +18,7 @@
 //   1. MSD radix select over the score key, 12/12/8 bits per level: each CTA
 //      counts its segment into a shared-memory histogram and all CTAs sum the
 //      C histograms through distributed shared memory, so every CTA finds the
-//      same bin.  Levels stop when that bin fits a candidate list (4096 keys)
+//      same bin.  Levels stop when that bin fits a candidate list (8192 keys)
 //      or is a single key.  Under sga_forward the indexer has already counted
 //      the first level, so that pass is skipped.
 //   2. One ballot pass builds, per 32 positions, an "above" word (keys whose
@@ -55,7 +55,7 @@ constexpr int kWarps = kThreads / 32;
 constexpr int kBits = kTopkHistBits;  // 12
 constexpr int kBins = kTopkHistBins;  // 4096
 constexpr int kBinsPerThread = kBins / kThreads;
-constexpr int kCandCap = 4096;
+constexpr int kCandCap = 8192;
 constexpr int kMaxCluster = 8;
 constexpr int kChunk = 8192;           // scores per ring slot (32 KB)
 constexpr int kRingSlots = 3;
@@ -71,6 +71,7 @@ constexpr int kResWarpSpan = kResSeg / kWarps;  // 1024 consecutive positions pe
 constexpr int kResSteps = kResWarpSpan / 32;    // 32 ballot steps per warp and pass
 constexpr size_t kResSmemBytes = kResSeg * 4 + 2 * kBins * 4 + kCandCap * 8;
 static_assert(kResSteps == 32, "lane j keeps the words of step j");
+static_assert(kSmemBytes + 2048 <= 232448 && kResSmemBytes + 2048 <= 232448, "shared memory budget");
 
 struct TopkParams {
   const float* scores;
