@@ -325,10 +325,10 @@ def test_forward_matches_oracle(B, T, L, pos):
 
 @pytest.mark.parametrize("k_range,L", [(0, 9000), (1, 20000)])
 def test_forward_wide_threshold_bin(k_range, L):
-    """Index keys all zero (every score equal) or in {-1, 0, 1} (heavy ties): the
-    bin of the K-th score holds more keys than the candidate list, so the
-    selection narrows it with passes over its positions and takes the lowest
-    positions among the ties."""
+    """Index keys all zero (every score equal: the K-th score's bin holds all
+    9,000 keys, more than the 8,192-key candidate list, so the selection
+    narrows it with passes over its positions) or in {-1, 0, 1} (heavy ties);
+    both take the lowest positions among the ties."""
     B = 2
     x = gen_small(B, 1, L, [[L - 1], [L // 2]], k_range=k_range, seed=7)
     ws = sga.alloc_workspace(sga.make_dims(B, 1, L), sga.OP_FORWARD)
