@@ -78,6 +78,7 @@ struct WarmupArgs {
   float* score;           // workspace [rows][K]
   float* loss_part;       // workspace [rows][K / 64]: each chunk's share of the loss
   float2* stats;          // workspace [rows][64][K / 64]: each chunk's (max z, sum exp(z - max)) per head
+  float2* score_stats;    // workspace [rows][K / 64]: each chunk's (max score, sum exp(score - max)) over its valid slots
   int* status;
   int n_q, kv_stride, top_k;
 };
@@ -273,13 +274,28 @@ __global__ void __launch_bounds__(kLogitThreads, 1) warmup_logits_kernel(WarmupA
   }
   sga::tc_fence_before();
   __syncthreads();
-  if (ok && t < kChunk)
-    p.score[static_cast<size_t>(row) * p.top_k + static_cast<size_t>(c) * kChunk + t] =
-        (sc_part[0][t] + sc_part[1][t]) + (sc_part[2][t] + sc_part[3][t]);
   if (warp == 0) {
     sga::tc_fence_after();
     sga::tmem_dealloc(tmem, kLogitTmemCols);
   }
+  // the score of slot t (warps 0 and 1), and the chunk's (max, sum of exponentials) over its valid slots
+  __shared__ float smax_w[2], ssum_w[2];
+  float sc = 0.f;
+  const bool valid = t < kChunk && slot_row[t] >= 0;
+  if (t < kChunk) {
+    sc = (sc_part[0][t] + sc_part[1][t]) + (sc_part[2][t] + sc_part[3][t]);
+    if (ok) p.score[static_cast<size_t>(row) * p.top_k + static_cast<size_t>(c) * kChunk + t] = sc;
+    const float m = warp_max(valid ? sc : -INFINITY);
+    if (lane == 0) smax_w[warp] = m;
+  }
+  __syncthreads();
+  const float cmax = fmaxf(smax_w[0], smax_w[1]);
+  if (t < kChunk) {
+    const float e = warp_sum(valid && cmax != -INFINITY ? expf(sc - cmax) : 0.f);
+    if (lane == 0) ssum_w[warp] = e;
+  }
+  __syncthreads();
+  if (ok && t == 0) p.score_stats[static_cast<size_t>(row) * nch + c] = make_float2(cmax, ssum_w[0] + ssum_w[1]);
 }
 
 // C: per (query, chunk), the objective for the chunk's slots, then their
@@ -361,18 +377,19 @@ __global__ void __launch_bounds__(kThreads, 2) warmup_grad_kernel(WarmupArgs p) 
       hinv[h] = l > 0.f ? 1.f / l : 0.f;
     }
   }
-  // ---- the indexer softmax over the query's valid slots (an empty slot has z = -inf in every head)
+  // ---- the indexer softmax's normaliser over the query's valid slots: the chunks' (max, sum) pairs merged
   const float* zr = p.z + static_cast<size_t>(row) * kHeads * K;
   const float* sr = p.score + static_cast<size_t>(row) * K;
-  float smax = -INFINITY;
-  for (int s = t; s < K; s += kThreads)
-    if (zr[s] != -INFINITY) smax = fmaxf(smax, sr[s]);
-  smax = block_reduce<true>(smax, red);
-  float ssum = 0.f;
-  if (smax != -INFINITY)
-    for (int s = t; s < K; s += kThreads)
-      if (zr[s] != -INFINITY) ssum += expf(sr[s] - smax);
-  ssum = block_reduce<false>(ssum, red);  // (its barriers also publish hm and hinv)
+  float smax = -INFINITY, ssum = 0.f;
+  {
+    const float2* st = p.score_stats + static_cast<size_t>(row) * nch;
+    for (int cc = t; cc < nch; cc += kThreads) smax = fmaxf(smax, st[cc].x);
+    smax = block_reduce<true>(smax, red);
+    if (smax != -INFINITY)
+      for (int cc = t; cc < nch; cc += kThreads)
+        if (st[cc].x != -INFINITY) ssum += st[cc].y * expf(st[cc].x - smax);
+    ssum = block_reduce<false>(ssum, red);  // (its barriers also publish hm and hinv)
+  }
   // ---- p(s) for the chunk's slots: thread (slot s, head group hg) sums 16 heads
   {
     const int s = t & (kChunk - 1), hg = t / kChunk;
@@ -380,9 +397,14 @@ __global__ void __launch_bounds__(kThreads, 2) warmup_grad_kernel(WarmupArgs p) 
     const float* zc = zr + static_cast<size_t>(c) * kChunk + s;
     float pp = 0.f;
     if (slot_row[s] >= 0) {
-#pragma unroll 4
-      for (int h = hg * kHeadsPerGroup; h < (hg + 1) * kHeadsPerGroup; ++h)
-        pp += expf(zc[static_cast<size_t>(h) * K] - hm[h]) * hinv[h];
+      float zv[kHeadsPerGroup];  // all loads in flight at once
+#pragma unroll
+      for (int i = 0; i < kHeadsPerGroup; ++i) zv[i] = zc[static_cast<size_t>(hg * kHeadsPerGroup + i) * K];
+#pragma unroll
+      for (int i = 0; i < kHeadsPerGroup; ++i) {
+        const int h = hg * kHeadsPerGroup + i;
+        pp += expf(zv[i] - hm[h]) * hinv[h];
+      }
     }
     pp_part[hg][s] = pp;
   }
@@ -530,7 +552,7 @@ __global__ void __launch_bounds__(kThreads) warmup_loss_kernel(WarmupArgs p, boo
 }
 
 struct WarmupLayout {
-  size_t z = 0, a = 0, score = 0, stats = 0, loss_part = 0, total = 0;
+  size_t z = 0, a = 0, score = 0, stats = 0, score_stats = 0, loss_part = 0, total = 0;
 };
 
 bool warmup_dims_ok(const sga_dims_t* d) {
@@ -552,6 +574,8 @@ WarmupLayout warmup_layout(const sga_dims_t& d) {
   off += align_up(rows * K * 4);
   l.stats = off;
   off += align_up(rows * kHeads * (K / kChunk) * 8);
+  l.score_stats = off;
+  off += align_up(rows * (K / kChunk) * 8);
   l.loss_part = off;
   off += align_up(rows * (K / kChunk) * 4);
   l.total = off;
@@ -602,7 +626,7 @@ sga_status_t sga_indexer_warmup(const sga_dims_t* dims, const sga_bf16_t* q_idx,
   }
   WarmupArgs a{q_idx, w, k_idx, q, kv, idx, loss, grad_q_idx, grad_w, grad_k_idx, at<float>(ws, l.z),
                at<float>(ws, l.a), at<float>(ws, l.score), at<float>(ws, l.loss_part), at<float2>(ws, l.stats),
-               at<int>(ws, 0), dims->n_q,
+               at<float2>(ws, l.score_stats), at<int>(ws, 0), dims->n_q,
                dims->kv_stride, dims->top_k};
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const int rows = dims->batch * dims->n_q;

@@ -196,9 +196,10 @@ def test_warmup_workspace_size(lib):
     d = sga.make_dims(2, 3, 5000, 2048)
     rows, K = 6, 2048
     # status block, then z and a ([rows][64][K] fp32 each), the scores ([rows][K] fp32), each 64-slot
-    # chunk's softmax statistics per head ([rows][64][K / 64] float pairs) and its loss term ([rows][K / 64])
+    # chunk's softmax statistics per head ([rows][64][K / 64] float pairs) and of its scores ([rows][K / 64]
+    # float pairs), and its loss term ([rows][K / 64])
     assert sga.indexer_warmup_workspace_size(d) == (256 + 2 * rows * 64 * K * 4 + rows * K * 4 + rows * 64 * 32 * 8
-                                                    + rows * 32 * 4)
+                                                    + rows * 32 * 8 + rows * 32 * 4)
 
 
 @pytest.mark.parametrize("dims", [(1, 1, 100, 100), (1, 1, 100, 0), (70000, 1, 100, 2048), (0, 1, 100, 2048)])
