@@ -50,11 +50,12 @@ using sga::host::at;
 using sga::host::kStatusBytes;
 constexpr size_t kAlign = sga::host::kWsAlign;
 
-// kernel A (tensor core): 22 swizzled boxes of 64 rows x 64 bf16, and the 1 KB alignment
+// kernel A (tensor core): 10 swizzled boxes of 64 rows x 64 bf16, and the 1 KB alignment
 constexpr int kLogitThreads = 128;
 constexpr int kBox = 64 * 128;
 constexpr uint32_t kLogitTmemCols = 128;  // z at column 0, a at column 64
-constexpr size_t kLogitsSmem = 1024 + 22 * kBox;
+constexpr int kLogitPhases = 3;  // Q and the latent rows: three 192-dim phases
+constexpr size_t kLogitsSmem = 1024 + 10 * kBox;
 // kernel C (tensor core): q_idx, the key rows and act's two parts in six boxes; the request
 // is sized so that at most two CTAs (256 tensor-memory columns each) share an SM
 constexpr uint32_t kGradTmemCols = 256;  // dq_idx at column 0, dk at column 128
@@ -120,19 +121,23 @@ __device__ void load_slot_rows(const WarmupArgs& p, int row, int c, int* slot_ro
 
 // A: logits, indexer dots, scores and the chunk's softmax statistics of one
 // chunk of 64 selected slots, on the tensor core.  All 128 threads gather the
-// query's 64 x 576 latent query, the chunk's 64 latent rows, the 64 x 128
-// indexer query and the chunk's 64 key rows into 128-byte-swizzled boxes of 64
-// rows x 64 dims (16-byte cp.async; empty slots are zero-filled); one thread
-// issues z = Q C^T (M = 64 heads, N = 64 slots, K = 576) and a = Q_idx K^T
+// query's 64 x 576 latent query and the chunk's 64 latent rows (in three
+// 192-dim phases), the 64 x 128 indexer query and the chunk's 64 key rows into
+// 128-byte-swizzled boxes of 64 rows x 64 dims (16-byte cp.async; empty slots
+// are zero-filled); one thread issues z = Q C^T (M = 64 heads, N = 64 slots,
+// K = 576, accumulated over the phases) and a = Q_idx K^T
 // (M = 64 indexer heads, K = 128) into tensor memory; each warp then reads 16
 // rows of both with the 16-lane x 256-bit shape (thread t: rows t/4 and 8 + t/4
 // of its quarter, columns 8k + 2(t%4) and +1).
-__global__ void __launch_bounds__(kLogitThreads, 1) warmup_logits_kernel(WarmupArgs p) {
+__global__ void __launch_bounds__(kLogitThreads, 2) warmup_logits_kernel(WarmupArgs p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  const uint32_t q_s = sga::smem_u32(smem);    // 9 boxes: the query's 64 heads x 576
-  const uint32_t kv_s = q_s + 9 * kBox;         // 9 boxes: the chunk's 64 latent rows
-  const uint32_t qi_s = kv_s + 9 * kBox;        // 2 boxes: 64 indexer heads x 128
+  // Q and the latent rows arrive in three phases of three 64-dim boxes each
+  // (the K = 576 contraction accumulates across them), so one CTA holds 80 KB
+  // and two share an SM: one's gathers overlap the other's MMAs and epilogue.
+  const uint32_t q_s = sga::smem_u32(smem);    // 3 boxes: the query's 64 heads x 192 dims of this phase
+  const uint32_t kv_s = q_s + 3 * kBox;         // 3 boxes: the chunk's 64 latent rows, same dims
+  const uint32_t qi_s = kv_s + 3 * kBox;        // 2 boxes: 64 indexer heads x 128
   const uint32_t ki_s = qi_s + 2 * kBox;        // 2 boxes: the chunk's 64 key rows
   __shared__ int slot_row[kChunk];
   __shared__ float sc_part[4][kChunk];
@@ -157,54 +162,74 @@ __global__ void __launch_bounds__(kLogitThreads, 1) warmup_logits_kernel(WarmupA
   __syncthreads();
   sga::tc_fence_after();
   const uint32_t tmem = tmem_slot;
-  {
-    // 16-byte pieces: a 576-wide row is 72 (box piece >> 3, part piece & 7); a 128-wide row 16
-    const uint16_t* qrow = p.q + static_cast<size_t>(row) * kHeads * kDq;
-    for (int e = t; e < kHeads * 72; e += kLogitThreads) {
-      const int r = e / 72, pc = e - r * 72;
-      sga::cp_async_16(q_s + (pc >> 3) * kBox + r * 128 + (((pc & 7) ^ (r & 7)) << 4), qrow + r * kDq + pc * 8, 16);
+  const uint16_t* qrow = p.q + static_cast<size_t>(row) * kHeads * kDq;
+  bool ok = true;
+  int committed = 0;  // MMA batches committed to mma_bar
+  for (int ph = 0; ph < kLogitPhases && ok; ++ph) {
+    if (ph > 0) {
+      // the previous phase's MMAs have read the buffers before they are refilled
+      ok = sga::mbar_wait(sga::smem_u32(&mma_bar), static_cast<uint32_t>((ph - 1) & 1), &abort_flag);
+      if (!ok) {
+        atomicCAS(p.status, 0, static_cast<int>(SGA_ERR_TIMEOUT));
+        abort_flag = 1;
+      }
+      ok = __syncthreads_and(ok) != 0;
+      if (!ok) break;
+      sga::tc_fence_after();
     }
-    for (int e = t; e < kChunk * 72; e += kLogitThreads) {
-      const int r = e / 72, pc = e - r * 72, sr = slot_row[r];
-      const uint16_t* src = p.kv + (seq_base + (sr >= 0 ? sr : 0)) * kDq + pc * 8;
+    // 16-byte pieces: this phase's 24 of a 576-wide row's 72 (box (piece >> 3) % 3, part piece & 7)
+    for (int e = t; e < kHeads * 24; e += kLogitThreads) {
+      const int r = e / 24, pc = e - r * 24, gp = 24 * ph + pc;
+      sga::cp_async_16(q_s + (pc >> 3) * kBox + r * 128 + (((pc & 7) ^ (r & 7)) << 4), qrow + r * kDq + gp * 8, 16);
+    }
+    for (int e = t; e < kChunk * 24; e += kLogitThreads) {
+      const int r = e / 24, pc = e - r * 24, gp = 24 * ph + pc, sr = slot_row[r];
+      const uint16_t* src = p.kv + (seq_base + (sr >= 0 ? sr : 0)) * kDq + gp * 8;
       sga::cp_async_16(kv_s + (pc >> 3) * kBox + r * 128 + (((pc & 7) ^ (r & 7)) << 4), src, sr >= 0 ? 16u : 0u);
     }
-    const uint16_t* qirow = p.q_idx + static_cast<size_t>(row) * kIdxHeads * kIdxDim;
-    for (int e = t; e < kIdxHeads * 16; e += kLogitThreads) {
-      const int r = e >> 4, pc = e & 15;
-      sga::cp_async_16(qi_s + (pc >> 3) * kBox + r * 128 + (((pc & 7) ^ (r & 7)) << 4), qirow + r * kIdxDim + pc * 8,
-                       16);
-    }
-    for (int e = t; e < kChunk * 16; e += kLogitThreads) {
-      const int r = e >> 4, pc = e & 15, sr = slot_row[r];
-      const uint16_t* src = p.k_idx + (seq_base + (sr >= 0 ? sr : 0)) * kIdxDim + pc * 8;
-      sga::cp_async_16(ki_s + (pc >> 3) * kBox + r * 128 + (((pc & 7) ^ (r & 7)) << 4), src, sr >= 0 ? 16u : 0u);
+    if (ph == 0) {
+      const uint16_t* qirow = p.q_idx + static_cast<size_t>(row) * kIdxHeads * kIdxDim;
+      for (int e = t; e < kIdxHeads * 16; e += kLogitThreads) {
+        const int r = e >> 4, pc = e & 15;
+        sga::cp_async_16(qi_s + (pc >> 3) * kBox + r * 128 + (((pc & 7) ^ (r & 7)) << 4),
+                         qirow + r * kIdxDim + pc * 8, 16);
+      }
+      for (int e = t; e < kChunk * 16; e += kLogitThreads) {
+        const int r = e >> 4, pc = e & 15, sr = slot_row[r];
+        const uint16_t* src = p.k_idx + (seq_base + (sr >= 0 ? sr : 0)) * kIdxDim + pc * 8;
+        sga::cp_async_16(ki_s + (pc >> 3) * kBox + r * 128 + (((pc & 7) ^ (r & 7)) << 4), src, sr >= 0 ? 16u : 0u);
+      }
     }
     asm volatile("cp.async.wait_all;" ::: "memory");
     sga::fence_proxy_async_smem();  // written by cp.async, read by the tensor core
-  }
-  __syncthreads();
-  if (t == 0) {
-    constexpr uint32_t idesc = sga::idesc_bf16_f32(kHeads, kChunk, false, false);
-    sga::tc_fence_after();
-    for (int bx = 0; bx < 9; ++bx)
+    __syncthreads();
+    if (t == 0) {
+      constexpr uint32_t idesc = sga::idesc_bf16_f32(kHeads, kChunk, false, false);
+      sga::tc_fence_after();
+      for (int bx = 0; bx < 3; ++bx)
 #pragma unroll
-      for (int kk = 0; kk < 4; ++kk)
-        sga::mma_bf16(tmem, sga::sdesc_sw128(q_s + bx * kBox + kk * 32, 16, 1024),
-                      sga::sdesc_sw128(kv_s + bx * kBox + kk * 32, 16, 1024), idesc, (bx | kk) ? 1u : 0u);
-    for (int bx = 0; bx < 2; ++bx)
+        for (int kk = 0; kk < 4; ++kk)
+          sga::mma_bf16(tmem, sga::sdesc_sw128(q_s + bx * kBox + kk * 32, 16, 1024),
+                        sga::sdesc_sw128(kv_s + bx * kBox + kk * 32, 16, 1024), idesc, (ph | bx | kk) ? 1u : 0u);
+      if (ph == 0) {
+        for (int bx = 0; bx < 2; ++bx)
 #pragma unroll
-      for (int kk = 0; kk < 4; ++kk)
-        sga::mma_bf16(tmem + kChunk, sga::sdesc_sw128(qi_s + bx * kBox + kk * 32, 16, 1024),
-                      sga::sdesc_sw128(ki_s + bx * kBox + kk * 32, 16, 1024), idesc, (bx | kk) ? 1u : 0u);
-    sga::mma_commit(sga::smem_u32(&mma_bar));
+          for (int kk = 0; kk < 4; ++kk)
+            sga::mma_bf16(tmem + kChunk, sga::sdesc_sw128(qi_s + bx * kBox + kk * 32, 16, 1024),
+                          sga::sdesc_sw128(ki_s + bx * kBox + kk * 32, 16, 1024), idesc, (bx | kk) ? 1u : 0u);
+      }
+      sga::mma_commit(sga::smem_u32(&mma_bar));
+    }
+    ++committed;
   }
-  bool ok = sga::mbar_wait(sga::smem_u32(&mma_bar), 0, &abort_flag);
-  if (!ok) {
-    atomicCAS(p.status, 0, static_cast<int>(SGA_ERR_TIMEOUT));
-    abort_flag = 1;
+  if (ok) {
+    ok = sga::mbar_wait(sga::smem_u32(&mma_bar), static_cast<uint32_t>((committed - 1) & 1), &abort_flag);
+    if (!ok) {
+      atomicCAS(p.status, 0, static_cast<int>(SGA_ERR_TIMEOUT));
+      abort_flag = 1;
+    }
+    ok = __syncthreads_and(ok) != 0;  // the epilogue's shuffles need whole warps
   }
-  ok = __syncthreads_and(ok) != 0;  // the epilogue's shuffles need whole warps
   sga::tc_fence_after();
   if (ok) {
     const uint32_t lane_addr = static_cast<uint32_t>(warp * 32) << 16;
@@ -268,9 +293,9 @@ __global__ void __launch_bounds__(kLogitThreads, 1) warmup_logits_kernel(WarmupA
         sc_part[warp][8 * k + 2 * m4 + 1] = sc[2 * k + 1];
       }
     }
-  } else if (t == 0) {
-    volatile int never = 0;
-    sga::mbar_wait(sga::smem_u32(&mma_bar), 0, &never);  // its MMAs must finish before tensor memory is freed
+  } else if (t == 0 && committed > 0) {
+    volatile int never = 0;  // the last committed batch's MMAs must finish before tensor memory is freed
+    sga::mbar_wait(sga::smem_u32(&mma_bar), static_cast<uint32_t>((committed - 1) & 1), &never);
   }
   sga::tc_fence_before();
   __syncthreads();
