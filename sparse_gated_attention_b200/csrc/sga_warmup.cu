@@ -17,12 +17,13 @@
 //   B  per query: clears the query's q_idx and w gradients;
 //   A  per (query, 64-slot chunk), on the tensor core: gathers the chunk's
 //      latent and key rows, writes the 64 head logits z, the 64 indexer dots
-//      a, the score of every slot (empty slots: z = -inf) and each head's
-//      (max, sum of exponentials) over the chunk to the workspace;
-//   C  per (query, chunk): the target's per-head statistics merged from the
-//      chunks', the indexer softmax's from all the query's scores; p, r,
-//      g = r - p and the loss terms of the chunk's slots; then the gradients,
-//      added with atomics;
+//      a, the score of every slot (empty slots: z = -inf), each head's
+//      (max, sum of exponentials) over the chunk and the same pair for the
+//      chunk's scores to the workspace;
+//   C  per (query, chunk): the target's per-head statistics and the indexer
+//      softmax's normaliser, merged from the chunks' pairs; p, r, g = r - p
+//      and the loss terms of the chunk's slots; then the gradients, on the
+//      tensor core, added with atomics;
 //   B  per query: the loss, the chunks' terms summed in chunk order.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -324,9 +325,9 @@ __global__ void __launch_bounds__(kLogitThreads, 2) warmup_logits_kernel(WarmupA
 }
 
 // C: per (query, chunk), the objective for the chunk's slots, then their
-// gradients.  The target's per-head statistics come merged from every
-// chunk's (max, sum) pair, the indexer softmax's from all of the query's
-// scores; then for each slot p(s), r(s), g_s = r(s) - p(s) and its loss term
+// gradients.  The target's per-head statistics and the indexer softmax's
+// normaliser come merged from every chunk's (max, sum) pairs; then for each
+// slot p(s), r(s), g_s = r(s) - p(s) and its loss term
 // (the chunk's share goes to the workspace, summed in chunk order by kernel
 // B).  With act[j][s] = g_s w_j [a_js > 0], carried as two bf16 parts (hi +
 // lo, about 16 mantissa bits), the tensor core computes
