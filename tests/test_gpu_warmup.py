@@ -47,3 +47,25 @@ def test_indexer_warmup_matches_oracle(B, T, L, pos):
     for k in ("grad_q_idx", "grad_w", "grad_k_idx"):
         r = rel_l2(got[k].cpu().numpy().astype(np.float64), want[k])
         assert r <= 1e-3, (k, r)
+
+
+@pytest.mark.parametrize("K", [64, 960])
+def test_indexer_warmup_other_top_k(K):
+    """Selections of one chunk (64 slots) and of 15 chunks: the per-chunk softmax
+    statistics are merged over that many chunks; three queries of one sequence
+    select overlapping rows, so their key gradients meet in the same rows."""
+    B, T, L = 1, 3, 2500
+    pos = [[2499, 1800, 900]]
+    wl = synth.custom(batch=B, n_q=T, ctx=L, first_pos=int(np.min(pos)))
+    x = synth.make_inputs(wl, device="cuda", seed=9)
+    q_pos = torch.as_tensor(np.asarray(pos, dtype=np.int32), device="cuda")
+    want = W.warmup_loss(x["q_idx"], x["w"], x["k_idx"], x["q"], x["kv"], q_pos.cpu(), k=K)
+    idx = torch.as_tensor(want["idx"], device="cuda")
+    ws = torch.zeros(sga.indexer_warmup_workspace_size(sga.make_dims(B, T, L, K)), dtype=torch.uint8, device="cuda")
+    got = sga.indexer_warmup(x["q_idx"], x["w"], x["k_idx"], x["q"], x["kv"], idx, ws=ws)
+    torch.cuda.synchronize()
+    assert sga.device_status(ws) == 0
+    np.testing.assert_allclose(got["loss"].cpu().numpy(), want["per_query"], rtol=1e-4)
+    for k in ("grad_q_idx", "grad_w", "grad_k_idx"):
+        r = rel_l2(got[k].cpu().numpy().astype(np.float64), want[k])
+        assert r <= 1e-3, (k, r)
