@@ -362,6 +362,23 @@ def test_forward_monotone_scores(order, L):
     assert_close(out.cpu().numpy(), want_out, f"forward, {order} scores")
 
 
+@pytest.mark.parametrize("K", [64, 512])
+def test_forward_other_top_k(K):
+    """The whole path with fewer selected positions per query: the top-k's
+    candidate refinement, the attention's chunk count and its split merge all
+    follow K; one query sits early enough that it has fewer than K positions."""
+    B, L = 3, 5000
+    pos = [[L - 1], [2500], [K // 2]]
+    x = gen_small(B, 1, L, pos, seed=13)
+    ws = sga.alloc_workspace(sga.make_dims(B, 1, L, K), sga.OP_FORWARD)
+    idx, out = sga.forward(x["q_idx"], x["w"], x["k_idx"], x["q"], x["kv"], x["gate"], x["q_pos"], top_k=K, ws=ws)
+    check_status(ws)
+    want_idx, want_out = oracle.forward(x["q_idx"], x["w"], x["k_idx"], x["q"], x["kv"], x["gate"],
+                                        x["q_pos"].cpu(), k=K)
+    np.testing.assert_array_equal(idx.cpu().numpy(), want_idx)
+    assert_close(out.cpu().numpy(), want_out, f"forward, top_k {K}")
+
+
 def test_forward_reuses_its_workspace():
     """The selection clears the indexer's histograms after reading them, on
     every exit (full selection, t + 1 <= K, bad position), so one zero-filled
