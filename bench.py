@@ -528,6 +528,7 @@ def main():
     out = torch.empty((B, T, 64, 512), dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream(dev)
     launches_per_step = 3  # indexer, top-k, attention (the attention's split merge needs no combine kernel)
+    fused_ok = T < 8 and L <= 262144  # the rows sga_forward_fused selects from candidates
 
     def fwd_step():
         sga.forward(x["q_idx"], x["w"], x["k_idx"], x["q"], x["kv"], x["gate"], x["q_pos"], top_k=K, idx_out=idx,
@@ -647,20 +648,43 @@ def main():
         sga.forward_fp8(xf["q_idx"], x["w"], xf["k_idx"], x["q"], x["kv"], x["gate"], x["q_pos"], top_k=K,
                         idx_out=idx, out=out, ws=ws_all, stream=stream)
 
-    for _ in range(max(args.warmup, 3)):
-        fp8_step()
-    torch.cuda.synchronize(dev)
-    if dist is not None:
-        dist.barrier()
-    s3, e3 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    s3.record(stream)
-    for _ in range(args.steps):
-        fp8_step()
-    e3.record(stream)
-    torch.cuda.synchronize(dev)
-    fp8_ms = max_over_ranks(dist, dev, s3.elapsed_time(e3))
-    if sga.device_status(ws_all) != 0:
-        raise RuntimeError("device status set during the E4M3 variant run")
+    def region_ms(step, ws, what):
+        """Warm-up, then `args.steps` calls timed as one region like the main one (max over ranks)."""
+        for _ in range(max(args.warmup, 3)):
+            step()
+        torch.cuda.synchronize(dev)
+        if dist is not None:
+            dist.barrier()
+        s3, e3 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s3.record(stream)
+        for _ in range(args.steps):
+            step()
+        e3.record(stream)
+        torch.cuda.synchronize(dev)
+        ms = max_over_ranks(dist, dev, s3.elapsed_time(e3))
+        if sga.device_status(ws) != 0:
+            raise RuntimeError(f"device status set during the {what} run")
+        return ms
+
+    fp8_ms = region_ms(fp8_step, ws_all, "E4M3 variant")
+
+    # ---- the fused selection (sga_forward_fused, an opt-in entry point with the
+    # same results): the indexer appends candidates instead of writing scores
+    fused_ms = fused8_ms = None
+    if fused_ok:
+        ws_fused = sga.alloc_workspace(dims, sga.OP_FORWARD_FUSED, dev)
+
+        def fused_step():
+            sga.forward_fused(x["q_idx"], x["w"], x["k_idx"], x["q"], x["kv"], x["gate"], x["q_pos"], top_k=K,
+                              idx_out=idx, out=out, ws=ws_fused, stream=stream)
+
+        def fused8_step():
+            sga.forward_fused_fp8(xf["q_idx"], x["w"], xf["k_idx"], x["q"], x["kv"], x["gate"], x["q_pos"],
+                                  top_k=K, idx_out=idx, out=out, ws=ws_fused, stream=stream)
+
+        fused_ms = region_ms(fused_step, ws_fused, "fused-selection variant")
+        fused8_ms = region_ms(fused8_step, ws_fused, "fused-selection E4M3 variant")
+        del ws_fused
     del xf
 
     # ---- one whole SGA layer (a separate configuration): h -> projections ->
@@ -731,6 +755,19 @@ def main():
         "path_roofline": {"achieved_gbs": fp8_gbs, "frac_of_8tbs": fp8_gbs / NOMINAL_HBM_GBS,
                           "frac_of_measured": fp8_gbs / peak, "bytes_per_query": ab8["total"]},
         "gpu_launches": launches_per_step * args.steps}}
+    if fused_ms is not None:
+        for key, ms, bpq, cfg in (("fused_selection", fused_ms, ab["total"], wl.name),
+                                  ("fused_selection_fp8_index_keys", fused8_ms, ab8["total"],
+                                   f"{wl.name} with q_idx and k_idx stored as E4M3")):
+            step_ms = ms / args.steps
+            gbs = bpq * rows / (step_ms * 1e-3) / 1e9
+            variants[key] = {
+                "value": whole_job_rate(rows, args.steps, world, ms), "unit": UNIT, "ms_per_step": step_ms,
+                "config": f"{cfg} through sga_forward_fused: the indexer appends the keys at or above a running "
+                          f"per-query threshold instead of writing scores; the same indices and outputs",
+                "path_roofline": {"achieved_gbs": gbs, "frac_of_8tbs": gbs / NOMINAL_HBM_GBS,
+                                  "frac_of_measured": gbs / peak, "bytes_per_query": bpq},
+                "gpu_launches": launches_per_step * args.steps}
     variants.update(decode_lines)
     if warm is not None:
         variants["indexer_warmup"] = warm

@@ -38,9 +38,10 @@
  *     error is kept until sga_clear_device_status.
  *   - Workspace: caller-allocated device memory of at least
  *     sga_workspace_size(dims, op) bytes, 256-byte aligned.  A zero-filled
- *     workspace starts with a clear status.  sga_forward also keeps per-query
- *     histograms in it: its workspace must be zero-filled before the first
- *     call, and every call leaves them zeroed for the next one.  After a
+ *     workspace starts with a clear status.  sga_forward (and its variants)
+ *     also keeps per-query histograms and counters in it: its workspace must
+ *     be zero-filled before the first call, and every call leaves them zeroed
+ *     for the next one.  After a
  *     device error, zero the whole workspace before using it again.  Calls
  *     that share a workspace must be ordered on one stream.
  *   - No C++ exception crosses this interface.
@@ -81,7 +82,8 @@ typedef enum {
   SGA_OP_INDEX_SCORES = 0,
   SGA_OP_TOPK_SELECT = 1,
   SGA_OP_SPARSE_MLA_ATTEND = 2,
-  SGA_OP_FORWARD = 3
+  SGA_OP_FORWARD = 3,
+  SGA_OP_FORWARD_FUSED = 4 /* sga_forward_fused and sga_forward_fused_fp8 */
 } sga_op_t;
 
 typedef struct {
@@ -109,7 +111,8 @@ SGA_API int32_t sga_abi_version(void);
 /* Human-readable name of a status code (static string). */
 SGA_API const char* sga_status_string(sga_status_t status);
 
-/* Bytes of workspace `op` needs for `dims`.  SGA_OP_FORWARD covers every op.
+/* Bytes of workspace `op` needs for `dims`.  SGA_OP_FORWARD covers ops 0-3;
+ * SGA_OP_FORWARD_FUSED covers only the fused forward calls.
  * Returns SGA_ERR_INVALID_ARG for bad dims or a null `bytes`. */
 SGA_API sga_status_t sga_workspace_size(const sga_dims_t* dims, sga_op_t op, size_t* bytes);
 
@@ -178,6 +181,28 @@ SGA_API sga_status_t sga_forward_fp8(const sga_dims_t* dims, const sga_fp8_e4m3_
                              const sga_fp8_e4m3_t* k_idx, const sga_bf16_t* q, const sga_bf16_t* kv,
                              const sga_bf16_t* gate, const int32_t* q_pos, int32_t* idx_out, float* out, void* ws,
                              size_t ws_bytes, sga_stream_t stream);
+
+/* The whole path with the selection fused into the indexer (archdb "A.X K2",
+ * token-selection field: the top 2,048 positions by indexer score).  The
+ * results are those of sga_forward / sga_forward_fp8 (the same indices, bit
+ * for bit, and the same outputs); only the work differs.  For queries of
+ * decode (T < 8) over L <= 262,144 positions the indexer writes no scores: it
+ * counts the first radix level of each query's selection as it goes, raises a
+ * per-query threshold from the counts so far (every key below it has at least
+ * K larger keys already counted), and appends only the keys at or above it,
+ * with their positions, to a candidate list in the workspace; the selection
+ * then reads the candidates instead of L scores.  Other dims take the path of
+ * sga_forward.  The workspace is sga_workspace_size(dims, SGA_OP_FORWARD_FUSED)
+ * bytes, zero-filled before the first call, as for sga_forward. */
+SGA_API sga_status_t sga_forward_fused(const sga_dims_t* dims, const sga_bf16_t* q_idx, const sga_bf16_t* w,
+                                       const sga_bf16_t* k_idx, const sga_bf16_t* q, const sga_bf16_t* kv,
+                                       const sga_bf16_t* gate, const int32_t* q_pos, int32_t* idx_out, float* out,
+                                       void* ws, size_t ws_bytes, sga_stream_t stream);
+SGA_API sga_status_t sga_forward_fused_fp8(const sga_dims_t* dims, const sga_fp8_e4m3_t* q_idx,
+                                           const sga_bf16_t* w, const sga_fp8_e4m3_t* k_idx, const sga_bf16_t* q,
+                                           const sga_bf16_t* kv, const sga_bf16_t* gate, const int32_t* q_pos,
+                                           int32_t* idx_out, float* out, void* ws, size_t ws_bytes,
+                                           sga_stream_t stream);
 
 /* Synchronises `stream` and returns in *device_status the first device-side
  * error recorded in the workspace (an sga_status_t value, SGA_OK if none). */

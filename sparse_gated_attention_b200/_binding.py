@@ -26,7 +26,7 @@ QK_DIM = 576
 V_DIM = 512
 TOP_K = 2048
 
-OP_INDEX_SCORES, OP_TOPK_SELECT, OP_SPARSE_MLA_ATTEND, OP_FORWARD = 0, 1, 2, 3
+OP_INDEX_SCORES, OP_TOPK_SELECT, OP_SPARSE_MLA_ATTEND, OP_FORWARD, OP_FORWARD_FUSED = 0, 1, 2, 3, 4
 LAYER_PROJECT, LAYER_OUTPUT, LAYER_FORWARD = 0, 1, 2
 # packed layer weights (see sga_layer_weights_t): rows of w_hq after W_DQ, rows of w_cq
 HQ_EXTRA = QK_DIM + INDEX_DIM + INDEX_HEADS  # 768
@@ -39,7 +39,7 @@ EXPORTED = ["sga_abi_version", "sga_status_string", "sga_workspace_size", "sga_i
             "sga_sparse_mla_attend", "sga_forward", "sga_get_device_status", "sga_clear_device_status",
             "sga_topk_select_noalloc", "sga_index_scores_fp8", "sga_forward_fp8", "sga_layer_workspace_size",
             "sga_layer_project", "sga_layer_output", "sga_layer_forward", "sga_indexer_warmup_workspace_size",
-            "sga_indexer_warmup", "sga_selftest_bounded_wait"]
+            "sga_indexer_warmup", "sga_selftest_bounded_wait", "sga_forward_fused", "sga_forward_fused_fp8"]
 NOALLOC_SCRATCH_BYTES = 256 + 4 * 1024 * 1024
 
 
@@ -89,6 +89,8 @@ def load_library(path: str | None = None) -> ctypes.CDLL:
         "sga_topk_select_noalloc": (ctypes.c_int, [D, P, P, P, P]),
         "sga_index_scores_fp8": (ctypes.c_int, [D, P, P, P, P, P, P, sz, P]),
         "sga_forward_fp8": (ctypes.c_int, [D, P, P, P, P, P, P, P, P, P, P, sz, P]),
+        "sga_forward_fused": (ctypes.c_int, [D, P, P, P, P, P, P, P, P, P, P, sz, P]),
+        "sga_forward_fused_fp8": (ctypes.c_int, [D, P, P, P, P, P, P, P, P, P, P, sz, P]),
         "sga_layer_workspace_size": (ctypes.c_int, [D, ctypes.POINTER(LayerWeights), ctypes.c_int,
                                                     ctypes.POINTER(sz)]),
         "sga_layer_project": (ctypes.c_int, [D, ctypes.POINTER(LayerWeights), P, P, P, P, P, P, P, P, P, sz, P]),
@@ -260,14 +262,17 @@ def sparse_mla_attend(q, kv, idx, gate=None, out=None, ws=None, stream=None):
     return out
 
 
-def forward(q_idx, w, k_idx, q, kv, gate, q_pos, top_k: int = TOP_K, idx_out=None, out=None, ws=None,
-            stream=None, return_idx: bool = True):
-    """The whole path.  Returns (idx [B,T,K] or None, out [B,T,64,512])."""
+def _forward_call(call: str, fp8: bool, op: int, q_idx, w, k_idx, q, kv, gate, q_pos, top_k, idx_out, out, ws,
+                  stream, return_idx):
     B, T = q_idx.shape[0], q_idx.shape[1]
     L = k_idx.shape[1]
-    _need(q_idx, "q_idx", torch.bfloat16, (B, T, INDEX_HEADS, INDEX_DIM))
+    if fp8:
+        q_idx = _need_fp8(q_idx, "q_idx", (B, T, INDEX_HEADS, INDEX_DIM))
+        k_idx = _need_fp8(k_idx, "k_idx", (B, L, INDEX_DIM))
+    else:
+        _need(q_idx, "q_idx", torch.bfloat16, (B, T, INDEX_HEADS, INDEX_DIM))
+        _need(k_idx, "k_idx", torch.bfloat16, (B, L, INDEX_DIM))
     _need(w, "w", torch.bfloat16, (B, T, INDEX_HEADS))
-    _need(k_idx, "k_idx", torch.bfloat16, (B, L, INDEX_DIM))
     _need(q, "q", torch.bfloat16, (B, T, HEADS, QK_DIM))
     _need(kv, "kv", torch.bfloat16, (B, L, QK_DIM))
     if gate is not None:
@@ -282,40 +287,41 @@ def forward(q_idx, w, k_idx, q, kv, gate, q_pos, top_k: int = TOP_K, idx_out=Non
         out = torch.empty((B, T, HEADS, V_DIM), dtype=torch.float32, device=q.device)
     _need(out, "out", torch.float32, (B, T, HEADS, V_DIM))
     if ws is None:
-        ws = alloc_workspace(dims, OP_FORWARD, q.device)
-    _check("sga_forward", load_library().sga_forward(
+        ws = alloc_workspace(dims, op, q.device)
+    _check(call, getattr(load_library(), call)(
         ctypes.byref(dims), _ptr(q_idx), _ptr(w), _ptr(k_idx), _ptr(q), _ptr(kv), _ptr(gate), _ptr(q_pos),
         _ptr(idx_out), _ptr(out), _ptr(ws), ws.numel(), _stream(stream)))
     return idx_out, out
+
+
+def forward(q_idx, w, k_idx, q, kv, gate, q_pos, top_k: int = TOP_K, idx_out=None, out=None, ws=None,
+            stream=None, return_idx: bool = True):
+    """The whole path.  Returns (idx [B,T,K] or None, out [B,T,64,512])."""
+    return _forward_call("sga_forward", False, OP_FORWARD, q_idx, w, k_idx, q, kv, gate, q_pos, top_k, idx_out,
+                         out, ws, stream, return_idx)
 
 
 def forward_fp8(q_idx, w, k_idx, q, kv, gate, q_pos, top_k: int = TOP_K, idx_out=None, out=None, ws=None,
                 stream=None, return_idx: bool = True):
     """The whole path with E4M3 indexer queries and keys (see sga_forward_fp8)."""
-    B, T = q_idx.shape[0], q_idx.shape[1]
-    L = k_idx.shape[1]
-    q_idx = _need_fp8(q_idx, "q_idx", (B, T, INDEX_HEADS, INDEX_DIM))
-    k_idx = _need_fp8(k_idx, "k_idx", (B, L, INDEX_DIM))
-    _need(w, "w", torch.bfloat16, (B, T, INDEX_HEADS))
-    _need(q, "q", torch.bfloat16, (B, T, HEADS, QK_DIM))
-    _need(kv, "kv", torch.bfloat16, (B, L, QK_DIM))
-    if gate is not None:
-        _need(gate, "gate", torch.bfloat16, (B, T, HEADS))
-    _need(q_pos, "q_pos", torch.int32, (B, T))
-    dims = make_dims(B, T, L, top_k)
-    if idx_out is None and return_idx:
-        idx_out = torch.empty((B, T, top_k), dtype=torch.int32, device=q.device)
-    if idx_out is not None:
-        _need(idx_out, "idx_out", torch.int32, (B, T, top_k))
-    if out is None:
-        out = torch.empty((B, T, HEADS, V_DIM), dtype=torch.float32, device=q.device)
-    _need(out, "out", torch.float32, (B, T, HEADS, V_DIM))
-    if ws is None:
-        ws = alloc_workspace(dims, OP_FORWARD, q.device)
-    _check("sga_forward_fp8", load_library().sga_forward_fp8(
-        ctypes.byref(dims), _ptr(q_idx), _ptr(w), _ptr(k_idx), _ptr(q), _ptr(kv), _ptr(gate), _ptr(q_pos),
-        _ptr(idx_out), _ptr(out), _ptr(ws), ws.numel(), _stream(stream)))
-    return idx_out, out
+    return _forward_call("sga_forward_fp8", True, OP_FORWARD, q_idx, w, k_idx, q, kv, gate, q_pos, top_k, idx_out,
+                         out, ws, stream, return_idx)
+
+
+def forward_fused(q_idx, w, k_idx, q, kv, gate, q_pos, top_k: int = TOP_K, idx_out=None, out=None, ws=None,
+                  stream=None, return_idx: bool = True):
+    """The whole path with the selection fused into the indexer (see
+    sga_forward_fused): the results of `forward`.  A workspace passed in is
+    sized for OP_FORWARD_FUSED."""
+    return _forward_call("sga_forward_fused", False, OP_FORWARD_FUSED, q_idx, w, k_idx, q, kv, gate, q_pos, top_k,
+                         idx_out, out, ws, stream, return_idx)
+
+
+def forward_fused_fp8(q_idx, w, k_idx, q, kv, gate, q_pos, top_k: int = TOP_K, idx_out=None, out=None, ws=None,
+                      stream=None, return_idx: bool = True):
+    """`forward_fused` with E4M3 indexer queries and keys: the results of `forward_fp8`."""
+    return _forward_call("sga_forward_fused_fp8", True, OP_FORWARD_FUSED, q_idx, w, k_idx, q, kv, gate, q_pos,
+                         top_k, idx_out, out, ws, stream, return_idx)
 
 
 # ----------------------------------------------------------------------------- one SGA layer

@@ -21,7 +21,7 @@ using host::kStatusBytes;
 constexpr size_t kAlign = host::kWsAlign;
 
 struct Layout {
-  size_t bitmap = 0, scores = 0, idx = 0, hist = 0, total = 0;
+  size_t bitmap = 0, scores = 0, idx = 0, hist = 0, cand = 0, cand_n = 0, total = 0;
 };
 
 bool dims_ok(const sga_dims_t* d) {
@@ -38,6 +38,21 @@ Layout make_layout(const sga_dims_t& d, sga_op_t op) {
   Layout l;
   const size_t rows = static_cast<size_t>(d.batch) * d.n_q;
   size_t off = kStatusBytes;
+  if (op == SGA_OP_FORWARD_FUSED && fused_topk_ok(d.n_q, d.kv_stride)) {
+    // no scores and no bitmaps: up to L candidates of 8 bytes per row, and the
+    // rows' candidate counters
+    l.idx = off;
+    off += align_up(rows * static_cast<size_t>(d.top_k) * 4);
+    l.hist = off;
+    off += align_up(rows * 4096 * 4);
+    l.cand = off;
+    off += align_up(rows * static_cast<size_t>(d.kv_stride) * 8);
+    l.cand_n = off;
+    off += align_up(rows * kCandNStride * 4);
+    l.total = off;
+    return l;
+  }
+  if (op == SGA_OP_FORWARD_FUSED) op = SGA_OP_FORWARD;  // rows the fused selection does not take
   if (op == SGA_OP_TOPK_SELECT || op == SGA_OP_FORWARD) {
     l.bitmap = off;
     off += align_up(rows * 2 * topk_bitmap_words(d.kv_stride) * 4);  // selection + tie bitmaps
@@ -148,17 +163,23 @@ sga_status_t index_scores_impl(const sga_dims_t* dims, const void* q_idx, const 
 
 sga_status_t forward_impl(const sga_dims_t* dims, const void* q_idx, const sga_bf16_t* w, const void* k_idx,
                           const sga_bf16_t* q, const sga_bf16_t* kv, const sga_bf16_t* gate, const int32_t* q_pos,
-                          int32_t* idx_out, float* out, void* ws, size_t ws_bytes, sga_stream_t stream, bool fp8) {
+                          int32_t* idx_out, float* out, void* ws, size_t ws_bytes, sga_stream_t stream, bool fp8,
+                          bool fused) {
   if (!dims_ok(dims)) return SGA_ERR_INVALID_ARG;
   if (!aligned(q_idx, 16) || !aligned(w, 16) || !aligned(k_idx, 16) || !aligned(q, 16) || !aligned(kv, 16) ||
       !aligned(q_pos, 4) || !aligned(out, 16) || (gate && !aligned(gate, 2)) || (idx_out && !aligned(idx_out, 16)))
     return SGA_ERR_INVALID_ARG;
   Layout l;
-  sga_status_t st = check_ws(ws, ws_bytes, *dims, SGA_OP_FORWARD, &l);
+  sga_status_t st = check_ws(ws, ws_bytes, *dims, fused ? SGA_OP_FORWARD_FUSED : SGA_OP_FORWARD, &l);
   if (st != SGA_OK) return st;
   int sms = 0;
   if ((st = device_info(&sms)) != SGA_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
+  // The fused selection: the indexer writes no scores; it keeps a running
+  // per-row threshold from the histogram counted so far and appends only the
+  // keys that can still be selected, and the selection reads those (clearing
+  // their counters for the next call).
+  const bool cand_mode = fused && fused_topk_ok(dims->n_q, dims->kv_stride);
   int* status = at<int>(ws, 0);
   float* scores = at<float>(ws, l.scores);
   int32_t* idx = idx_out ? idx_out : at<int32_t>(ws, l.idx);
@@ -171,13 +192,25 @@ sga_status_t forward_impl(const sga_dims_t* dims, const void* q_idx, const sga_b
   {
     host::NvtxRange range("sga.index_scores");
     IndexArgs ia{q_idx, w, k_idx, q_pos, scores, hist, status, dims->batch, dims->n_q, dims->kv_stride, fp8};
+    if (cand_mode) {
+      ia.scores = nullptr;
+      ia.cand = at<uint64_t>(ws, l.cand);
+      ia.cand_n = at<uint32_t>(ws, l.cand_n);
+      ia.top_k = dims->top_k;
+    }
     e = launch_index_scores(ia, sms, s);
   }
   if (e != cudaSuccess) return from_cuda(e);
   {
     host::NvtxRange range("sga.topk_select");
-    TopkArgs ta{scores, q_pos, idx, at<uint32_t>(ws, l.bitmap), hist, status, rows, dims->kv_stride, dims->top_k};
-    e = launch_topk(ta, s);
+    if (cand_mode) {
+      TopkCandArgs ca{at<uint64_t>(ws, l.cand), at<uint32_t>(ws, l.cand_n), hist, q_pos, idx, status, rows,
+                      dims->kv_stride, dims->top_k};
+      e = launch_topk_candidates(ca, s);
+    } else {
+      TopkArgs ta{scores, q_pos, idx, at<uint32_t>(ws, l.bitmap), hist, status, rows, dims->kv_stride, dims->top_k};
+      e = launch_topk(ta, s);
+    }
   }
   if (e != cudaSuccess) return from_cuda(e);
   host::NvtxRange range("sga.sparse_mla_attend");
@@ -207,7 +240,7 @@ const char* sga_status_string(sga_status_t s) {
 }
 
 sga_status_t sga_workspace_size(const sga_dims_t* dims, sga_op_t op, size_t* bytes) {
-  if (!dims_ok(dims) || !bytes || op < SGA_OP_INDEX_SCORES || op > SGA_OP_FORWARD) return SGA_ERR_INVALID_ARG;
+  if (!dims_ok(dims) || !bytes || op < SGA_OP_INDEX_SCORES || op > SGA_OP_FORWARD_FUSED) return SGA_ERR_INVALID_ARG;
   *bytes = make_layout(*dims, op).total;
   return SGA_OK;
 }
@@ -262,14 +295,28 @@ sga_status_t sga_forward(const sga_dims_t* dims, const sga_bf16_t* q_idx, const 
                          const sga_bf16_t* k_idx, const sga_bf16_t* q, const sga_bf16_t* kv,
                          const sga_bf16_t* gate, const int32_t* q_pos, int32_t* idx_out, float* out, void* ws,
                          size_t ws_bytes, sga_stream_t stream) {
-  return forward_impl(dims, q_idx, w, k_idx, q, kv, gate, q_pos, idx_out, out, ws, ws_bytes, stream, false);
+  return forward_impl(dims, q_idx, w, k_idx, q, kv, gate, q_pos, idx_out, out, ws, ws_bytes, stream, false, false);
 }
 
 sga_status_t sga_forward_fp8(const sga_dims_t* dims, const sga_fp8_e4m3_t* q_idx, const sga_bf16_t* w,
                              const sga_fp8_e4m3_t* k_idx, const sga_bf16_t* q, const sga_bf16_t* kv,
                              const sga_bf16_t* gate, const int32_t* q_pos, int32_t* idx_out, float* out, void* ws,
                              size_t ws_bytes, sga_stream_t stream) {
-  return forward_impl(dims, q_idx, w, k_idx, q, kv, gate, q_pos, idx_out, out, ws, ws_bytes, stream, true);
+  return forward_impl(dims, q_idx, w, k_idx, q, kv, gate, q_pos, idx_out, out, ws, ws_bytes, stream, true, false);
+}
+
+sga_status_t sga_forward_fused(const sga_dims_t* dims, const sga_bf16_t* q_idx, const sga_bf16_t* w,
+                               const sga_bf16_t* k_idx, const sga_bf16_t* q, const sga_bf16_t* kv,
+                               const sga_bf16_t* gate, const int32_t* q_pos, int32_t* idx_out, float* out,
+                               void* ws, size_t ws_bytes, sga_stream_t stream) {
+  return forward_impl(dims, q_idx, w, k_idx, q, kv, gate, q_pos, idx_out, out, ws, ws_bytes, stream, false, true);
+}
+
+sga_status_t sga_forward_fused_fp8(const sga_dims_t* dims, const sga_fp8_e4m3_t* q_idx, const sga_bf16_t* w,
+                                   const sga_fp8_e4m3_t* k_idx, const sga_bf16_t* q, const sga_bf16_t* kv,
+                                   const sga_bf16_t* gate, const int32_t* q_pos, int32_t* idx_out, float* out,
+                                   void* ws, size_t ws_bytes, sga_stream_t stream) {
+  return forward_impl(dims, q_idx, w, k_idx, q, kv, gate, q_pos, idx_out, out, ws, ws_bytes, stream, true, true);
 }
 
 sga_status_t sga_get_device_status(const void* ws, sga_stream_t stream, int32_t* device_status) {

@@ -40,6 +40,8 @@ constexpr int kQBox = kHeads * 128;  // one 128-byte-wide column strip of a quer
 constexpr int kTmemCols = 512;  // TMEM accumulators fill all 512 columns
 constexpr int kEpiGroups = 2;   // epilogue warp groups, taking alternate tiles
 constexpr int kThreads = 64 + kEpiGroups * 128;
+constexpr int kThrWarp = 2 + 4 * kEpiGroups;  // the candidate threshold warp (candidate mode only)
+constexpr int kCandThreads = kThreads + 32;
 constexpr int kHistBytes = kTopkHistBins * 4;
 constexpr int kEpiThreads = 128;
 
@@ -62,7 +64,7 @@ struct IndexCfg {
   static_assert((kAcc & (kAcc - 1)) == 0, "the epilogue indexes accumulators with a mask");
   static constexpr int kNumBars = 2 * kStages + 4 + 2 * kAcc + 1;
   static constexpr size_t kSmemBytes =
-      1024 + kStages * kAStage + 2 * kQBuf + kEpiGroups * kHistBytes + kNumBars * 8 + 16;
+      1024 + kStages * kAStage + 2 * kQBuf + kEpiGroups * kHistBytes + kNumBars * 8 + 32;
   static constexpr uint32_t kIdesc = kFp8 ? idesc_e4m3_f32(kKeys, kHeads) : idesc_bf16_f32(kKeys, kHeads, false, false);
 };
 static_assert(IndexCfg<false>::kSmemBytes <= 232448 && IndexCfg<true>::kSmemBytes <= 232448, "shared memory budget");
@@ -71,11 +73,66 @@ struct IndexParams {
   const uint16_t* w;
   const int32_t* q_pos;
   float* scores;
-  uint32_t* hist;  // [rows][kTopkHistBins] or null
+  uint32_t* hist;    // [rows][kTopkHistBins] or null
+  uint64_t* cand;    // candidate mode: [rows][kv_stride] selection candidates
+  uint32_t* cand_n;  // candidate mode: [rows][kCandNStride]
   int* status;
-  int n_q, kv_stride, tiles_per_row;
+  int n_q, kv_stride, tiles_per_row, top_k;
   long long total_tiles;
 };
+
+// A bin below which no key of a row can be among its top_k, from the row's
+// global histogram as far as it has been counted: the highest bin b with at
+// least top_k counted keys in bins >= b, or 0 while fewer are counted.  Every
+// counted key is a real key of the row, so at least top_k keys of the row are
+// larger than any key in a lower bin.  One warp reads the bins from the top,
+// 1,024 per round (lane l: 32 bins, lane 0 the highest), and stops at the
+// round that reaches top_k.
+__device__ __noinline__ uint32_t candidate_threshold(const uint32_t* hrow, uint32_t top_k) {
+  const int lane = threadIdx.x & 31;
+  uint32_t carry = 0;
+  for (int round = 0; round < kTopkHistBins / 1024; ++round) {
+    const int base = kTopkHistBins - 1024 * (round + 1) + 32 * (31 - lane);  // this lane's lowest bin
+    const uint4* hp = reinterpret_cast<const uint4*>(hrow + base);
+    uint32_t h[32];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const uint4 v = __ldcg(hp + i);
+      h[4 * i] = v.x;
+      h[4 * i + 1] = v.y;
+      h[4 * i + 2] = v.z;
+      h[4 * i + 3] = v.w;
+    }
+    uint32_t sum = 0;
+#pragma unroll
+    for (int k = 0; k < 32; ++k) sum += h[k];
+    uint32_t incl = sum;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t y = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    const uint32_t hi = carry + incl, lo = hi - sum;  // counted keys above and at this lane's bins
+    uint32_t b = 0;
+    if (lo < top_k && top_k <= hi) {
+      uint32_t run = lo;
+      bool found = false;
+#pragma unroll
+      for (int k = 31; k >= 0; --k) {
+        run += h[k];
+        if (!found && run >= top_k) {
+          b = static_cast<uint32_t>(base + k);
+          found = true;
+        }
+      }
+    }
+    const uint32_t hit = __ballot_sync(0xFFFFFFFFu, lo < top_k && top_k <= hi);
+    if (hit != 0u) return __shfl_sync(0xFFFFFFFFu, b, __ffs(hit) - 1);
+    carry += __shfl_sync(0xFFFFFFFFu, incl, 31);
+  }
+  return 0u;
+}
+
 
 // Walks work items j = (query row, 128-key tile) in order: one division at
 // the start, then a key step per item; the query position is read only when
@@ -102,8 +159,13 @@ struct TileCursor {
   __device__ __forceinline__ bool live(const IndexParams& p) const { return !bad_position(p) && key0 <= t; }
 };
 
-template <bool kFp8>
-__global__ void __launch_bounds__(kThreads, 1)
+// kCand: instead of scores, every key that can still be among its row's top_k
+// is appended to the row's candidate list (order key, position), and a
+// threshold warp keeps a bin below which keys are dropped, from the row's
+// global histogram as counted so far (the epilogue adds its counts every 8
+// tiles).  The candidate mode needs the histogram.
+template <bool kFp8, bool kCand>
+__global__ void __launch_bounds__(kCand ? kCandThreads : kThreads, 1)
     sga_index_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap qmap,
                      IndexParams p) {
   using C = IndexCfg<kFp8>;
@@ -125,6 +187,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t done_bar = bar0 + 8u * (2 * kStages + 4 + 2 * kAcc);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + kNumBars);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  // candidate mode: the row the epilogue works on, the groups that have
+  // finished, and the threshold warp's latest (row << 32 | bin)
+  int* row_s = reinterpret_cast<int*>(tmem_slot + 2);
+  int* done_s = row_s + 1;
+  volatile unsigned long long* thr_tag = reinterpret_cast<volatile unsigned long long*>(tmem_slot + 4);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -144,6 +211,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     mbar_init(done_bar, 1);
     *abort_flag = 0;
+    *row_s = -1;
+    *done_s = 0;
+    *thr_tag = ~0ull;
     fence_barrier_init();
   }
   if (warp == 0 && lane == 0) {
@@ -298,6 +368,34 @@ __global__ void __launch_bounds__(kThreads, 1)
       volatile int never = 0;
       mbar_wait(done_bar, 0, &never);
     }
+  } else if (kCand && warp == kThrWarp) {
+    // ------------------------------------------------------------ candidate threshold
+    // Every few microseconds: the row the epilogue works on, that row's global
+    // histogram as counted so far, and, when it rises, the threshold published
+    // for the epilogue (which drops keys in lower bins).  Ends when both
+    // epilogue groups have finished, or after the wait budget.
+    if constexpr (kCand) {
+      const long long t_start = clock64();
+      int trow = -1;
+      uint32_t tbin = 0;
+      while (*reinterpret_cast<volatile int*>(done_s) < kEpiGroups && clock64() - t_start < kWaitBudgetCycles) {
+        const int r = *reinterpret_cast<volatile int*>(row_s);
+        if (r >= 0) {
+          if (r != trow) {
+            trow = r;
+            tbin = 0;
+          }
+          const uint32_t b =
+              candidate_threshold(p.hist + static_cast<size_t>(r) * kTopkHistBins, static_cast<uint32_t>(p.top_k));
+          if (b > tbin) {
+            tbin = b;
+            if (lane == 0) *thr_tag = (static_cast<unsigned long long>(static_cast<uint32_t>(r)) << 32) | b;
+          }
+        }
+        // about 3 us until the next look, in short sleeps so the CTA is not held up at its end
+        for (int i = 0; i < 8 && *reinterpret_cast<volatile int*>(done_s) < kEpiGroups; ++i) __nanosleep(400);
+      }
+    }
   } else {
     // ------------------------------------------------------------ epilogue
     // Two groups of four warps take alternate tiles (group g reads the
@@ -308,10 +406,39 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int et = threadIdx.x - 64 - kEpiThreads * group;
     const int bar_id = 1 + group;
     uint32_t* hist_g = hist_s + group * kTopkHistBins;
-    const bool with_hist = p.hist != nullptr;
+    const bool with_hist = kCand || p.hist != nullptr;
     int an = 0;  // live tiles seen (both groups' ones): accumulator an % kAcc
     int cur_row = -1;
-    float wv[kHeads];
+    float wv[kCand ? 1 : kHeads];          // the row's head weights
+    uint32_t wpk[kCand ? kHeads / 2 : 1];  // candidate mode: as bf16 pairs (head 2i low, 2i + 1 high)
+    // Candidate mode: every 8 of its tiles the group adds its counts to the
+    // row's global histogram (each bin read and cleared atomically, so no
+    // barrier), and before each tile it takes the threshold warp's latest bin
+    // for the row; keys in lower bins are dropped.  A warp's candidates of one
+    // tile half are stored one group tile later: the counter update's result
+    // is read only then, so its round trip to L2 overlaps the next tile.
+    uint32_t thr = 0;  // bins below thr hold no key of the row's top_k
+    int gtiles = 0;
+    uint32_t pend_m[C::kHalves], pend_base[C::kHalves];
+    uint64_t pend_val[C::kHalves];
+    int pend_row = 0;
+#pragma unroll
+    for (int hh = 0; hh < C::kHalves; ++hh) pend_m[hh] = 0u;
+    auto store_pending = [&]() {
+#pragma unroll
+      for (int hh = 0; hh < C::kHalves; ++hh) {
+        if (pend_m[hh] != 0u) {
+          const uint32_t base = __shfl_sync(0xFFFFFFFFu, pend_base[hh], 0);
+          const uint32_t below = pend_m[hh] & ((1u << lane) - 1u);
+          const uint32_t slot = base + static_cast<uint32_t>(__popc(below));
+          const bool mine = (pend_m[hh] >> lane) & 1u;
+          SGA_DCHECK(p.status, !mine || slot < static_cast<uint32_t>(p.kv_stride));
+          if (mine && slot < static_cast<uint32_t>(p.kv_stride))
+            p.cand[static_cast<size_t>(pend_row) * p.kv_stride + slot] = pend_val[hh];
+          pend_m[hh] = 0u;
+        }
+      }
+    };
     // Adds the shared histogram of `r` to global memory and clears it.
     auto flush_hist = [&](int r) {
       named_barrier(bar_id, kEpiThreads);
@@ -339,6 +466,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int row = cur.row, key0 = cur.key0, t = cur.t;
       if (row != cur_row) {
         if (with_hist && cur_row >= 0) flush_hist(cur_row);
+        if constexpr (kCand) {
+          thr = 0;
+          gtiles = 0;
+          if (et == 0) atomicMax(row_s, row);
+        }
         const uint4* wp = reinterpret_cast<const uint4*>(p.w + static_cast<size_t>(row) * kHeads);
 #pragma unroll
         for (int c = 0; c < kHeads / 8; ++c) {
@@ -346,8 +478,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t x[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
-            wv[8 * c + 2 * e] = __uint_as_float(x[e] << 16);
-            wv[8 * c + 2 * e + 1] = __uint_as_float(x[e] & 0xFFFF0000u);
+            if constexpr (kCand) {
+              wpk[4 * c + e] = x[e];
+            } else {
+              wv[8 * c + 2 * e] = __uint_as_float(x[e] << 16);
+              wv[8 * c + 2 * e + 1] = __uint_as_float(x[e] & 0xFFFF0000u);
+            }
           }
         }
         cur_row = row;
@@ -358,33 +494,88 @@ __global__ void __launch_bounds__(kThreads, 1)
         *abort_flag = 1;
         break;
       }
+      if constexpr (kCand) {
+        store_pending();
+        const unsigned long long tv = *thr_tag;
+        if (static_cast<uint32_t>(tv >> 32) == static_cast<uint32_t>(row)) thr = max(thr, static_cast<uint32_t>(tv));
+      }
       tc_fence_after();
 #pragma unroll
       for (int hh = 0; hh < C::kHalves; ++hh) {
-        float v[64];
         const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
                                static_cast<uint32_t>(acc * C::kAccCols + hh * kHeads);
-        tmem_ld64(taddr, v);
-        if (hh == C::kHalves - 1) {
-          tc_fence_before();
-          mbar_arrive(accempty(acc));
-        }
         // head sum as four independent chains (one warp per scheduler: the chain
         // latency, not issue, bounds the epilogue); integer-valued inputs keep
         // every partial sum exact, so the order does not change the score
         float ps[4] = {0.f, 0.f, 0.f, 0.f};
+        if constexpr (kCand) {
+          // the 64 head dots are read 32 at a time (fewer live registers)
 #pragma unroll
-        for (int h = 0; h < 64; ++h) ps[h & 3] = fmaf(wv[h], fmaxf(v[h], 0.f), ps[h & 3]);
+          for (int part = 0; part < 2; ++part) {
+            float v[32];
+            tmem_ld32(taddr + 32 * part, v);
+            if (hh == C::kHalves - 1 && part == 1) {
+              tc_fence_before();
+              mbar_arrive(accempty(acc));
+            }
+#pragma unroll
+            for (int h = 0; h < 32; ++h) {
+              const uint32_t wp2 = wpk[16 * part + (h >> 1)];
+              const float wh = __uint_as_float((h & 1) ? (wp2 & 0xFFFF0000u) : (wp2 << 16));
+              ps[h & 3] = fmaf(wh, fmaxf(v[h], 0.f), ps[h & 3]);
+            }
+          }
+        } else {
+          float v[64];
+          tmem_ld64(taddr, v);
+          if (hh == C::kHalves - 1) {
+            tc_fence_before();
+            mbar_arrive(accempty(acc));
+          }
+#pragma unroll
+          for (int h = 0; h < 64; ++h) ps[h & 3] = fmaf(wv[h], fmaxf(v[h], 0.f), ps[h & 3]);
+        }
         const float s = (ps[0] + ps[1]) + (ps[2] + ps[3]);
         const int key = key0 + hh * kKeys + quarter * 32 + lane;
-        if (key <= t) {
+        if constexpr (kCand) {
+          // this warp's surviving keys are appended with one counter update
+          const uint32_t kb = order_bits(s);
+          if (key <= t) atomicAdd(hist_g + (kb >> (32 - kTopkHistBits)), 1u);
+          const bool c = key <= t && (kb >> (32 - kTopkHistBits)) >= thr;
+          const uint32_t m = __ballot_sync(0xFFFFFFFFu, c);
+          pend_m[hh] = m;
+          pend_val[hh] = (static_cast<uint64_t>(kb) << 32) | static_cast<uint32_t>(key);
+          pend_base[hh] = 0u;
+          if (lane == 0 && m != 0u)
+            pend_base[hh] =
+                atomicAdd(p.cand_n + static_cast<size_t>(row) * kCandNStride, static_cast<uint32_t>(__popc(m)));
+          pend_row = row;
+        } else if (key <= t) {
           p.scores[static_cast<size_t>(row) * p.kv_stride + key] = s;
           if (with_hist) atomicAdd(hist_g + (order_bits(s) >> (32 - kTopkHistBits)), 1u);
         }
       }
       ++an;
+      if (kCand && (++gtiles & 7) == 0) {
+        // this thread's bins: eight runs of four, read 16 bytes at a time
+        uint32_t* grow = p.hist + static_cast<size_t>(row) * kTopkHistBins;
+#pragma unroll
+        for (int i = 0; i < kTopkHistBins / (4 * kEpiThreads); ++i) {
+          const int b0 = 4 * (et + kEpiThreads * i);
+          const uint4 q = *reinterpret_cast<const uint4*>(hist_g + b0);
+          if ((q.x | q.y | q.z | q.w) != 0u) {
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const uint32_t v = atomicExch(hist_g + b0 + e, 0u);
+              if (v != 0u) atomicAdd(grow + b0 + e, v);
+            }
+          }
+        }
+      }
     }
+    if constexpr (kCand) store_pending();
     if (with_hist && cur_row >= 0) flush_hist(cur_row);
+    if (kCand && et == 0) atomicAdd(done_s, 1);
   }
 
   tc_fence_before();
@@ -838,7 +1029,10 @@ cudaError_t launch_index_scores(const IndexArgs& a, int num_sms, cudaStream_t st
   e = make_tmap_2d(&qmap, a.fp8, a.q_idx, kDim, static_cast<uint64_t>(rows) * kHeads, kDim * esize, strip, kHeads);
   if (e != cudaSuccess) return e;
   if (prefill) return launch_prefill(a, num_sms, stream, kmap, qmap);
-  auto kernel = a.fp8 ? sga_index_kernel<true> : sga_index_kernel<false>;
+  const bool cand = a.cand != nullptr;
+  if (cand && (a.hist == nullptr || a.cand_n == nullptr || a.kv_stride > kFusedTopkMaxL)) return cudaErrorInvalidValue;
+  auto kernel = cand ? (a.fp8 ? sga_index_kernel<true, true> : sga_index_kernel<false, true>)
+                     : (a.fp8 ? sga_index_kernel<true, false> : sga_index_kernel<false, false>);
   const size_t smem = a.fp8 ? IndexCfg<true>::kSmemBytes : IndexCfg<false>::kSmemBytes;
   e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e != cudaSuccess) return e;
@@ -847,15 +1041,18 @@ cudaError_t launch_index_scores(const IndexArgs& a, int num_sms, cudaStream_t st
   p.q_pos = a.q_pos;
   p.scores = a.scores;
   p.hist = a.hist;
+  p.cand = a.cand;
+  p.cand_n = a.cand_n;
   p.status = a.status;
   p.n_q = a.n_q;
   p.kv_stride = a.kv_stride;
   p.tiles_per_row = tiles_per_row;
+  p.top_k = a.top_k;
   p.total_tiles = total;
   const int grid = static_cast<int>(total < num_sms ? total : num_sms);
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(grid));
-  cfg.blockDim = dim3(kThreads);
+  cfg.blockDim = dim3(cand ? kCandThreads : kThreads);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];

@@ -13,16 +13,30 @@ struct IndexArgs {
   const uint16_t* w;      // [rows][64]
   const void* k_idx;      // [B][L][128] bf16, or E4M3 bytes when fp8
   const int32_t* q_pos;   // [rows]
-  float* scores;          // [rows][L]
+  float* scores;          // [rows][L]; not written when `cand` is set
   uint32_t* hist;         // [rows][4096] first-level top-k histogram (all zero on entry) or null
   int* status;
   int batch, n_q, kv_stride;
   bool fp8;               // indexer queries and keys in E4M3
+  // Selection candidates instead of scores (decode only, with `hist`; see
+  // fused_topk_ok): row r appends (order key << 32 | position) to
+  // cand[r][0 .. L) for every key that can still be among its top_k, counting
+  // them in cand_n[r * kCandNStride] (zero on entry).
+  uint64_t* cand = nullptr;
+  uint32_t* cand_n = nullptr;
+  int top_k = 0;
 };
 // n_q >= 8 queries per sequence take the prefill kernel (query blocks x key
 // tiles), which counts no histogram: `hist` is then ignored.
 cudaError_t launch_index_scores(const IndexArgs& a, int num_sms, cudaStream_t stream);
 bool index_uses_prefill(int n_q);
+// The fused selection (the indexer emits candidates, a per-row kernel selects
+// from them) takes decode rows of at most kFusedTopkMaxL positions.
+constexpr int kFusedTopkMaxL = 262144;
+// Candidate counters are kCandNStride words apart: one 128-byte line per row,
+// so the rows' counter updates spread over L2 slices.
+constexpr int kCandNStride = 32;
+inline bool fused_topk_ok(int n_q, int kv_stride) { return !index_uses_prefill(n_q) && kv_stride <= kFusedTopkMaxL; }
 
 // ---- top-k (step 2) ------------------------------------------------------------
 struct TopkArgs {
@@ -37,6 +51,19 @@ struct TopkArgs {
 size_t topk_bitmap_words(int kv_stride);
 int topk_cluster_size(int rows);
 cudaError_t launch_topk(const TopkArgs& a, cudaStream_t stream);
+
+// The selection from the indexer's candidates (rows of at most kFusedTopkMaxL
+// positions): one CTA per row; clears hist[r] and cand_n[r] for the next call.
+struct TopkCandArgs {
+  const uint64_t* cand;  // [rows][L]: (order key << 32 | position), cand_n[r] of them
+  uint32_t* cand_n;      // [rows][kCandNStride], word 0 of each row
+  uint32_t* hist;        // [rows][4096] the rows' complete first-level histograms
+  const int32_t* q_pos;  // [rows]
+  int32_t* idx;          // [rows][K]
+  int* status;
+  int rows, kv_stride, top_k;
+};
+cudaError_t launch_topk_candidates(const TopkCandArgs& a, cudaStream_t stream);
 
 // ---- sparse attention + gate (steps 3-4) -----------------------------------------
 struct AttendArgs {

@@ -870,6 +870,207 @@ __global__ void __launch_bounds__(kThreads, 1) sga_topk_resident_kernel(TopkPara
   }
 }
 
+
+// ---- selection from the indexer's candidates
+// One CTA per row.  The indexer kept every key of the row that can still be
+// among its top K, with its position, and counted the whole row's first radix
+// level, so the bin of the K-th key comes from that histogram.  While the bin
+// holds more keys than the list takes, further levels narrow it with passes
+// over the candidates.  Then one pass marks the candidates above the bin in a
+// position bitmap and lists the ones inside it; the list is refined to the
+// exact K-th key K*, its keys above K* join the bitmap and its keys equal to
+// K* form a tie bitmap, and both are emitted in position order, the lowest
+// positions first among the ties.
+constexpr int kFMaxWords = kFusedTopkMaxL / 32;
+constexpr int kFWordsPerThread = kFMaxWords / kThreads;
+constexpr int kFBatch = 8;  // candidate loads in flight per thread
+constexpr int kFListCap = 8192;  // keys of the K-th key's bin listed without a further level
+constexpr size_t kFSmemBytes = 2 * kFMaxWords * 4 + kBins * 4 + kFListCap * 8;
+static_assert(kFMaxWords % kThreads == 0, "whole bitmap words per thread");
+
+struct TopkCandParams {
+  const uint64_t* cand;
+  uint32_t* cand_n;
+  uint32_t* hist;
+  const int32_t* q_pos;
+  int32_t* idx;
+  int* status;
+  int kv_stride, top_k;
+};
+
+__global__ void __launch_bounds__(kThreads, 1) sga_topk_cand_kernel(TopkCandParams p) {
+  extern __shared__ __align__(128) uint8_t smem_raw[];
+  uint32_t* selw = reinterpret_cast<uint32_t*>(smem_raw);        // [kFMaxWords] selected positions
+  uint32_t* tiew = selw + kFMaxWords;                             // [kFMaxWords] positions of keys equal to K*
+  uint32_t* ghist = tiew + kFMaxWords;                            // [kBins]
+  uint64_t* list = reinterpret_cast<uint64_t*>(ghist + kBins);   // [kFListCap] the K-th key's bin
+  __shared__ uint32_t warp_buf[kWarps], warp_buf2[kWarps];
+  __shared__ Narrow narrow;
+  __shared__ uint32_t list_n;
+
+  const int row = blockIdx.x;
+  const int tid = threadIdx.x, lane = tid & 31;
+  const int K = p.top_k;
+  int32_t* out = p.idx + static_cast<size_t>(row) * K;
+  grid_dependency_wait();  // candidates, counts and histograms come from the indexer
+  grid_launch_dependents();
+  uint32_t* hist_row = p.hist + static_cast<size_t>(row) * kBins;
+  const int t = __ldg(p.q_pos + row);
+  const bool bad = t < 0 || t >= p.kv_stride;
+  const int n = bad ? 0 : t + 1;
+  uint32_t nc = __ldcg(p.cand_n + static_cast<size_t>(row) * kCandNStride);
+  __syncthreads();  // every thread has read the count before it is cleared for the next call
+  if (tid == 0) p.cand_n[static_cast<size_t>(row) * kCandNStride] = 0u;
+  SGA_DCHECK(p.status, nc <= static_cast<uint32_t>(n));
+  nc = min(nc, static_cast<uint32_t>(n));
+  if (bad || n <= K) {
+    if (bad && tid == 0) record_status(p.status, kStatusDeviceArg);
+    for (int j = tid; j < K; j += kThreads) out[j] = j < n ? j : -1;
+    for (int b = tid; b < kBins; b += kThreads) hist_row[b] = 0;
+    return;
+  }
+  const int words = (n + 31) >> 5;
+  reinterpret_cast<uint4*>(ghist)[tid] = __ldcg(reinterpret_cast<const uint4*>(hist_row) + tid);
+  for (int w = tid; w < words; w += kThreads) {
+    selw[w] = 0u;
+    tiew[w] = 0u;
+  }
+  if (tid == 0) list_n = 0u;
+  __syncthreads();
+  for (int b = tid; b < kBins; b += kThreads) hist_row[b] = 0;  // read above; ready for the next call
+
+  const uint64_t* cr = p.cand + static_cast<size_t>(row) * p.kv_stride;
+  const Narrow nr = find_bin(ghist, static_cast<uint32_t>(K), warp_buf, &narrow);
+  uint32_t prefix = nr.digit << (32 - kBits);
+  uint32_t mask = ~((1u << (32 - kBits)) - 1u);
+  uint32_t need = static_cast<uint32_t>(K) - nr.above;
+  uint32_t count = nr.count;
+  int shift = 32 - kBits;
+  // ---- 1. while the bin holds more keys than the list takes: one more level
+  // over the candidates (every key of the bin is a candidate)
+  while (count > static_cast<uint32_t>(kFListCap) && shift > 0) {
+    const int width = shift >= kBits ? kBits : shift;
+    shift -= width;
+    const uint32_t dmask = (1u << width) - 1u;
+    for (int b = tid; b < kBins; b += kThreads) ghist[b] = 0;
+    __syncthreads();
+    for (uint32_t i0 = 0; i0 < nc; i0 += kFBatch * kThreads) {
+      uint32_t kk[kFBatch];
+#pragma unroll
+      for (int u = 0; u < kFBatch; ++u) {
+        const uint32_t i = i0 + u * kThreads + tid;
+        kk[u] = i < nc ? static_cast<uint32_t>(__ldcg(cr + i) >> 32) : 0u;
+      }
+#pragma unroll
+      for (int u = 0; u < kFBatch; ++u)
+        if (i0 + u * kThreads + tid < nc && (kk[u] & mask) == prefix)
+          atomicAdd(ghist + ((kk[u] >> shift) & dmask), 1u);
+    }
+    __syncthreads();
+    const Narrow nb = find_bin(ghist, need, warp_buf, &narrow);
+    prefix |= nb.digit << shift;
+    mask |= dmask << shift;
+    need -= nb.above;
+    count = nb.count;
+  }
+  // ---- 2. one pass: keys above the bin join the bitmap, keys inside it are
+  // listed (or, once all 32 bits are fixed, are the ties themselves)
+  const bool listing = shift > 0;
+  for (uint32_t i0 = 0; i0 < nc; i0 += kFBatch * kThreads) {
+    uint64_t cb[kFBatch];
+#pragma unroll
+    for (int u = 0; u < kFBatch; ++u) {
+      const uint32_t i = i0 + u * kThreads + tid;
+      cb[u] = i < nc ? __ldcg(cr + i) : 0ull;
+    }
+    uint32_t inm = 0;  // which of this thread's batch entries lie in the bin
+#pragma unroll
+    for (int u = 0; u < kFBatch; ++u) {
+      const uint32_t k = static_cast<uint32_t>(cb[u] >> 32), pos = static_cast<uint32_t>(cb[u]);
+      const bool valid = i0 + u * kThreads + tid < nc && pos <= static_cast<uint32_t>(t);
+      SGA_DCHECK(p.status, i0 + u * kThreads + tid >= nc || pos <= static_cast<uint32_t>(t));
+      const bool in = valid && (k & mask) == prefix;
+      if (valid && (k & mask) > prefix) atomicOr(selw + (pos >> 5), 1u << (pos & 31));
+      if (in && !listing) atomicOr(tiew + (pos >> 5), 1u << (pos & 31));
+      inm |= static_cast<uint32_t>(in) << u;
+    }
+    if (listing) {
+      // one list update per warp and batch: a warp scan of the lanes' counts
+      const uint32_t cnt = static_cast<uint32_t>(__popc(inm));
+      uint32_t incl = cnt;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t y = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+        if (lane >= o) incl += y;
+      }
+      uint32_t base = 0;
+      const uint32_t wtotal = __shfl_sync(0xFFFFFFFFu, incl, 31);
+      if (lane == 0 && wtotal != 0u) base = atomicAdd(&list_n, wtotal);
+      uint32_t slot = __shfl_sync(0xFFFFFFFFu, base, 0) + incl - cnt;
+#pragma unroll
+      for (int u = 0; u < kFBatch; ++u) {
+        if ((inm >> u) & 1u) {
+          SGA_DCHECK(p.status, slot < static_cast<uint32_t>(kFListCap));
+          if (slot < static_cast<uint32_t>(kFListCap)) list[slot] = cb[u];
+          ++slot;
+        }
+      }
+    }
+  }
+  __syncthreads();  // bitmap and list complete
+  // ---- 3. the exact K-th key K*, and the listed keys split against it
+  if (listing) {
+    const uint32_t ln = min(list_n, static_cast<uint32_t>(kFListCap));
+    SGA_DCHECK(p.status, ln == count);
+    uint64_t kmask;
+    const uint32_t kstar = static_cast<uint32_t>(
+        refine_candidates(list, ln, ghist, prefix, mask, shift, need, warp_buf, &narrow, kmask) >> 32);
+    for (uint32_t i = tid; i < ln; i += kThreads) {
+      const uint64_t c = list[i];
+      const uint32_t k = static_cast<uint32_t>(c >> 32), pos = static_cast<uint32_t>(c);
+      if (k > kstar) atomicOr(selw + (pos >> 5), 1u << (pos & 31));
+      if (k == kstar) atomicOr(tiew + (pos >> 5), 1u << (pos & 31));
+    }
+    __syncthreads();
+  }
+  // ---- 4. emission in position order: the selected words plus the first `need` ties
+  const int w0 = tid * kFWordsPerThread;
+  uint32_t sw[kFWordsPerThread], tw[kFWordsPerThread];
+  uint32_t cs = 0, ct = 0;
+#pragma unroll
+  for (int i = 0; i < kFWordsPerThread; ++i) {
+    const bool inw = w0 + i < words;
+    sw[i] = inw ? selw[w0 + i] : 0u;
+    tw[i] = inw ? tiew[w0 + i] : 0u;
+    cs += __popc(sw[i]);
+    ct += __popc(tw[i]);
+  }
+  uint32_t sel_all, tie_all;
+  const uint32_t s_incl = block_inclusive_scan(cs, warp_buf, sel_all);
+  const uint32_t t_incl = block_inclusive_scan(ct, warp_buf2, tie_all);
+  SGA_DCHECK(p.status, sel_all + need == static_cast<uint32_t>(K) && tie_all >= need);
+  const uint32_t tb = t_incl - ct;  // ties in the words of lower threads
+  uint32_t pos = (s_incl - cs) + min(tb, need);
+  uint32_t ties_left = tb < need ? need - tb : 0u;
+#pragma unroll
+  for (int i = 0; i < kFWordsPerThread; ++i) {
+    uint32_t t2 = tw[i], keep = 0;
+    while (t2 && ties_left) {
+      const uint32_t low = t2 & (0u - t2);
+      keep |= low;
+      t2 ^= low;
+      --ties_left;
+    }
+    for (uint32_t m = sw[i] | keep; m; m &= m - 1) {
+      const int b = __ffs(m) - 1;
+      if (pos < static_cast<uint32_t>(K)) out[pos] = (w0 + i) * 32 + b;
+      ++pos;
+    }
+  }
+  const uint32_t emitted = min(sel_all + min(tie_all, need), static_cast<uint32_t>(K));
+  for (int j = static_cast<int>(emitted) + tid; j < K; j += kThreads) out[j] = -1;
+}
+
 }  // namespace
 
 // Words of one bitmap per row; the workspace holds two per row (selected, ties).
@@ -920,6 +1121,34 @@ cudaError_t launch_topk(const TopkArgs& a, cudaStream_t stream) {
   cfg.attrs = attr;
   cfg.numAttrs = 2;
   return cudaLaunchKernelEx(&cfg, kernel, p);
+}
+
+cudaError_t launch_topk_candidates(const TopkCandArgs& a, cudaStream_t stream) {
+  if (a.rows == 0) return cudaSuccess;
+  if (a.kv_stride > kFusedTopkMaxL) return cudaErrorInvalidValue;
+  cudaError_t e = cudaFuncSetAttribute(sga_topk_cand_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(kFSmemBytes));
+  if (e != cudaSuccess) return e;
+  TopkCandParams p;
+  p.cand = a.cand;
+  p.cand_n = a.cand_n;
+  p.hist = a.hist;
+  p.q_pos = a.q_pos;
+  p.idx = a.idx;
+  p.status = a.status;
+  p.kv_stride = a.kv_stride;
+  p.top_k = a.top_k;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(a.rows));
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = kFSmemBytes;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, sga_topk_cand_kernel, p);
 }
 
 }  // namespace sga

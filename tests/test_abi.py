@@ -71,6 +71,18 @@ def test_workspace_sizes(lib):
     # prefill: 4096 queries fill the GPU without splitting
     p = sga.make_dims(1, 4096, 131072)
     assert sga.workspace_size(p, sga.OP_SPARSE_MLA_ATTEND) == 256
+    # the fused selection: no scores and no bitmaps; 8-byte candidates, the
+    # histograms and one 128-byte counter line per query
+    fused_ws = sga.workspace_size(d, sga.OP_FORWARD_FUSED)
+    assert fused_ws == 256 + 32 * 2048 * 4 + 32 * 4096 * 4 + 32 * 131072 * 8 + 32 * 128
+    # rows the fused selection does not take (prefill; L above 262,144) use the plain layout
+    assert sga.workspace_size(p, sga.OP_FORWARD_FUSED) == sga.workspace_size(p, sga.OP_FORWARD)
+    big = sga.make_dims(2, 1, 262144 + 32)
+    assert sga.workspace_size(big, sga.OP_FORWARD_FUSED) == sga.workspace_size(big, sga.OP_FORWARD)
+    edge = sga.make_dims(2, 1, 262144)
+    assert sga.workspace_size(edge, sga.OP_FORWARD_FUSED) != sga.workspace_size(edge, sga.OP_FORWARD)
+    with pytest.raises(sga.SGAError):
+        sga.workspace_size(d, sga.OP_FORWARD_FUSED + 1)
 
 
 @pytest.mark.parametrize("dims", [(0, 1, 100, 2048), (1, 0, 100, 2048), (1, 1, 0, 2048), (1, 1, 100, 100),
