@@ -56,6 +56,9 @@ def parse_args():
                     help="skip the whole-layer variant (the projections either side of the path)")
     ap.add_argument("--layer-only", action="store_true",
                     help="run only the whole-layer variant and print it (a profiling case)")
+    ap.add_argument("--fused-only", action="store_true",
+                    help="run only the fused-selection variant (sga_forward_fused, bf16 and E4M3) and print it "
+                         "(a profiling case)")
     ap.add_argument("--prefill-only", action="store_true",
                     help="run only the chunked-prefill variant and print it (a profiling case)")
     ap.add_argument("--prefill-queries", type=int, default=0, help="prefill variant: new queries (default 4096)")
@@ -423,6 +426,44 @@ def layer_variant(sga, synth, args, dev, stream, dist, rank, x, dims, idx) -> di
     return {"ms": layer_ms, "weight_bytes": weight_bytes, "act_bytes": h.numel() * 2 + y.numel() * 4}
 
 
+def fused_variant(sga, synth, args, wl, x, dev, stream, dist, xf=None, idx=None, out=None) -> dict:
+    """The whole path through sga_forward_fused and sga_forward_fused_fp8 on `wl`, each timed like
+    the main region (warm-up, then `args.steps` calls as one region, max over ranks); total ms."""
+    B, T, L, K = wl.batch, wl.n_q, wl.ctx, wl.top_k
+    dims = sga.make_dims(B, T, L, K)
+    if xf is None:
+        xf = {"q_idx": synth.to_e4m3(x["q_idx"]), "k_idx": synth.to_e4m3(x["k_idx"])}
+    if idx is None:
+        idx = torch.empty((B, T, K), dtype=torch.int32, device=dev)
+    if out is None:
+        out = torch.empty((B, T, 64, 512), dtype=torch.float32, device=dev)
+    ws = sga.alloc_workspace(dims, sga.OP_FORWARD_FUSED, dev)
+    steps = {
+        "bf16": lambda: sga.forward_fused(x["q_idx"], x["w"], x["k_idx"], x["q"], x["kv"], x["gate"], x["q_pos"],
+                                          top_k=K, idx_out=idx, out=out, ws=ws, stream=stream),
+        "fp8": lambda: sga.forward_fused_fp8(xf["q_idx"], x["w"], xf["k_idx"], x["q"], x["kv"], x["gate"],
+                                             x["q_pos"], top_k=K, idx_out=idx, out=out, ws=ws, stream=stream),
+    }
+    res = {}
+    for name, step in steps.items():
+        for _ in range(max(args.warmup, 3)):
+            step()
+        torch.cuda.synchronize(dev)
+        if dist is not None:
+            dist.barrier()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(args.steps):
+            step()
+        b.record(stream)
+        torch.cuda.synchronize(dev)
+        res[name] = max_over_ranks(dist, dev, a.elapsed_time(b))
+        if sga.device_status(ws) != 0:
+            raise RuntimeError(f"device status set during the fused-selection {name} run")
+    del ws
+    return res
+
+
 def warmup_objective_variant(sga, args, dev, stream, dist, rank, x, dims, idx, peak) -> dict:
     """The indexer's sparse warm-up objective and its gradients (a training-time
     variant; sga_indexer_warmup) over the headline step's own selection, timed
@@ -505,6 +546,16 @@ def main():
         if rank == 0:
             print(json.dumps({"variant": "sga_layer", "ms_per_step": res["ms"] / args.steps,
                               "weight_bytes": res["weight_bytes"]}), flush=True)
+        return
+    if args.fused_only:
+        xo = synth.make_inputs(wl, device=dev, seed=rank)
+        res = fused_variant(sga, synth, args, wl, xo, dev, torch.cuda.current_stream(dev), dist)
+        if dist is not None:
+            dist.barrier()
+            dist.destroy_process_group()
+        if rank == 0:
+            print(json.dumps({"variant": "fused_selection", "workload": wl.name,
+                              "ms_per_step": {k: v / args.steps for k, v in res.items()}}), flush=True)
         return
     if args.prefill_only:
         res = prefill_variant(sga, synth, args, dev, torch.cuda.current_stream(dev), dist, rank)
@@ -672,19 +723,8 @@ def main():
     # same results): the indexer appends candidates instead of writing scores
     fused_ms = fused8_ms = None
     if fused_ok:
-        ws_fused = sga.alloc_workspace(dims, sga.OP_FORWARD_FUSED, dev)
-
-        def fused_step():
-            sga.forward_fused(x["q_idx"], x["w"], x["k_idx"], x["q"], x["kv"], x["gate"], x["q_pos"], top_k=K,
-                              idx_out=idx, out=out, ws=ws_fused, stream=stream)
-
-        def fused8_step():
-            sga.forward_fused_fp8(xf["q_idx"], x["w"], xf["k_idx"], x["q"], x["kv"], x["gate"], x["q_pos"],
-                                  top_k=K, idx_out=idx, out=out, ws=ws_fused, stream=stream)
-
-        fused_ms = region_ms(fused_step, ws_fused, "fused-selection variant")
-        fused8_ms = region_ms(fused8_step, ws_fused, "fused-selection E4M3 variant")
-        del ws_fused
+        fr = fused_variant(sga, synth, args, wl, x, dev, stream, dist, xf=xf, idx=idx, out=out)
+        fused_ms, fused8_ms = fr["bf16"], fr["fp8"]
     del xf
 
     # ---- one whole SGA layer (a separate configuration): h -> projections ->

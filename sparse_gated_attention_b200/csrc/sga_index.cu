@@ -409,8 +409,7 @@ __global__ void __launch_bounds__(kCand ? kCandThreads : kThreads, 1)
     const bool with_hist = kCand || p.hist != nullptr;
     int an = 0;  // live tiles seen (both groups' ones): accumulator an % kAcc
     int cur_row = -1;
-    float wv[kCand ? 1 : kHeads];          // the row's head weights
-    uint32_t wpk[kCand ? kHeads / 2 : 1];  // candidate mode: as bf16 pairs (head 2i low, 2i + 1 high)
+    float wv[kHeads];  // the row's head weights
     // Candidate mode: every 8 of its tiles the group adds its counts to the
     // row's global histogram (each bin read and cleared atomically, so no
     // barrier), and before each tile it takes the threshold warp's latest bin
@@ -478,12 +477,8 @@ __global__ void __launch_bounds__(kCand ? kCandThreads : kThreads, 1)
           const uint32_t x[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
-            if constexpr (kCand) {
-              wpk[4 * c + e] = x[e];
-            } else {
-              wv[8 * c + 2 * e] = __uint_as_float(x[e] << 16);
-              wv[8 * c + 2 * e + 1] = __uint_as_float(x[e] & 0xFFFF0000u);
-            }
+            wv[8 * c + 2 * e] = __uint_as_float(x[e] << 16);
+            wv[8 * c + 2 * e + 1] = __uint_as_float(x[e] & 0xFFFF0000u);
           }
         }
         cur_row = row;
@@ -502,39 +497,20 @@ __global__ void __launch_bounds__(kCand ? kCandThreads : kThreads, 1)
       tc_fence_after();
 #pragma unroll
       for (int hh = 0; hh < C::kHalves; ++hh) {
+        float v[64];
         const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
                                static_cast<uint32_t>(acc * C::kAccCols + hh * kHeads);
+        tmem_ld64(taddr, v);
+        if (hh == C::kHalves - 1) {
+          tc_fence_before();
+          mbar_arrive(accempty(acc));
+        }
         // head sum as four independent chains (one warp per scheduler: the chain
         // latency, not issue, bounds the epilogue); integer-valued inputs keep
         // every partial sum exact, so the order does not change the score
         float ps[4] = {0.f, 0.f, 0.f, 0.f};
-        if constexpr (kCand) {
-          // the 64 head dots are read 32 at a time (fewer live registers)
 #pragma unroll
-          for (int part = 0; part < 2; ++part) {
-            float v[32];
-            tmem_ld32(taddr + 32 * part, v);
-            if (hh == C::kHalves - 1 && part == 1) {
-              tc_fence_before();
-              mbar_arrive(accempty(acc));
-            }
-#pragma unroll
-            for (int h = 0; h < 32; ++h) {
-              const uint32_t wp2 = wpk[16 * part + (h >> 1)];
-              const float wh = __uint_as_float((h & 1) ? (wp2 & 0xFFFF0000u) : (wp2 << 16));
-              ps[h & 3] = fmaf(wh, fmaxf(v[h], 0.f), ps[h & 3]);
-            }
-          }
-        } else {
-          float v[64];
-          tmem_ld64(taddr, v);
-          if (hh == C::kHalves - 1) {
-            tc_fence_before();
-            mbar_arrive(accempty(acc));
-          }
-#pragma unroll
-          for (int h = 0; h < 64; ++h) ps[h & 3] = fmaf(wv[h], fmaxf(v[h], 0.f), ps[h & 3]);
-        }
+        for (int h = 0; h < 64; ++h) ps[h & 3] = fmaf(wv[h], fmaxf(v[h], 0.f), ps[h & 3]);
         const float s = (ps[0] + ps[1]) + (ps[2] + ps[3]);
         const int key = key0 + hh * kKeys + quarter * 32 + lane;
         if constexpr (kCand) {
