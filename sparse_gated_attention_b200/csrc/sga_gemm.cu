@@ -8,9 +8,11 @@
 // for the packed projections).  With 32 new tokens the weights are the whole
 // cost (230 MB for one layer against 2.3 MB of activations), so the design is
 // a weight stream:
-//   * the weights are the M = 128 operand, read once through a TMA ring of
-//     128 x 64 tiles (128-byte swizzle; MN-major weights as two 64-wide
-//     strips); the tokens are N (padded to 16, at most 128 per work item);
+//   * the weights are the M = 128 operand, read once through a TMA ring whose
+//     stages hold 128 x 128 tiles as two 128 x 64 boxes (128-byte swizzle;
+//     MN-major weights as 64-wide strips), so one barrier round trip moves
+//     32 KB of weights; the tokens are N (padded to 16, at most 128 per work
+//     item);
 //   * a work item is (batch, 128-row tile, token block, K split); a persistent
 //     grid walks the items, and split K keeps every SM streaming when there are
 //     fewer tiles than SMs (its partial sums go to the workspace and the
@@ -28,9 +30,11 @@ namespace sga {
 namespace {
 
 constexpr int kGM = 128;                    // weight rows per tile: MMA M
-constexpr int kGStrip = 64;                 // K elements per 128-byte strip
-constexpr int kGABytes = kGM * 128;         // 16 KB
-constexpr int kGRingBytes = 6 * (kGABytes + kGemmMaxN * 128);  // 192 KB
+constexpr int kGBox = 64;                   // K elements per 128-byte box row
+constexpr int kGStrip = 2 * kGBox;          // K elements per ring stage
+constexpr int kGHalf = kGM * 128;           // one 128 x 64 weight box: 16 KB
+constexpr int kGABytes = 2 * kGHalf;        // the weights of one stage: 32 KB
+constexpr int kGRingBytes = 208 * 1024;     // 5 stages at 32 tokens, 3 at 128
 constexpr int kGMaxStages = 16;
 constexpr int kGThreads = 192;
 constexpr int kGAccCols = kGemmMaxN;        // one accumulator: 128 lanes x up to 128 columns
@@ -114,7 +118,8 @@ __global__ void __launch_bounds__(kGThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
-  const uint32_t b_bytes = static_cast<uint32_t>(p.n_pad) * 128u;
+  const uint32_t b_half = static_cast<uint32_t>(p.n_pad) * 128u;  // one 64-wide token box
+  const uint32_t b_bytes = 2u * b_half;
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
@@ -123,18 +128,24 @@ __global__ void __launch_bounds__(kGThreads, 1)
       const uint64_t pol_x = policy_evict_last();   // tokens are re-read by every tile
       auto load_w = [&](int st, const Item& it, int ks) {
         const uint32_t a_dst = ring + st * stage_bytes;
-        if constexpr (kMnMajor) {
-          // two 64-wide strips of the m tile, 64 k rows each
-          const int y = it.b * p.w_rows_per_batch + ks * kGStrip;
-          tma_load_2d(a_dst, &wmap, full(st), it.t * kGM, y, pol_w);
-          tma_load_2d(a_dst + kGABytes / 2, &wmap, full(st), it.t * kGM + 64, y, pol_w);
-        } else {
-          tma_load_2d(a_dst, &wmap, full(st), ks * kGStrip, it.b * p.w_rows_per_batch + it.t * kGM, pol_w);
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          if constexpr (kMnMajor) {
+            // per 64 k rows, two 64-wide strips of the m tile (8 KB each)
+            const int y = it.b * p.w_rows_per_batch + ks * kGStrip + h * kGBox;
+            tma_load_2d(a_dst + h * kGHalf, &wmap, full(st), it.t * kGM, y, pol_w);
+            tma_load_2d(a_dst + h * kGHalf + kGHalf / 2, &wmap, full(st), it.t * kGM + 64, y, pol_w);
+          } else {
+            tma_load_2d(a_dst + h * kGHalf, &wmap, full(st), ks * kGStrip + h * kGBox,
+                        it.b * p.w_rows_per_batch + it.t * kGM, pol_w);
+          }
         }
       };
       auto load_x = [&](int st, const Item& it, int ks) {
-        tma_load_2d(ring + st * stage_bytes + kGABytes, &xmap, full(st), it.b * p.x_col_per_batch + ks * kGStrip,
-                    it.nb * kGemmMaxN, pol_x);
+#pragma unroll
+        for (int h = 0; h < 2; ++h)
+          tma_load_2d(ring + st * stage_bytes + kGABytes + h * b_half, &xmap, full(st),
+                      it.b * p.x_col_per_batch + ks * kGStrip + h * kGBox, it.nb * kGemmMaxN, pol_x);
       };
       // This CTA's (item, K strip) sequence.
       long long j = blockIdx.x;
@@ -222,11 +233,13 @@ __global__ void __launch_bounds__(kGThreads, 1)
           tc_fence_after();
           const uint32_t a = ring + st * stage_bytes;
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk) {
-            // 16 K elements per MMA: 32 bytes along a K-major row, or 16 rows of an MN-major strip
-            const uint64_t adesc = kMnMajor ? sdesc_sw128(a + kk * 2048, kGABytes / 2, 1024)
-                                            : sdesc_sw128(a + kk * 32, 16, 1024);
-            const uint64_t bdesc = sdesc_sw128(a + kGABytes + kk * 32, 16, 1024);
+          for (int kk = 0; kk < 8; ++kk) {
+            // 16 K elements per MMA: 32 bytes along a K-major row, or 16 rows of an MN-major strip;
+            // MMAs 0-3 read the stage's first 64-wide box, 4-7 its second
+            const uint32_t ah = a + static_cast<uint32_t>((kk >> 2) * kGHalf);
+            const uint64_t adesc = kMnMajor ? sdesc_sw128(ah + (kk & 3) * 2048, kGHalf / 2, 1024)
+                                            : sdesc_sw128(ah + (kk & 3) * 32, 16, 1024);
+            const uint64_t bdesc = sdesc_sw128(a + kGABytes + (kk >> 2) * b_half + (kk & 3) * 32, 16, 1024);
             mma_bf16(d, adesc, bdesc, idesc, (ks > it.ks0 || kk > 0) ? 1u : 0u);
           }
           mma_commit(empty(st));
@@ -300,8 +313,8 @@ __global__ void __launch_bounds__(kGThreads, 1)
 
 }  // namespace
 
-// The K split with the least time on the busiest SM, counted in weight strips
-// (16 KB each): ceil(items / SMs) items of ceil(k_strips / S) strips, plus the
+// The K split with the least time on the busiest SM, counted in ring stages
+// (32 KB of weights each): ceil(items / SMs) items of ceil(k_strips / S) stages, plus the
 // fp32 partial sums each extra split writes and its consumer reads back, spread
 // over the SMs.  S is at most 8; ties go to the smaller S.
 int gemm_splits(int m, int n, int k, int batch, int num_sms) {
@@ -335,9 +348,13 @@ cudaError_t launch_gemm(const GemmArgs& a, int num_sms, cudaStream_t stream) {
   p.n_blocks = (a.n + kGemmMaxN - 1) / kGemmMaxN;
   p.k_strips = (a.k + kGStrip - 1) / kGStrip;
   if (a.splits > p.k_strips) return cudaErrorInvalidValue;
+  // A stage spans 128 of K.  Past the end of K a K-major weight box reads zeros,
+  // but an MN-major one, or the token box of a batch other than the last, would
+  // read the next batch's rows: those shapes need K a multiple of 128.
+  if ((a.w_mn_major || a.batch > 1) && a.k % kGStrip != 0) return cudaErrorInvalidValue;
   const int n_in_block = a.n < kGemmMaxN ? a.n : kGemmMaxN;
   p.n_pad = (n_in_block + 15) / 16 * 16;
-  p.stage_bytes = kGABytes + p.n_pad * 128;  // a multiple of 2 KB: every stage keeps the 1 KB swizzle alignment
+  p.stage_bytes = kGABytes + 2 * p.n_pad * 128;  // a multiple of 4 KB: every box keeps the 1 KB swizzle alignment
   p.stages = kGRingBytes / p.stage_bytes;
   if (p.stages > kGMaxStages) p.stages = kGMaxStages;
   p.items = static_cast<long long>(a.batch) * p.m_tiles * p.n_blocks * a.splits;
@@ -354,7 +371,7 @@ cudaError_t launch_gemm(const GemmArgs& a, int num_sms, cudaStream_t stream) {
   if (a.w_mn_major) {
     // rows: batch * k (k index), columns: m; box 64 m x 64 k rows
     e = make_tmap_bf16_2d(&wmap, a.w, a.m, static_cast<uint64_t>(a.batch) * a.k, static_cast<uint64_t>(a.m) * 2, 64,
-                          kGStrip);
+                          kGBox);
   } else {
     // rows: batch * m, columns: k; box 64 k x 128 m rows
     e = make_tmap_bf16_2d(&wmap, a.w, a.k, static_cast<uint64_t>(a.batch) * a.m, static_cast<uint64_t>(a.k) * 2, 64,
