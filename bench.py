@@ -56,6 +56,9 @@ def parse_args():
                     help="skip the whole-layer variant (the projections either side of the path)")
     ap.add_argument("--layer-only", action="store_true",
                     help="run only the whole-layer variant and print it (a profiling case)")
+    ap.add_argument("--warmup-only", action="store_true",
+                    help="run only the indexer's warm-up objective over the workload's own selection and print it "
+                         "(a profiling case)")
     ap.add_argument("--fused-only", action="store_true",
                     help="run only the fused-selection variant (sga_forward_fused, bf16 and E4M3) and print it "
                          "(a profiling case)")
@@ -546,6 +549,20 @@ def main():
         if rank == 0:
             print(json.dumps({"variant": "sga_layer", "ms_per_step": res["ms"] / args.steps,
                               "weight_bytes": res["weight_bytes"]}), flush=True)
+        return
+    if args.warmup_only:
+        xo = synth.make_inputs(wl, device=dev, seed=rank)
+        do = sga.make_dims(wl.batch, wl.n_q, wl.ctx, wl.top_k)
+        io, _ = sga.forward(xo["q_idx"], xo["w"], xo["k_idx"], xo["q"], xo["kv"], xo["gate"], xo["q_pos"],
+                            top_k=wl.top_k)
+        res = warmup_objective_variant(sga, args, dev, torch.cuda.current_stream(dev), dist, rank, xo, do, io,
+                                       measured_peaks()[0])
+        if dist is not None:
+            dist.barrier()
+            dist.destroy_process_group()
+        if rank == 0:
+            print(json.dumps({"variant": "indexer_warmup", "workload": wl.name, "ms_per_step": res["ms_per_step"]}),
+                  flush=True)
         return
     if args.fused_only:
         xo = synth.make_inputs(wl, device=dev, seed=rank)
