@@ -514,10 +514,13 @@ __global__ void __launch_bounds__(kCand ? kCandThreads : kThreads, 1)
         const float s = (ps[0] + ps[1]) + (ps[2] + ps[3]);
         const int key = key0 + hh * kKeys + quarter * 32 + lane;
         if constexpr (kCand) {
-          // this warp's surviving keys are appended with one counter update
+          // this warp's surviving keys are counted and appended with one
+          // counter update.  Keys below the threshold are not counted: every
+          // threshold lies at or below the K-th key's bin, and neither a later
+          // threshold nor the selection reads the counts of lower bins.
           const uint32_t kb = order_bits(s);
-          if (key <= t) atomicAdd(hist_g + (kb >> (32 - kTopkHistBits)), 1u);
           const bool c = key <= t && (kb >> (32 - kTopkHistBits)) >= thr;
+          if (c) atomicAdd(hist_g + (kb >> (32 - kTopkHistBits)), 1u);
           const uint32_t m = __ballot_sync(0xFFFFFFFFu, c);
           pend_m[hh] = m;
           pend_val[hh] = (static_cast<uint64_t>(kb) << 32) | static_cast<uint32_t>(key);

@@ -21,7 +21,8 @@ struct IndexArgs {
   // Selection candidates instead of scores (decode only, with `hist`; see
   // fused_topk_ok): row r appends (order key << 32 | position) to
   // cand[r][0 .. L) for every key that can still be among its top_k, counting
-  // them in cand_n[r * kCandNStride] (zero on entry).
+  // them in cand_n[r * kCandNStride] (zero on entry).  `hist` then counts only
+  // those keys: exact for every bin at or above the K-th key's bin.
   uint64_t* cand = nullptr;
   uint32_t* cand_n = nullptr;
   int top_k = 0;
@@ -57,7 +58,7 @@ cudaError_t launch_topk(const TopkArgs& a, cudaStream_t stream);
 struct TopkCandArgs {
   const uint64_t* cand;  // [rows][L]: (order key << 32 | position), cand_n[r] of them
   uint32_t* cand_n;      // [rows][kCandNStride], word 0 of each row
-  uint32_t* hist;        // [rows][4096] the rows' complete first-level histograms
+  uint32_t* hist;        // [rows][4096] first-level histograms, exact at and above the K-th key's bin
   const int32_t* q_pos;  // [rows]
   int32_t* idx;          // [rows][K]
   int* status;

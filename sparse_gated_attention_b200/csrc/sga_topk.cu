@@ -873,14 +873,14 @@ __global__ void __launch_bounds__(kThreads, 1) sga_topk_resident_kernel(TopkPara
 
 // ---- selection from the indexer's candidates
 // One CTA per row.  The indexer kept every key of the row that can still be
-// among its top K, with its position, and counted the whole row's first radix
-// level, so the bin of the K-th key comes from that histogram.  While the bin
-// holds more keys than the list takes, further levels narrow it with passes
-// over the candidates.  Then one pass marks the candidates above the bin in a
-// position bitmap and lists the ones inside it; the list is refined to the
-// exact K-th key K*, its keys above K* join the bitmap and its keys equal to
-// K* form a tie bitmap, and both are emitted in position order, the lowest
-// positions first among the ties.
+// among its top K, with its position, and counted the first radix level of
+// those keys, which is exact at and above the K-th key's bin, so that bin
+// comes from the histogram.  While the bin holds more keys than the list
+// takes, further levels narrow it with passes over the candidates.  Then one
+// pass marks the candidates above the bin in a position bitmap and lists the
+// ones inside it; the list is refined to the exact K-th key K*, its keys above
+// K* join the bitmap and its keys equal to K* form a tie bitmap, and both are
+// emitted in position order, the lowest positions first among the ties.
 constexpr int kFMaxWords = kFusedTopkMaxL / 32;
 constexpr int kFWordsPerThread = kFMaxWords / kThreads;
 constexpr int kFBatch = 8;  // candidate loads in flight per thread
