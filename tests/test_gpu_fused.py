@@ -70,29 +70,35 @@ def test_fused_matches_oracle(fp8, B, T, L, pos):
     assert_close(out.cpu().numpy(), want_out, f"fused forward, fp8 {fp8}")
 
 
+@pytest.mark.parametrize("fp8", [False, True])
 @pytest.mark.parametrize("k_range,L", [(0, 9000), (1, 20000)])
-def test_fused_wide_threshold_bin(k_range, L):
+def test_fused_wide_threshold_bin(k_range, L, fp8):
     """Every score equal (no threshold ever drops a key, and the K-th key's
     bin holds all 9,000 candidates: the selection narrows it with passes over
     the list down to all 32 bits), or heavy ties; the lowest positions among
-    the ties are taken."""
+    the ties are taken.  Keys in {-1, 0, 1} are exact in E4M3."""
     B = 2
     x = gen_small(B, 1, L, [[L - 1], [L // 2]], k_range=k_range, seed=7)
+    if fp8:
+        x = _as_fp8(x)
     ws = sga.alloc_workspace(sga.make_dims(B, 1, L), sga.OP_FORWARD_FUSED)
-    idx, out = _fused(x, False, ws)
+    idx, out = _fused(x, fp8, ws)
     check_status(ws)
-    want_idx, want_out = _oracle(x, False)
+    want_idx, want_out = _oracle(x, fp8)
     np.testing.assert_array_equal(idx.cpu().numpy(), want_idx)
     assert_close(out.cpu().numpy(), want_out, f"fused forward, k_range {k_range}")
 
 
+@pytest.mark.parametrize("fp8", [False, True])
 @pytest.mark.parametrize("order,L", [("rising", 20000), ("falling", 20000), ("rising", 70000),
                                      ("falling", 70000)])
-def test_fused_monotone_scores(order, L):
+def test_fused_monotone_scores(order, L, fp8):
     """Scores that fall with the position put the top K first, so the
     threshold rises early and drops most later keys; rising scores keep it low
     until the end.  Runs of equal scores split the K-th key's run.  The second
-    call checks that the first left the counters and histograms cleared."""
+    call checks that the first left the counters and histograms cleared.  In
+    E4M3 the key values 0..249 round onto the format's grid, which merges runs
+    into longer ties; both sides use the same codes."""
     B = 2
     run = L // 250 + 1
     x = gen_small(B, 1, L, [[L - 1], [L // 2]], seed=11)
@@ -101,11 +107,13 @@ def test_fused_monotone_scores(order, L):
         c = c.max() - c
     x["k_idx"] = c.to(torch.bfloat16).view(1, L, 1).expand(B, L, 128).contiguous()
     x["q_idx"] = torch.ones_like(x["q_idx"])
+    if fp8:
+        x = _as_fp8(x)
     ws = sga.alloc_workspace(sga.make_dims(B, 1, L), sga.OP_FORWARD_FUSED)
     for _ in range(2):
-        idx, out = _fused(x, False, ws)
+        idx, out = _fused(x, fp8, ws)
         check_status(ws)
-    want_idx, want_out = _oracle(x, False)
+    want_idx, want_out = _oracle(x, fp8)
     np.testing.assert_array_equal(idx.cpu().numpy(), want_idx)
     assert_close(out.cpu().numpy(), want_out, f"fused forward, {order} scores")
 
