@@ -183,3 +183,20 @@ def test_fused_workload_equals_plain_path(name, fp8):
                                 sel(x["gate"]), sel(x["q_pos"]), k=wl.top_k)
         np.testing.assert_array_equal(idx[b].cpu().numpy(), want_idx[0])
         assert_close(out[b].cpu().numpy(), want_out[0], f"{name} seq {b}")
+
+
+def test_fused_above_the_candidate_length_limit():
+    """Rows longer than 262,144 positions take sga_forward's kernels (the
+    candidate lists hold at most that many keys); the results are the same."""
+    B, L = 1, 262144 + 64
+    x = gen_small(B, 1, L, [[L - 1]], k_range=1, seed=17)
+    ws = sga.alloc_workspace(sga.make_dims(B, 1, L), sga.OP_FORWARD_FUSED)
+    assert ws.numel() == sga.workspace_size(sga.make_dims(B, 1, L), sga.OP_FORWARD)
+    idx, out = _fused(x, False, ws)
+    check_status(ws)
+    ws0 = sga.alloc_workspace(sga.make_dims(B, 1, L), sga.OP_FORWARD)
+    idx0, out0 = sga.forward(x["q_idx"], x["w"], x["k_idx"], x["q"], x["kv"], x["gate"], x["q_pos"], ws=ws0)
+    assert torch.equal(idx, idx0) and torch.equal(out, out0)
+    want_idx, want_out = _oracle(x, False)
+    np.testing.assert_array_equal(idx.cpu().numpy(), want_idx)
+    assert_close(out.cpu().numpy(), want_out, "fused forward above the length limit")
