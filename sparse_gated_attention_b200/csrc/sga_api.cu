@@ -164,10 +164,11 @@ sga_status_t index_scores_impl(const sga_dims_t* dims, const void* q_idx, const 
 sga_status_t forward_impl(const sga_dims_t* dims, const void* q_idx, const sga_bf16_t* w, const void* k_idx,
                           const sga_bf16_t* q, const sga_bf16_t* kv, const sga_bf16_t* gate, const int32_t* q_pos,
                           int32_t* idx_out, float* out, void* ws, size_t ws_bytes, sga_stream_t stream, bool fp8,
-                          bool fused) {
+                          bool fused, uint16_t* out_bf16 = nullptr) {
   if (!dims_ok(dims)) return SGA_ERR_INVALID_ARG;
   if (!aligned(q_idx, 16) || !aligned(w, 16) || !aligned(k_idx, 16) || !aligned(q, 16) || !aligned(kv, 16) ||
-      !aligned(q_pos, 4) || !aligned(out, 16) || (gate && !aligned(gate, 2)) || (idx_out && !aligned(idx_out, 16)))
+      !aligned(q_pos, 4) || !aligned(out, 16) || (gate && !aligned(gate, 2)) || (idx_out && !aligned(idx_out, 16)) ||
+      (out_bf16 && !aligned(out_bf16, 8)))
     return SGA_ERR_INVALID_ARG;
   Layout l;
   sga_status_t st = check_ws(ws, ws_bytes, *dims, fused ? SGA_OP_FORWARD_FUSED : SGA_OP_FORWARD, &l);
@@ -215,10 +216,21 @@ sga_status_t forward_impl(const sga_dims_t* dims, const void* q_idx, const sga_b
   if (e != cudaSuccess) return from_cuda(e);
   host::NvtxRange range("sga.sparse_mla_attend");
   AttendArgs aa{q, kv, idx, gate, out, status, dims->batch, dims->n_q, dims->kv_stride, dims->top_k};
+  aa.out_bf16 = out_bf16;
   return from_cuda(launch_attend(aa, s));
 }
 
 }  // namespace
+
+namespace sga {
+sga_status_t forward_bf16_copy(const sga_dims_t* dims, const sga_bf16_t* q_idx, const sga_bf16_t* w,
+                               const sga_bf16_t* k_idx, const sga_bf16_t* q, const sga_bf16_t* kv,
+                               const sga_bf16_t* gate, const int32_t* q_pos, int32_t* idx_out, float* out,
+                               uint16_t* out_bf16, void* ws, size_t ws_bytes, sga_stream_t stream) {
+  return forward_impl(dims, q_idx, w, k_idx, q, kv, gate, q_pos, idx_out, out, ws, ws_bytes, stream, false, false,
+                      out_bf16);
+}
+}  // namespace sga
 
 
 extern "C" {

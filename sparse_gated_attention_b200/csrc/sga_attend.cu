@@ -101,6 +101,7 @@ struct AttendParams {
   const int32_t* idx;
   const uint16_t* gate;
   float* out;
+  uint16_t* out_bf16;  // or null
   int* status;
   int n_q, kv_stride, top_k, splits, chunks_per_split;
   float scale_log2;
@@ -604,9 +605,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_ld32(tmem + lane_addr + blk * kHeads + c * 32, o);
         float* col;
         if (S == 1) {
-          col = p.out + static_cast<size_t>(row) * kHeads * kDv + static_cast<size_t>(c * 32) * kDv + dim;
+          const size_t off = static_cast<size_t>(row) * kHeads * kDv + static_cast<size_t>(c * 32) * kDv + dim;
+          col = p.out + off;
 #pragma unroll
           for (int i = 0; i < 32; ++i) col[static_cast<size_t>(i) * kDv] = o[i] * hf[i];
+          if (p.out_bf16 != nullptr) {
+#pragma unroll
+            for (int i = 0; i < 32; ++i)
+              p.out_bf16[off + static_cast<size_t>(i) * kDv] = __bfloat16_as_ushort(__float2bfloat16_rn(o[i] * hf[i]));
+          }
         } else {
           const int v = dim >> 2;
           const int owner = ((v + 1) * S - 1) / (kDv / 4);  // the r with v0(r) <= v < v0(r + 1)
@@ -634,6 +641,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         acc.w += x.w;
       }
       *reinterpret_cast<float4*>(orow + h * kDv + 4 * (v0 + dv)) = acc;
+      if (p.out_bf16 != nullptr) {
+        const uint32_t lo = pack_bf16(acc.x, acc.y), hi = pack_bf16(acc.z, acc.w);
+        *reinterpret_cast<uint2*>(p.out_bf16 + static_cast<size_t>(row) * kHeads * kDv + h * kDv + 4 * (v0 + dv)) =
+            make_uint2(lo, hi);
+      }
     }
   }
 
@@ -676,6 +688,7 @@ cudaError_t launch_attend(const AttendArgs& a, cudaStream_t stream) {
   p.idx = a.idx;
   p.gate = a.gate;
   p.out = a.out;
+  p.out_bf16 = a.out_bf16;
   p.status = a.status;
   p.n_q = a.n_q;
   p.kv_stride = a.kv_stride;

@@ -5,7 +5,17 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include "../../include/sga.h"
+
 namespace sga {
+
+// sga_forward that also writes the attention output rounded to bf16 (nearest
+// even) into out_bf16 [rows][64][512] (8-byte aligned): the whole layer's W_UV
+// input, without a conversion pass.  Arguments otherwise as sga_forward's.
+sga_status_t forward_bf16_copy(const sga_dims_t* dims, const sga_bf16_t* q_idx, const sga_bf16_t* w,
+                               const sga_bf16_t* k_idx, const sga_bf16_t* q, const sga_bf16_t* kv,
+                               const sga_bf16_t* gate, const int32_t* q_pos, int32_t* idx_out, float* out,
+                               uint16_t* out_bf16, void* ws, size_t ws_bytes, sga_stream_t stream);
 
 // ---- indexer (step 1) --------------------------------------------------------
 struct IndexArgs {
@@ -75,6 +85,7 @@ struct AttendArgs {
   float* out;            // [rows][64][512]
   int* status;
   int batch, n_q, kv_stride, top_k;
+  uint16_t* out_bf16 = nullptr;  // [rows][64][512]: out rounded to bf16 (nearest even) as well, or null
 };
 int attend_splits(int rows, int top_k);
 cudaError_t launch_attend(const AttendArgs& a, cudaStream_t stream);

@@ -424,8 +424,9 @@ sga_status_t project_impl(const sga_dims_t& d, const sga_layer_weights_t* W, con
 }
 
 // out -> bf16, G4 (W_UV per head, bf16 out), G5 (o_proj) and the sum of its partials.
+// With out_b_ready, out_b already holds bf16(out) (written by the attention) and the conversion is skipped.
 sga_status_t output_impl(const sga_dims_t& d, const sga_layer_weights_t* W, const float* out, float* y, void* ws,
-                         const LayerLayout& l, int sms, cudaStream_t s) {
+                         const LayerLayout& l, int sms, cudaStream_t s, bool out_b_ready = false) {
   const int rows = d.batch * d.n_q;
   int* status = at<int>(ws, 0);
   uint16_t* out_b = at<uint16_t>(ws, l.out_b);
@@ -433,7 +434,9 @@ sga_status_t output_impl(const sga_dims_t& d, const sga_layer_weights_t* W, cons
   cudaError_t e;
   {
     sga::host::NvtxRange range("sga.layer.g4_uv");
-    if ((e = launch_convert(out, kLatent, out_b, kLatent, rows * kHeads, kLatent, s)) != cudaSuccess) return from_cuda(e);
+    if (!out_b_ready &&
+        (e = launch_convert(out, kLatent, out_b, kLatent, rows * kHeads, kLatent, s)) != cudaSuccess)
+      return from_cuda(e);
     // G4: o[r][h][i] = bf16(sum_j W_UV[h][i][j] out[r][h][j]): W_UV[h] is [128 i][512 j] (K-major)
     sga::GemmArgs ga{W->w_uv, out_b, kVHead, rows, kLatent, kHeads, false, kHeads * kLatent, kLatent, 1, nullptr, o_b,
                      kOWidth, kVHead, status};
@@ -530,9 +533,11 @@ sga_status_t sga_layer_forward(const sga_dims_t* dims, const sga_layer_weights_t
   if (st != SGA_OK) return st;
   size_t path_bytes = 0;
   sga_workspace_size(dims, SGA_OP_FORWARD, &path_bytes);
-  st = sga_forward(dims, q_idx, w, k_idx_cache, q, kv_cache, gate, q_pos, idx_out, out, ws, path_bytes, stream);
+  // the attention also writes its output in bf16 for W_UV: no conversion pass
+  st = sga::forward_bf16_copy(dims, q_idx, w, k_idx_cache, q, kv_cache, gate, q_pos, idx_out, out,
+                              at<uint16_t>(ws, l.out_b), ws, path_bytes, stream);
   if (st != SGA_OK) return st;
-  return output_impl(*dims, weights, out, y, ws, l, sms, s);
+  return output_impl(*dims, weights, out, y, ws, l, sms, s, true);
 }
 
 }  // extern "C"
