@@ -841,9 +841,9 @@ def main():
             "path_roofline": {"achieved_gbs": layer_gbs, "frac_of_8tbs": layer_gbs / NOMINAL_HBM_GBS,
                               "frac_of_measured": layer_gbs / peak, "bytes_per_step": layer_bytes,
                               "weight_bytes": layer["weight_bytes"]},
-            # own kernels per step: five GEMMs, two projection preps, the out conversion, the
-            # G5 partial sum, the path's three
-            "gpu_launches": 12 * args.steps}
+            # own kernels per step: five GEMMs, two projection preps, the G5 partial sum, the
+            # path's three (the attention also writes the bf16 copy of its output for W_UV)
+            "gpu_launches": 11 * args.steps}
 
     cpu = None
     if not args.no_cpu_baseline and world == 1:
