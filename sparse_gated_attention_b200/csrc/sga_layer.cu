@@ -133,8 +133,10 @@ struct Partials {
   }
 };
 
-constexpr int kPrepHParts = 4;  // blocks per token
-constexpr int kPrepQParts = 8;
+// Blocks per token: enough threads that each takes one or two items, so the
+// summed split partials of an item are the only memory round trips in its chain.
+constexpr int kPrepHParts = 9;   // 2,272 items per token with R = 1536
+constexpr int kPrepQParts = 36;  // 18,496 items per token
 
 // Blocks (token, part): c_q, w and the token's cache rows (c_kv, rotated
 // k_rope, k_idx), the elements of a token dealt round-robin over its parts.
