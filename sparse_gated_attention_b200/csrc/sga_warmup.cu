@@ -387,20 +387,28 @@ __global__ void __launch_bounds__(kThreads, 2) warmup_grad_kernel(WarmupArgs p) 
       sga::cp_async_16(ki_s + (pc >> 3) * kBox + r * 128 + (((pc & 7) ^ (r & 7)) << 4), src, sr >= 0 ? 16u : 0u);
     }
   }
-  // ---- the target's per-head statistics: the chunks' (max, sum) pairs merged
-  for (int h = warp; h < kHeads; h += kThreads / 32) {
-    const float2* st = p.stats + (static_cast<size_t>(row) * kHeads + h) * nch;
-    float m = -INFINITY;
-    for (int cc = lane; cc < nch; cc += 32) m = fmaxf(m, st[cc].x);
-    m = warp_max(m);
-    float l = 0.f;
-    if (m != -INFINITY)
-      for (int cc = lane; cc < nch; cc += 32)
-        if (st[cc].x != -INFINITY) l += st[cc].y * expf(st[cc].x - m);
-    l = warp_sum(l);
-    if (lane == 0) {
-      hm[h] = m;
-      hinv[h] = l > 0.f ? 1.f / l : 0.f;
+  // ---- the target's per-head statistics: the chunks' (max, sum) pairs merged.  A query has at
+  // most 32 chunks, one pair per lane; a warp loads all of its heads' pairs before reducing any.
+  {
+    constexpr int kHeadsPerWarp = kHeads / (kThreads / 32);
+    static_assert(SGA_MAX_TOP_K / kChunk <= 32, "one chunk per lane");
+    float2 v[kHeadsPerWarp];
+#pragma unroll
+    for (int i = 0; i < kHeadsPerWarp; ++i) {
+      const int h = warp + i * (kThreads / 32);
+      v[i] = lane < nch ? p.stats[(static_cast<size_t>(row) * kHeads + h) * nch + lane] : make_float2(-INFINITY, 0.f);
+    }
+#pragma unroll
+    for (int i = 0; i < kHeadsPerWarp; ++i) {
+      const int h = warp + i * (kThreads / 32);
+      const float m = warp_max(v[i].x);
+      float l = 0.f;
+      if (m != -INFINITY && v[i].x != -INFINITY) l = v[i].y * expf(v[i].x - m);
+      l = warp_sum(l);
+      if (lane == 0) {
+        hm[h] = m;
+        hinv[h] = l > 0.f ? 1.f / l : 0.f;
+      }
     }
   }
   // ---- the indexer softmax's normaliser over the query's valid slots: the chunks' (max, sum) pairs merged
