@@ -573,10 +573,12 @@ __global__ void __launch_bounds__(kThreads, 2) warmup_grad_kernel(WarmupArgs p) 
 __global__ void __launch_bounds__(kThreads) warmup_loss_kernel(WarmupArgs p, bool clear_grads) {
   const int row = blockIdx.x, t = threadIdx.x;
   const int nch = p.top_k / kChunk;
-  if (t == 0 && !clear_grads) {
+  if (t < 32 && !clear_grads) {
+    // all of the query's terms loaded at once (at most 32 chunks, one per lane), then summed in chunk order
+    const float v = t < nch ? p.loss_part[static_cast<size_t>(row) * nch + t] : 0.f;
     float sum = 0.f;
-    for (int cc = 0; cc < nch; ++cc) sum += p.loss_part[static_cast<size_t>(row) * nch + cc];
-    p.loss[row] = sum;
+    for (int cc = 0; cc < nch; ++cc) sum += __shfl_sync(0xFFFFFFFFu, v, cc);
+    if (t == 0) p.loss[row] = sum;
   }
   if (clear_grads) {
     for (int e = t; e < kIdxHeads * kIdxDim; e += kThreads)
