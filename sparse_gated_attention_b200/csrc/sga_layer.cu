@@ -122,13 +122,22 @@ struct PrepHArgs {
 };
 
 // The sum of a GEMM output's `splits` partials, in split order.
+// Split partials of one GEMM output element (at most kMaxGemmSplits of them,
+// the bound gemm_splits keeps): all loads issued before the first add, then
+// added in split order.
+constexpr int kMaxGemmSplits = 8;
 struct Partials {
   const float* base;
   int splits;
   size_t stride;
   __device__ __forceinline__ float operator[](size_t i) const {
-    float v = base[i];
-    for (int s = 1; s < splits; ++s) v += base[static_cast<size_t>(s) * stride + i];
+    float u[kMaxGemmSplits];
+#pragma unroll
+    for (int s = 0; s < kMaxGemmSplits; ++s) u[s] = s < splits ? base[static_cast<size_t>(s) * stride + i] : 0.f;
+    float v = u[0];
+#pragma unroll
+    for (int s = 1; s < kMaxGemmSplits; ++s)
+      if (s < splits) v += u[s];
     return v;
   }
 };
@@ -255,13 +264,21 @@ __global__ void sum_partials_kernel(const float* part, int splits, size_t stride
   const size_t n4 = count / 4;
   for (size_t e = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; e < n4;
        e += static_cast<size_t>(gridDim.x) * blockDim.x) {
-    float4 v = reinterpret_cast<const float4*>(part)[e];
-    for (int s = 1; s < splits; ++s) {
-      const float4 u = reinterpret_cast<const float4*>(part + static_cast<size_t>(s) * stride)[e];
-      v.x += u.x;
-      v.y += u.y;
-      v.z += u.z;
-      v.w += u.w;
+    // every split's partial loaded before the first add, then added in split order
+    float4 u[kMaxGemmSplits];
+#pragma unroll
+    for (int s = 0; s < kMaxGemmSplits; ++s)
+      u[s] = s < splits ? reinterpret_cast<const float4*>(part + static_cast<size_t>(s) * stride)[e]
+                        : make_float4(0.f, 0.f, 0.f, 0.f);
+    float4 v = u[0];
+#pragma unroll
+    for (int s = 1; s < kMaxGemmSplits; ++s) {
+      if (s < splits) {
+        v.x += u[s].x;
+        v.y += u[s].y;
+        v.z += u[s].z;
+        v.w += u[s].w;
+      }
     }
     reinterpret_cast<float4*>(y)[e] = v;
   }
