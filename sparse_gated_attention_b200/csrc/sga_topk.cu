@@ -84,6 +84,32 @@ struct TopkParams {
   long long words_per_row;
 };
 
+// ghist = the sum of every cluster CTA's lhist.  Thread t takes bins 4t .. 4t + 3:
+// one 16-byte shared-memory load per CTA, four CTAs' loads issued before any
+// is added.
+__device__ __forceinline__ void cluster_hist_sum(cg::cluster_group& cluster, const uint32_t* lhist, uint32_t* ghist,
+                                                 int C) {
+  static_assert(kBins == 4 * kThreads, "four bins per thread");
+  const int tid = threadIdx.x;
+  constexpr int kInFlight = 4;
+  uint4 acc = make_uint4(0u, 0u, 0u, 0u);
+  for (int r0 = 0; r0 < C; r0 += kInFlight) {
+    uint4 v[kInFlight];
+#pragma unroll
+    for (int k = 0; k < kInFlight; ++k)
+      v[k] = r0 + k < C ? reinterpret_cast<const uint4*>(cluster.map_shared_rank(lhist, r0 + k))[tid]
+                        : make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+    for (int k = 0; k < kInFlight; ++k) {
+      acc.x += v[k].x;
+      acc.y += v[k].y;
+      acc.z += v[k].z;
+      acc.w += v[k].w;
+    }
+  }
+  reinterpret_cast<uint4*>(ghist)[tid] = acc;
+}
+
 // Inclusive block scan of one value per thread; also returns the block total.
 __device__ __forceinline__ uint32_t block_inclusive_scan(uint32_t v, uint32_t* warp_buf, uint32_t& total) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -423,11 +449,7 @@ __global__ void __launch_bounds__(kThreads, 1) sga_topk_stream_kernel(TopkParams
       }
       if (kVec) consumed += nch;
       cluster.sync();
-      for (int b = tid; b < kBins; b += kThreads) {
-        uint32_t acc = 0;
-        for (int r = 0; r < C; ++r) acc += cluster.map_shared_rank(lhist, r)[b];
-        ghist[b] = acc;
-      }
+      cluster_hist_sum(cluster, lhist, ghist, C);
       cluster.sync();  // every CTA has read every histogram
     }
     first = false;
@@ -724,11 +746,7 @@ __global__ void __launch_bounds__(kThreads, 1) sga_topk_resident_kernel(TopkPara
         }
       }
       cluster.sync();
-      for (int b = tid; b < kBins; b += kThreads) {
-        uint32_t acc = 0;
-        for (int r = 0; r < C; ++r) acc += cluster.map_shared_rank(lhist, r)[b];
-        ghist[b] = acc;
-      }
+      cluster_hist_sum(cluster, lhist, ghist, C);
       cluster.sync();  // every CTA has read every histogram
     }
     first = false;
