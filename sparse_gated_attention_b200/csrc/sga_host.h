@@ -2,6 +2,7 @@
 // the status block at the start of every workspace, pointer checks.
 #pragma once
 
+#include <cuda_runtime.h>
 #include <nvtx3/nvToolsExt.h>
 #include <stddef.h>
 #include <stdint.h>
@@ -31,6 +32,26 @@ struct NvtxRange {
   NvtxRange(const NvtxRange&) = delete;
   NvtxRange& operator=(const NvtxRange&) = delete;
 };
+
+// Launches `kernel` with programmatic dependent launch: its grid may be
+// scheduled once every CTA of the previous kernel on the stream has called
+// griddepcontrol.launch_dependents (or exited), so its set-up overlaps that
+// kernel's tail; its griddepcontrol.wait orders the reads that depend on it.
+template <class... Params, class... Args>
+cudaError_t launch_pdl(void (*kernel)(Params...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                       Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
 
 }  // namespace host
 }  // namespace sga

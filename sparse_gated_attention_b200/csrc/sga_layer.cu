@@ -287,16 +287,7 @@ __global__ void sum_partials_kernel(const float* part, int splits, size_t stride
 // Launches `kernel` on `grid` x 256 threads with programmatic dependent launch.
 template <class... Params, class... Args>
 cudaError_t launch_pdl(void (*kernel)(Params...), dim3 grid, cudaStream_t s, Args... args) {
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = grid;
-  cfg.blockDim = dim3(256);
-  cfg.stream = s;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, kernel, args...);
+  return sga::host::launch_pdl(kernel, grid, dim3(256), 0, s, args...);
 }
 
 cudaError_t launch_convert(const float* src, int src_ld, uint16_t* dst, int dst_ld, int n_rows, int n_cols,

@@ -49,6 +49,7 @@ using sga::host::align_up;
 using sga::host::aligned;
 using sga::host::at;
 using sga::host::kStatusBytes;
+using sga::host::launch_pdl;
 constexpr size_t kAlign = sga::host::kWsAlign;
 
 // kernel A (tensor core): 10 swizzled boxes of 64 rows x 64 bf16, and the 1 KB alignment
@@ -163,6 +164,10 @@ __global__ void __launch_bounds__(kLogitThreads, 2) warmup_logits_kernel(WarmupA
   __syncthreads();
   sga::tc_fence_after();
   const uint32_t tmem = tmem_slot;
+  // This kernel reads only the caller's inputs, and its writes go to regions
+  // whose last reader (the previous call's kernel C) finished before this grid
+  // could start; its tensor memory is held, so kernel C may be scheduled now.
+  sga::grid_launch_dependents();
   const uint16_t* qrow = p.q + static_cast<size_t>(row) * kHeads * kDq;
   bool ok = true;
   int committed = 0;  // MMA batches committed to mma_bar
@@ -322,6 +327,9 @@ __global__ void __launch_bounds__(kLogitThreads, 2) warmup_logits_kernel(WarmupA
   }
   __syncthreads();
   if (ok && t == 0) p.score_stats[static_cast<size_t>(row) * nch + c] = make_float2(cmax, ssum_w[0] + ssum_w[1]);
+  // not done before the first kernel B is: kernel C, which waits for this
+  // grid, adds into the gradients that kernel B clears
+  sga::grid_dependency_wait();
 }
 
 // C: per (query, chunk), the objective for the chunk's slots, then their
@@ -387,6 +395,11 @@ __global__ void __launch_bounds__(kThreads, 2) warmup_grad_kernel(WarmupArgs p) 
       sga::cp_async_16(ki_s + (pc >> 3) * kBox + r * 128 + (((pc & 7) ^ (r & 7)) << 4), src, sr >= 0 ? 16u : 0u);
     }
   }
+  // The above reads the caller's inputs only; the statistics, z, a and the
+  // scores below come from kernel A, and the gradients added into at the end
+  // were cleared by the first kernel B.
+  sga::grid_dependency_wait();
+  sga::grid_launch_dependents();
   // ---- the target's per-head statistics: the chunks' (max, sum) pairs merged.  A query has at
   // most 32 chunks, one pair per lane; a warp loads all of its heads' pairs before reducing any.
   {
@@ -573,6 +586,9 @@ __global__ void __launch_bounds__(kThreads, 2) warmup_grad_kernel(WarmupArgs p) 
 __global__ void __launch_bounds__(kThreads) warmup_loss_kernel(WarmupArgs p, bool clear_grads) {
   const int row = blockIdx.x, t = threadIdx.x;
   const int nch = p.top_k / kChunk;
+  // the terms come from kernel C; the gradients cleared here may still be read by earlier work
+  sga::grid_dependency_wait();
+  sga::grid_launch_dependents();
   if (t < 32 && !clear_grads) {
     // all of the query's terms loaded at once (at most 32 chunks, one per lane), then summed in chunk order
     const float v = t < nch ? p.loss_part[static_cast<size_t>(row) * nch + t] : 0.f;
@@ -667,14 +683,17 @@ sga_status_t sga_indexer_warmup(const sga_dims_t* dims, const sga_bf16_t* q_idx,
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const int rows = dims->batch * dims->n_q;
   const dim3 grid(dims->top_k / kChunk, rows);
-  warmup_loss_kernel<<<rows, kThreads, 0, s>>>(a, true);
-  if (cudaGetLastError() != cudaSuccess) return SGA_ERR_CUDA;
-  warmup_logits_kernel<<<grid, kLogitThreads, kLogitsSmem, s>>>(a);
-  if (cudaGetLastError() != cudaSuccess) return SGA_ERR_CUDA;
-  warmup_grad_kernel<<<grid, kThreads, kGradSmem, s>>>(a);
-  if (cudaGetLastError() != cudaSuccess) return SGA_ERR_CUDA;
-  warmup_loss_kernel<<<rows, kThreads, 0, s>>>(a, false);
-  return cudaGetLastError() == cudaSuccess ? SGA_OK : SGA_ERR_CUDA;
+  // Every launch is programmatic: each kernel's set-up overlaps the previous
+  // kernel's tail, and its grid_dependency_wait orders what depends on it.
+  cudaError_t e = launch_pdl(warmup_loss_kernel, dim3(rows), dim3(kThreads), 0, s, a, true);
+  if (e == cudaSuccess) e = launch_pdl(warmup_logits_kernel, grid, dim3(kLogitThreads), kLogitsSmem, s, a);
+  if (e == cudaSuccess) e = launch_pdl(warmup_grad_kernel, grid, dim3(kThreads), kGradSmem, s, a);
+  if (e == cudaSuccess) e = launch_pdl(warmup_loss_kernel, dim3(rows), dim3(kThreads), 0, s, a, false);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return SGA_ERR_CUDA;
+  }
+  return SGA_OK;
 }
 
 }  // extern "C"
