@@ -69,3 +69,33 @@ def test_indexer_warmup_other_top_k(K):
     for k in ("grad_q_idx", "grad_w", "grad_k_idx"):
         r = rel_l2(got[k].cpu().numpy().astype(np.float64), want[k])
         assert r <= 1e-3, (k, r)
+
+
+def test_indexer_warmup_back_to_back_calls():
+    """Two calls on one stream with one workspace and no synchronisation between
+    them, the second call's selection coming straight from sga_forward on the same
+    stream.  The launches overlap through programmatic dependent launch: the
+    second call's kernels must still see the forward's indices, and must not
+    overwrite the workspace's logits and statistics before the first call's
+    gradient kernel has read them.  Both results are checked against the oracle."""
+    B, T, L = 2, 1, 3000
+    wl = synth.custom(batch=B, n_q=T, ctx=L, first_pos=L - 1)
+    x1 = synth.make_inputs(wl, device="cuda", seed=11)
+    x2 = synth.make_inputs(wl, device="cuda", seed=12)
+    want1 = W.warmup_loss(x1["q_idx"], x1["w"], x1["k_idx"], x1["q"], x1["kv"], x1["q_pos"].cpu())
+    want2 = W.warmup_loss(x2["q_idx"], x2["w"], x2["k_idx"], x2["q"], x2["kv"], x2["q_pos"].cpu())
+    idx1 = torch.as_tensor(want1["idx"], device="cuda")
+    ws = torch.zeros(sga.indexer_warmup_workspace_size(sga.make_dims(B, T, L)), dtype=torch.uint8, device="cuda")
+    fws = sga.alloc_workspace(sga.make_dims(B, T, L), sga.OP_FORWARD, "cuda")
+    torch.cuda.synchronize()
+    got1 = sga.indexer_warmup(x1["q_idx"], x1["w"], x1["k_idx"], x1["q"], x1["kv"], idx1, ws=ws)
+    idx2, _ = sga.forward(x2["q_idx"], x2["w"], x2["k_idx"], x2["q"], x2["kv"], x2["gate"], x2["q_pos"], ws=fws)
+    got2 = sga.indexer_warmup(x2["q_idx"], x2["w"], x2["k_idx"], x2["q"], x2["kv"], idx2, ws=ws)
+    torch.cuda.synchronize()
+    assert sga.device_status(ws) == 0 and sga.device_status(fws) == 0
+    np.testing.assert_array_equal(idx2.cpu().numpy(), want2["idx"])
+    for got, want in ((got1, want1), (got2, want2)):
+        np.testing.assert_allclose(got["loss"].cpu().numpy(), want["per_query"], rtol=1e-4)
+        for k in ("grad_q_idx", "grad_w", "grad_k_idx"):
+            r = rel_l2(got[k].cpu().numpy().astype(np.float64), want[k])
+            assert r <= 1e-3, (k, r)
