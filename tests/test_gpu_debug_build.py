@@ -2,7 +2,8 @@
 device-side invariant checks compiled in: gathered rows inside their sequence,
 emitted slots and positions inside their row, the selection's candidate list
 within its capacity, GEMM work items inside their tensors, prefill query blocks
-inside their sequence) runs a forward, a prefill-shaped forward, a long-row
+inside their sequence) runs a forward, a prefill-shaped forward, the fused
+selection with bf16 and E4M3 keys, the indexer's warm-up objective, a long-row
 top-k and a layer forward in a process of its own.  Every check must hold
 (the workspace status stays SGA_OK) and the results must match the oracle as
 the release build's do."""
@@ -44,6 +45,32 @@ for B, T, L, seed in [(3, 1, 9000, 0), (2, 12, 6000, 1)]:
     want_idx, want_out = oracle.forward(x["q_idx"], x["w"], x["k_idx"], x["q"], x["kv"], x["gate"], x["q_pos"].cpu())
     assert np.array_equal(idx.cpu().numpy(), want_idx)
     assert close(out.cpu().numpy(), want_out)
+
+# the fused selection (candidate lists within their capacity), bf16 and E4M3 keys, on the decode case
+B, T, L = 3, 1, 9000
+wl = synth.custom(batch=B, n_q=T, ctx=L, first_pos=L - T)
+x = synth.make_inputs(wl, device="cuda", seed=0)
+want_idx, want_out = oracle.forward(x["q_idx"], x["w"], x["k_idx"], x["q"], x["kv"], x["gate"], x["q_pos"].cpu())
+ws = sga.alloc_workspace(sga.make_dims(B, T, L), sga.OP_FORWARD_FUSED)
+for fp8 in (False, True):
+    qi, ki = (synth.to_e4m3(x["q_idx"]), synth.to_e4m3(x["k_idx"])) if fp8 else (x["q_idx"], x["k_idx"])
+    call = sga.forward_fused_fp8 if fp8 else sga.forward_fused
+    idx, out = call(qi, x["w"], ki, x["q"], x["kv"], x["gate"], x["q_pos"], ws=ws)
+    assert sga.device_status(ws) == 0, ("fused", fp8, sga.device_status(ws))
+    assert np.array_equal(idx.cpu().numpy(), want_idx), ("fused", fp8)  # integer inputs: E4M3 codes are exact
+    assert close(out.cpu().numpy(), want_out), ("fused", fp8)
+
+# the indexer's warm-up objective over the oracle's selection
+from oracle import warmup as warmup_oracle
+want = warmup_oracle.warmup_loss(x["q_idx"], x["w"], x["k_idx"], x["q"], x["kv"], x["q_pos"].cpu())
+wws = torch.zeros(sga.indexer_warmup_workspace_size(sga.make_dims(B, T, L)), dtype=torch.uint8, device="cuda")
+got = sga.indexer_warmup(x["q_idx"], x["w"], x["k_idx"], x["q"], x["kv"], torch.as_tensor(want["idx"], device="cuda"),
+                         ws=wws)
+assert sga.device_status(wws) == 0
+assert np.allclose(got["loss"].cpu().numpy(), want["per_query"], rtol=1e-4, atol=0)
+for k in ("grad_q_idx", "grad_w", "grad_k_idx"):
+    g_ = got[k].cpu().numpy().astype(np.float64)
+    assert np.linalg.norm(g_ - want[k]) <= 1e-3 * np.linalg.norm(want[k]), k
 
 # a long row: the streaming top-k with its words in the workspace
 g = torch.Generator(device="cuda").manual_seed(2)
