@@ -395,6 +395,36 @@ def prefill_variant(sga, synth, args, dev, stream, dist, rank) -> dict:
             "gpu_launches": 3}
 
 
+def graph_replay_ms(make_step, args, dev, dist) -> float:
+    """`args.steps` calls of a step captured in one CUDA graph and replayed, as a
+    serving loop launches its decode steps.  make_step(stream) returns the step
+    bound to a stream; its one-time set-up must have run before (outside the
+    capture).  Untimed replays cover at least 3 warm-up steps, then one replay
+    is timed between CUDA events on the capture stream (max over ranks)."""
+    gs = torch.cuda.Stream(dev)
+    gs.wait_stream(torch.cuda.current_stream(dev))
+    step = make_step(gs)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=gs):
+        for _ in range(args.steps):
+            step()
+    with torch.cuda.stream(gs):
+        for _ in range(max(1, -(-3 // args.steps))):
+            graph.replay()
+    torch.cuda.synchronize(dev)
+    if dist is not None:
+        dist.barrier()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(gs):
+        a.record(gs)
+        graph.replay()
+        b.record(gs)
+    torch.cuda.synchronize(dev)
+    ms = max_over_ranks(dist, dev, a.elapsed_time(b))
+    del graph
+    return ms
+
+
 def layer_variant(sga, synth, args, dev, stream, dist, rank, x, dims, idx) -> dict:
     """One whole SGA layer (a separate configuration): h -> projections -> the path
     -> W_UV, o_proj, on the workload's caches (the new tokens' rows are rewritten
@@ -407,9 +437,9 @@ def layer_variant(sga, synth, args, dev, stream, dist, rank, x, dims, idx) -> di
     ws_layer = sga.alloc_layer_workspace(dims, sga.layer_weights(lw_t), sga.LAYER_FORWARD, dev)
     y = torch.empty((B, T, synth.D_MODEL), dtype=torch.float32, device=dev)
 
-    def layer_step():
+    def layer_step(st=stream):
         sga.layer_forward(lw_t, h, x["q_pos"], x["kv"], x["k_idx"], top_k=K, idx_out=idx, y=y, ws=ws_layer,
-                          stream=stream)
+                          stream=st)
 
     for _ in range(max(args.warmup, 3)):
         layer_step()
@@ -425,8 +455,16 @@ def layer_variant(sga, synth, args, dev, stream, dist, rank, x, dims, idx) -> di
     layer_ms = max_over_ranks(dist, dev, s4.elapsed_time(e4))
     if sga.device_status(ws_layer) != 0:
         raise RuntimeError("device status set during the layer variant run")
+    try:
+        graph_ms = graph_replay_ms(lambda st: (lambda: layer_step(st)), args, dev, dist)
+        if sga.device_status(ws_layer) != 0:
+            raise RuntimeError("device status set during the layer's graph replay")
+    except (RuntimeError, TypeError, ValueError) as exc:
+        torch.cuda.synchronize(dev)
+        graph_ms = f"{type(exc).__name__}: {exc}"
     weight_bytes = sum(t.numel() * t.element_size() for t in lw_t.values())
-    return {"ms": layer_ms, "weight_bytes": weight_bytes, "act_bytes": h.numel() * 2 + y.numel() * 4}
+    return {"ms": layer_ms, "graph_ms": graph_ms, "weight_bytes": weight_bytes,
+            "act_bytes": h.numel() * 2 + y.numel() * 4}
 
 
 def fused_variant(sga, synth, args, wl, x, dev, stream, dist, xf=None, idx=None, out=None) -> dict:
@@ -547,7 +585,9 @@ def main():
         il = torch.empty((wl_l.batch, wl_l.n_q, wl_l.top_k), dtype=torch.int32, device=dev)
         res = layer_variant(sga, synth, args, dev, torch.cuda.current_stream(dev), dist, rank, xl, dl, il)
         if rank == 0:
+            g = res["graph_ms"]
             print(json.dumps({"variant": "sga_layer", "ms_per_step": res["ms"] / args.steps,
+                              "graph_replay_ms_per_step": g / args.steps if isinstance(g, float) else g,
                               "weight_bytes": res["weight_bytes"]}), flush=True)
         return
     if args.warmup_only:
@@ -736,6 +776,18 @@ def main():
 
     fp8_ms = region_ms(fp8_step, ws_all, "E4M3 variant")
 
+    # ---- the headline step replayed from a CUDA graph (the same sga_forward calls,
+    # captured once): what a serving loop that launches through graphs sees
+    try:
+        graph_ms = graph_replay_ms(lambda st: (lambda: sga.forward(
+            x["q_idx"], x["w"], x["k_idx"], x["q"], x["kv"], x["gate"], x["q_pos"], top_k=K, idx_out=idx, out=out,
+            ws=ws_all, stream=st)), args, dev, dist)
+        if sga.device_status(ws_all) != 0:
+            raise RuntimeError("device status set during the graph replay")
+    except (RuntimeError, TypeError, ValueError) as exc:
+        torch.cuda.synchronize(dev)
+        graph_ms = f"{type(exc).__name__}: {exc}"
+
     # ---- the fused selection (sga_forward_fused, an opt-in entry point with the
     # same results): the indexer appends candidates instead of writing scores
     fused_ms = fused8_ms = None
@@ -812,6 +864,18 @@ def main():
         "path_roofline": {"achieved_gbs": fp8_gbs, "frac_of_8tbs": fp8_gbs / NOMINAL_HBM_GBS,
                           "frac_of_measured": fp8_gbs / peak, "bytes_per_query": ab8["total"]},
         "gpu_launches": launches_per_step * args.steps}}
+    if isinstance(graph_ms, float):
+        g_step_ms = graph_ms / args.steps
+        g_gbs = ab["total"] * rows / (g_step_ms * 1e-3) / 1e9
+        variants["graph_replay"] = {
+            "value": whole_job_rate(rows, args.steps, world, graph_ms), "unit": UNIT, "ms_per_step": g_step_ms,
+            "config": f"{wl.name}: the headline's {args.steps} sga_forward calls captured in one CUDA graph and "
+                      f"replayed (the launches become graph kernel nodes with their programmatic dependencies)",
+            "path_roofline": {"achieved_gbs": g_gbs, "frac_of_8tbs": g_gbs / NOMINAL_HBM_GBS,
+                              "frac_of_measured": g_gbs / peak, "bytes_per_query": ab["total"]},
+            "gpu_launches": launches_per_step * args.steps}
+    else:
+        variants["graph_replay"] = {"error": graph_ms}
     if fused_ms is not None:
         for key, ms, bpq, cfg in (("fused_selection", fused_ms, ab["total"], wl.name),
                                   ("fused_selection_fp8_index_keys", fused8_ms, ab8["total"],
@@ -844,6 +908,10 @@ def main():
             # own kernels per step: five GEMMs, two projection preps, the G5 partial sum, the
             # path's three (the attention also writes the bf16 copy of its output for W_UV)
             "gpu_launches": 11 * args.steps}
+        if isinstance(layer["graph_ms"], float):
+            variants["sga_layer"]["graph_replay_ms_per_step"] = layer["graph_ms"] / args.steps
+        else:
+            variants["sga_layer"]["graph_replay_error"] = layer["graph_ms"]
 
     cpu = None
     if not args.no_cpu_baseline and world == 1:
