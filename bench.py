@@ -405,7 +405,8 @@ def graph_replay_ms(make_step, args, dev, dist) -> float:
     gs.wait_stream(torch.cuda.current_stream(dev))
     step = make_step(gs)
     graph = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(graph, stream=gs):
+    # thread-local capture: other threads' CUDA calls (a process group's watchdog) stay legal meanwhile
+    with torch.cuda.graph(graph, stream=gs, capture_error_mode="thread_local"):
         for _ in range(args.steps):
             step()
     with torch.cuda.stream(gs):
